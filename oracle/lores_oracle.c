@@ -1,0 +1,316 @@
+/*
+ * lores_oracle.c -- plain, slow CPU oracle for one LoReS decode step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or
+ * calls this file.  It is used by the test-suite, by the smoke check and by
+ * the CPU-baseline leg of the benchmark.  It shares no source with the CUDA
+ * library: every definition below is written out again from the method's
+ * description and from the arithmetic definition of the state format.
+ *
+ * Sources (page titles; "Quantizing Recurrent Language Models Is Easier Than
+ * You Think", summary page):
+ *   - General recurrence form, Introduction:  S_t = S_{t-1} diag(a_t)
+ *     (I - delta beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
+ *   - Key properties, Intra-State Quantization: the state is dequantized,
+ *     updated and requantized on every decode step.
+ *   - Proposition 1: symmetric absmax scale s_G = max|S_G| / r with
+ *     r = 2^(b-1) - 1; value-axis grouping (one scale per value row, here
+ *     optionally split into key blocks of G entries).
+ *   - Proposition 3 / Table 6: stochastic rounding of the requantization.
+ *   - Table 5 text and the abstract: decay-based mixed precision per head.
+ *
+ * Readings where the pages are silent (each is a choice, not a page fact):
+ *   - Scales are recomputed from the updated state on every step.
+ *   - The readout o_t uses the updated fp32 state before requantization.
+ *   - Products and sums are fp32 with the association written below; the
+ *     dot product S'k uses a fixed order (16-column sequential chunks, then a
+ *     pairwise combine of the chunk sums) so that two implementations that
+ *     follow it agree bit for bit.  The readout is summed in double.
+ *   - Stochastic rounding adds an 8-bit dither on a grid of 1/256 of a code
+ *     step: t = fma(x, r/m, 49152 + d/256); code = floor(t - 49152).  49152 is
+ *     1.5 * 2^15, whose float spacing is exactly 1/256, so the fma rounds
+ *     x*r/m to the nearest 1/256 and adds d/256 exactly.  With d uniform in
+ *     0..255 the code is unbiased up to that 1/512-step rounding.
+ *   - The dither bytes come from SplitMix64 (Steele, Lea, Flood 2014) and the
+ *     MurmurHash3 32-bit finalizer (Appleby), keyed on seed, step, sequence,
+ *     head, row and column.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -frounding-math -fPIC -shared
+ * (no fast-math; fmaf is used only where the definition says fma).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Counter-based random bits                                                */
+/* ------------------------------------------------------------------------ */
+
+/* SplitMix64 output for generator state z (state advanced by the golden
+ * gamma, then the variant-13 mixer).  Steele, Lea & Flood, "Fast splittable
+ * pseudorandom number generators", OOPSLA 2014; constants as published by
+ * Vigna for splitmix64. */
+uint64_t lo_splitmix64(uint64_t z)
+{
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+/* MurmurHash3 32-bit finalizer (Appleby). */
+uint32_t lo_fmix32(uint32_t h)
+{
+    h ^= h >> 16;
+    h *= 0x85EBCA6Bu;
+    h ^= h >> 13;
+    h *= 0xC2B2AE35u;
+    h ^= h >> 16;
+    return h;
+}
+
+/* 32-bit key of one decode step of one handle. */
+uint32_t lo_step_key(uint64_t seed, uint64_t step)
+{
+    uint64_t k = lo_splitmix64(seed ^ lo_splitmix64(step));
+    return (uint32_t)(k ^ (k >> 32));
+}
+
+/* 32-bit key of one (sequence, head) tile: tile_index = b * H + h. */
+uint32_t lo_tile_key(uint32_t step_key, uint32_t tile_index)
+{
+    return lo_fmix32(step_key + 0x85EBCA77u * (tile_index + 1u));
+}
+
+/* Dither byte d in 0..255 for state element (i, j) of a tile.  Four
+ * consecutive columns share one 32-bit hash; column j takes byte j mod 4. */
+uint32_t lo_dither(uint32_t tile_key, int d_k, int i, int j)
+{
+    uint32_t n = (uint32_t)i * (uint32_t)(d_k / 4) + (uint32_t)(j / 4);
+    uint32_t h = lo_fmix32(tile_key + 0x9E3779B9u * (n + 1u));
+    return (h >> (8 * (j % 4))) & 0xFFu;
+}
+
+/* ------------------------------------------------------------------------ */
+/* State layout                                                             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int d_k, d_v;      /* state is d_v x d_k (value rows, key columns)       */
+    int group;         /* key entries per scale, divides d_k                 */
+    int bits;          /* 8, 4, or 32 (unquantized fp32 state)               */
+    int delta;         /* 0 or 1: delta correction on/off                     */
+    int diag;          /* 0: scalar decay; 1: decay per key column           */
+    int stochastic;    /* 1: stochastic rounding; 0: round to nearest        */
+} lo_cfg;
+
+static int code_max(int bits) { return (1 << (bits - 1)) - 1; }
+
+/* Read code (i, j) from a packed tile.  int8: one byte per code, two's
+ * complement.  int4: two codes per byte, even column in the low nibble, odd
+ * column in the high nibble, two's complement nibbles. */
+static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
+{
+    if (c->bits == 8)
+        return (int)(int8_t)codes[(size_t)i * c->d_k + j];
+    uint8_t byte = codes[(size_t)i * (c->d_k / 2) + j / 2];
+    int nib = (j % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+static void put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code)
+{
+    if (c->bits == 8) {
+        codes[(size_t)i * c->d_k + j] = (uint8_t)(int8_t)code;
+        return;
+    }
+    size_t at = (size_t)i * (c->d_k / 2) + j / 2;
+    uint8_t nib = (uint8_t)(code & 0xF);
+    if (j % 2 == 0)
+        codes[at] = (uint8_t)((codes[at] & 0xF0) | nib);
+    else
+        codes[at] = (uint8_t)((codes[at] & 0x0F) | (nib << 4));
+}
+
+int lo_get_code(const lo_cfg *c, const uint8_t *codes, int i, int j) { return get_code(c, codes, i, j); }
+void lo_put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code) { put_code(c, codes, i, j, code); }
+
+/* ------------------------------------------------------------------------ */
+/* Fixed-order dot product                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* sum_j a_j b_j for n = 16*C, C a power of two <= 16: each chunk of 16
+ * consecutive terms is a sequential fma chain from zero; the C chunk sums
+ * are then combined pairwise, partner at distance C/2, C/4, ..., 1. */
+float lo_dot_c16(const float *a, const float *b, int n)
+{
+    float p[16], nxt[16];
+    int C = n / 16;
+    for (int c = 0; c < C; c++) {
+        float acc = 0.0f;
+        for (int e = 0; e < 16; e++)
+            acc = fmaf(a[16 * c + e], b[16 * c + e], acc);
+        p[c] = acc;
+    }
+    for (int stride = C / 2; stride >= 1; stride /= 2) {
+        for (int l = 0; l < C; l++)
+            nxt[l] = p[l] + p[l ^ stride];
+        memcpy(p, nxt, sizeof(float) * C);
+    }
+    return p[0];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Requantization of one value row (Proposition 1 scale, SR or RTN)         */
+/* ------------------------------------------------------------------------ */
+
+/* x: the updated fp32 row (d_k entries).  Writes the row's codes and its
+ * d_k/G scales.  A row that holds a non-finite entry is stored as zero
+ * (scales 0, codes 0) and reported with return value 1. */
+static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_key,
+                          uint8_t *codes, float *scales)
+{
+    const int r = code_max(c->bits);
+    const int ng = c->d_k / c->group;
+    int bad = 0;
+    for (int j = 0; j < c->d_k; j++)
+        if (!isfinite(x[j]))
+            bad = 1;
+    for (int g = 0; g < ng; g++) {
+        float m = 0.0f;
+        for (int j = g * c->group; j < (g + 1) * c->group; j++)
+            if (fabsf(x[j]) > m)
+                m = fabsf(x[j]);
+        float inv = 0.0f, s = 0.0f;
+        if (!bad && m > 0.0f) {
+            inv = (float)r / m;            /* round to nearest */
+            if (isfinite(inv))
+                s = m / (float)r;          /* round to nearest */
+            else
+                inv = 0.0f;                /* m too small to scale: store as zero */
+        }
+        scales[(size_t)i * ng + g] = s;
+        for (int j = g * c->group; j < (g + 1) * c->group; j++) {
+            int code = 0;
+            if (!bad && inv != 0.0f) {
+                float d = c->stochastic ? (float)lo_dither(tile_key, c->d_k, i, j) : 128.0f;
+                float t = fmaf(x[j], inv, 49152.0f + d / 256.0f);
+                code = (int)floorf(t - 49152.0f);
+            }
+            put_code(c, codes, i, j, code);
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One decode step of one (sequence, head) tile                             */
+/* ------------------------------------------------------------------------ */
+
+/* state: packed codes (bits 8/4) or float[d_v*d_k] (bits 32), updated in place.
+ * scales: float[d_v * d_k/G] (ignored for bits 32), updated in place.
+ * q, k: d_k floats; v: d_v floats; alpha: 1 float (scalar decay) or d_k
+ * floats (diag); beta: scalar.  o_out: d_v doubles.  x_out (optional, may be
+ * NULL): the updated fp32 state before requantization, d_v*d_k floats.
+ * Returns 1 if any row held a non-finite value, else 0. */
+int lo_tile_step(const lo_cfg *c, void *state, float *scales,
+                 const float *q, const float *k, const float *v,
+                 const float *alpha, float beta, uint32_t tile_key,
+                 double *o_out, float *x_out)
+{
+    const int dk = c->d_k, ng = dk / c->group;
+    float *Sp = malloc(sizeof(float) * dk);   /* S_{t-1} diag(alpha), one row */
+    float *x = malloc(sizeof(float) * dk);    /* S_t, one row                 */
+    int flag = 0;
+    for (int i = 0; i < c->d_v; i++) {
+        /* dequantize and decay: entry (i, j) is c_ij * (s_ig * alpha_j) */
+        for (int j = 0; j < dk; j++) {
+            float aj = c->diag ? alpha[j] : alpha[0];
+            if (c->bits == 32) {
+                Sp[j] = ((float *)state)[(size_t)i * dk + j] * aj;
+            } else {
+                float s = scales[(size_t)i * ng + j / c->group];
+                Sp[j] = (float)get_code(c, (uint8_t *)state, i, j) * (s * aj);
+            }
+        }
+        /* write: w_i = beta (v_i - delta u_i), u_i = (S' k)_i */
+        float w;
+        if (c->delta) {
+            float u = lo_dot_c16(Sp, k, dk);
+            w = beta * (v[i] - u);
+        } else {
+            w = beta * v[i];
+        }
+        for (int j = 0; j < dk; j++)
+            x[j] = fmaf(w, k[j], Sp[j]);
+        /* readout o_i = (S_t q)_i from the fp32 state */
+        double o = 0.0;
+        for (int j = 0; j < dk; j++)
+            o += (double)x[j] * (double)q[j];
+        o_out[i] = o;
+        if (x_out)
+            memcpy(x_out + (size_t)i * dk, x, sizeof(float) * dk);
+        /* requantize (or store the fp32 state) */
+        if (c->bits == 32) {
+            for (int j = 0; j < dk; j++) {
+                if (!isfinite(x[j]))
+                    flag = 1;
+                ((float *)state)[(size_t)i * dk + j] = x[j];
+            }
+        } else {
+            flag |= requantize_row(c, x, i, tile_key, (uint8_t *)state, scales);
+        }
+    }
+    free(Sp);
+    free(x);
+    return flag;
+}
+
+/* Quantize an fp32 tile S (d_v x d_k) into codes and scales with the same
+ * quantizer as the decode step.  Returns 1 if a row was non-finite. */
+int lo_tile_quantize(const lo_cfg *c, const float *S, uint8_t *codes, float *scales,
+                     uint32_t tile_key)
+{
+    int flag = 0;
+    for (int i = 0; i < c->d_v; i++)
+        flag |= requantize_row(c, S + (size_t)i * c->d_k, i, tile_key, codes, scales);
+    return flag;
+}
+
+/* Dequantize a tile: S_ij = c_ij * s_ig. */
+void lo_tile_dequant(const lo_cfg *c, const uint8_t *codes, const float *scales, float *S)
+{
+    const int ng = c->d_k / c->group;
+    for (int i = 0; i < c->d_v; i++)
+        for (int j = 0; j < c->d_k; j++)
+            S[(size_t)i * c->d_k + j] =
+                (float)get_code(c, codes, i, j) * scales[(size_t)i * ng + j / c->group];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decay-based mixed precision (create time)                                */
+/* ------------------------------------------------------------------------ */
+
+/* The round(frac_high * H) heads with the largest mean decay (slowest to
+ * forget) get bits_high, the rest bits_low.  Equal decays: lower head index
+ * first.  Plain selection, one head at a time. */
+void lo_assign_bits_by_decay(const float *mean_decay, int H, float frac_high,
+                             int bits_high, int bits_low, int *out_bits)
+{
+    int n_high = (int)floor((double)frac_high * (double)H + 0.5);
+    if (n_high < 0) n_high = 0;
+    if (n_high > H) n_high = H;
+    char *taken = calloc((size_t)H, 1);
+    for (int h = 0; h < H; h++)
+        out_bits[h] = bits_low;
+    for (int n = 0; n < n_high; n++) {
+        int best = -1;
+        for (int h = 0; h < H; h++)
+            if (!taken[h] && (best < 0 || mean_decay[h] > mean_decay[best]))
+                best = h;
+        taken[best] = 1;
+        out_bits[best] = bits_high;
+    }
+    free(taken);
+}

@@ -1,0 +1,184 @@
+"""ctypes front end of the CPU oracle (test infrastructure only).
+
+Every arithmetic step lives in lores_oracle.c; this module only moves numpy
+arrays in and out and loops over tiles and steps.  Layouts follow the state
+format: codes of one (sequence, head) tile are row-major [d_v][d_k] (int8) or
+[d_v][d_k/2] bytes (int4, even column in the low nibble); scales are
+[d_v][d_k/G] fp32; the fp32 state is [d_v][d_k].
+"""
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class LoCfg(C.Structure):
+    _fields_ = [("d_k", C.c_int), ("d_v", C.c_int), ("group", C.c_int), ("bits", C.c_int),
+                ("delta", C.c_int), ("diag", C.c_int), ("stochastic", C.c_int)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        L.lo_splitmix64.restype = C.c_uint64
+        L.lo_splitmix64.argtypes = [C.c_uint64]
+        L.lo_fmix32.restype = C.c_uint32
+        L.lo_fmix32.argtypes = [C.c_uint32]
+        L.lo_step_key.restype = C.c_uint32
+        L.lo_step_key.argtypes = [C.c_uint64, C.c_uint64]
+        L.lo_tile_key.restype = C.c_uint32
+        L.lo_tile_key.argtypes = [C.c_uint32, C.c_uint32]
+        L.lo_dither.restype = C.c_uint32
+        L.lo_dither.argtypes = [C.c_uint32, C.c_int, C.c_int, C.c_int]
+        L.lo_dot_c16.restype = C.c_float
+        L.lo_dot_c16.argtypes = [C.c_void_p, C.c_void_p, C.c_int]
+        L.lo_get_code.restype = C.c_int
+        L.lo_get_code.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_int, C.c_int]
+        L.lo_put_code.restype = None
+        L.lo_put_code.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_int, C.c_int, C.c_int]
+        L.lo_tile_step.restype = C.c_int
+        L.lo_tile_step.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_void_p, C.c_void_p,
+                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_float, C.c_uint32,
+                                   C.c_void_p, C.c_void_p]
+        L.lo_tile_quantize.restype = C.c_int
+        L.lo_tile_quantize.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_uint32]
+        L.lo_tile_dequant.restype = None
+        L.lo_tile_dequant.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_void_p, C.c_void_p]
+        L.lo_assign_bits_by_decay.restype = None
+        L.lo_assign_bits_by_decay.argtypes = [C.c_void_p, C.c_int, C.c_float, C.c_int, C.c_int,
+                                              C.c_void_p]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def _f32(a):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return a
+
+
+class TileCfg:
+    """Shape and recipe of one (sequence, head) tile."""
+
+    def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1):
+        self.d_k, self.d_v = int(d_k), int(d_v)
+        self.group = int(group if group else d_k)
+        self.bits, self.delta, self.diag, self.stochastic = int(bits), int(delta), int(diag), int(stochastic)
+        self.c = LoCfg(self.d_k, self.d_v, self.group, self.bits, self.delta, self.diag,
+                       self.stochastic)
+
+    @property
+    def n_groups(self):
+        return self.d_k // self.group
+
+    def code_bytes(self):
+        if self.bits == 32:
+            return self.d_v * self.d_k * 4
+        return self.d_v * self.d_k * self.bits // 8
+
+    def zero_state(self):
+        """(state, scales) of an all-zero tile."""
+        if self.bits == 32:
+            return np.zeros((self.d_v, self.d_k), np.float32), np.zeros((self.d_v, self.n_groups), np.float32)
+        return (np.zeros(self.code_bytes(), np.uint8),
+                np.zeros((self.d_v, self.n_groups), np.float32))
+
+
+# --- random bits ------------------------------------------------------------
+
+def splitmix64(z):
+    return int(lib().lo_splitmix64(z & (2**64 - 1)))
+
+
+def fmix32(h):
+    return int(lib().lo_fmix32(h & 0xFFFFFFFF))
+
+
+def step_key(seed, step):
+    return int(lib().lo_step_key(seed & (2**64 - 1), step & (2**64 - 1)))
+
+
+def tile_key(skey, tile_index):
+    return int(lib().lo_tile_key(skey, tile_index & 0xFFFFFFFF))
+
+
+def dither(tkey, d_k, i, j):
+    return int(lib().lo_dither(tkey, d_k, i, j))
+
+
+def dot_c16(a, b):
+    a, b = _f32(a), _f32(b)
+    return float(lib().lo_dot_c16(_p(a), _p(b), a.size))
+
+
+# --- codes ------------------------------------------------------------------
+
+def unpack_codes(cfg: TileCfg, codes):
+    """Packed tile bytes -> int array [d_v, d_k] (int8 or int4 layouts)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty((cfg.d_v, cfg.d_k), np.int32)
+    L = lib()
+    for i in range(cfg.d_v):
+        for j in range(cfg.d_k):
+            out[i, j] = L.lo_get_code(C.byref(cfg.c), _p(codes), i, j)
+    return out
+
+
+def pack_codes(cfg: TileCfg, ints):
+    """int array [d_v, d_k] -> packed tile bytes."""
+    codes = np.zeros(cfg.code_bytes(), np.uint8)
+    L = lib()
+    for i in range(cfg.d_v):
+        for j in range(cfg.d_k):
+            L.lo_put_code(C.byref(cfg.c), _p(codes), i, j, int(ints[i, j]))
+    return codes
+
+
+# --- steps ------------------------------------------------------------------
+
+def tile_step(cfg: TileCfg, state, scales, q, k, v, alpha, beta, tkey, want_x=False):
+    """One decode step of one tile, in place on (state, scales).
+
+    Returns (o [d_v] float64, flag, x or None)."""
+    assert state.flags.c_contiguous and scales.flags.c_contiguous
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    alpha = _f32(np.atleast_1d(alpha))
+    o = np.empty(cfg.d_v, np.float64)
+    x = np.empty((cfg.d_v, cfg.d_k), np.float32) if want_x else None
+    flag = lib().lo_tile_step(C.byref(cfg.c), _p(state), _p(scales), _p(q), _p(k), _p(v),
+                              _p(alpha), float(np.float32(beta)), tkey, _p(o),
+                              _p(x) if want_x else None)
+    return o, int(flag), x
+
+
+def tile_quantize(cfg: TileCfg, S, tkey):
+    S = _f32(S)
+    codes = np.zeros(cfg.code_bytes(), np.uint8)
+    scales = np.zeros((cfg.d_v, cfg.n_groups), np.float32)
+    flag = lib().lo_tile_quantize(C.byref(cfg.c), _p(S), _p(codes), _p(scales), tkey)
+    return codes, scales, int(flag)
+
+
+def tile_dequant(cfg: TileCfg, codes, scales):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = _f32(scales)
+    S = np.empty((cfg.d_v, cfg.d_k), np.float32)
+    lib().lo_tile_dequant(C.byref(cfg.c), _p(codes), _p(scales), _p(S))
+    return S
+
+
+def assign_bits_by_decay(mean_decay, frac_high, bits_high=8, bits_low=4):
+    d = _f32(mean_decay)
+    out = np.empty(d.size, np.int32)
+    lib().lo_assign_bits_by_decay(_p(d), d.size, float(frac_high), bits_high, bits_low, _p(out))
+    return out

@@ -1,0 +1,476 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself: every expected value is a closed
+form of the recurrence, an fp64 brute-force product, an invariant the pages
+state (delta-rule projection, Propositions 1-3, the absmax scale), a
+published known-answer vector, or a hand-derived worked example of the state
+format.  Page references are to "Quantizing Recurrent Language Models Is
+Easier Than You Think" (summary page).
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+def unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def draw(T, d_k, d_v, seed, diag=False, alpha_lo=0.5, beta_hi=2.0):
+    """Seeded inputs inside the recurrence's domain (General recurrence form):
+    unit q, k; beta in (0, 2); alpha in (0, 1]."""
+    g = rng(seed)
+    q = unit(g.standard_normal((T, d_k))).astype(np.float32)
+    k = unit(g.standard_normal((T, d_k))).astype(np.float32)
+    v = g.standard_normal((T, d_v)).astype(np.float32)
+    beta = g.uniform(0.05, beta_hi * 0.95, T).astype(np.float32)
+    shape = (T, d_k) if diag else (T, 1)
+    alpha = g.uniform(alpha_lo, 1.0, shape).astype(np.float32)
+    return q, k, v, alpha, beta
+
+
+def run_fp32(cfg, q, k, v, alpha, beta, S0=None):
+    S = np.zeros((cfg.d_v, cfg.d_k), np.float32) if S0 is None else S0.astype(np.float32).copy()
+    sc = np.zeros((cfg.d_v, cfg.n_groups), np.float32)
+    Ss, os_ = [], []
+    for t in range(q.shape[0]):
+        o, flag, _ = O.tile_step(cfg, S, sc, q[t], k[t], v[t], alpha[t], beta[t], 0)
+        assert flag == 0
+        Ss.append(S.copy())
+        os_.append(o)
+    return Ss, os_
+
+
+def recur64(S, a, k, v, beta, delta):
+    """fp64 brute force: S diag(a) (I - delta beta k k^T) + beta v k^T."""
+    d_k = S.shape[1]
+    a = np.broadcast_to(np.asarray(a, np.float64), (d_k,))
+    k = k.astype(np.float64)
+    A = np.diag(a) @ (np.eye(d_k) - delta * float(beta) * np.outer(k, k))
+    return S.astype(np.float64) @ A + float(beta) * np.outer(v.astype(np.float64), k)
+
+
+# --------------------------------------------------------------------------
+# Random bits: published known-answer vectors and uniformity
+# --------------------------------------------------------------------------
+
+def test_rng_known_answers():
+    n = 0
+    for line in open(os.path.join(GOLDEN, "rng_kat.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        fn, arg, want = line.split()
+        if fn == "splitmix64":
+            z = (int(arg) * 0x9E3779B97F4A7C15) % 2**64
+            assert O.splitmix64(z) == int(want, 16)
+        else:
+            assert O.fmix32(int(arg, 16)) == int(want, 16)
+        n += 1
+    assert n == 7
+
+
+def test_dither_bytes_uniform_and_keyed():
+    # chi-square over 256 bins on 2^17 dithers from many tiles, steps and elements
+    counts = np.zeros(256)
+    for step in range(8):
+        sk = O.step_key(11, step)
+        for tile in range(4):
+            tk = O.tile_key(sk, tile)
+            for i in range(32):
+                for j in range(128):
+                    counts[O.dither(tk, 128, i, j)] += 1
+    n = counts.sum()
+    chi2 = ((counts - n / 256) ** 2 / (n / 256)).sum()
+    # 255 dof: mean 255, sd ~22.6; 6 sd bound
+    assert chi2 < 255 + 6 * 22.6, chi2
+    # different steps / tiles / seeds give different keys
+    keys = {O.tile_key(O.step_key(s, t), b) for s in range(3) for t in range(50) for b in range(40)}
+    assert len(keys) == 3 * 50 * 40
+
+
+def test_dither_adjacent_columns_independent():
+    # the four bytes of one hash feed four columns: their pairwise correlation is ~0
+    sk = O.step_key(5, 9)
+    tk = O.tile_key(sk, 3)
+    d = np.array([[O.dither(tk, 128, i, j) for j in range(128)] for i in range(128)], float)
+    for off in (1, 2, 3, 4):
+        c = np.corrcoef(d[:, :-off].ravel(), d[:, off:].ravel())[0, 1]
+        assert abs(c) < 0.03, (off, c)
+
+
+# --------------------------------------------------------------------------
+# Fixed-order dot product
+# --------------------------------------------------------------------------
+
+def test_dot_exact_on_integers():
+    g = rng(1)
+    for n in (16, 32, 64, 128, 256):
+        a = g.integers(-50, 50, n).astype(np.float32)
+        b = g.integers(-50, 50, n).astype(np.float32)
+        assert O.dot_c16(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
+
+
+def test_dot_error_bound():
+    # |fl(a.b) - a.b| <= gamma_n sum|a_j b_j| (Higham, Accuracy and Stability, 3.1)
+    g = rng(2)
+    for n in (16, 64, 128, 256):
+        a = g.standard_normal(n).astype(np.float32)
+        b = g.standard_normal(n).astype(np.float32)
+        exact = sum(Fraction(float(x)) * Fraction(float(y)) for x, y in zip(a, b))
+        u = 2.0 ** -24
+        bound = n * u / (1 - n * u) * float(np.sum(np.abs(a.astype(np.float64) * b)))
+        assert abs(float(Fraction(O.dot_c16(a, b)) - exact)) <= bound
+
+
+def test_dot_combine_order_worked_example():
+    # Chunk sums p = [2^24, 1, -2^24, 1] (one nonzero term per 16-column chunk).
+    # Partner at distance C/2 first: [p0+p2, p1+p3] = [0, 2], then 0 + 2 = 2.
+    # (A left-to-right sum would lose the first 1 and give 1.)
+    a = np.zeros(64, np.float32)
+    b = np.ones(64, np.float32)
+    a[0], a[16], a[32], a[48] = 2.0 ** 24, 1.0, -(2.0 ** 24), 1.0
+    assert O.dot_c16(a, b) == 2.0
+
+
+# --------------------------------------------------------------------------
+# The recurrence (General recurrence form), quantization off (fp32 state)
+# --------------------------------------------------------------------------
+
+def test_closed_form_no_decay_no_delta():
+    # alpha = 1, delta = 0: S_T = sum_t beta_t v_t k_t^T and o_t = S_t q_t
+    T, d = 40, 32
+    cfg = O.TileCfg(d, d, bits=32, delta=0)
+    q, k, v, _, beta = draw(T, d, d, 3)
+    alpha = np.ones((T, 1), np.float32)
+    Ss, os_ = run_fp32(cfg, q, k, v, alpha, beta)
+    S = np.zeros((d, d))
+    for t in range(T):
+        S += float(beta[t]) * np.outer(v[t].astype(np.float64), k[t].astype(np.float64))
+        np.testing.assert_allclose(Ss[t], S, rtol=0, atol=1e-5 * np.abs(S).max())
+        o = S @ q[t].astype(np.float64)
+        assert np.linalg.norm(os_[t] - o) <= 1e-5 * np.linalg.norm(o)
+
+
+@pytest.mark.parametrize("diag", [0, 1])
+def test_closed_form_decayed_linear_attention(diag):
+    # delta = 0: S_T[:, j] = sum_t (prod_{tau > t} alpha_tau,j) beta_t v_t k_t,j
+    T, dk, dv = 30, 32, 16
+    cfg = O.TileCfg(dk, dv, bits=32, delta=0, diag=diag)
+    q, k, v, alpha, beta = draw(T, dk, dv, 4 + diag, diag=bool(diag), alpha_lo=0.7)
+    Ss, _ = run_fp32(cfg, q, k, v, alpha, beta)
+    a = np.broadcast_to(alpha.astype(np.float64), (T, dk))
+    S = np.zeros((dv, dk))
+    for t in range(T):
+        w = np.prod(a[t + 1:], axis=0)
+        S += float(beta[t]) * np.outer(v[t].astype(np.float64), k[t] * w)
+    np.testing.assert_allclose(Ss[-1], S, rtol=0, atol=2e-6 * np.abs(S).max() * T)
+
+
+def test_delta_rule_projection_invariant():
+    # delta = 1, beta = 1, unit k: (I - k k^T) annihilates k, so S_t k_t = v_t
+    T, d = 40, 64
+    cfg = O.TileCfg(d, d, bits=32, delta=1, diag=1)
+    q, k, v, alpha, _ = draw(T, d, d, 6, diag=True)
+    beta = np.ones(T, np.float32)
+    Ss, _ = run_fp32(cfg, q, k, v, alpha, beta)
+    for t in range(T):
+        r = Ss[t].astype(np.float64) @ k[t].astype(np.float64) - v[t]
+        assert np.linalg.norm(r) <= 1e-5 * np.linalg.norm(v[t])
+
+
+@pytest.mark.parametrize("delta,diag", [(1, 0), (1, 1), (0, 1)])
+def test_brute_force_recurrence_fp32_state(delta, diag):
+    T, d = 24, 16
+    cfg = O.TileCfg(d, d, bits=32, delta=delta, diag=diag)
+    q, k, v, alpha, beta = draw(T, d, d, 7 + delta + 2 * diag, diag=bool(diag))
+    S0 = rng(8).standard_normal((d, d)).astype(np.float32)
+    Ss, os_ = run_fp32(cfg, q, k, v, alpha, beta, S0=S0)
+    S = S0.astype(np.float64)
+    for t in range(T):
+        S = recur64(S, alpha[t], k[t], v[t], beta[t], delta)
+        np.testing.assert_allclose(Ss[t], S, rtol=0, atol=1e-5 * max(1.0, np.abs(S).max()))
+        np.testing.assert_allclose(os_[t], S @ q[t].astype(np.float64), rtol=0,
+                                   atol=1e-5 * max(1.0, np.abs(S).max()))
+
+
+# --------------------------------------------------------------------------
+# Quantized step: dequantize -> update -> requantize (Key properties, item 3)
+# --------------------------------------------------------------------------
+
+def quantized_case(bits, group, d_k=32, d_v=16, seed=9, delta=1, diag=1):
+    g = rng(seed)
+    cfg = O.TileCfg(d_k, d_v, group=group, bits=bits, delta=delta, diag=diag)
+    r = (1 << (bits - 1)) - 1
+    ints = g.integers(-r, r + 1, (d_v, d_k))
+    codes = O.pack_codes(cfg, ints)
+    scales = g.uniform(0.01, 0.1, (d_v, cfg.n_groups)).astype(np.float32)
+    return cfg, ints, codes, scales
+
+
+@pytest.mark.parametrize("bits,group,delta,diag", [(8, 32, 1, 1), (8, 16, 0, 0), (4, 32, 1, 0),
+                                                    (4, 16, 1, 1), (8, 8, 1, 1)])
+def test_quantized_step_matches_fp64_update(bits, group, delta, diag):
+    d_k = 32
+    if d_k % group:
+        pytest.skip()
+    cfg, ints, codes, scales = quantized_case(bits, group, delta=delta, diag=diag)
+    q, k, v, alpha, beta = draw(1, cfg.d_k, cfg.d_v, 10, diag=bool(diag))
+    # fp64 reference: dequantize with the scale of each entry's group, then update
+    S_hat = ints * np.repeat(scales.astype(np.float64), group, axis=1)
+    X = recur64(S_hat, alpha[0], k[0], v[0], beta[0], delta)
+    o, flag, x = O.tile_step(cfg, codes, scales, q[0], k[0], v[0], alpha[0], beta[0],
+                             O.tile_key(O.step_key(1, 2), 3), want_x=True)
+    assert flag == 0
+    np.testing.assert_allclose(x, X, rtol=0, atol=1e-5 * np.abs(X).max())
+    np.testing.assert_allclose(o, X @ q[0].astype(np.float64), rtol=0, atol=1e-5 * np.abs(X).max())
+
+
+@pytest.mark.parametrize("bits,group,sr", [(8, 128, 1), (8, 32, 1), (4, 128, 1), (4, 16, 1),
+                                            (8, 128, 0), (4, 32, 0)])
+def test_absmax_quantizer_invariants(bits, group, sr):
+    # Proposition 1's scale: s_G = max|S_G| / r, r = 2^(b-1) - 1, codes in [-r, r]
+    d_k, d_v = 128, 64
+    cfg = O.TileCfg(d_k, d_v, group=group, bits=bits, stochastic=sr)
+    r = (1 << (bits - 1)) - 1
+    g = rng(12 + bits + group)
+    X = (g.standard_normal((d_v, d_k)) * np.exp(g.uniform(-8, 8, (d_v, 1)))).astype(np.float32)
+    X[3, :] = 0.0                                # an all-zero row
+    X[5, :group] = 0.0                           # an all-zero group
+    codes, scales, flag = O.tile_quantize(cfg, X, O.tile_key(O.step_key(2, 7), 1))
+    assert flag == 0
+    C_ = O.unpack_codes(cfg, codes)
+    assert C_.min() >= -r and C_.max() <= r
+    for i in range(d_v):
+        for gi in range(cfg.n_groups):
+            xs = X[i, gi * group:(gi + 1) * group]
+            cs = C_[i, gi * group:(gi + 1) * group]
+            m = np.float32(np.abs(xs).max())
+            s = scales[i, gi]
+            if m == 0:
+                assert s == 0 and not cs.any()
+                continue
+            assert s == np.float32(m / np.float32(r))
+            assert np.abs(cs).max() == r            # the group's max code is r exactly
+            err = np.abs(cs * np.float64(s) - xs)
+            lim = (1.0 if sr else 0.5 + 2.0 ** -8) * float(s) * (1 + 1e-6)
+            assert err.max() <= lim
+
+
+def test_int4_and_int8_packing_worked_example():
+    # int4: even column in the low nibble, odd in the high one, two's complement.
+    cfg4 = O.TileCfg(16, 1, bits=4)
+    ints = np.array([[1, -1, 7, -7, 0, 3, -3, 2, 5, -5, 6, -6, 4, -4, 1, 0]])
+    b = O.pack_codes(cfg4, ints)
+    assert b[0] == 0xF1 and b[1] == 0x97 and b[2] == 0x30 and b[3] == 0x2D
+    assert (O.unpack_codes(cfg4, b) == ints).all()
+    cfg8 = O.TileCfg(16, 16, bits=8)
+    allc = np.arange(-127, 129)[:256].reshape(16, 16).clip(-127, 127)
+    b8 = O.pack_codes(cfg8, allc)
+    assert b8.view(np.int8).reshape(16, 16).tolist() == allc.tolist()
+    assert (O.unpack_codes(cfg8, b8) == allc).all()
+    all4 = np.tile(np.arange(-7, 8), 2)[:16].reshape(1, 16)
+    assert (O.unpack_codes(cfg4, O.pack_codes(cfg4, all4)) == all4).all()
+
+
+def test_stochastic_rounding_unbiased_and_variance():
+    # mean over 10^4 keys of code*s converges to x (Proposition 3's premise);
+    # per-element variance is f(1-f) s^2 for fractional part f
+    d_k, d_v = 16, 4
+    cfg = O.TileCfg(d_k, d_v, bits=8)
+    g = rng(13)
+    X = g.standard_normal((d_v, d_k)).astype(np.float32)
+    N = 10000
+    acc = np.zeros((d_v, d_k))
+    acc2 = np.zeros((d_v, d_k))
+    for n in range(N):
+        codes, scales, _ = O.tile_quantize(cfg, X, O.tile_key(O.step_key(n, 0), 0))
+        Y = O.unpack_codes(cfg, codes) * scales.astype(np.float64)
+        acc += Y
+        acc2 += Y * Y
+    mean = acc / N
+    var = acc2 / N - mean ** 2
+    s = (np.abs(X).max(axis=1, keepdims=True) / 127.0)
+    f = (X / s) - np.floor(X / s)
+    sd = np.sqrt(f * (1 - f)) * s
+    bias_bound = s * 2.0 ** -9                      # the 1/256 grid rounds by <= 1/512 step
+    assert (np.abs(mean - X) <= 4.5 * sd / np.sqrt(N) + bias_bound + 1e-12).all()
+    np.testing.assert_allclose(var, (f * (1 - f)) * s ** 2, rtol=0, atol=0.08 * float(s.max()) ** 2)
+
+
+def test_round_to_nearest_mode_is_deterministic_nearest():
+    d_k, d_v = 32, 8
+    cfg = O.TileCfg(d_k, d_v, bits=8, stochastic=0)
+    X = rng(14).standard_normal((d_v, d_k)).astype(np.float32)
+    c1, s1, _ = O.tile_quantize(cfg, X, 1)
+    c2, s2, _ = O.tile_quantize(cfg, X, 999)
+    assert (c1 == c2).all() and (s1 == s2).all()
+    Y = O.unpack_codes(cfg, c1)
+    nearest = np.rint(X.astype(np.float64) / s1.astype(np.float64))
+    # equal except where x/s sits within 1/512 of a half step
+    frac = np.abs(X / s1 - np.floor(X / s1) - 0.5)
+    assert ((Y == nearest) | (frac < 2.0 ** -8)).all()
+
+
+def test_nonfinite_row_is_zeroed_and_flagged():
+    d_k, d_v = 32, 8
+    cfg = O.TileCfg(d_k, d_v, bits=8)
+    X = rng(15).standard_normal((d_v, d_k)).astype(np.float32)
+    X[2, 5] = np.nan
+    X[6, 0] = np.inf
+    codes, scales, flag = O.tile_quantize(cfg, X, 7)
+    assert flag == 1
+    C_ = O.unpack_codes(cfg, codes)
+    assert not C_[2].any() and not C_[6].any() and scales[2, 0] == 0 and scales[6, 0] == 0
+    assert C_[[0, 1, 3, 4, 5, 7]].any(axis=1).all()
+
+
+def test_step_requantization_equals_quantizer():
+    # the step's requantization is the same quantizer as the state loader
+    cfg, ints, codes, scales = quantized_case(8, 32, d_k=64, d_v=8, seed=16)
+    q, k, v, alpha, beta = draw(1, 64, 8, 17, diag=True)
+    tk = O.tile_key(O.step_key(3, 4), 5)
+    c1, s1 = codes.copy(), scales.copy()
+    _, _, x = O.tile_step(cfg, c1, s1, q[0], k[0], v[0], alpha[0], beta[0], tk, want_x=True)
+    c2, s2, _ = O.tile_quantize(cfg, x, tk)
+    assert (c1 == c2).all() and (s1 == s2).all()
+
+
+# --------------------------------------------------------------------------
+# Error recursion and Propositions 1-3
+# --------------------------------------------------------------------------
+
+def trajectories(bits, T, d, seed, delta, diag, alpha_lo=0.8, sr=1):
+    """Quantized and fp32 trajectories from the same inputs and zero state.
+    Returns lists of S_hat_t (dequantized), X_t (pre-quantization), S_fp_t."""
+    q, k, v, alpha, beta = draw(T, d, d, seed, diag=bool(diag), alpha_lo=alpha_lo)
+    cq = O.TileCfg(d, d, bits=bits, delta=delta, diag=diag, stochastic=sr)
+    cf = O.TileCfg(d, d, bits=32, delta=delta, diag=diag)
+    codes, sc = cq.zero_state()
+    Sf = np.zeros((d, d), np.float32)
+    scf = np.zeros((d, 1), np.float32)
+    S_hat, X, S_fp = [], [], []
+    for t in range(T):
+        tk = O.tile_key(O.step_key(seed, t), 0)
+        _, _, x = O.tile_step(cq, codes, sc, q[t], k[t], v[t], alpha[t], beta[t], tk, want_x=True)
+        O.tile_step(cf, Sf, scf, q[t], k[t], v[t], alpha[t], beta[t], 0)
+        S_hat.append(O.tile_dequant(cq, codes, sc).astype(np.float64))
+        X.append(x.astype(np.float64))
+        S_fp.append(Sf.astype(np.float64).copy())
+    return (q, k, v, alpha, beta), S_hat, X, S_fp
+
+
+@pytest.mark.parametrize("delta,diag", [(1, 0), (1, 1), (0, 0)])
+def test_error_recursion_identity(delta, diag):
+    # E_t = E_{t-1} diag(alpha_t)(I - delta beta_t k_t k_t^T) + eps_t with
+    # E_t = S_hat_t - S_fp_t and eps_t = S_hat_t - X_t (this step's rounding)
+    T, d = 30, 32
+    (q, k, v, alpha, beta), S_hat, X, S_fp = trajectories(8, T, d, 20 + delta + diag, delta, diag)
+    E_prev = np.zeros((d, d))
+    for t in range(T):
+        eps = S_hat[t] - X[t]
+        a = np.broadcast_to(alpha[t].astype(np.float64), (d,))
+        A = np.diag(a) @ (np.eye(d) - delta * float(beta[t]) * np.outer(k[t], k[t]))
+        E = S_hat[t] - S_fp[t]
+        pred = E_prev @ A + eps
+        scale = max(np.abs(S_fp[t]).max(), 1e-30)
+        assert np.abs(E - pred).max() <= 1e-5 * scale, t
+        E_prev = E
+
+
+def test_proposition2_decaying_error_bound():
+    # ||E_t||_F <= sum_tau alpha^(t - tau) ||eps_tau||_F for alpha < 1 bounding the decay
+    T, d = 60, 32
+    (q, k, v, alpha, beta), S_hat, X, S_fp = trajectories(4, T, d, 30, 1, 1, alpha_lo=0.6)
+    amax = float(alpha.max())
+    assert amax < 1.0
+    bound = 0.0
+    for t in range(T):
+        eps = np.linalg.norm(S_hat[t] - X[t])
+        bound = amax * bound + eps
+        E = np.linalg.norm(S_hat[t] - S_fp[t])
+        assert E <= bound * (1 + 1e-4) + 1e-5 * np.abs(S_fp[t]).max(), t
+
+
+def test_proposition1_value_axis_readout_error():
+    # RTN with one scale per value row: E[e_i^2] = M_i^2 / (12 r^2) for the readout
+    # error e = (S_hat - S) q with unit q (uniform rounding-error model)
+    d_k, d_v, n = 128, 32, 400
+    cfg = O.TileCfg(d_k, d_v, bits=4, stochastic=0)
+    g = rng(40)
+    num = np.zeros(d_v)
+    den = np.zeros(d_v)
+    for it in range(n):
+        S = (g.standard_normal((d_v, d_k)) * g.uniform(0.1, 10, (d_v, 1))).astype(np.float32)
+        q = unit(g.standard_normal(d_k))
+        codes, sc, _ = O.tile_quantize(cfg, S, 0)
+        e = (O.tile_dequant(cfg, codes, sc).astype(np.float64) - S) @ q
+        M = np.abs(S).max(axis=1).astype(np.float64)
+        num += e ** 2
+        den += M ** 2 / (12 * 7 ** 2)
+    ratio = num.sum() / den.sum()
+    assert 0.9 < ratio < 1.1, ratio
+
+
+def test_proposition3_sr_cross_terms_vanish():
+    # delta = 0, scalar decay: E||E_t^SR||^2 = sum gamma^2 E||eps||^2 (no cross terms),
+    # while RTN's cross terms reinforce.  A repeated token with a small write makes
+    # consecutive RTN rounding errors nearly identical, the case the proposition targets.
+    T, d, a, b = 40, 16, 0.97, 0.05
+    g = rng(50)
+    k = unit(g.standard_normal(d)).astype(np.float32)
+    v = g.standard_normal(d).astype(np.float32)
+    q = k.copy()
+    S0 = g.standard_normal((d, d)).astype(np.float32)
+    cf = O.TileCfg(d, d, bits=32, delta=0)
+
+    def run(sr, seed):
+        cq = O.TileCfg(d, d, bits=4, delta=0, stochastic=sr)
+        codes, sc, _ = O.tile_quantize(cq, S0, O.tile_key(O.step_key(seed, 10 ** 6), 0))
+        Sf = O.tile_dequant(cq, codes, sc)
+        scf = np.zeros((d, 1), np.float32)
+        eps = []
+        for t in range(T):
+            tk = O.tile_key(O.step_key(seed, t), 0)
+            _, _, x = O.tile_step(cq, codes, sc, q, k, v, a, b, tk, want_x=True)
+            O.tile_step(cf, Sf, scf, q, k, v, a, b, 0)
+            eps.append(O.tile_dequant(cq, codes, sc).astype(np.float64) - x)
+        E = O.tile_dequant(cq, codes, sc).astype(np.float64) - Sf
+        gam = [np.float64(a) ** (T - 1 - t) for t in range(T)]
+        return np.sum(E * E), sum(gm ** 2 * np.sum(e * e) for gm, e in zip(gam, eps))
+
+    ratios = []
+    for s in range(60):
+        e, dsum = run(1, s)
+        ratios.append(e / dsum)
+    # SR: ratio 1 in expectation (spread ~0.15 per run, so test the mean of 60)
+    assert 0.85 < np.mean(ratios) < 1.15, np.mean(ratios)
+    e_rtn, d_rtn = run(0, 0)
+    assert e_rtn / d_rtn > 5.0, e_rtn / d_rtn
+
+
+# --------------------------------------------------------------------------
+# Decay-based mixed precision (Table 5 text)
+# --------------------------------------------------------------------------
+
+def test_assign_bits_by_decay_worked_examples():
+    # slowest-decaying (largest mean decay) heads are promoted
+    assert O.assign_bits_by_decay([0.5, 0.9, 0.99, 0.7], 0.5).tolist() == [4, 8, 8, 4]
+    # ties go to the lower head index
+    assert O.assign_bits_by_decay([0.9, 0.9, 0.9, 0.1], 0.5).tolist() == [8, 8, 4, 4]
+    # 25% of 32 heads -> 8 heads
+    d = np.linspace(0.5, 0.9999, 32).astype(np.float32)
+    b = O.assign_bits_by_decay(d, 0.25)
+    assert (b[24:] == 8).all() and (b[:24] == 4).all()
+    assert O.assign_bits_by_decay([0.3, 0.2], 0.0).tolist() == [4, 4]
+    assert O.assign_bits_by_decay([0.3, 0.2], 1.0).tolist() == [8, 8]
