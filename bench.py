@@ -1,0 +1,422 @@
+"""Benchmark of the LoReS decode step on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    (N > 1: launch with torch.distributed.run, one rank per GPU)
+
+Workload (default): the 48-layer throughput sweep point at batch 256 per GPU, 32 heads,
+d_k = d_v = 128, delta rule, scalar per-head decay, int8 state with one fp32 scale per
+value row, stochastic rounding.  Each layer is its own handle with its own state and
+inputs.  One step = one decode token through all 48 layers = 48 kernel launches.
+Inputs are synthetic (seeded), resident in HBM; each layer's state (294 MB) exceeds the
+126 MB L2, so no flush is needed between steps.
+
+Metric: state updates per second, one update = one (sequence, head, layer, token).
+Every rank runs its own batch (sequences are independent: weak scaling, no collective
+on the data path); time is the max over ranks.
+
+The JSON line also carries: roofline of the decode kernel against the measured HBM
+copy bandwidth, an end-to-end number through the host-buffer C-ABI call, the clocks
+seen during the timed region, and the CPU oracle's rate on a bounded sample.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "state-update steps/s (seq x head x token) and achieved HBM GB/s as % of B200 peak"
+UNIT = "state-updates/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=256, help="sequences per GPU")
+    ap.add_argument("--layers", type=int, default=48)
+    ap.add_argument("--variant", default="int8", choices=["int8", "mixed", "fp32"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+# workload description and algorithmic bytes
+# ---------------------------------------------------------------------------------------
+
+def workload(args):
+    from bit_recurrent_state_lores_b200 import synth
+    return synth.workload("sweep", B=args.batch, layers=args.layers)
+
+
+def layer_bits(args, wl, layer):
+    from bit_recurrent_state_lores_b200 import synth
+    from bit_recurrent_state_lores_b200 import lores as L
+    if args.variant == "int8":
+        return [8] * wl.H
+    if args.variant == "fp32":
+        return [32] * wl.H
+    hp = synth.head_params(layer_workload(wl, layer))
+    return L.lores_assign_bits_by_decay(hp["mean_decay"], 0.25, 8, 4)
+
+
+def layer_workload(wl, layer):
+    from bit_recurrent_state_lores_b200 import synth
+    return synth.replace(wl, seed=wl.seed * 1000 + layer)
+
+
+def tile_bytes(wl, bits):
+    """Algorithmic bytes of one (sequence, head) update: codes + scales + q, k, v, alpha,
+    beta read; codes + scales + o written (fp32 heads: the fp32 state, no scales)."""
+    code = wl.d_v * wl.d_k * bits // 8
+    scales = 0 if bits == 32 else wl.d_v * (wl.d_k // wl.G) * 4
+    alpha = wl.d_k * 4 if wl.diag else 4
+    read = code + scales + 2 * wl.d_k * 4 + wl.d_v * 4 + alpha + 4
+    write = code + scales + wl.d_v * 4
+    return read + write
+
+
+def launch_bytes(wl, bits):
+    return wl.B * sum(tile_bytes(wl, b) for b in bits)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("lores.cu", "lores_device.cuh"):
+        h.update(open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(variant, batch):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    except Exception:
+        return None
+    e = d.get(f"{variant}-b{batch}")
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [r for (ts, r) in self.rows if t0 - 0.15 <= ts <= t1 + 0.15 and len(r) >= 10]
+        note = "samples inside the timed region"
+        if not rows:
+            rows = [r for (ts, r) in self.rows if len(r) >= 10][-5:]
+            note = "timed region shorter than the sampling period: nearest samples"
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max((num(r[4]) or 0) for r in rows),
+                "note": note}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline key)
+# ---------------------------------------------------------------------------------------
+
+def time_oracle(wl, variant_bits, seconds, steps=None):
+    """Run the oracle's decode step on a bounded sample of the workload: tiles of layer 0,
+    batch 1, all heads, for successive steps until `seconds` elapse (or `steps` steps).
+    Returns (rate in state-updates/s, tiles done, elapsed s, description)."""
+    import numpy as np
+    from bit_recurrent_state_lores_b200 import synth
+    from oracle import oracle as O
+
+    wl0 = synth.replace(layer_workload(wl, 0), B=1)
+    hp = synth.head_params(wl0)
+    cfgs = [O.TileCfg(wl0.d_k, wl0.d_v, group=wl0.G, bits=b, delta=wl0.delta, diag=wl0.diag)
+            for b in variant_bits]
+    states = [c.zero_state() for c in cfgs]
+    done, elapsed, t = 0, 0.0, 0
+    while (steps is None and elapsed < seconds) or (steps is not None and t < steps):
+        q, k, v, a, b = [x.numpy() for x in synth.step_inputs(wl0, t, hp, device="cpu")]
+        sk = O.step_key(wl0.seed, t)
+        t0 = time.perf_counter()
+        for hh, cfg in enumerate(cfgs):
+            st, sc = states[hh]
+            O.tile_step(cfg, st, sc, q[0, hh], k[0, hh], v[0, hh], a[0, hh], b[0, hh],
+                        O.tile_key(sk, hh))
+        elapsed += time.perf_counter() - t0
+        done += len(cfgs)
+        t += 1
+    desc = (f"oracle decode step, single thread: layer 0, batch 1, {wl0.H} heads "
+            f"{wl0.d_v}x{wl0.d_k}, {t} steps ({done} (seq,head) updates, {elapsed:.1f} s)")
+    return done / elapsed, done, elapsed, desc
+
+
+def cpu_cores_used():
+    return 1
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from bit_recurrent_state_lores_b200 import lores as L
+    from bit_recurrent_state_lores_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workload(args)
+    layers = []
+    for layer in range(wl.layers):
+        wll = layer_workload(wl, layer)
+        bits = layer_bits(args, wl, layer)
+        hp = synth.head_params(wll)
+        h = L.lores_create(wl.B, wl.H, wl.d_k, wl.d_v, group_size=0, delta=wl.delta,
+                           decay_diag=wl.diag, head_bits=bits, stochastic=1,
+                           seed=(wll.seed << 8) + rank, device=local_rank)
+        inputs = [synth.step_inputs(wll, 10_000 * rank + p, hp, device=dev) for p in range(2)]
+        o = torch.empty(wl.B, wl.H, wl.d_v, device=dev)
+        layers.append((h, bits, inputs, o))
+    bytes_per_launch = [launch_bytes(wl, bits) for (_, bits, _, _) in layers]
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def one_step(step, ev=None):
+        for li, (h, bits, inp, o) in enumerate(layers):
+            q, k, v, a, b = inp[step & 1]
+            if ev is not None:
+                ev[li][0].record(stream)
+            L.lores_decode_step(h, q, k, v, a, b, o, step, sptr)
+            if ev is not None:
+                ev[li][1].record(stream)
+
+    for s in range(args.warmup):
+        one_step(s)
+    torch.cuda.synchronize(dev)
+    for (h, _, _, _) in layers:
+        st = L.lores_check_errors(h, sptr)
+        assert st == L.LORES_OK, L.lores_status_string(st)
+
+    clocks = None if args.no_clocks else ClockSampler(local_rank)
+    if clocks:
+        time.sleep(0.3)
+    K = args.steps
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+            for _ in layers] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start.record(stream)
+    for n in range(K):
+        one_step(args.warmup + n, evs[n])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    launch_ms = [evs[n][li][0].elapsed_time(evs[n][li][1]) for n in range(K)
+                 for li in range(len(layers))]
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clock_summary = None
+    if clocks:
+        time.sleep(0.2)
+        clocks.stop()
+        clock_summary = clocks.summary(t_wall0, t_wall1)
+    for (h, _, _, _) in layers:
+        st = L.lores_check_errors(h, sptr)
+        assert st == L.LORES_OK, L.lores_status_string(st)
+
+    units = world * wl.B * wl.H * wl.layers * K
+    value = units / (ms / 1e3)
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    avg_bytes = statistics.mean(bytes_per_launch)
+    peak, peak_kind = measured_peak()
+    achieved = avg_bytes / avg_launch_s / 1e9
+    traffic = profiled_traffic(args.variant, wl.B)
+
+    # ---- end to end through the host-buffer C-ABI call --------------------------------
+    e2e = None
+    if not args.no_e2e:
+        hin = []
+        for (h, bits, inp, o) in layers:
+            hin.append([x.cpu().pin_memory() for x in inp[0]] +
+                       [torch.empty(wl.B, wl.H, wl.d_v).pin_memory()])
+        Ke = max(1, args.e2e_steps)
+        h2d = sum(sum(x.numel() * 4 for x in hi[:5]) for hi in hin)
+        d2h = sum(hi[5].numel() * 4 for hi in hin)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        s0.record(stream)
+        for n in range(Ke):
+            for li, (h, _, _, _) in enumerate(layers):
+                q, k, v, a, b, o = hin[li]
+                L.lores_decode_step_host(h, q, k, v, a, b, o, 1_000_000 + n, sptr)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * wl.B * wl.H * wl.layers * Ke / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+               "api": "lores_decode_step_host (pinned host buffers)"}
+
+    for (h, _, _, _) in layers:
+        L.lores_destroy(h)
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            rate, done, el, desc = time_oracle(wl, layers[0][1], args.cpu_seconds)
+            cpu = {"value": rate, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
+                   "sample": desc}
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32+s8" if args.variant == "int8"
+            else ("f32+s8/s4" if args.variant == "mixed" else "f32"),
+            "data": "synthetic (seeded generators shaped like the 48-layer GDN-style sweep)",
+            "config": {"workload": f"sweep-{args.variant}-b{wl.B}-L{wl.layers}",
+                       "batch_per_gpu": wl.B, "heads": wl.H, "d_k": wl.d_k, "d_v": wl.d_v,
+                       "layers": wl.layers, "delta": wl.delta, "decay": "scalar per head",
+                       "group_size": wl.G, "rounding": "stochastic",
+                       "parallelism": f"dp{world} (sequences; no collective)",
+                       "l2": "state per layer > 126 MB L2 (inputs larger than L2; no flush)"},
+            "gpu_launches": wl.layers * K,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "kernel": "lores::decode_step_kernel<128,false,true>",
+                         "bytes_per_launch": avg_bytes, "avg_launch_us": avg_launch_s * 1e6,
+                         "frac_of_8TBps": achieved / 8000.0},
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clock_summary,
+        }
+    return result
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: same metric, timed on host cores."""
+    if rank != 0:
+        return None
+    wl = workload(args)
+    bits = layer_bits(args, wl, 0)
+    K = args.steps
+    per_step_budget = max(0.2, min(2.0, 120.0 / max(1, K + args.warmup)))
+    time_oracle(wl, bits, per_step_budget * args.warmup) if args.warmup else None
+    rate, done, el, desc = time_oracle(wl, bits, per_step_budget * K)
+    return {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+s8", "data": "synthetic",
+        "config": {"workload": f"sweep-{args.variant}-b{wl.B}-L{wl.layers}",
+                   "batch_per_gpu": wl.B, "heads": wl.H, "d_k": wl.d_k, "d_v": wl.d_v,
+                   "layers": wl.layers},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cpu_cores_used(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,867 @@
+// lores.cu -- LoReS quantized recurrent-state decode step: kernels and C ABI (sm_100a).
+//
+// One decode step of a linear-recurrence layer ("Quantizing Recurrent Language Models Is
+// Easier Than You Think", summary page: General recurrence form; Key properties item 3;
+// Proposition 1; Table 5 text; Proposition 3 / Table 6):
+//   S_t = S_{t-1} diag(alpha_t) (I - delta beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t
+// with S_{t-1} dequantized from int8/int4 codes and per-(value row, key block) fp32
+// scales, and S_t requantized with stochastic rounding, all in one pass over the state.
+//
+// Work decomposition.  Every value row of every (sequence, head) tile is independent.
+// A work unit is a block of rows of one tile; a persistent CTA (4 warps) walks its
+// share of units round robin.  For each unit one elected thread issues bulk async
+// copies (TMA, non-tensor form) of the unit's codes, scales, k, q, v (and per-column
+// alpha) into a 2-deep shared-memory ring, so the next unit streams in while the
+// current one is computed.  In a warp, d_k/16 lanes own one row, 16 consecutive
+// columns each; dot products and the group absmax reduce across those lanes with
+// shuffles.  Codes go back with 16-byte (int8) / 8-byte (int4) stores.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "lores.h"
+#include "lores_device.cuh"
+
+namespace lores {
+
+// One work unit inside a sequence's block.
+struct __align__(16) UnitDesc {
+  int32_t head;
+  int32_t row0;
+  int32_t nrows;
+  int32_t bits;          // 8, 4 or 32
+  int64_t code_off;      // byte offset of row0 of this head inside one sequence's block
+  int64_t pad;
+};
+
+struct StepParams {
+  uint8_t *codes;        // [B][seq_bytes]
+  float *scales;         // [B][H][d_v][ng]
+  const float *q, *k, *v, *alpha, *beta;
+  float *o;
+  unsigned *flag;
+  const UnitDesc *units; // [units_per_seq]
+  long long seq_bytes;
+  long long total_units;
+  int H, d_v, ng, G, units_per_seq;
+  uint32_t step_key;
+  int stochastic;
+  // stage layout (bytes from the stage start)
+  int st_scales, st_k, st_q, st_v, st_a, stage_bytes;
+};
+
+// Bytes of one row of a tile with `bits`-bit entries.
+__host__ __device__ inline int row_bytes(int dk, int bits) { return dk * bits / 8; }
+
+// -------------------------------------------------------------------------------------
+// producer: stage one unit's inputs into shared memory
+// -------------------------------------------------------------------------------------
+template <int DK, bool DIAG>
+__device__ __forceinline__ void issue_unit(const StepParams &p, long long u, uint8_t *stage,
+                                           uint64_t *bar) {
+  const long long b = u / p.units_per_seq;
+  const UnitDesc d = p.units[u % p.units_per_seq];
+  const long long tile = b * p.H + d.head;
+  const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
+  const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
+  const unsigned vbytes = (unsigned)(d.nrows * 4);
+  const unsigned vec = DK * 4;
+  const unsigned total = cbytes + sbytes + vbytes + 2 * vec + (DIAG ? vec : 0);
+  mbar_expect_tx(bar, total);
+  bulk_g2s(stage, p.codes + b * p.seq_bytes + d.code_off, cbytes, bar);
+  if (sbytes)
+    bulk_g2s(stage + p.st_scales, p.scales + (tile * p.d_v + d.row0) * p.ng, sbytes, bar);
+  bulk_g2s(stage + p.st_k, p.k + tile * DK, vec, bar);
+  bulk_g2s(stage + p.st_q, p.q + tile * DK, vec, bar);
+  bulk_g2s(stage + p.st_v, p.v + tile * p.d_v + d.row0, vbytes, bar);
+  if (DIAG) bulk_g2s(stage + p.st_a, p.alpha + tile * DK, vec, bar);
+}
+
+// -------------------------------------------------------------------------------------
+// consumer: one unit (rows [row0, row0 + nrows) of one tile) from its stage
+// -------------------------------------------------------------------------------------
+template <int DK, bool DIAG, bool DELTA, int BITS>
+__device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, long long b,
+                                             const UnitDesc &d) {
+  constexpr int LPR = DK / 16;            // lanes per row
+  constexpr int RPW = 32 / LPR;           // rows per warp pass
+  constexpr int RB = DK * BITS / 8;       // bytes per row
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lir = lane % LPR, riw = lane / LPR;
+  const int col0 = lir * 16;
+  const int lpg = p.G / 16;
+  const int g = col0 / p.G;
+  const long long tile = b * p.H + d.head;
+
+  const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
+  const float *sq = reinterpret_cast<const float *>(stage + p.st_q);
+  const float *sv = reinterpret_cast<const float *>(stage + p.st_v);
+  const float *ss = reinterpret_cast<const float *>(stage + p.st_scales);
+  float kk[16], qq[16], aa[16];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float4 k4 = *reinterpret_cast<const float4 *>(sk + col0 + 4 * c);
+    const float4 q4 = *reinterpret_cast<const float4 *>(sq + col0 + 4 * c);
+    kk[4 * c] = k4.x; kk[4 * c + 1] = k4.y; kk[4 * c + 2] = k4.z; kk[4 * c + 3] = k4.w;
+    qq[4 * c] = q4.x; qq[4 * c + 1] = q4.y; qq[4 * c + 2] = q4.z; qq[4 * c + 3] = q4.w;
+    if (DIAG) {
+      const float4 a4 =
+          *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(stage + p.st_a) +
+                                            col0 + 4 * c);
+      aa[4 * c] = a4.x; aa[4 * c + 1] = a4.y; aa[4 * c + 2] = a4.z; aa[4 * c + 3] = a4.w;
+    }
+  }
+  const float alpha_s = DIAG ? 0.0f : __ldg(p.alpha + tile);
+  const float beta = __ldg(p.beta + tile);
+  const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
+
+  uint8_t *gcodes = p.codes + b * p.seq_bytes + d.code_off;
+  float *gscales = p.scales + (tile * p.d_v + d.row0) * p.ng;
+  float *go = p.o + tile * p.d_v + d.row0;
+
+  for (int base = warp * RPW; base < d.nrows; base += kWarps * RPW) {
+    const int lr = base + riw;                 // row inside the unit
+    const bool active = lr < d.nrows;
+    const int lrr = active ? lr : 0;           // keep shared loads in bounds
+
+    // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
+    float sp[16];
+    if (BITS == 32) {
+      const float *srow = reinterpret_cast<const float *>(stage + (size_t)lrr * RB) + col0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float4 s4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
+        const float sv4[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          sp[4 * c + e] = __fmul_rn(sv4[e], DIAG ? aa[4 * c + e] : alpha_s);
+      }
+    } else {
+      float cf[16];
+      if (BITS == 8)
+        unpack_i8(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
+      else
+        unpack_i4(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
+      const float s_in = ss[lrr * p.ng + g];
+      const float a_row = __fmul_rn(s_in, alpha_s);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(cf[e], DIAG ? __fmul_rn(s_in, aa[e]) : a_row);
+    }
+
+    // ---- write: w = beta (v - delta (S'k)), x = S' + w k^T ----------------------------
+    const float vr = sv[lrr];
+    float w;
+    if (DELTA) {
+      float u = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) u = __fmaf_rn(sp[e], kk[e], u);
+#pragma unroll
+      for (int st = LPR / 2; st >= 1; st >>= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
+      w = __fmul_rn(beta, __fsub_rn(vr, u));
+    } else {
+      w = __fmul_rn(beta, vr);
+    }
+    float x[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(w, kk[e], sp[e]);
+
+    // ---- readout o = S_t q -----------------------------------------------------------
+    float oacc = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) oacc = __fmaf_rn(x[e], qq[e], oacc);
+#pragma unroll
+    for (int st = LPR / 2; st >= 1; st >>= 1) oacc = __fadd_rn(oacc, __shfl_xor_sync(kFull, oacc, st));
+
+    // ---- requantize and store --------------------------------------------------------
+    const int row = d.row0 + lrr;              // row inside the tile (dither counter)
+    bool row_bad;
+    if (BITS == 32) {
+      float m = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
+      const bool lbad = !(m <= 3.402823466e38f);
+      const unsigned bal = __ballot_sync(kFull, lbad);
+      const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
+      row_bad = (bal & rowmask) != 0u;
+      if (active) {
+        float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          __stcs(dst + c, make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
+      }
+    } else {
+      uint32_t words[4];
+      float s_new;
+      const uint32_t n0 = (uint32_t)row * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
+      row_bad = requantize16<LPR>(x, BITS, lpg, lane, tkey, n0, p.stochastic, words, s_new);
+      if (active) {
+        if (BITS == 8)
+          __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
+                 make_uint4(words[0], words[1], words[2], words[3]));
+        else
+          __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8),
+                 make_uint2(words[0], words[1]));
+        if (lir % lpg == 0) gscales[(size_t)lr * p.ng + g] = s_new;
+      }
+    }
+    if (active && lir == 0) {
+      go[lr] = oacc;
+      if (row_bad) atomicOr(p.flag, kFlagNonFinite);
+    }
+  }
+}
+
+template <int DK, bool DIAG, bool DELTA>
+__global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+  uint8_t *stages = smem + 128;
+
+  const long long first = blockIdx.x;
+  const long long stride = gridDim.x;
+  if (first >= p.total_units) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      const long long u = first + s * stride;
+      if (u < p.total_units) issue_unit<DK, DIAG>(p, u, stages + s * p.stage_bytes, &bars[s]);
+    }
+  }
+
+  int n = 0;
+  for (long long u = first; u < p.total_units; u += stride, ++n) {
+    const int s = n % kStages;
+    uint8_t *stage = stages + s * p.stage_bytes;
+    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1));
+    if (__syncthreads_or(!ok)) {
+      // Give up: record it, let the other stage's copy (if any) land, and leave.
+      if (threadIdx.x == 0) {
+        atomicOr(p.flag, kFlagTimeout);
+        const long long un = u + stride;
+        if (un < p.total_units)
+          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
+      }
+      __syncthreads();
+      return;
+    }
+    const long long b = u / p.units_per_seq;
+    const UnitDesc d = p.units[u % p.units_per_seq];
+    if (d.bits == 8)
+      compute_unit<DK, DIAG, DELTA, 8>(p, stage, b, d);
+    else if (d.bits == 4)
+      compute_unit<DK, DIAG, DELTA, 4>(p, stage, b, d);
+    else
+      compute_unit<DK, DIAG, DELTA, 32>(p, stage, b, d);
+    __syncthreads();                                   // every thread is done with `stage`
+    if (threadIdx.x == 0) {
+      const long long un = u + kStages * stride;
+      if (un < p.total_units) {
+        fence_proxy_async();
+        issue_unit<DK, DIAG>(p, un, stage, &bars[s]);
+      }
+    }
+  }
+}
+
+// -------------------------------------------------------------------------------------
+// state loader: quantize an fp32 state [B][H][d_v][d_k] with the step's quantizer
+// -------------------------------------------------------------------------------------
+struct LoadParams {
+  const float *S;
+  uint8_t *codes;
+  float *scales;
+  const int32_t *head_bits;     // device [H]
+  const int64_t *head_off;      // device [H]
+  long long seq_bytes;
+  long long rows;               // B * H * d_v
+  int H, d_v, ng, G;
+  uint32_t step_key;
+  int stochastic;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p) {
+  constexpr int LPR = DK / 16, RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lir = lane % LPR, riw = lane / LPR, col0 = lir * 16;
+  const long long gr = ((long long)blockIdx.x * kWarps + warp) * RPW + riw;   // global row
+  const bool active = gr < p.rows;
+  const long long grr = active ? gr : 0;
+  const int row = (int)(grr % p.d_v);
+  const long long tile = grr / p.d_v;
+  const int head = (int)(tile % p.H);
+  const long long b = tile / p.H;
+  // Rows of one warp may belong to different tiles (and bit widths): every lane runs the
+  // quantizer (it shuffles across the warp) and each lane stores per its own row.
+  const int bits = __ldg(p.head_bits + head);
+  float x[16];
+  const float *src = p.S + grr * DK + col0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float4 f = __ldg(reinterpret_cast<const float4 *>(src) + c);
+    x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
+  }
+  uint8_t *tilecodes = p.codes + b * p.seq_bytes + __ldg(p.head_off + head);
+  const int g = col0 / p.G, lpg = p.G / 16;
+  const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
+  const uint32_t n0 = (uint32_t)row * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
+  uint32_t words[4];
+  float s_new;
+  requantize16<LPR>(x, bits == 4 ? 4 : 8, lpg, lane, tkey, n0, p.stochastic, words, s_new);
+  if (!active) return;
+  if (bits == 32) {
+    float4 *dst = reinterpret_cast<float4 *>(tilecodes + (size_t)row * DK * 4) + lir * 4;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+    return;
+  }
+  if (bits == 8)
+    *reinterpret_cast<uint4 *>(tilecodes + (size_t)row * DK + lir * 16) =
+        make_uint4(words[0], words[1], words[2], words[3]);
+  else
+    *reinterpret_cast<uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8) =
+        make_uint2(words[0], words[1]);
+  if (lir % lpg == 0) p.scales[grr * p.ng + g] = s_new;
+}
+
+// -------------------------------------------------------------------------------------
+// dequantize the state into fp32 [B][H][d_v][d_k]
+// -------------------------------------------------------------------------------------
+template <int DK>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, float *out) {
+  constexpr int LPR = DK / 16;
+  const long long t = (long long)blockIdx.x * kThreads + threadIdx.x;
+  if (t >= p.rows * LPR) return;
+  const long long grr = t / LPR;
+  const int lir = (int)(t % LPR), col0 = lir * 16;
+  const int row = (int)(grr % p.d_v);
+  const long long tile = grr / p.d_v;
+  const int head = (int)(tile % p.H);
+  const long long b = tile / p.H;
+  const int bits = p.head_bits[head];
+  const uint8_t *tilecodes = p.codes + b * p.seq_bytes + p.head_off[head];
+  float y[16];
+  if (bits == 32) {
+    const float4 *src = reinterpret_cast<const float4 *>(tilecodes + (size_t)row * DK * 4) + lir * 4;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float4 f = src[c];
+      y[4 * c] = f.x; y[4 * c + 1] = f.y; y[4 * c + 2] = f.z; y[4 * c + 3] = f.w;
+    }
+  } else {
+    float cf[16];
+    if (bits == 8)
+      unpack_i8(*reinterpret_cast<const uint4 *>(tilecodes + (size_t)row * DK + lir * 16), cf);
+    else
+      unpack_i4(*reinterpret_cast<const uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8), cf);
+    const float s = p.scales[grr * p.ng + col0 / p.G];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(cf[e], s);
+  }
+  float4 *dst = reinterpret_cast<float4 *>(out + grr * DK + col0);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+}
+
+// -------------------------------------------------------------------------------------
+// host side
+// -------------------------------------------------------------------------------------
+
+// Step key: SplitMix64 (Steele, Lea & Flood 2014; Vigna's constants) of the seed xor
+// SplitMix64 of the step, folded to 32 bits.
+static uint64_t splitmix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+static uint32_t step_key_of(uint64_t seed, uint64_t step) {
+  const uint64_t k = splitmix64(seed ^ splitmix64(step));
+  return (uint32_t)(k ^ (k >> 32));
+}
+
+using StepFn = void (*)(const StepParams);
+using LoadFn = void (*)(const LoadParams);
+using DequantFn = void (*)(const LoadParams, float *);
+
+template <int DK>
+static StepFn pick_step(bool diag, bool delta) {
+  if (diag) return delta ? decode_step_kernel<DK, true, true> : decode_step_kernel<DK, true, false>;
+  return delta ? decode_step_kernel<DK, false, true> : decode_step_kernel<DK, false, false>;
+}
+static StepFn step_kernel_for(int dk, bool diag, bool delta) {
+  switch (dk) {
+    case 16: return pick_step<16>(diag, delta);
+    case 32: return pick_step<32>(diag, delta);
+    case 64: return pick_step<64>(diag, delta);
+    case 128: return pick_step<128>(diag, delta);
+    case 256: return pick_step<256>(diag, delta);
+  }
+  return nullptr;
+}
+static LoadFn load_kernel_for(int dk) {
+  switch (dk) {
+    case 16: return load_state_kernel<16>;
+    case 32: return load_state_kernel<32>;
+    case 64: return load_state_kernel<64>;
+    case 128: return load_state_kernel<128>;
+    case 256: return load_state_kernel<256>;
+  }
+  return nullptr;
+}
+static DequantFn dequant_kernel_for(int dk) {
+  switch (dk) {
+    case 16: return dequant_kernel<16>;
+    case 32: return dequant_kernel<32>;
+    case 64: return dequant_kernel<64>;
+    case 128: return dequant_kernel<128>;
+    case 256: return dequant_kernel<256>;
+  }
+  return nullptr;
+}
+
+}  // namespace lores
+
+using namespace lores;
+
+struct lores_handle {
+  lores_config cfg;
+  std::vector<int32_t> bits;       // [H]
+  std::vector<int64_t> head_off;   // [H]
+  int G = 0, ng = 0;
+  long long seq_bytes = 0;
+  uint8_t *codes = nullptr;
+  float *scales = nullptr;
+  unsigned *flag = nullptr;
+  UnitDesc *units = nullptr;
+  int32_t *d_bits = nullptr;
+  int64_t *d_head_off = nullptr;
+  int units_per_seq = 0;
+  int grid = 0;
+  int smem = 0;
+  StepParams sp{};
+  StepFn step_fn = nullptr;
+  // staging for lores_decode_step_host
+  float *stage_in = nullptr;
+  float *stage_o = nullptr;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lores_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LORES_OK;
+  if (e == cudaErrorMemoryAllocation) {
+    (void)cudaGetLastError();
+    return LORES_ERR_OOM;
+  }
+  return LORES_ERR_CUDA;
+}
+
+void free_all(lores_handle *h) {
+  cudaFree(h->codes);
+  cudaFree(h->scales);
+  cudaFree(h->flag);
+  cudaFree(h->units);
+  cudaFree(h->d_bits);
+  cudaFree(h->d_head_off);
+  cudaFree(h->stage_in);
+  cudaFree(h->stage_o);
+}
+
+LoadParams load_params(const lores_handle *h) {
+  LoadParams p{};
+  p.codes = h->codes;
+  p.scales = h->scales;
+  p.head_bits = h->d_bits;
+  p.head_off = h->d_head_off;
+  p.seq_bytes = h->seq_bytes;
+  p.rows = (long long)h->cfg.batch * h->cfg.heads * h->cfg.d_v;
+  p.H = h->cfg.heads;
+  p.d_v = h->cfg.d_v;
+  p.ng = h->ng;
+  p.G = h->G;
+  p.stochastic = h->cfg.stochastic;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lores_status_string(lores_status s) {
+  switch (s) {
+    case LORES_OK: return "ok";
+    case LORES_ERR_INVALID_ARG: return "invalid argument";
+    case LORES_ERR_OOM: return "out of memory";
+    case LORES_ERR_CUDA: return "CUDA error";
+    case LORES_ERR_NONFINITE: return "non-finite state";
+    case LORES_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LORES_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+lores_status lores_assign_bits_by_decay(const float *mean_decay, int32_t H, float frac_high,
+                                        int32_t bits_high, int32_t bits_low, int32_t *out_bits) {
+  auto okbits = [](int b) { return b == 4 || b == 8 || b == 32; };
+  if (!mean_decay || !out_bits || H < 1 || !(frac_high >= 0.0f && frac_high <= 1.0f) ||
+      !okbits(bits_high) || !okbits(bits_low))
+    return LORES_ERR_INVALID_ARG;
+  std::vector<int> order(H);
+  for (int h = 0; h < H; ++h) order[h] = h;
+  // largest mean decay first; equal decays keep head order (stable sort)
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int b) { return mean_decay[a] > mean_decay[b]; });
+  long long n_high = (long long)((double)frac_high * (double)H + 0.5);
+  n_high = std::max(0LL, std::min<long long>(n_high, H));
+  for (int h = 0; h < H; ++h) out_bits[h] = bits_low;
+  for (long long n = 0; n < n_high; ++n) out_bits[order[n]] = bits_high;
+  return LORES_OK;
+}
+
+lores_status lores_create(const lores_config *cfg, lores_handle **out) {
+  if (!out) return LORES_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return LORES_ERR_INVALID_ARG;
+  const lores_config c = *cfg;
+  const int dk = c.d_k, dv = c.d_v;
+  if (c.batch < 1 || c.heads < 1 || c.heads > 65536) return LORES_ERR_INVALID_ARG;
+  if (!(dk == 16 || dk == 32 || dk == 64 || dk == 128 || dk == 256)) return LORES_ERR_INVALID_ARG;
+  if (dv < 4 || dv > 4096 || dv % 4) return LORES_ERR_INVALID_ARG;
+  const int G = c.group_size == 0 ? dk : c.group_size;
+  if (G < 16 || G % 16 || dk % G) return LORES_ERR_INVALID_ARG;
+  if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
+      (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
+    return LORES_ERR_INVALID_ARG;
+  std::vector<int32_t> bits(c.heads, 8);
+  if (c.head_bits)
+    for (int h = 0; h < c.heads; ++h) {
+      bits[h] = c.head_bits[h];
+      if (bits[h] != 8 && bits[h] != 4 && bits[h] != 32) return LORES_ERR_INVALID_ARG;
+    }
+
+  DeviceGuard guard(c.device);
+  if (!guard.ok) {
+    (void)cudaGetLastError();
+    return LORES_ERR_CUDA;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, c.device) != cudaSuccess) return LORES_ERR_CUDA;
+  if (prop.major < 10) return LORES_ERR_UNSUPPORTED;
+
+  lores_handle *h = new (std::nothrow) lores_handle();
+  if (!h) return LORES_ERR_OOM;
+  h->cfg = c;
+  h->cfg.head_bits = nullptr;           // the caller's array is not kept
+  h->bits = bits;
+  h->G = G;
+  h->ng = dk / G;
+  h->head_off.resize(c.heads);
+  long long off = 0;
+  for (int hh = 0; hh < c.heads; ++hh) {
+    h->head_off[hh] = off;
+    off += (long long)dv * row_bytes(dk, bits[hh]);
+  }
+  h->seq_bytes = off;
+
+  // ---- work units: row blocks sized so one stage holds <= 16 KB of state ------------
+  const int LPR = dk / 16, rows_per_pass = kWarps * (32 / LPR);
+  auto rows_for = [&](int b) {
+    int R = 16384 / row_bytes(dk, b);
+    R = std::min(R, 1024 / h->ng);           // scales <= 4 KB per stage
+    R = std::min(R, 1024);                   // v slice <= 4 KB
+    if (R >= rows_per_pass) R -= R % rows_per_pass;
+    R -= R % 4;
+    return std::max(4, std::min(R, dv));
+  };
+  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta);
+  // occupancy is computed for the largest stage; split rows if one wave is not filled
+  int R8 = rows_for(8), R4 = rows_for(4), R32 = rows_for(32);
+  int split = 1;
+  auto build_units = [&](std::vector<UnitDesc> &u) {
+    u.clear();
+    for (int hh = 0; hh < c.heads; ++hh) {
+      const int b = bits[hh];
+      int R = b == 8 ? R8 : (b == 4 ? R4 : R32);
+      R = std::max(4, (R / split) - ((R / split) % 4));
+      for (int r0 = 0; r0 < dv; r0 += R) {
+        UnitDesc d{};
+        d.head = hh;
+        d.row0 = r0;
+        d.nrows = std::min(R, dv - r0);
+        d.bits = b;
+        d.code_off = h->head_off[hh] + (long long)r0 * row_bytes(dk, b);
+        u.push_back(d);
+      }
+    }
+  };
+  auto stage_bytes_for = [&](const std::vector<UnitDesc> &u, int *sc, int *sv) {
+    int cmax = 0, smax = 0, vmax = 0;
+    for (const UnitDesc &d : u) {
+      cmax = std::max(cmax, d.nrows * row_bytes(dk, d.bits));
+      if (d.bits != 32) smax = std::max(smax, d.nrows * h->ng * 4);
+      vmax = std::max(vmax, d.nrows * 4);
+    }
+    *sc = cmax;
+    *sv = smax;
+    return cmax + smax + vmax + 2 * dk * 4 + (c.decay_diag ? dk * 4 : 0);
+  };
+  std::vector<UnitDesc> units;
+  int ctas_per_sm = 1;
+  for (;;) {
+    build_units(units);
+    int cbytes, sbytes;
+    const int stage = stage_bytes_for(units, &cbytes, &sbytes);
+    const int smem = 128 + kStages * stage;
+    // the attribute is per kernel and shared by all handles: only ever raise it
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+        (fa.maxDynamicSharedSizeBytes < smem &&
+         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+             cudaSuccess)) {
+      delete h;
+      return LORES_ERR_CUDA;
+    }
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, fn, kThreads, smem) !=
+            cudaSuccess ||
+        ctas_per_sm < 1) {
+      delete h;
+      return LORES_ERR_CUDA;
+    }
+    const long long total = (long long)c.batch * (long long)units.size();
+    const long long slots = (long long)ctas_per_sm * prop.multiProcessorCount;
+    int maxR = 0;
+    for (const UnitDesc &d : units) maxR = std::max(maxR, d.nrows);
+    if (total >= slots || maxR <= rows_per_pass || maxR <= 4 || split >= 64) {
+      h->smem = smem;
+      h->sp.st_scales = cbytes;
+      h->sp.st_k = cbytes + sbytes;
+      h->sp.st_q = h->sp.st_k + dk * 4;
+      h->sp.st_a = h->sp.st_q + dk * 4;
+      h->sp.st_v = h->sp.st_a + (c.decay_diag ? dk * 4 : 0);
+      h->sp.stage_bytes = stage;
+      h->grid = (int)std::min<long long>(total, slots);
+      break;
+    }
+    split *= 2;
+  }
+  h->units_per_seq = (int)units.size();
+  h->step_fn = fn;
+
+  const long long code_bytes = (long long)c.batch * h->seq_bytes;
+  const long long scale_count = (long long)c.batch * c.heads * dv * h->ng;
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = cudaMalloc(&h->codes, (size_t)code_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&h->scales, (size_t)scale_count * 4);
+  if (e == cudaSuccess) e = cudaMalloc(&h->flag, 16);
+  if (e == cudaSuccess) e = cudaMalloc(&h->units, units.size() * sizeof(UnitDesc));
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_bits, c.heads * sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_head_off, c.heads * sizeof(int64_t));
+  if (e == cudaSuccess) e = cudaMemset(h->codes, 0, (size_t)code_bytes);
+  if (e == cudaSuccess) e = cudaMemset(h->scales, 0, (size_t)scale_count * 4);
+  if (e == cudaSuccess) e = cudaMemset(h->flag, 0, 16);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->units, units.data(), units.size() * sizeof(UnitDesc), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->d_bits, bits.data(), c.heads * sizeof(int32_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->d_head_off, h->head_off.data(), c.heads * sizeof(int64_t),
+                   cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    const lores_status st = cuda_status(e);
+    free_all(h);
+    delete h;
+    return st;
+  }
+
+  StepParams &p = h->sp;
+  p.codes = h->codes;
+  p.scales = h->scales;
+  p.flag = h->flag;
+  p.units = h->units;
+  p.seq_bytes = h->seq_bytes;
+  p.total_units = (long long)c.batch * h->units_per_seq;
+  p.H = c.heads;
+  p.d_v = dv;
+  p.ng = h->ng;
+  p.G = G;
+  p.units_per_seq = h->units_per_seq;
+  p.stochastic = c.stochastic;
+  *out = h;
+  return LORES_OK;
+}
+
+lores_status lores_destroy(lores_handle *h) {
+  if (!h) return LORES_OK;
+  DeviceGuard guard(h->cfg.device);
+  free_all(h);
+  delete h;
+  return LORES_OK;
+}
+
+lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, const float *v,
+                               const float *alpha, const float *beta, float *o, uint64_t step,
+                               void *stream) {
+  if (!h || !q || !k || !v || !alpha || !beta || !o) return LORES_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (h->cfg.decay_diag ? !aligned16(alpha) : (reinterpret_cast<uintptr_t>(alpha) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(o) & 3u))
+    return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  StepParams p = h->sp;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.step_key = step_key_of(h->cfg.seed, step);
+  h->step_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+lores_status lores_decode_step_host(lores_handle *h, const float *q, const float *k,
+                                    const float *v, const float *alpha, const float *beta,
+                                    float *o, uint64_t step, void *stream) {
+  if (!h || !q || !k || !v || !alpha || !beta || !o) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  const lores_config &c = h->cfg;
+  const size_t BH = (size_t)c.batch * c.heads;
+  const size_t nk = BH * c.d_k, nv = BH * c.d_v, na = c.decay_diag ? BH * c.d_k : BH;
+  // staging: q | k | v | alpha | beta, each region padded to 16 bytes
+  auto pad4 = [](size_t n) { return (n + 3) & ~size_t(3); };
+  const size_t oq = 0, ok_ = oq + pad4(nk), ov = ok_ + pad4(nk), oa = ov + pad4(nv),
+               ob = oa + pad4(na), total = ob + pad4(BH);
+  cudaError_t e = cudaSuccess;
+  if (!h->stage_in) e = cudaMalloc(&h->stage_in, total * 4);
+  if (e == cudaSuccess && !h->stage_o) e = cudaMalloc(&h->stage_o, nv * 4);
+  if (e != cudaSuccess) return cuda_status(e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *d = h->stage_in;
+  e = cudaMemcpyAsync(d + oq, q, nk * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d + ok_, k, nk * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d + ov, v, nv * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d + oa, alpha, na * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d + ob, beta, BH * 4, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  lores_status st =
+      lores_decode_step(h, d + oq, d + ok_, d + ov, d + oa, d + ob, h->stage_o, step, stream);
+  if (st != LORES_OK) return st;
+  e = cudaMemcpyAsync(o, h->stage_o, nv * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+lores_status lores_dequant_state(lores_handle *h, float *out, void *stream) {
+  if (!h || !out || !aligned16(out)) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  LoadParams p = load_params(h);
+  const long long threads = p.rows * (h->cfg.d_k / 16);
+  const int blocks = (int)((threads + kThreads - 1) / kThreads);
+  dequant_kernel_for(h->cfg.d_k)<<<blocks, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p, out);
+  return cuda_status(cudaGetLastError());
+}
+
+lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, void *stream) {
+  if (!h || !S || !aligned16(S)) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  LoadParams p = load_params(h);
+  p.S = S;
+  p.step_key = step_key_of(h->cfg.seed, step);
+  const int rpw = 32 / (h->cfg.d_k / 16);
+  const long long warps = (p.rows + rpw - 1) / rpw;
+  const int blocks = (int)((warps + kWarps - 1) / kWarps);
+  load_kernel_for(h->cfg.d_k)<<<blocks, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+lores_status lores_export_codes(lores_handle *h, void *codes, float *scales, void *stream) {
+  if (!h) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (codes)
+    e = cudaMemcpyAsync(codes, h->codes, (size_t)h->cfg.batch * h->seq_bytes, cudaMemcpyDefault, s);
+  if (e == cudaSuccess && scales)
+    e = cudaMemcpyAsync(scales, h->scales,
+                        (size_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng * 4,
+                        cudaMemcpyDefault, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+lores_status lores_load_codes(lores_handle *h, const void *codes, const float *scales,
+                              void *stream) {
+  if (!h || !codes || !scales) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e =
+      cudaMemcpyAsync(h->codes, codes, (size_t)h->cfg.batch * h->seq_bytes, cudaMemcpyDefault, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->scales, scales,
+                        (size_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng * 4,
+                        cudaMemcpyDefault, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t *head_offsets) {
+  if (!h || !out) return LORES_ERR_INVALID_ARG;
+  out->code_bytes = (int64_t)h->cfg.batch * h->seq_bytes;
+  out->seq_code_bytes = h->seq_bytes;
+  out->scale_count = (int64_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng;
+  out->n_groups = h->ng;
+  out->units_per_step = (int32_t)((long long)h->cfg.batch * h->units_per_seq);
+  out->grid = h->grid;
+  out->smem_bytes = h->smem;
+  if (head_offsets)
+    for (int hh = 0; hh < h->cfg.heads; ++hh) head_offsets[hh] = h->head_off[hh];
+  return LORES_OK;
+}
+
+lores_status lores_check_errors(lores_handle *h, void *stream) {
+  if (!h) return LORES_ERR_INVALID_ARG;
+  DeviceGuard guard(h->cfg.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned f = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&f, h->flag, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->flag, 0, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (f & kFlagTimeout) return LORES_ERR_TIMEOUT;
+  if (f & kFlagNonFinite) return LORES_ERR_NONFINITE;
+  return LORES_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+// lores_device.cuh -- device building blocks of the LoReS decode step (sm_100a).
+//
+// Arithmetic of one state row, shared by the decode kernel and the state loader.
+// The element order and every fp32 rounding follow the state format definition:
+//   entry of S_{t-1} diag(alpha):   c_ij * (s_ig * alpha_j)
+//   u_i = (S'k)_i:                  16-column fma chains, then pairwise combine with the
+//                                   partner lane at distance C/2, ..., 1
+//   w_i = beta (v_i - u_i)  [delta] or beta v_i;   x_ij = fma(w_i, k_j, S'_ij)
+//   requantize per group:           m = max|x|, inv = r / m, s = m / r (round to nearest),
+//                                   t = fma(x, inv, 49152 + d/256), code = floor(t - 49152)
+// ("Quantizing Recurrent Language Models Is Easier Than You Think": General recurrence
+// form; Key properties item 3; Proposition 1; Proposition 3.)
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace lores {
+
+constexpr int kThreads = 128;          // 4 warps per CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 2;             // smem ring depth per CTA
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Flag bits of the handle's sticky device word.
+constexpr unsigned kFlagNonFinite = 1u;
+constexpr unsigned kFlagTimeout = 2u;
+
+// Bounded waits: every spin on an mbarrier gives up after this many polls.
+constexpr unsigned kMaxPolls = 1u << 24;
+
+// -------------------------------------------------------------------------------------
+// random bits (MurmurHash3 32-bit finalizer, Appleby)
+// -------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85EBCA6Bu;
+  h ^= h >> 13;
+  h *= 0xC2B2AE35u;
+  h ^= h >> 16;
+  return h;
+}
+
+__device__ __forceinline__ uint32_t tile_key(uint32_t step_key, uint32_t tile_index) {
+  return fmix32(step_key + 0x85EBCA77u * (tile_index + 1u));
+}
+
+// max(m, |x|) that propagates NaN (PTX max.NaN), so a group max is non-finite
+// exactly when some entry is.
+__device__ __forceinline__ float max_abs_nan(float m, float x) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(fabsf(x)));
+  return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// -------------------------------------------------------------------------------------
+// mbarrier + bulk async copy (TMA, non-tensor form; no multicast)
+// -------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; returns false if the phase did not complete within kMaxPolls polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
+  for (unsigned n = 0; n < kMaxPolls; ++n)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+// global -> shared bulk copy completing on `bar`; dst, src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// -------------------------------------------------------------------------------------
+// code <-> float
+// -------------------------------------------------------------------------------------
+// 16 int8 codes (two's complement) -> exact floats: bias to offset binary, drop each
+// byte into the mantissa of 2^23, subtract 2^23 + 128.
+__device__ __forceinline__ void unpack_i8(const uint4 &cw, float (&c)[16]) {
+  const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
+                         cw.w ^ 0x80808080u};
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    c[e] = __fsub_rn(__uint_as_float(__byte_perm(w[e >> 2], 0x4B000000u, 0x7650u | (e & 3))),
+                     8388736.0f);
+}
+// 16 int4 codes (two's complement nibbles, even column low) -> exact floats.
+__device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
+  const uint32_t w[2] = {cw.x, cw.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t lo = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // even columns
+    const uint32_t hi = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // odd columns
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      c[8 * h + 2 * p] =
+          __fsub_rn(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u | p)), 8388616.0f);
+      c[8 * h + 2 * p + 1] =
+          __fsub_rn(__uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u | p)), 8388616.0f);
+    }
+  }
+}
+// t holds 49152 + code + frac in fp32: its byte 1 is the code (two's complement).
+__device__ __forceinline__ uint4 pack_i8(const uint32_t (&t)[16]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t lo = __byte_perm(t[4 * q], t[4 * q + 1], 0x0051u);
+    const uint32_t hi = __byte_perm(t[4 * q + 2], t[4 * q + 3], 0x0051u);
+    w[q] = __byte_perm(lo, hi, 0x5410u);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ uint2 pack_i4(const uint32_t (&t)[16]) {
+  uint32_t m[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p)
+    m[p] = (t[2 * p] & 0x0F00u) | ((t[2 * p + 1] << 4) & 0xF000u);   // byte 1 = (odd<<4)|even
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t lo = __byte_perm(m[4 * h], m[4 * h + 1], 0x0051u);
+    const uint32_t hi = __byte_perm(m[4 * h + 2], m[4 * h + 3], 0x0051u);
+    w[h] = __byte_perm(lo, hi, 0x5410u);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// -------------------------------------------------------------------------------------
+// requantize one lane's 16 entries of a value row
+// -------------------------------------------------------------------------------------
+// LPR lanes hold one row (16 consecutive columns each); LPG = G/16 lanes share a group.
+// Returns the row's "non-finite" verdict (same on all lanes of the row).  Writes the
+// lane's packed codes into `words` (int8: 4 words, int4: 2 words) and the lane's group
+// scale into `s_out`.  `bits` (8 or 4) may differ between rows of one warp; every lane
+// of the warp must call this function together (it shuffles across the warp).
+template <int LPR>
+__device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
+                                             uint32_t tkey, uint32_t n0, int stochastic,
+                                             uint32_t (&words)[4], float &s_out) {
+  const float r = (bits == 8) ? 127.0f : 7.0f;
+  float m = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
+  for (int st = 1; st < lpg; st <<= 1) m = max_nan(m, __shfl_xor_sync(kFull, m, st));
+  const bool gbad = !(m <= 3.402823466e38f);            // inf or NaN in the group
+  const unsigned bal = __ballot_sync(kFull, gbad);
+  const int riw = (lane % 32) / LPR;
+  const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
+  const bool row_bad = (bal & rowmask) != 0u;
+
+  float inv = 0.0f, s = 0.0f;
+  if (!row_bad && m > 0.0f) {
+    inv = __fdiv_rn(r, m);
+    if (inv <= 3.402823466e38f)
+      s = __fdiv_rn(m, r);
+    else
+      inv = 0.0f;                                        // m too small to scale: zero group
+  }
+  uint32_t t[16];
+  if (stochastic) {
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) h[q] = fmix32(tkey + 0x9E3779B9u * (n0 + q + 1u));
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float g = __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)));
+      t[e] = __float_as_uint(__fmaf_rn(x[e], inv, g));
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, 49152.5f));
+  }
+  if (bits == 8) {
+    const uint4 w = pack_i8(t);
+    words[0] = w.x; words[1] = w.y; words[2] = w.z; words[3] = w.w;
+  } else {
+    const uint2 w = pack_i4(t);
+    words[0] = w.x; words[1] = w.y; words[2] = 0u; words[3] = 0u;
+  }
+  if (row_bad) {
+    words[0] = words[1] = words[2] = words[3] = 0u;
+    s = 0.0f;
+  }
+  s_out = s;
+  return row_bad;
+}
+
+}  // namespace lores

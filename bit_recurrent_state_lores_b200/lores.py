@@ -1,0 +1,181 @@
+"""Thin ctypes binding of liblores.so (include/lores.h): same names, argument
+marshalling only.  Every step of the decode path runs in the library's kernels.
+
+Pointers may be given as ints or as torch tensors (their data_ptr() is passed);
+`stream` may be a torch.cuda.Stream, an int handle, or None for the current torch
+stream.  A non-OK status raises LoresError, except from lores_check_errors, which
+returns the status so that callers can test for NONFINITE.
+"""
+import ctypes as C
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblores.so")
+
+LORES_OK = 0
+LORES_ERR_INVALID_ARG = 1
+LORES_ERR_OOM = 2
+LORES_ERR_CUDA = 3
+LORES_ERR_NONFINITE = 4
+LORES_ERR_UNSUPPORTED = 5
+LORES_ERR_TIMEOUT = 6
+
+
+class LoresError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = int(status)
+        super().__init__(f"{where}: {lores_status_string(status)} ({status})")
+
+
+class lores_config(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("heads", C.c_int32), ("d_k", C.c_int32),
+                ("d_v", C.c_int32), ("group_size", C.c_int32), ("delta", C.c_int32),
+                ("decay_diag", C.c_int32), ("head_bits", C.POINTER(C.c_int32)),
+                ("stochastic", C.c_int32), ("seed", C.c_uint64), ("device", C.c_int32)]
+
+
+class lores_layout(C.Structure):
+    _fields_ = [("code_bytes", C.c_int64), ("seq_code_bytes", C.c_int64),
+                ("scale_count", C.c_int64), ("n_groups", C.c_int32),
+                ("units_per_step", C.c_int32), ("grid", C.c_int32), ("smem_bytes", C.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m "
+                          "bit_recurrent_state_lores_b200.build` (needs nvcc)")
+    L = C.CDLL(LIB_PATH)
+    P, U64, I32, F32 = C.c_void_p, C.c_uint64, C.c_int32, C.c_float
+    sig = {
+        "lores_create": (I32, [C.POINTER(lores_config), C.POINTER(P)]),
+        "lores_destroy": (I32, [P]),
+        "lores_decode_step": (I32, [P, P, P, P, P, P, P, U64, P]),
+        "lores_decode_step_host": (I32, [P, P, P, P, P, P, P, U64, P]),
+        "lores_dequant_state": (I32, [P, P, P]),
+        "lores_load_state": (I32, [P, P, U64, P]),
+        "lores_export_codes": (I32, [P, P, P, P]),
+        "lores_load_codes": (I32, [P, P, P, P]),
+        "lores_get_layout": (I32, [P, C.POINTER(lores_layout), P]),
+        "lores_check_errors": (I32, [P, P]),
+        "lores_assign_bits_by_decay": (I32, [P, I32, F32, I32, I32, P]),
+        "lores_status_string": (C.c_char_p, [I32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    return L
+
+
+_lib = _load()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if hasattr(x, "ctypes"):            # numpy array (host memory)
+        return x.ctypes.data
+    raise TypeError(f"cannot pass {type(x)} as a pointer")
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st, where):
+    if st != LORES_OK:
+        raise LoresError(st, where)
+
+
+def lores_status_string(status):
+    return _lib.lores_status_string(int(status)).decode()
+
+
+def lores_create(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
+                 stochastic=1, seed=0, device=0):
+    """Returns an opaque handle (int)."""
+    hb = None
+    if head_bits is not None:
+        arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
+        hb = C.cast(arr, C.POINTER(C.c_int32))
+    cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
+                       seed & (2**64 - 1), device)
+    out = C.c_void_p()
+    _check(_lib.lores_create(C.byref(cfg), C.byref(out)), "lores_create")
+    return out.value
+
+
+def lores_destroy(h):
+    _check(_lib.lores_destroy(h), "lores_destroy")
+
+
+def lores_decode_step(h, q, k, v, alpha, beta, o, step, stream=None):
+    _check(_lib.lores_decode_step(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                  _ptr(o), step & (2**64 - 1), _stream(stream)),
+           "lores_decode_step")
+
+
+def lores_decode_step_host(h, q, k, v, alpha, beta, o, step, stream=None):
+    _check(_lib.lores_decode_step_host(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                       _ptr(o), step & (2**64 - 1), _stream(stream)),
+           "lores_decode_step_host")
+
+
+def lores_dequant_state(h, out, stream=None):
+    _check(_lib.lores_dequant_state(h, _ptr(out), _stream(stream)), "lores_dequant_state")
+
+
+def lores_load_state(h, S, step, stream=None):
+    _check(_lib.lores_load_state(h, _ptr(S), step & (2**64 - 1), _stream(stream)),
+           "lores_load_state")
+
+
+def lores_export_codes(h, codes, scales, stream=None):
+    _check(_lib.lores_export_codes(h, _ptr(codes), _ptr(scales), _stream(stream)),
+           "lores_export_codes")
+
+
+def lores_load_codes(h, codes, scales, stream=None):
+    _check(_lib.lores_load_codes(h, _ptr(codes), _ptr(scales), _stream(stream)),
+           "lores_load_codes")
+
+
+def lores_get_layout(h, heads=None):
+    """Returns (lores_layout, head_offsets list or None)."""
+    lay = lores_layout()
+    offs = (C.c_int64 * heads)() if heads else None
+    _check(_lib.lores_get_layout(h, C.byref(lay), C.cast(offs, C.c_void_p) if offs else None),
+           "lores_get_layout")
+    return lay, (list(offs) if offs else None)
+
+
+def lores_check_errors(h, stream=None):
+    """Returns the status (LORES_OK, LORES_ERR_NONFINITE or LORES_ERR_TIMEOUT); raises
+    on other failures."""
+    st = _lib.lores_check_errors(h, _stream(stream))
+    if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT):
+        raise LoresError(st, "lores_check_errors")
+    return st
+
+
+def lores_assign_bits_by_decay(mean_decay, frac_high, bits_high=8, bits_low=4):
+    H = len(mean_decay)
+    d = (C.c_float * H)(*[float(x) for x in mean_decay])
+    out = (C.c_int32 * H)()
+    _check(_lib.lores_assign_bits_by_decay(C.cast(d, C.c_void_p), H, float(frac_high), bits_high,
+                                           bits_low, C.cast(out, C.c_void_p)),
+           "lores_assign_bits_by_decay")
+    return list(out)
+
+
+def raw_library():
+    """The loaded CDLL (for callers that marshal arguments themselves)."""
+    return _lib

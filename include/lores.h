@@ -1,0 +1,167 @@
+/*
+ * lores.h -- C ABI of the LoReS quantized recurrent-state decode step (B200, sm_100a).
+ *
+ * One decode step of a linear-recurrence layer, for every sequence and head of a
+ * batch, fused into one read and one write of the quantized state:
+ *
+ *   dequantize  S_hat = code * scale                       (value-axis groups)
+ *   update      S_t = S_hat diag(alpha_t) (I - delta beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   readout     o_t = S_t q_t                              (from the fp32 S_t)
+ *   requantize  per group of G key entries of one value row: s = max|S_t| / r,
+ *               r = 2^(b-1) - 1, stochastic rounding (or round to nearest)
+ *
+ * Sources: "Quantizing Recurrent Language Models Is Easier Than You Think"
+ * (summary page): General recurrence form (Introduction); Key properties item 3
+ * (dequantize -> update -> requantize each step); Proposition 1 (absmax scale,
+ * value-axis grouping); Table 5 text (decay-based mixed precision per head);
+ * Proposition 3 / Table 6 (stochastic rounding).
+ *
+ * Conventions for every call:
+ *  - Every function returns a lores_status; nothing aborts, throws or traps.
+ *  - Device pointers are plain CUDA device addresses (for example a torch tensor's
+ *    data_ptr()).  Unless a call says otherwise they are owned by the caller, must be
+ *    fp32, contiguous, row-major with the shapes given, and stay valid until the
+ *    stream has executed the call.  Vector inputs q, k, v, alpha (per column) and the
+ *    outputs of dequant/load must be 16-byte aligned; misaligned or NULL pointers
+ *    return LORES_ERR_INVALID_ARG before anything is launched.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Calls that launch work are asynchronous unless stated.
+ *  - A handle is not thread-safe: two calls on one handle that overlap on the GPU
+ *    (different streams, no ordering) race on the state.
+ *  - CUDA failures map to LORES_ERR_CUDA.  Values that the device finds non-finite
+ *    raise a sticky flag that lores_check_errors reports.
+ *
+ * Shapes: B = batch, H = heads, d_k = key dim (16, 32, 64, 128 or 256), d_v = value
+ * dim (multiple of 4, at most 4096), G = group_size (multiple of 16 dividing d_k).
+ */
+#ifndef LORES_H
+#define LORES_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LORES_OK = 0,
+    LORES_ERR_INVALID_ARG = 1,   /* bad shape, value, NULL or misaligned pointer          */
+    LORES_ERR_OOM = 2,           /* a device or host allocation failed                   */
+    LORES_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed                 */
+    LORES_ERR_NONFINITE = 4,     /* a state row became non-finite (inf or NaN)            */
+    LORES_ERR_UNSUPPORTED = 5,   /* well-formed but not supported (bits, d_k, device)     */
+    LORES_ERR_TIMEOUT = 6        /* a kernel gave up waiting on its own copies            */
+} lores_status;
+
+typedef struct lores_handle lores_handle;
+
+/* Create-time description of one recurrent layer's state for a batch. */
+typedef struct {
+    int32_t batch;          /* B >= 1 sequences                                              */
+    int32_t heads;          /* H >= 1                                                        */
+    int32_t d_k;            /* key dim: 16, 32, 64, 128 or 256                               */
+    int32_t d_v;            /* value dim: multiple of 4, 4..4096                             */
+    int32_t group_size;     /* G: key entries per scale; 0 means d_k (one scale per row)     */
+    int32_t delta;          /* 1: delta-rule correction (GDN, KDA); 0: none (Mamba-2)        */
+    int32_t decay_diag;     /* 0: alpha is one scalar per (seq, head); 1: one per key column */
+    const int32_t *head_bits; /* host [H], each 8, 4 or 32 (fp32, unquantized); NULL: all 8 */
+    int32_t stochastic;     /* 1: stochastic rounding (LoReS); 0: round to nearest           */
+    uint64_t seed;          /* key of the rounding dither                                    */
+    int32_t device;         /* CUDA device ordinal                                           */
+} lores_config;
+
+/* Sizes of the handle's state, for export/import buffers. */
+typedef struct {
+    int64_t code_bytes;        /* bytes of the whole code pool = batch * seq_code_bytes      */
+    int64_t seq_code_bytes;    /* bytes of one sequence: all heads' tiles back to back       */
+    int64_t scale_count;       /* fp32 scales: batch * heads * d_v * n_groups                */
+    int32_t n_groups;          /* d_k / G                                                    */
+    int32_t units_per_step;    /* work units (sequence, head, row block) of one step         */
+    int32_t grid;              /* CTAs of the decode kernel                                  */
+    int32_t smem_bytes;        /* dynamic shared memory per CTA of the decode kernel         */
+} lores_layout;
+
+/* Create a handle: validate `cfg`, allocate the code pool, the scales and the
+ * handle's bookkeeping on cfg->device, and zero the state (the zero state has
+ * scale 0 and code 0 everywhere).  The head precision map is fixed for the life of
+ * the handle (Table 5 text: precision follows the head's decay).  On success
+ * *out receives the handle; on failure *out is NULL.  Errors: INVALID_ARG
+ * (shapes, bits, group size), UNSUPPORTED (device without sm_100), OOM, CUDA. */
+lores_status lores_create(const lores_config *cfg, lores_handle **out);
+
+/* Release every allocation of the handle.  NULL is accepted and returns LORES_OK.
+ * The caller must make sure no work on the handle is still queued. */
+lores_status lores_destroy(lores_handle *h);
+
+/* One decode step for all B*H (sequence, head) pairs, in place on the handle's
+ * state (General recurrence form; dequantize -> update -> requantize).
+ *   q, k   [B, H, d_k] unit-norm fp32 (not renormalised here)
+ *   v      [B, H, d_v]
+ *   alpha  [B, H] (decay_diag = 0) or [B, H, d_k] (decay_diag = 1), in (0, 1]
+ *   beta   [B, H], in (0, 2)
+ *   o      [B, H, d_v] output, o_t = S_t q_t from the updated fp32 state
+ *   step   the rounding counter: the dither of step t is a pure function of
+ *          (seed, step, sequence, head, row, column), so replaying the same steps
+ *          from the same state reproduces the state bit for bit.
+ * A row whose updated state holds inf or NaN is stored as zero (scales 0, codes 0)
+ * and raises the sticky NONFINITE flag.  Asynchronous on `stream`. */
+lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, const float *v,
+                               const float *alpha, const float *beta, float *o,
+                               uint64_t step, void *stream);
+
+/* The same step with HOST buffers of the same shapes (pinned or pageable).  The
+ * call copies the inputs to device staging buffers owned by the handle (allocated
+ * on first use), runs the step, copies o back, and returns after `stream` has
+ * finished, so `o` is valid on return. */
+lores_status lores_decode_step_host(lores_handle *h, const float *q, const float *k,
+                                    const float *v, const float *alpha, const float *beta,
+                                    float *o, uint64_t step, void *stream);
+
+/* Write the dequantized state, out[B, H, d_v, d_k] = code * scale (fp32 heads:
+ * the state itself), to device memory `out`.  Asynchronous. */
+lores_status lores_dequant_state(lores_handle *h, float *out, void *stream);
+
+/* Replace the state by the quantization of the fp32 state S[B, H, d_v, d_k]
+ * (device memory), with the decode step's own quantizer and the dither of `step`
+ * (fp32 heads copy S).  Used to start from a warmed-up fp32 state.  Asynchronous. */
+lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, void *stream);
+
+/* Copy the raw state out: codes (layout_.code_bytes bytes; per sequence the heads'
+ * tiles back to back in head order; a tile is row-major [d_v][d_k] int8, or
+ * [d_v][d_k/2] bytes of int4 with the even column in the low nibble, or
+ * [d_v][d_k] fp32) and scales [B, H, d_v, n_groups] fp32.  Either pointer may be
+ * host or device memory (unified addressing); either may be NULL to skip it.
+ * Returns after the copies have finished on `stream`. */
+lores_status lores_export_codes(lores_handle *h, void *codes, float *scales, void *stream);
+
+/* Inverse of lores_export_codes: overwrite the state with the given codes and
+ * scales (host or device memory).  Returns after the copies have finished. */
+lores_status lores_load_codes(lores_handle *h, const void *codes, const float *scales,
+                              void *stream);
+
+/* Fill *out with the handle's sizes.  head_offsets (may be NULL) receives H int64
+ * byte offsets of each head's tile inside one sequence's block. */
+lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t *head_offsets);
+
+/* Wait for `stream`, then read and clear the handle's sticky device flag.
+ * Returns LORES_ERR_TIMEOUT if a kernel gave up waiting on its own copies (its
+ * outputs for that call are incomplete), else LORES_ERR_NONFINITE if any row
+ * became non-finite since the last check, else LORES_OK. */
+lores_status lores_check_errors(lores_handle *h, void *stream);
+
+/* Decay-based mixed precision (Table 5 text): the round(frac_high * H) heads with
+ * the largest mean decay (slowest to forget) get bits_high, the others bits_low;
+ * equal decays go to the lower head index.  Host only; mean_decay and out_bits
+ * are host arrays of H entries.  Errors: INVALID_ARG for NULL, H < 1, frac outside
+ * [0, 1] or bits outside {4, 8, 32}. */
+lores_status lores_assign_bits_by_decay(const float *mean_decay, int32_t H, float frac_high,
+                                        int32_t bits_high, int32_t bits_low, int32_t *out_bits);
+
+/* Static English name of a status code. */
+const char *lores_status_string(lores_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORES_H */
