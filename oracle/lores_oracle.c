@@ -21,15 +21,25 @@
  *
  * Readings where the pages are silent (each is a choice, not a page fact):
  *   - Scales are recomputed from the updated state on every step.
- *   - The readout o_t uses the updated fp32 state before requantization.
+ *   - The readout o_t = S_t q_t uses S_t = S' + w k^T (S' = S_{t-1} diag(alpha)
+ *     in fp32, w in fp32) evaluated exactly, i.e. before requantization and before
+ *     the fp32 rounding of the stored entries.
  *   - Products and sums are fp32 with the association written below; the
- *     dot product S'k uses a fixed order (16-column sequential chunks, then a
- *     pairwise combine of the chunk sums) so that two implementations that
- *     follow it agree bit for bit.  The readout is summed in double.
+ *     dot product S'k uses a fixed order (4-column sequential chunks, then a
+ *     pairwise combine of the chunk sums, nearest partners first) so that two
+ *     implementations that follow it agree bit for bit.  The readout is summed
+ *     in double.
+ *   - Scale and its inverse: s = m * fl(1/r); inv = r * y, where y ~ 1/m comes
+ *     from three Newton-Raphson steps y <- y + y(1 - m y) (fma form) started
+ *     from the exponent-reflected seed bits(y0) = 0x7F000000 - bits(m).  The
+ *     relative error of inv is below 1e-6, far inside what the quantizer's
+ *     range argument needs (2^-16).  Group maxima outside [2^-100, 2^100] are
+ *     not scaled: below, the group is stored as zero; above, the row is
+ *     treated as overflow (stored as zero and flagged).
  *   - Stochastic rounding adds an 8-bit dither on a grid of 1/256 of a code
- *     step: t = fma(x, r/m, 49152 + d/256); code = floor(t - 49152).  49152 is
+ *     step: t = fma(x, inv, 49152 + d/256); code = floor(t - 49152).  49152 is
  *     1.5 * 2^15, whose float spacing is exactly 1/256, so the fma rounds
- *     x*r/m to the nearest 1/256 and adds d/256 exactly.  With d uniform in
+ *     x*inv to the nearest 1/256 and adds d/256 exactly.  With d uniform in
  *     0..255 the code is unbiased up to that 1/512-step rounding.
  *   - The dither bytes come from SplitMix64 (Steele, Lea, Flood 2014) and the
  *     MurmurHash3 32-bit finalizer (Appleby), keyed on seed, step, sequence,
@@ -140,20 +150,20 @@ void lo_put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code) { put_
 /* Fixed-order dot product                                                  */
 /* ------------------------------------------------------------------------ */
 
-/* sum_j a_j b_j for n = 16*C, C a power of two <= 16: each chunk of 16
- * consecutive terms is a sequential fma chain from zero; the C chunk sums
- * are then combined pairwise, partner at distance C/2, C/4, ..., 1. */
-float lo_dot_c16(const float *a, const float *b, int n)
+/* sum_j a_j b_j for n = 4*C, C a power of two <= 64: each chunk of 4
+ * consecutive terms is a sequential fma chain from zero; the C chunk sums are
+ * then combined pairwise, partner at distance 1, then 2, 4, ..., C/2. */
+float lo_dot_c4(const float *a, const float *b, int n)
 {
-    float p[16], nxt[16];
-    int C = n / 16;
+    float p[64], nxt[64];
+    int C = n / 4;
     for (int c = 0; c < C; c++) {
         float acc = 0.0f;
-        for (int e = 0; e < 16; e++)
-            acc = fmaf(a[16 * c + e], b[16 * c + e], acc);
+        for (int e = 0; e < 4; e++)
+            acc = fmaf(a[4 * c + e], b[4 * c + e], acc);
         p[c] = acc;
     }
-    for (int stride = C / 2; stride >= 1; stride /= 2) {
+    for (int stride = 1; stride < C; stride *= 2) {
         for (int l = 0; l < C; l++)
             nxt[l] = p[l] + p[l ^ stride];
         memcpy(p, nxt, sizeof(float) * C);
@@ -161,39 +171,60 @@ float lo_dot_c16(const float *a, const float *b, int n)
     return p[0];
 }
 
+/* Approximate 1/m for m in [2^-100, 2^100]: seed from reflecting the exponent
+ * field (exact for powers of two, within 12.5% otherwise), then three
+ * Newton-Raphson steps for f(y) = 1/y - m, written y <- y + y (1 - m y) with
+ * fmas.  Each step squares the relative error: 1.3e-1 -> 1.6e-2 -> 2.4e-4 -> ~1e-7. */
+float lo_recip_nr(float m)
+{
+    uint32_t bm, by;
+    float y;
+    memcpy(&bm, &m, 4);
+    by = 0x7F000000u - bm;
+    memcpy(&y, &by, 4);
+    for (int it = 0; it < 3; it++) {
+        float e = fmaf(-m, y, 1.0f);
+        y = fmaf(y, e, y);
+    }
+    return y;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Requantization of one value row (Proposition 1 scale, SR or RTN)         */
 /* ------------------------------------------------------------------------ */
 
 /* x: the updated fp32 row (d_k entries).  Writes the row's codes and its
- * d_k/G scales.  A row that holds a non-finite entry is stored as zero
- * (scales 0, codes 0) and reported with return value 1. */
+ * d_k/G scales.  A row that holds a non-finite entry (or one above 2^100) is
+ * stored as zero (scales 0, codes 0) and reported with return value 1. */
 static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_key,
                           uint8_t *codes, float *scales)
 {
     const int r = code_max(c->bits);
+    const float inv_r = (c->bits == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   /* fl(1/r) */
+    const float m_lo = 0x1p-100f, m_hi = 0x1p100f;
     const int ng = c->d_k / c->group;
     int bad = 0;
     for (int j = 0; j < c->d_k; j++)
         if (!isfinite(x[j]))
             bad = 1;
+    for (int g = 0; g < ng && !bad; g++)
+        for (int j = g * c->group; j < (g + 1) * c->group; j++)
+            if (fabsf(x[j]) > m_hi)
+                bad = 1;                  /* overflow: treated like a non-finite row */
     for (int g = 0; g < ng; g++) {
         float m = 0.0f;
         for (int j = g * c->group; j < (g + 1) * c->group; j++)
             if (fabsf(x[j]) > m)
                 m = fabsf(x[j]);
         float inv = 0.0f, s = 0.0f;
-        if (!bad && m > 0.0f) {
-            inv = (float)r / m;            /* round to nearest */
-            if (isfinite(inv))
-                s = m / (float)r;          /* round to nearest */
-            else
-                inv = 0.0f;                /* m too small to scale: store as zero */
+        if (!bad && m >= m_lo) {
+            inv = (float)r * lo_recip_nr(m);
+            s = m * inv_r;
         }
         scales[(size_t)i * ng + g] = s;
         for (int j = g * c->group; j < (g + 1) * c->group; j++) {
             int code = 0;
-            if (!bad && inv != 0.0f) {
+            if (inv != 0.0f) {
                 float d = c->stochastic ? (float)lo_dither(tile_key, c->d_k, i, j) : 128.0f;
                 float t = fmaf(x[j], inv, 49152.0f + d / 256.0f);
                 code = (int)floorf(t - 49152.0f);
@@ -237,17 +268,18 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
         /* write: w_i = beta (v_i - delta u_i), u_i = (S' k)_i */
         float w;
         if (c->delta) {
-            float u = lo_dot_c16(Sp, k, dk);
+            float u = lo_dot_c4(Sp, k, dk);
             w = beta * (v[i] - u);
         } else {
             w = beta * v[i];
         }
         for (int j = 0; j < dk; j++)
             x[j] = fmaf(w, k[j], Sp[j]);
-        /* readout o_i = (S_t q)_i from the fp32 state */
+        /* readout o_i = (S_t q)_i with S_t = S' + w k^T evaluated exactly (in double)
+         * from the fp32 S' and w, before any rounding of the stored state */
         double o = 0.0;
         for (int j = 0; j < dk; j++)
-            o += (double)x[j] * (double)q[j];
+            o += ((double)Sp[j] + (double)w * (double)k[j]) * (double)q[j];
         o_out[i] = o;
         if (x_out)
             memcpy(x_out + (size_t)i * dk, x, sizeof(float) * dk);

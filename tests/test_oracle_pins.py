@@ -118,7 +118,7 @@ def test_dot_exact_on_integers():
     for n in (16, 32, 64, 128, 256):
         a = g.integers(-50, 50, n).astype(np.float32)
         b = g.integers(-50, 50, n).astype(np.float32)
-        assert O.dot_c16(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
+        assert O.dot_c4(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
 
 
 def test_dot_error_bound():
@@ -130,17 +130,32 @@ def test_dot_error_bound():
         exact = sum(Fraction(float(x)) * Fraction(float(y)) for x, y in zip(a, b))
         u = 2.0 ** -24
         bound = n * u / (1 - n * u) * float(np.sum(np.abs(a.astype(np.float64) * b)))
-        assert abs(float(Fraction(O.dot_c16(a, b)) - exact)) <= bound
+        assert abs(float(Fraction(O.dot_c4(a, b)) - exact)) <= bound
 
 
 def test_dot_combine_order_worked_example():
-    # Chunk sums p = [2^24, 1, -2^24, 1] (one nonzero term per 16-column chunk).
-    # Partner at distance C/2 first: [p0+p2, p1+p3] = [0, 2], then 0 + 2 = 2.
-    # (A left-to-right sum would lose the first 1 and give 1.)
-    a = np.zeros(64, np.float32)
-    b = np.ones(64, np.float32)
-    a[0], a[16], a[32], a[48] = 2.0 ** 24, 1.0, -(2.0 ** 24), 1.0
-    assert O.dot_c16(a, b) == 2.0
+    # Chunk sums p = [1, 2^24, 1, -2^24] (one nonzero term per 4-column chunk).
+    # Nearest partner first: [p0+p1, p2+p3] = [2^24 (the 1 is lost: tie to even),
+    # 1 - 2^24 (exact)], then 2^24 + (1 - 2^24) = 1.  (Left to right would give 0;
+    # the far partner first would give [p0+p2, p1+p3] = [2, 0] -> 2.)
+    a = np.zeros(16, np.float32)
+    b = np.ones(16, np.float32)
+    a[0], a[4], a[8], a[12] = 1.0, 2.0 ** 24, 1.0, -(2.0 ** 24)
+    assert O.dot_c4(a, b) == 1.0
+
+
+def test_newton_reciprocal_error_bound():
+    # three Newton-Raphson steps from the exponent-reflected seed: |m y - 1| <= 2^-21
+    g = rng(60)
+    ms = np.concatenate([2.0 ** g.uniform(-100, 100, 20000), 1 + np.arange(0, 1, 1 / 4096),
+                         [2.0 ** -100, 2.0 ** 100, 1.5, 1.9999999]]).astype(np.float32)
+    worst = 0.0
+    for m in ms:
+        y = O.recip_nr(m)
+        worst = max(worst, abs(float(m) * y - 1.0))
+    assert worst <= 2.0 ** -21, worst
+    for k in range(-100, 101, 7):                     # exact on powers of two
+        assert O.recip_nr(2.0 ** k) == 2.0 ** -k
 
 
 # --------------------------------------------------------------------------
@@ -260,7 +275,9 @@ def test_absmax_quantizer_invariants(bits, group, sr):
             if m == 0:
                 assert s == 0 and not cs.any()
                 continue
-            assert s == np.float32(m / np.float32(r))
+            # s = m * fl(1/r): two roundings, so |s r / m - 1| <= 2^-24 + 2^-24 (+ tiny)
+            assert s == np.float32(m * (np.float32(1) / np.float32(r)))
+            assert abs(float(s) * r / float(m) - 1.0) <= 2.0 ** -23 * (1 + 1e-6)
             assert np.abs(cs).max() == r            # the group's max code is r exactly
             err = np.abs(cs * np.float64(s) - xs)
             lim = (1.0 if sr else 0.5 + 2.0 ** -8) * float(s) * (1 + 1e-6)
@@ -320,6 +337,21 @@ def test_round_to_nearest_mode_is_deterministic_nearest():
     # equal except where x/s sits within 1/512 of a half step
     frac = np.abs(X / s1 - np.floor(X / s1) - 0.5)
     assert ((Y == nearest) | (frac < 2.0 ** -8)).all()
+
+
+def test_scale_range_rules():
+    # group maxima below 2^-100 are stored as zero; above 2^100 the row is overflow
+    d_k, d_v = 32, 4
+    cfg = O.TileCfg(d_k, d_v, group=16, bits=8)
+    X = rng(16).standard_normal((d_v, d_k)).astype(np.float32)
+    X[0, :16] *= np.float32(2.0 ** -104)              # tiny group, rest of the row normal
+    X[1, 3] = np.float32(2.0 ** 101)                  # overflow row
+    codes, scales, flag = O.tile_quantize(cfg, X, 3)
+    C_ = O.unpack_codes(cfg, codes)
+    assert flag == 1
+    assert scales[0, 0] == 0 and not C_[0, :16].any() and np.abs(C_[0, 16:]).max() == 127
+    assert not C_[1].any() and not scales[1].any()
+    assert np.abs(C_[2:]).max() == 127
 
 
 def test_nonfinite_row_is_zeroed_and_flagged():
