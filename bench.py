@@ -217,6 +217,36 @@ def cpu_cores_used():
 
 
 # ---------------------------------------------------------------------------------------
+# ranks (one process per GPU; sequences are independent, so ranks share nothing)
+# ---------------------------------------------------------------------------------------
+
+def rank_seed(layer_seed, rank):
+    """Rounding-dither seed of one layer on one rank: every rank decodes its own batch."""
+    return (layer_seed << 8) + rank
+
+
+def rank_input_step(rank, p):
+    """Generator step index of input set p on `rank` (distinct inputs per rank)."""
+    return 10_000 * rank + p
+
+
+def reduce_max(x, device):
+    """Max of a float over ranks (the job time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, batch, heads, layers, steps, max_ms):
+    """Whole-job state updates per second: every rank's units over the slowest rank's time."""
+    return world * batch * heads * layers * steps / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------
 
@@ -236,8 +266,9 @@ def run_ours(args, rank, world, local_rank):
         hp = synth.head_params(wll)
         h = L.lores_create(wl.B, wl.H, wl.d_k, wl.d_v, group_size=0, delta=wl.delta,
                            decay_diag=wl.diag, head_bits=bits, stochastic=1,
-                           seed=(wll.seed << 8) + rank, device=local_rank)
-        inputs = [synth.step_inputs(wll, 10_000 * rank + p, hp, device=dev) for p in range(2)]
+                           seed=rank_seed(wll.seed, rank), device=local_rank)
+        inputs = [synth.step_inputs(wll, rank_input_step(rank, p), hp, device=dev)
+                  for p in range(2)]
         o = torch.empty(wl.B, wl.H, wl.d_v, device=dev)
         layers.append((h, bits, inputs, o))
     bytes_per_launch = [launch_bytes(wl, bits) for (_, bits, _, _) in layers]
@@ -283,10 +314,7 @@ def run_ours(args, rank, world, local_rank):
     ms = start.elapsed_time(end)
     launch_ms = [evs[n][li][0].elapsed_time(evs[n][li][1]) for n in range(K)
                  for li in range(len(layers))]
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, dev)
     clock_summary = None
     if clocks:
         time.sleep(0.2)
@@ -296,8 +324,7 @@ def run_ours(args, rank, world, local_rank):
         st = L.lores_check_errors(h, sptr)
         assert st == L.LORES_OK, L.lores_status_string(st)
 
-    units = world * wl.B * wl.H * wl.layers * K
-    value = units / (ms / 1e3)
+    value = job_rate(world, wl.B, wl.H, wl.layers, K, ms)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     avg_bytes = statistics.mean(bytes_per_launch)
     peak, peak_kind = measured_peak()
@@ -326,12 +353,8 @@ def run_ours(args, rank, world, local_rank):
                 L.lores_decode_step_host(h, q, k, v, a, b, o, 1_000_000 + n, sptr)
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * wl.B * wl.H * wl.layers * Ke / (ems / 1e3), "unit": UNIT,
+        ems = reduce_max(s0.elapsed_time(s1), dev)
+        e2e = {"value": job_rate(world, wl.B, wl.H, wl.layers, Ke, ems), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
                "api": "lores_decode_step_host (pinned host buffers)"}
 

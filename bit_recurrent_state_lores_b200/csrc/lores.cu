@@ -29,7 +29,7 @@
 
 namespace lores {
 
-// One work unit inside a sequence's block.
+// One work unit: a block of rows of one (sequence, head) tile, processed by one warp.
 struct __align__(16) UnitDesc {
   int32_t head;
   int32_t row0;
@@ -50,22 +50,33 @@ struct StepParams {
   long long total_units;
   int H, d_v, ng, G, units_per_seq;
   uint32_t step_key;
-  int stochastic;
-  // stage layout (bytes from the stage start)
-  int st_scales, st_k, st_q, st_v, st_a, stage_bytes;
+  // shared memory layout: [unit table][warp 0 area][warp 1 area]...; a warp area is
+  // [2 mbarriers | pad to 64][readout partials][row w][stage 0][stage 1]
+  int table_bytes;       // bytes of the unit table copy (0: read the table from global)
+  int warp_bytes;        // bytes of one warp area
+  int opart_floats;      // readout partials per warp (max rows * lanes per row)
+  int ow_floats;         // row w per warp (max rows)
+  int st_scales, st_k, st_q, st_v, st_a, stage_bytes;   // stage layout
 };
 
 // Bytes of one row of a tile with `bits`-bit entries.
-__host__ __device__ inline int row_bytes(int dk, int bits) { return dk * bits / 8; }
+__host__ __device__ constexpr int row_bytes(int dk, int bits) { return dk * bits / 8; }
+
+// Rows of a full unit: 4 KB of state, a whole number of warp passes (32/(d_k/16) rows).
+__host__ __device__ constexpr int full_rows(int dk, int bits) {
+  return (4096 / row_bytes(dk, bits)) < (32 / (dk / 16))
+             ? (32 / (dk / 16))
+             : (4096 / row_bytes(dk, bits)) - (4096 / row_bytes(dk, bits)) % (32 / (dk / 16));
+}
 
 // -------------------------------------------------------------------------------------
-// producer: stage one unit's inputs into shared memory
+// producer (one lane of the warp): stage one unit's inputs into the warp's ring slot
 // -------------------------------------------------------------------------------------
 template <int DK, bool DIAG>
-__device__ __forceinline__ void issue_unit(const StepParams &p, long long u, uint8_t *stage,
-                                           uint64_t *bar) {
+__device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *tbl, long long u,
+                                           uint8_t *stage, uint64_t *bar) {
   const long long b = u / p.units_per_seq;
-  const UnitDesc d = p.units[u % p.units_per_seq];
+  const UnitDesc d = tbl[u % p.units_per_seq];
   const long long tile = b * p.H + d.head;
   const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
   const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
@@ -83,19 +94,27 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, long long u, uin
 }
 
 // -------------------------------------------------------------------------------------
-// consumer: one unit (rows [row0, row0 + nrows) of one tile) from its stage
+// consumer (the whole warp): rows [row0, row0 + nrows) of one tile from a stage
 // -------------------------------------------------------------------------------------
-template <int DK, bool DIAG, bool DELTA, int BITS>
+// Lane layout: LPR = d_k/16 lanes own a row, 16 consecutive columns each; a warp pass
+// covers RPW = 32/LPR rows.  FULL: every pass is complete (nrows % RPW == 0).
+// The readout is reduced per warp: each lane leaves its share of S'q in opart, lane 0
+// of the row leaves w in ow, and after the rows each lane forms o for one row as
+// sum(opart) + w (k.q).
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL>
 __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, long long b,
-                                             const UnitDesc &d) {
+                                             const UnitDesc &d, float alpha_s, float beta,
+                                             float *opart, float *ow) {
   constexpr int LPR = DK / 16;            // lanes per row
   constexpr int RPW = 32 / LPR;           // rows per warp pass
   constexpr int RB = DK * BITS / 8;       // bytes per row
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int lir = lane % LPR, riw = lane / LPR;
   const int col0 = lir * 16;
-  const int lpg = p.G / 16;
-  const int g = col0 / p.G;
+  const int lpg = p.G / 16;                               // lanes per scale group (power of 2)
+  const int g = lir / lpg;                                 // this lane's group in the row
+  const bool scale_writer = (lir & (lpg - 1)) == 0;
+  const int ng = p.ng;
   const long long tile = b * p.H + d.head;
 
   const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
@@ -116,17 +135,25 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
       aa[4 * c] = a4.x; aa[4 * c + 1] = a4.y; aa[4 * c + 2] = a4.z; aa[4 * c + 3] = a4.w;
     }
   }
-  const float alpha_s = DIAG ? 0.0f : __ldg(p.alpha + tile);
-  const float beta = __ldg(p.beta + tile);
+  // k.q in double (strided columns, warp butterfly): the readout is o = S'q + w (k.q),
+  // which keeps the step-0 readout (S' = 0) exact even for nearly orthogonal k and q.
+  double kqd = 0.0;
+#pragma unroll
+  for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sq[j], kqd);
+#pragma unroll
+  for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
+  const float kq = (float)kqd;
   const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
 
   uint8_t *gcodes = p.codes + b * p.seq_bytes + d.code_off;
-  float *gscales = p.scales + (tile * p.d_v + d.row0) * p.ng;
-  float *go = p.o + tile * p.d_v + d.row0;
+  float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
+  constexpr int kFullPasses = full_rows(DK, BITS) / RPW;
+  const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
 
-  for (int base = warp * RPW; base < d.nrows; base += kWarps * RPW) {
-    const int lr = base + riw;                 // row inside the unit
-    const bool active = lr < d.nrows;
+#pragma unroll(FULL ? 4 : 1)
+  for (int n = 0; n < npass; ++n) {
+    const int lr = n * RPW + riw;              // row inside the unit
+    const bool active = FULL || lr < d.nrows;
     const int lrr = active ? lr : 0;           // keep shared loads in bounds
 
     // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
@@ -147,7 +174,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
         unpack_i8(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
       else
         unpack_i4(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
-      const float s_in = ss[lrr * p.ng + g];
+      const float s_in = ss[lrr * ng + g];
       const float a_row = __fmul_rn(s_in, alpha_s);
 #pragma unroll
       for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(cf[e], DIAG ? __fmul_rn(s_in, aa[e]) : a_row);
@@ -157,11 +184,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     const float vr = sv[lrr];
     float w;
     if (DELTA) {
-      float u = 0.0f;
+      float u = dot16_c4(sp, kk);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) u = __fmaf_rn(sp[e], kk[e], u);
-#pragma unroll
-      for (int st = LPR / 2; st >= 1; st >>= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
+      for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
       w = __fmul_rn(beta, __fsub_rn(vr, u));
     } else {
       w = __fmul_rn(beta, vr);
@@ -170,35 +195,32 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
 #pragma unroll
     for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(w, kk[e], sp[e]);
 
-    // ---- readout o = S_t q -----------------------------------------------------------
-    float oacc = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) oacc = __fmaf_rn(x[e], qq[e], oacc);
-#pragma unroll
-    for (int st = LPR / 2; st >= 1; st >>= 1) oacc = __fadd_rn(oacc, __shfl_xor_sync(kFull, oacc, st));
+    // ---- readout share: this lane's part of S'q ----------------------------------------
+    const float opv = dot16_c4(sp, qq);
+    if (active) {
+      opart[lr * LPR + lir] = opv;
+      if (lir == 0) ow[lr] = w;
+    }
 
     // ---- requantize and store --------------------------------------------------------
-    const int row = d.row0 + lrr;              // row inside the tile (dither counter)
-    bool row_bad;
     if (BITS == 32) {
       float m = 0.0f;
 #pragma unroll
       for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
       const bool lbad = !(m <= 3.402823466e38f);
-      const unsigned bal = __ballot_sync(kFull, lbad);
-      const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
-      row_bad = (bal & rowmask) != 0u;
       if (active) {
         float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           __stcs(dst + c, make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
       }
+      if (__any_sync(kFull, lbad) && lbad && active) atomicOr(p.flag, kFlagNonFinite);
     } else {
       uint32_t words[4];
       float s_new;
-      const uint32_t n0 = (uint32_t)row * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
-      row_bad = requantize16<LPR>(x, BITS, lpg, lane, tkey, n0, p.stochastic, words, s_new);
+      const uint32_t n0 = (uint32_t)(d.row0 + lrr) * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
+      const bool row_bad =
+          requantize16<LPR>(x, BITS, lpg, lane, tkey, n0, SR ? 1 : 0, words, s_new);
       if (active) {
         if (BITS == 8)
           __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
@@ -206,70 +228,119 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
         else
           __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8),
                  make_uint2(words[0], words[1]));
-        if (lir % lpg == 0) gscales[(size_t)lr * p.ng + g] = s_new;
+        if (scale_writer) gscales[lr * ng + g] = s_new;
       }
-    }
-    if (active && lir == 0) {
-      go[lr] = oacc;
-      if (row_bad) atomicOr(p.flag, kFlagNonFinite);
+      if (row_bad && active && lir == 0) atomicOr(p.flag, kFlagNonFinite);
     }
   }
+
+  // ---- readout: o_i = sum of the row's lane shares + w_i (k.q) -------------------------
+  __syncwarp();
+  float *go = p.o + tile * p.d_v + d.row0;
+  for (int r = lane; r < d.nrows; r += 32) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
+    go[r] = __fmaf_rn(ow[r], kq, acc);
+  }
+  __syncwarp();
 }
 
-template <int DK, bool DIAG, bool DELTA>
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS>
+__device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *stage, long long b,
+                                            const UnitDesc &d, float alpha_s, float beta,
+                                            float *opart, float *ow) {
+  if (d.nrows == full_rows(DK, BITS))
+    compute_unit<DK, DIAG, DELTA, SR, BITS, true>(p, stage, b, d, alpha_s, beta, opart, ow);
+  else
+    compute_unit<DK, DIAG, DELTA, SR, BITS, false>(p, stage, b, d, alpha_s, beta, opart, ow);
+}
+
+// Persistent kernel: every warp runs its own pipeline over units gw, gw + W, gw + 2W, ...
+// (gw = global warp index, W = warps in the grid), with a 2-slot ring of bulk copies
+// whose producer is the warp's lane 0.  Warps never wait on one another.
+template <int DK, bool DIAG, bool DELTA, bool SR>
 __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-  uint8_t *stages = smem + 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  UnitDesc *stbl = reinterpret_cast<UnitDesc *>(smem);
+  uint8_t *wa = smem + p.table_bytes + warp * p.warp_bytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wa);
+  float *opart = reinterpret_cast<float *>(wa + 64);
+  float *ow = opart + p.opart_floats;
+  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
 
-  const long long first = blockIdx.x;
-  const long long stride = gridDim.x;
+  const UnitDesc *tbl = p.units;
+  if (p.table_bytes) {
+    for (int i = threadIdx.x; i < p.units_per_seq; i += kThreads) stbl[i] = p.units[i];
+    tbl = stbl;
+  }
+  __syncthreads();                                  // the only CTA-wide barrier
+
+  const long long first = (long long)blockIdx.x * kWarps + warp;
+  const long long stride = (long long)gridDim.x * kWarps;
   if (first >= p.total_units) return;
 
-  if (threadIdx.x == 0) {
+  if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       const long long u = first + s * stride;
-      if (u < p.total_units) issue_unit<DK, DIAG>(p, u, stages + s * p.stage_bytes, &bars[s]);
+      if (u < p.total_units) issue_unit<DK, DIAG>(p, tbl, u, stages + s * p.stage_bytes, &bars[s]);
     }
+  }
+  __syncwarp();
+
+  // per-tile scalars of the current unit; the next unit's are loaded one unit ahead
+  auto tile_of = [&](long long u) {
+    return (u / p.units_per_seq) * p.H + tbl[u % p.units_per_seq].head;
+  };
+  float alpha_cur = 0.0f, beta_cur;
+  {
+    const long long t0 = tile_of(first);
+    beta_cur = __ldg(p.beta + t0);
+    if (!DIAG) alpha_cur = __ldg(p.alpha + t0);
   }
 
   int n = 0;
   for (long long u = first; u < p.total_units; u += stride, ++n) {
     const int s = n % kStages;
     uint8_t *stage = stages + s * p.stage_bytes;
+    float alpha_nx = 0.0f, beta_nx = 0.0f;
+    if (u + stride < p.total_units) {
+      const long long tn = tile_of(u + stride);
+      beta_nx = __ldg(p.beta + tn);
+      if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
+    }
     const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1));
-    if (__syncthreads_or(!ok)) {
-      // Give up: record it, let the other stage's copy (if any) land, and leave.
-      if (threadIdx.x == 0) {
+    if (!__all_sync(kFull, ok)) {
+      // Give up: record it, let the other slot's copy (if any) land, and leave.
+      if (lane == 0) {
         atomicOr(p.flag, kFlagTimeout);
-        const long long un = u + stride;
-        if (un < p.total_units)
+        if (u + stride < p.total_units)
           (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
       }
-      __syncthreads();
+      __syncwarp();
       return;
     }
     const long long b = u / p.units_per_seq;
-    const UnitDesc d = p.units[u % p.units_per_seq];
+    const UnitDesc d = tbl[u % p.units_per_seq];
     if (d.bits == 8)
-      compute_unit<DK, DIAG, DELTA, 8>(p, stage, b, d);
+      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
     else if (d.bits == 4)
-      compute_unit<DK, DIAG, DELTA, 4>(p, stage, b, d);
+      compute_any<DK, DIAG, DELTA, SR, 4>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
     else
-      compute_unit<DK, DIAG, DELTA, 32>(p, stage, b, d);
-    __syncthreads();                                   // every thread is done with `stage`
-    if (threadIdx.x == 0) {
+      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
+    // compute_any ends with __syncwarp: every lane is done reading this slot
+    if (lane == 0) {
       const long long un = u + kStages * stride;
       if (un < p.total_units) {
         fence_proxy_async();
-        issue_unit<DK, DIAG>(p, un, stage, &bars[s]);
+        issue_unit<DK, DIAG>(p, tbl, un, stage, &bars[s]);
       }
     }
+    alpha_cur = alpha_nx;
+    beta_cur = beta_nx;
   }
 }
 
@@ -394,18 +465,23 @@ using StepFn = void (*)(const StepParams);
 using LoadFn = void (*)(const LoadParams);
 using DequantFn = void (*)(const LoadParams, float *);
 
-template <int DK>
+template <int DK, bool SR>
 static StepFn pick_step(bool diag, bool delta) {
-  if (diag) return delta ? decode_step_kernel<DK, true, true> : decode_step_kernel<DK, true, false>;
-  return delta ? decode_step_kernel<DK, false, true> : decode_step_kernel<DK, false, false>;
+  if (diag)
+    return delta ? decode_step_kernel<DK, true, true, SR> : decode_step_kernel<DK, true, false, SR>;
+  return delta ? decode_step_kernel<DK, false, true, SR> : decode_step_kernel<DK, false, false, SR>;
 }
-static StepFn step_kernel_for(int dk, bool diag, bool delta) {
+template <int DK>
+static StepFn pick_step(bool diag, bool delta, bool sr) {
+  return sr ? pick_step<DK, true>(diag, delta) : pick_step<DK, false>(diag, delta);
+}
+static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
   switch (dk) {
-    case 16: return pick_step<16>(diag, delta);
-    case 32: return pick_step<32>(diag, delta);
-    case 64: return pick_step<64>(diag, delta);
-    case 128: return pick_step<128>(diag, delta);
-    case 256: return pick_step<256>(diag, delta);
+    case 16: return pick_step<16>(diag, delta, sr);
+    case 32: return pick_step<32>(diag, delta, sr);
+    case 64: return pick_step<64>(diag, delta, sr);
+    case 128: return pick_step<128>(diag, delta, sr);
+    case 256: return pick_step<256>(diag, delta, sr);
   }
   return nullptr;
 }
@@ -588,26 +664,24 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   }
   h->seq_bytes = off;
 
-  // ---- work units: row blocks sized so one stage holds <= 16 KB of state ------------
-  const int LPR = dk / 16, rows_per_pass = kWarps * (32 / LPR);
-  auto rows_for = [&](int b) {
-    int R = 16384 / row_bytes(dk, b);
-    R = std::min(R, 1024 / h->ng);           // scales <= 4 KB per stage
-    R = std::min(R, 1024);                   // v slice <= 4 KB
-    if (R >= rows_per_pass) R -= R % rows_per_pass;
-    R -= R % 4;
-    return std::max(4, std::min(R, dv));
-  };
-  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta);
-  // occupancy is computed for the largest stage; split rows if one wave is not filled
-  int R8 = rows_for(8), R4 = rows_for(4), R32 = rows_for(32);
+  // ---- work units: row blocks of one tile, ~4 KB of state each, one warp per unit -----
+  // A unit's row count is a multiple of the warp pass (32/LPR rows) where the head's
+  // d_v allows; the last unit of a head takes the remainder.  Small batches split
+  // units further (down to one pass) until every warp of one wave has work.
+  const int LPR = dk / 16, rpw = 32 / LPR;
+  auto rows_for = [&](int b) { return std::min(full_rows(dk, b), dv); };
+  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  const int R8 = rows_for(8), R4 = rows_for(4), R32 = rows_for(32);
   int split = 1;
   auto build_units = [&](std::vector<UnitDesc> &u) {
     u.clear();
     for (int hh = 0; hh < c.heads; ++hh) {
       const int b = bits[hh];
       int R = b == 8 ? R8 : (b == 4 ? R4 : R32);
-      R = std::max(4, (R / split) - ((R / split) % 4));
+      int Rs = R / split;
+      Rs -= Rs % std::min(rpw, R);
+      Rs -= Rs % 4;
+      R = std::max(Rs, std::min(4, R));
       for (int r0 = 0; r0 < dv; r0 += R) {
         UnitDesc d{};
         d.head = hh;
@@ -619,24 +693,26 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       }
     }
   };
-  auto stage_bytes_for = [&](const std::vector<UnitDesc> &u, int *sc, int *sv) {
-    int cmax = 0, smax = 0, vmax = 0;
-    for (const UnitDesc &d : u) {
-      cmax = std::max(cmax, d.nrows * row_bytes(dk, d.bits));
-      if (d.bits != 32) smax = std::max(smax, d.nrows * h->ng * 4);
-      vmax = std::max(vmax, d.nrows * 4);
-    }
-    *sc = cmax;
-    *sv = smax;
-    return cmax + smax + vmax + 2 * dk * 4 + (c.decay_diag ? dk * 4 : 0);
-  };
   std::vector<UnitDesc> units;
   int ctas_per_sm = 1;
   for (;;) {
     build_units(units);
-    int cbytes, sbytes;
-    const int stage = stage_bytes_for(units, &cbytes, &sbytes);
-    const int smem = 128 + kStages * stage;
+    int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
+    for (const UnitDesc &d : units) {
+      cmax = std::max(cmax, d.nrows * row_bytes(dk, d.bits));
+      if (d.bits != 32) smax = std::max(smax, d.nrows * h->ng * 4);
+      vmax = std::max(vmax, d.nrows * 4);
+      maxrows = std::max(maxrows, d.nrows);
+    }
+    auto up16 = [](int x) { return (x + 15) & ~15; };
+    const int stage = up16(cmax) + up16(smax) + up16(vmax) + 2 * dk * 4 +
+                      (c.decay_diag ? dk * 4 : 0);
+    const int opart_floats = ((maxrows * LPR + 31) / 32) * 32;     // 128-byte multiples
+    const int ow_floats = ((maxrows + 31) / 32) * 32;
+    const int warp_bytes = ((64 + 4 * (opart_floats + ow_floats) + kStages * stage + 127) / 128) * 128;
+    const int table = (int)units.size() * (int)sizeof(UnitDesc) <= 16384
+                          ? (((int)units.size() * (int)sizeof(UnitDesc) + 127) / 128) * 128 : 0;
+    const int smem = table + kWarps * warp_bytes;
     // the attribute is per kernel and shared by all handles: only ever raise it
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
@@ -653,18 +729,21 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       return LORES_ERR_CUDA;
     }
     const long long total = (long long)c.batch * (long long)units.size();
-    const long long slots = (long long)ctas_per_sm * prop.multiProcessorCount;
-    int maxR = 0;
-    for (const UnitDesc &d : units) maxR = std::max(maxR, d.nrows);
-    if (total >= slots || maxR <= rows_per_pass || maxR <= 4 || split >= 64) {
+    const long long warp_slots = (long long)ctas_per_sm * prop.multiProcessorCount * kWarps;
+    if (total >= warp_slots || maxrows <= rpw || maxrows <= 4 || split >= 64) {
       h->smem = smem;
-      h->sp.st_scales = cbytes;
-      h->sp.st_k = cbytes + sbytes;
+      h->sp.table_bytes = table;
+      h->sp.warp_bytes = warp_bytes;
+      h->sp.opart_floats = opart_floats;
+      h->sp.ow_floats = ow_floats;
+      h->sp.st_scales = up16(cmax);
+      h->sp.st_v = h->sp.st_scales + up16(smax);
+      h->sp.st_k = h->sp.st_v + up16(vmax);
       h->sp.st_q = h->sp.st_k + dk * 4;
       h->sp.st_a = h->sp.st_q + dk * 4;
-      h->sp.st_v = h->sp.st_a + (c.decay_diag ? dk * 4 : 0);
       h->sp.stage_bytes = stage;
-      h->grid = (int)std::min<long long>(total, slots);
+      const long long ctas = (total + kWarps - 1) / kWarps;
+      h->grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * prop.multiProcessorCount);
       break;
     }
     split *= 2;
@@ -710,7 +789,6 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   p.ng = h->ng;
   p.G = G;
   p.units_per_seq = h->units_per_seq;
-  p.stochastic = c.stochastic;
   *out = h;
   return LORES_OK;
 }

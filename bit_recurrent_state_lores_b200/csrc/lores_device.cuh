@@ -3,11 +3,12 @@
 // Arithmetic of one state row, shared by the decode kernel and the state loader.
 // The element order and every fp32 rounding follow the state format definition:
 //   entry of S_{t-1} diag(alpha):   c_ij * (s_ig * alpha_j)
-//   u_i = (S'k)_i:                  16-column fma chains, then pairwise combine with the
-//                                   partner lane at distance C/2, ..., 1
+//   u_i = (S'k)_i:                  4-column fma chains, combined pairwise with the nearest
+//                                   partner first (distance 1, 2, 4, ... in chunks)
 //   w_i = beta (v_i - u_i)  [delta] or beta v_i;   x_ij = fma(w_i, k_j, S'_ij)
-//   requantize per group:           m = max|x|, inv = r / m, s = m / r (round to nearest),
-//                                   t = fma(x, inv, 49152 + d/256), code = floor(t - 49152)
+//   requantize per group:           m = max|x|; y = Newton reciprocal of m; inv = r * y;
+//                                   s = m * fl(1/r); t = fma(x, inv, 49152 + d/256);
+//                                   code = floor(t - 49152)
 // ("Quantizing Recurrent Language Models Is Easier Than You Think": General recurrence
 // form; Key properties item 3; Proposition 1; Proposition 3.)
 #pragma once
@@ -161,36 +162,77 @@ __device__ __forceinline__ uint2 pack_i4(const uint32_t (&t)[16]) {
 }
 
 // -------------------------------------------------------------------------------------
+// reductions over the lane's 16 entries
+// -------------------------------------------------------------------------------------
+// sum_e a_e b_e over the lane's 16 columns in the fixed order: four 4-column fma chains,
+// then (c0 + c1) + (c2 + c3).  Chunk c of the lane is columns 4c .. 4c+3.
+__device__ __forceinline__ float dot16_c4(const float (&a)[16], const float (&b)[16]) {
+  float p[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float acc = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc = __fmaf_rn(a[4 * c + e], b[4 * c + e], acc);
+    p[c] = acc;
+  }
+  return __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
+}
+
+// Newton-Raphson reciprocal of m in [2^-100, 2^100]: seed by reflecting the exponent
+// field (bits 0x7F000000 - bits(m), exact for powers of two, within 12.5% otherwise),
+// then three steps y <- y + y (1 - m y); relative error < 2^-21.
+__device__ __forceinline__ float recip_nr(float m) {
+  float y = __uint_as_float(0x7F000000u - __float_as_uint(m));
+#pragma unroll
+  for (int it = 0; it < 3; ++it) {
+    const float e = __fmaf_rn(-m, y, 1.0f);
+    y = __fmaf_rn(y, e, y);
+  }
+  return y;
+}
+
+// -------------------------------------------------------------------------------------
 // requantize one lane's 16 entries of a value row
 // -------------------------------------------------------------------------------------
 // LPR lanes hold one row (16 consecutive columns each); LPG = G/16 lanes share a group.
-// Returns the row's "non-finite" verdict (same on all lanes of the row).  Writes the
-// lane's packed codes into `words` (int8: 4 words, int4: 2 words) and the lane's group
-// scale into `s_out`.  `bits` (8 or 4) may differ between rows of one warp; every lane
-// of the warp must call this function together (it shuffles across the warp).
+// Returns the row's "non-finite" verdict (same on all lanes of the row): a row with an
+// entry that is inf, NaN or above 2^100 is stored as zero.  Writes the lane's packed
+// codes into `words` (int8: 4 words, int4: 2 words) and the lane's group scale into
+// `s_out`.  `bits` (8 or 4) may differ between rows of one warp; every lane of the warp
+// must call this function together (it shuffles and votes across the warp).
 template <int LPR>
 __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
                                              uint32_t tkey, uint32_t n0, int stochastic,
                                              uint32_t (&words)[4], float &s_out) {
   const float r = (bits == 8) ? 127.0f : 7.0f;
-  float m = 0.0f;
+  const float inv_r = (bits == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
+  float mq[4];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
-  for (int st = 1; st < lpg; st <<= 1) m = max_nan(m, __shfl_xor_sync(kFull, m, st));
-  const bool gbad = !(m <= 3.402823466e38f);            // inf or NaN in the group
-  const unsigned bal = __ballot_sync(kFull, gbad);
-  const int riw = (lane % 32) / LPR;
-  const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
-  const bool row_bad = (bal & rowmask) != 0u;
-
-  float inv = 0.0f, s = 0.0f;
-  if (!row_bad && m > 0.0f) {
-    inv = __fdiv_rn(r, m);
-    if (inv <= 3.402823466e38f)
-      s = __fdiv_rn(m, r);
-    else
-      inv = 0.0f;                                        // m too small to scale: zero group
+  for (int c = 0; c < 4; ++c)
+    mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[4 * c]), x[4 * c + 1]), x[4 * c + 2]),
+                        x[4 * c + 3]);
+  float m = max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
+  // group max over the lpg lanes of the group: the levels are fixed at compile time
+  // (log2 LPR); levels at or beyond the group width keep the lane's own value.
+#pragma unroll
+  for (int st = 1; st < LPR; st <<= 1) {
+    const float mo = __shfl_xor_sync(kFull, m, st);
+    m = (st < lpg) ? max_nan(m, mo) : m;
   }
+  const bool gbad = !(m <= 0x1p100f);                    // inf, NaN or overflow
+  const bool any_bad = __any_sync(kFull, gbad);
+  bool row_bad = false;
+  if (any_bad) {
+    const unsigned bal = __ballot_sync(kFull, gbad);
+    const int riw = lane / LPR;
+    const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
+    row_bad = (bal & rowmask) != 0u;
+  }
+  const bool scaled = m >= 0x1p-100f && !gbad;           // below 2^-100: zero group
+  const float y = recip_nr(scaled ? m : 1.0f);
+  const float inv = scaled ? __fmul_rn(r, y) : 0.0f;
+  float s = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+
   uint32_t t[16];
   if (stochastic) {
     uint32_t h[4];
@@ -212,7 +254,7 @@ __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int
     const uint2 w = pack_i4(t);
     words[0] = w.x; words[1] = w.y; words[2] = 0u; words[3] = 0u;
   }
-  if (row_bad) {
+  if (any_bad && row_bad) {
     words[0] = words[1] = words[2] = words[3] = 0u;
     s = 0.0f;
   }
