@@ -21,6 +21,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -943,3 +944,176 @@ lores_status lores_check_errors(lores_handle *h, void *stream) {
 }
 
 }  // extern "C"
+
+// -------------------------------------------------------------------------------------
+// Decode step without any allocation
+// -------------------------------------------------------------------------------------
+// Some callers cannot let a library allocate device memory: a serving engine that
+// plans every buffer from its own pool up front (a cudaMalloc there can stall the
+// device and fragment the pool), or an application held to a fixed device-memory
+// budget.  For them, lores_decode_step_noalloc runs the same decode kernel on state
+// buffers the caller owns, and keeps the kernel's own bookkeeping (the work-unit table
+// and the error word) in the fixed array below instead of in allocated memory.  The
+// array is part of the module image: every GPU that loads this library holds it until
+// the process exits.
+namespace {
+
+constexpr int kNoAllocMaxUnits = 2048;                 // work units of one sequence, at most
+constexpr size_t kNoAllocTableBytes = kNoAllocMaxUnits * sizeof(UnitDesc);
+constexpr size_t kNoAllocScratchBytes = kNoAllocTableBytes + 256;   // table, then error word
+constexpr int kNoAllocMaxDevices = 64;
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_scratch_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on `device` (the current device).  In host code the
+// array's name only stands in for the symbol, so the address is looked up once per device.
+lores_status noalloc_scratch(int device, unsigned char **out) {
+  if (device >= kNoAllocMaxDevices) return LORES_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_scratch_ptr[device]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      (void)cudaGetLastError();
+      return LORES_ERR_CUDA;
+    }
+    g_noalloc_scratch_ptr[device] = ptr;
+  }
+  *out = static_cast<unsigned char *>(g_noalloc_scratch_ptr[device]);
+  return LORES_OK;
+}
+
+}  // namespace
+
+extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void *codes,
+                                                  float *scales, const float *q, const float *k,
+                                                  const float *v, const float *alpha,
+                                                  const float *beta, float *o, uint64_t step,
+                                                  uint32_t *flags_out, void *stream) {
+  if (!cfg || !codes || !scales || !q || !k || !v || !alpha || !beta || !o)
+    return LORES_ERR_INVALID_ARG;
+  const lores_config c = *cfg;
+  const int dk = c.d_k, dv = c.d_v;
+  if (c.batch < 1 || c.heads < 1 || c.heads > 65536) return LORES_ERR_INVALID_ARG;
+  if (!(dk == 16 || dk == 32 || dk == 64 || dk == 128 || dk == 256)) return LORES_ERR_INVALID_ARG;
+  if (dv < 4 || dv > 4096 || dv % 4) return LORES_ERR_INVALID_ARG;
+  const int G = c.group_size == 0 ? dk : c.group_size;
+  if (G < 16 || G % 16 || dk % G) return LORES_ERR_INVALID_ARG;
+  if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
+      (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
+    return LORES_ERR_INVALID_ARG;
+  for (int hh = 0; c.head_bits && hh < c.heads; ++hh)
+    if (c.head_bits[hh] != 8 && c.head_bits[hh] != 4 && c.head_bits[hh] != 32)
+      return LORES_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (c.decay_diag ? !aligned16(alpha) : (reinterpret_cast<uintptr_t>(alpha) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(o) & 3u))
+    return LORES_ERR_INVALID_ARG;
+
+  // Work units of one sequence, planned on the stack: full units of ~4 KB of state, the
+  // last unit of each head takes the remainder (the same plan as a handle at full batch).
+  UnitDesc units[kNoAllocMaxUnits];
+  int nunits = 0;
+  long long seq_bytes = 0;
+  int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
+  const int ng = dk / G, LPR = dk / 16;
+  for (int hh = 0; hh < c.heads; ++hh) {
+    const int b = c.head_bits ? c.head_bits[hh] : 8;
+    const int R = std::min(full_rows(dk, b), dv);
+    for (int r0 = 0; r0 < dv; r0 += R) {
+      if (nunits == kNoAllocMaxUnits) return LORES_ERR_UNSUPPORTED;   // beyond the fixed table
+      UnitDesc &d = units[nunits++];
+      d = UnitDesc{};
+      d.head = hh;
+      d.row0 = r0;
+      d.nrows = std::min(R, dv - r0);
+      d.bits = b;
+      d.code_off = seq_bytes + (long long)r0 * row_bytes(dk, b);
+      cmax = std::max(cmax, d.nrows * row_bytes(dk, b));
+      if (b != 32) smax = std::max(smax, d.nrows * ng * 4);
+      vmax = std::max(vmax, d.nrows * 4);
+      maxrows = std::max(maxrows, d.nrows);
+    }
+    seq_bytes += (long long)dv * row_bytes(dk, b);
+  }
+
+  DeviceGuard guard(c.device);
+  if (!guard.ok) {
+    (void)cudaGetLastError();
+    return LORES_ERR_CUDA;
+  }
+  unsigned char *scratch = nullptr;
+  lores_status st = noalloc_scratch(c.device, &scratch);
+  if (st != LORES_OK) return st;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c.device) != cudaSuccess)
+    return LORES_ERR_CUDA;
+
+  auto up16 = [](int x) { return (x + 15) & ~15; };
+  StepParams p{};
+  const int stage = up16(cmax) + up16(smax) + up16(vmax) + 2 * dk * 4 + (c.decay_diag ? dk * 4 : 0);
+  p.opart_floats = ((maxrows * LPR + 31) / 32) * 32;
+  p.ow_floats = ((maxrows + 31) / 32) * 32;
+  p.warp_bytes = ((64 + 4 * (p.opart_floats + p.ow_floats) + kStages * stage + 127) / 128) * 128;
+  p.table_bytes = nunits * (int)sizeof(UnitDesc) <= 16384
+                      ? ((nunits * (int)sizeof(UnitDesc) + 127) / 128) * 128 : 0;
+  p.st_scales = up16(cmax);
+  p.st_v = p.st_scales + up16(smax);
+  p.st_k = p.st_v + up16(vmax);
+  p.st_q = p.st_k + dk * 4;
+  p.st_a = p.st_q + dk * 4;
+  p.stage_bytes = stage;
+  const int smem = p.table_bytes + kWarps * p.warp_bytes;
+  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+      (fa.maxDynamicSharedSizeBytes < smem &&
+       cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess))
+    return LORES_ERR_CUDA;
+  int ctas_per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, fn, kThreads, smem) !=
+          cudaSuccess ||
+      ctas_per_sm < 1)
+    return LORES_ERR_CUDA;
+
+  p.codes = static_cast<uint8_t *>(codes);
+  p.scales = scales;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.units = reinterpret_cast<const UnitDesc *>(scratch);
+  p.flag = reinterpret_cast<unsigned *>(scratch + kNoAllocTableBytes);
+  p.seq_bytes = seq_bytes;
+  p.total_units = (long long)c.batch * nunits;
+  p.H = c.heads;
+  p.d_v = dv;
+  p.ng = ng;
+  p.G = G;
+  p.units_per_seq = nunits;
+  p.step_key = step_key_of(c.seed, step);
+  const long long ctas = (p.total_units + kWarps - 1) / kWarps;
+  const int grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * sms);
+
+  // The scratch keeps whatever the previous call left: the table is rewritten and the
+  // error word cleared on this stream before the launch.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(scratch, units, nunits * sizeof(UnitDesc),
+                                  cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(scratch + kNoAllocTableBytes, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  fn<<<grid, kThreads, smem, s>>>(p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && flags_out)
+    e = cudaMemcpyAsync(flags_out, scratch + kNoAllocTableBytes, sizeof(uint32_t),
+                        cudaMemcpyDefault, s);
+  return cuda_status(e);
+}

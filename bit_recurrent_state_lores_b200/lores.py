@@ -51,6 +51,8 @@ def _load():
         "lores_destroy": (I32, [P]),
         "lores_decode_step": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_host": (I32, [P, P, P, P, P, P, P, U64, P]),
+        "lores_decode_step_noalloc": (I32, [C.POINTER(lores_config), P, P, P, P, P, P, P, P, U64,
+                                            P, P]),
         "lores_dequant_state": (I32, [P, P, P]),
         "lores_load_state": (I32, [P, P, U64, P]),
         "lores_export_codes": (I32, [P, P, P, P]),
@@ -127,6 +129,30 @@ def lores_decode_step_host(h, q, k, v, alpha, beta, o, step, stream=None):
     _check(_lib.lores_decode_step_host(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                        _ptr(o), step & (2**64 - 1), _stream(stream)),
            "lores_decode_step_host")
+
+
+def lores_decode_step_noalloc(cfg, codes, scales, q, k, v, alpha, beta, o, step,
+                              flags_out=None, stream=None):
+    """The decode step on caller-owned state buffers, allocating nothing (see
+    include/lores.h).  `cfg` is a lores_config (make_config builds one)."""
+    _check(_lib.lores_decode_step_noalloc(C.byref(cfg), _ptr(codes), _ptr(scales), _ptr(q),
+                                          _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
+                                          step & (2**64 - 1), _ptr(flags_out), _stream(stream)),
+           "lores_decode_step_noalloc")
+
+
+def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
+                stochastic=1, seed=0, device=0):
+    """A lores_config; the head_bits array is kept alive on the returned object."""
+    hb = None
+    arr = None
+    if head_bits is not None:
+        arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
+        hb = C.cast(arr, C.POINTER(C.c_int32))
+    cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
+                       seed & (2**64 - 1), device)
+    cfg._head_bits_keepalive = arr
+    return cfg
 
 
 def lores_dequant_state(h, out, stream=None):

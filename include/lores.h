@@ -117,6 +117,43 @@ lores_status lores_decode_step_host(lores_handle *h, const float *q, const float
                                     const float *v, const float *alpha, const float *beta,
                                     float *o, uint64_t step, void *stream);
 
+/* The decode step for callers that must not let this library allocate device memory:
+ * for example a serving engine that hands out every buffer from its own pre-planned
+ * pool (a cudaMalloc inside a step can stall the device and fragment that pool), or an
+ * application held to a fixed device-memory budget.  The paper has no counterpart to
+ * this call; it only changes who owns the memory.
+ *
+ * There is no handle: cfg describes the layer (as for lores_create), and the caller
+ * owns the state as two device buffers, updated in place:
+ *   codes   the code pool in the handle's export layout: per sequence, the heads'
+ *           tiles back to back in head order (int8 tile d_v*d_k bytes, int4 d_v*d_k/2,
+ *           fp32 4*d_v*d_k), 16-byte aligned; all zero for a zero state
+ *   scales  [B, H, d_v, d_k/G] fp32, 16-byte aligned
+ * q, k, v, alpha, beta, o, step as for lores_decode_step.  flags_out (may be NULL):
+ * host or device address that receives this call's error bits (1 = a row became
+ * non-finite, 2 = the kernel gave up a wait) when the stream reaches the copy.
+ * Results are the same as lores_decode_step's on a handle whose state equals these
+ * buffers.
+ *
+ * The call allocates nothing: it never calls cudaMalloc, cudaFree or any allocating
+ * library routine.  The kernel's bookkeeping (its work-unit table and error word) lives
+ * in one fixed array of 64 KB + 256 B compiled into the library, which every GPU that
+ * loads the library holds until the process exits.  That fixes a limit: one sequence
+ * may span at most 2048 work units (a unit is up to 4 KB of one head's state, so e.g.
+ * 32 heads of 128 x 128 int8 use 128); beyond it the call returns
+ * LORES_ERR_UNSUPPORTED before launching anything.  The array is shared by every call
+ * and keeps the last call's contents; each call rewrites the table and clears the
+ * error word on its own stream, so calls that overlap on the GPU (different streams,
+ * no ordering between them) race on it.  The first call on each device looks up the
+ * array's device address; make that first call before any stream capture.
+ * Asynchronous on `stream` (the table upload from host memory may wait for the
+ * stream's earlier work).  Errors: INVALID_ARG (shapes, NULL or misaligned pointers),
+ * UNSUPPORTED (too many units, device ordinal >= 64), CUDA. */
+lores_status lores_decode_step_noalloc(const lores_config *cfg, void *codes, float *scales,
+                                       const float *q, const float *k, const float *v,
+                                       const float *alpha, const float *beta, float *o,
+                                       uint64_t step, uint32_t *flags_out, void *stream);
+
 /* Write the dequantized state, out[B, H, d_v, d_k] = code * scale (fp32 heads:
  * the state itself), to device memory `out`.  Asynchronous. */
 lores_status lores_dequant_state(lores_handle *h, float *out, void *stream);
