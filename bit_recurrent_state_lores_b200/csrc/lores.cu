@@ -150,6 +150,12 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
   constexpr int kFullPasses = full_rows(DK, BITS) / RPW;
   const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
+  // dither counter of the lane's first quad in pass 0: n0 = (row0 + riw) d_k/4 + 4 lir;
+  // each pass moves RPW rows, i.e. RPW d_k/4 quads
+  const uint32_t cbase0 =
+      tkey + 0x9E3779B9u * ((uint32_t)(d.row0 + riw) * (uint32_t)(DK / 4) + (uint32_t)lir * 4u + 1u);
+  constexpr uint32_t kCtrPerPass = 0x9E3779B9u * (uint32_t)(RPW * DK / 4);
+  uint32_t badmask = 0;                        // bit n: this lane's group was bad in pass n
 
 #pragma unroll(FULL ? 4 : 1)
   for (int n = 0; n < npass; ++n) {
@@ -203,25 +209,23 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
       if (lir == 0) ow[lr] = w;
     }
 
-    // ---- requantize and store --------------------------------------------------------
+    // ---- requantize and store (bad rows are fixed up after the passes) ------------------
+    bool gbad;
     if (BITS == 32) {
       float m = 0.0f;
 #pragma unroll
       for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
-      const bool lbad = !(m <= 3.402823466e38f);
+      gbad = !(m <= 3.402823466e38f);
       if (active) {
         float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           __stcs(dst + c, make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
       }
-      if (__any_sync(kFull, lbad) && lbad && active) atomicOr(p.flag, kFlagNonFinite);
     } else {
       uint32_t words[4];
       float s_new;
-      const uint32_t n0 = (uint32_t)(d.row0 + lrr) * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
-      const bool row_bad =
-          requantize16<LPR>(x, BITS, lpg, lane, tkey, n0, SR ? 1 : 0, words, s_new);
+      gbad = requantize16_nb<LPR, BITS, SR>(x, lpg, cbase0 + kCtrPerPass * (uint32_t)n, words, s_new);
       if (active) {
         if (BITS == 8)
           __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
@@ -231,7 +235,27 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
                  make_uint2(words[0], words[1]));
         if (scale_writer) gscales[lr * ng + g] = s_new;
       }
-      if (row_bad && active && lir == 0) atomicOr(p.flag, kFlagNonFinite);
+    }
+    badmask |= (gbad && active ? 1u : 0u) << n;
+  }
+
+  // ---- rare: rows with a non-finite (or overflowing) entry -----------------------------
+  // A row is bad if any of its groups is; quantized rows are stored as zero.  The lane
+  // that wrote a word rewrites it, so no ordering between lanes is needed.
+  if (__any_sync(kFull, badmask != 0u)) {
+    const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
+    for (int n = 0; n < npass; ++n) {
+      const unsigned bal = __ballot_sync(kFull, (badmask >> n) & 1u);
+      const int lr = n * RPW + riw;
+      if ((bal & rowmask) == 0u || !(FULL || lr < d.nrows)) continue;
+      if (BITS != 32) {
+        if (BITS == 8)
+          __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16), make_uint4(0, 0, 0, 0));
+        else
+          __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8), make_uint2(0, 0));
+        if (scale_writer) gscales[lr * ng + g] = 0.0f;
+      }
+      if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
     }
   }
 

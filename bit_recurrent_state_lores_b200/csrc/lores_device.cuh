@@ -200,6 +200,56 @@ __device__ __forceinline__ float recip_nr(float m) {
 // codes into `words` (int8: 4 words, int4: 2 words) and the lane's group scale into
 // `s_out`.  `bits` (8 or 4) may differ between rows of one warp; every lane of the warp
 // must call this function together (it shuffles and votes across the warp).
+// Requantize one lane's 16 entries without any branch or vote: returns this lane's
+// group verdict (true: an entry of the group is inf, NaN or above 2^100).  A row with
+// a bad group must then be zeroed by the caller (see zero_bad_rows); its codes and
+// scale written here are not meaningful.  cbase = tile key + golden * (n0 + 1) where
+// n0 is the quad index of the lane's first column (see the dither definition).
+template <int LPR, int BITS, bool SR>
+__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int lpg, uint32_t cbase,
+                                                uint32_t (&words)[4], float &s_out) {
+  constexpr float r = (BITS == 8) ? 127.0f : 7.0f;
+  constexpr float inv_r = (BITS == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
+  float mq[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[4 * c]), x[4 * c + 1]), x[4 * c + 2]),
+                        x[4 * c + 3]);
+  float m = max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
+#pragma unroll
+  for (int st = 1; st < LPR; st <<= 1) {
+    const float mo = __shfl_xor_sync(kFull, m, st);
+    m = (st < lpg) ? max_nan(m, mo) : m;
+  }
+  const bool gbad = !(m <= 0x1p100f);                    // inf, NaN or overflow
+  const bool scaled = m >= 0x1p-100f && !gbad;           // below 2^-100: zero group
+  const float y = recip_nr(scaled ? m : 1.0f);
+  const float inv = scaled ? __fmul_rn(r, y) : 0.0f;
+  s_out = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+  uint32_t t[16];
+  if (SR) {
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float g = __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)));
+      t[e] = __float_as_uint(__fmaf_rn(x[e], inv, g));
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, 49152.5f));
+  }
+  if (BITS == 8) {
+    const uint4 w = pack_i8(t);
+    words[0] = w.x; words[1] = w.y; words[2] = w.z; words[3] = w.w;
+  } else {
+    const uint2 w = pack_i4(t);
+    words[0] = w.x; words[1] = w.y; words[2] = 0u; words[3] = 0u;
+  }
+  return gbad;
+}
+
 template <int LPR>
 __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
                                              uint32_t tkey, uint32_t n0, int stochastic,
