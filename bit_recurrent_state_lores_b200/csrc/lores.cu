@@ -49,7 +49,7 @@ struct StepParams {
   const UnitDesc *units; // [units_per_seq]
   long long seq_bytes;
   long long total_units;
-  int H, d_v, ng, G, units_per_seq;
+  int B, H, d_v, ng, G, units_per_seq;
   uint32_t step_key;
   // shared memory layout: [unit table][warp 0 area][warp 1 area]...; a warp area is
   // [2 mbarriers | pad to 64][readout partials][row w][stage 0][stage 1]
@@ -74,18 +74,17 @@ __host__ __device__ constexpr int full_rows(int dk, int bits) {
 // producer (one lane of the warp): stage one unit's inputs into the warp's ring slot
 // -------------------------------------------------------------------------------------
 template <int DK, bool DIAG>
-__device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *tbl, long long u,
+__device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *tbl, int b, int ub,
                                            uint8_t *stage, uint64_t *bar) {
-  const long long b = u / p.units_per_seq;
-  const UnitDesc d = tbl[u % p.units_per_seq];
-  const long long tile = b * p.H + d.head;
+  const UnitDesc d = tbl[ub];
+  const long long tile = (long long)b * p.H + d.head;
   const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
   const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
   const unsigned vbytes = (unsigned)(d.nrows * 4);
   const unsigned vec = DK * 4;
   const unsigned total = cbytes + sbytes + vbytes + 2 * vec + (DIAG ? vec : 0);
   mbar_expect_tx(bar, total);
-  bulk_g2s(stage, p.codes + b * p.seq_bytes + d.code_off, cbytes, bar);
+  bulk_g2s(stage, p.codes + (long long)b * p.seq_bytes + d.code_off, cbytes, bar);
   if (sbytes)
     bulk_g2s(stage + p.st_scales, p.scales + (tile * p.d_v + d.row0) * p.ng, sbytes, bar);
   bulk_g2s(stage + p.st_k, p.k + tile * DK, vec, bar);
@@ -103,7 +102,7 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
 // of the row leaves w in ow, and after the rows each lane forms o for one row as
 // sum(opart) + w (k.q).
 template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL>
-__device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, long long b,
+__device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow) {
   constexpr int LPR = DK / 16;            // lanes per row
@@ -116,7 +115,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   const int g = lir / lpg;                                 // this lane's group in the row
   const bool scale_writer = (lir & (lpg - 1)) == 0;
   const int ng = p.ng;
-  const long long tile = b * p.H + d.head;
+  const long long tile = (long long)b * p.H + d.head;
 
   const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
   const float *sq = reinterpret_cast<const float *>(stage + p.st_q);
@@ -146,7 +145,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   const float kq = (float)kqd;
   const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
 
-  uint8_t *gcodes = p.codes + b * p.seq_bytes + d.code_off;
+  uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
   float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
   constexpr int kFullPasses = full_rows(DK, BITS) / RPW;
   const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
@@ -272,7 +271,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
 }
 
 template <int DK, bool DIAG, bool DELTA, bool SR, int BITS>
-__device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *stage, long long b,
+__device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *stage, int b,
                                             const UnitDesc &d, float alpha_s, float beta,
                                             float *opart, float *ow) {
   if (d.nrows == full_rows(DK, BITS))
@@ -280,6 +279,20 @@ __device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *
   else
     compute_unit<DK, DIAG, DELTA, SR, BITS, false>(p, stage, b, d, alpha_s, beta, opart, ow);
 }
+
+// Position of a unit in (sequence b, unit index ub within the sequence), advanced by a
+// fixed stride without divisions.
+struct UnitPos {
+  int b, ub;
+  __device__ __forceinline__ void advance(int sb, int su, int ups) {
+    ub += su;
+    b += sb;
+    if (ub >= ups) {
+      ub -= ups;
+      ++b;
+    }
+  }
+};
 
 // Persistent kernel: every warp runs its own pipeline over units gw, gw + W, gw + 2W, ...
 // (gw = global warp index, W = warps in the grid), with a 2-slot ring of bulk copies
@@ -296,44 +309,48 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
   uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
 
   const UnitDesc *tbl = p.units;
+  const int ups = p.units_per_seq;
   if (p.table_bytes) {
-    for (int i = threadIdx.x; i < p.units_per_seq; i += kThreads) stbl[i] = p.units[i];
+    for (int i = threadIdx.x; i < ups; i += kThreads) stbl[i] = p.units[i];
     tbl = stbl;
   }
   __syncthreads();                                  // the only CTA-wide barrier
 
   const long long first = (long long)blockIdx.x * kWarps + warp;
-  const long long stride = (long long)gridDim.x * kWarps;
   if (first >= p.total_units) return;
+  const long long stride = (long long)gridDim.x * kWarps;
+  const int sb = (int)(stride / ups), su = (int)(stride % ups);
+  UnitPos cur{(int)(first / ups), (int)(first % ups)};
 
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    for (int s = 0; s < kStages; ++s) {
-      const long long u = first + s * stride;
-      if (u < p.total_units) issue_unit<DK, DIAG>(p, tbl, u, stages + s * p.stage_bytes, &bars[s]);
+    UnitPos q = cur;
+    for (int s = 0; s < kStages && q.b < p.B; ++s) {
+      issue_unit<DK, DIAG>(p, tbl, q.b, q.ub, stages + s * p.stage_bytes, &bars[s]);
+      q.advance(sb, su, ups);
     }
   }
   __syncwarp();
+  UnitPos nxt = cur;                                // the unit after `cur`
+  nxt.advance(sb, su, ups);
+  UnitPos fill = nxt;                               // the unit that refills the slot just used
+  fill.advance(sb, su, ups);
 
   // per-tile scalars of the current unit; the next unit's are loaded one unit ahead
-  auto tile_of = [&](long long u) {
-    return (u / p.units_per_seq) * p.H + tbl[u % p.units_per_seq].head;
-  };
   float alpha_cur = 0.0f, beta_cur;
   {
-    const long long t0 = tile_of(first);
+    const long long t0 = (long long)cur.b * p.H + tbl[cur.ub].head;
     beta_cur = __ldg(p.beta + t0);
     if (!DIAG) alpha_cur = __ldg(p.alpha + t0);
   }
 
-  int n = 0;
-  for (long long u = first; u < p.total_units; u += stride, ++n) {
+  for (int n = 0; cur.b < p.B; ++n) {
     const int s = n % kStages;
     uint8_t *stage = stages + s * p.stage_bytes;
     float alpha_nx = 0.0f, beta_nx = 0.0f;
-    if (u + stride < p.total_units) {
-      const long long tn = tile_of(u + stride);
+    if (nxt.b < p.B) {
+      const long long tn = (long long)nxt.b * p.H + tbl[nxt.ub].head;
       beta_nx = __ldg(p.beta + tn);
       if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
     }
@@ -342,28 +359,27 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       // Give up: record it, let the other slot's copy (if any) land, and leave.
       if (lane == 0) {
         atomicOr(p.flag, kFlagTimeout);
-        if (u + stride < p.total_units)
+        if (nxt.b < p.B)
           (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
       }
       __syncwarp();
       return;
     }
-    const long long b = u / p.units_per_seq;
-    const UnitDesc d = tbl[u % p.units_per_seq];
+    const UnitDesc d = tbl[cur.ub];
     if (d.bits == 8)
-      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
+      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     else if (d.bits == 4)
-      compute_any<DK, DIAG, DELTA, SR, 4>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
+      compute_any<DK, DIAG, DELTA, SR, 4>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     else
-      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, b, d, alpha_cur, beta_cur, opart, ow);
+      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     // compute_any ends with __syncwarp: every lane is done reading this slot
-    if (lane == 0) {
-      const long long un = u + kStages * stride;
-      if (un < p.total_units) {
-        fence_proxy_async();
-        issue_unit<DK, DIAG>(p, tbl, un, stage, &bars[s]);
-      }
+    if (lane == 0 && fill.b < p.B) {
+      fence_proxy_async();
+      issue_unit<DK, DIAG>(p, tbl, fill.b, fill.ub, stage, &bars[s]);
     }
+    cur = nxt;
+    nxt.advance(sb, su, ups);
+    fill.advance(sb, su, ups);
     alpha_cur = alpha_nx;
     beta_cur = beta_nx;
   }
@@ -809,6 +825,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   p.units = h->units;
   p.seq_bytes = h->seq_bytes;
   p.total_units = (long long)c.batch * h->units_per_seq;
+  p.B = c.batch;
   p.H = c.heads;
   p.d_v = dv;
   p.ng = h->ng;
@@ -1118,6 +1135,7 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   p.flag = reinterpret_cast<unsigned *>(scratch + kNoAllocTableBytes);
   p.seq_bytes = seq_bytes;
   p.total_units = (long long)c.batch * nunits;
+  p.B = c.batch;
   p.H = c.heads;
   p.d_v = dv;
   p.ng = ng;
