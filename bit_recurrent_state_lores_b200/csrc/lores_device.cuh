@@ -13,6 +13,7 @@
 // form; Key properties item 3; Proposition 1; Proposition 3.)
 #pragma once
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace lores {
@@ -109,15 +110,24 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned by
 // -------------------------------------------------------------------------------------
 // code <-> float
 // -------------------------------------------------------------------------------------
-// 16 int8 codes (two's complement) -> exact floats: bias to offset binary, drop each
-// byte into the mantissa of 2^23, subtract 2^23 + 128.
+// 16 int8 codes (two's complement) -> exact floats.  Bias to offset binary, drop pairs
+// of bytes into the mantissas of an fp16 pair (1024 + b: fp16 spacing is 1 there),
+// subtract 1024 + 128 from both halves (exact), widen each half to fp32.
 __device__ __forceinline__ void unpack_i8(const uint4 &cw, float (&c)[16]) {
   const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
                          cw.w ^ 0x80808080u};
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
 #pragma unroll
-  for (int e = 0; e < 16; ++e)
-    c[e] = __fsub_rn(__uint_as_float(__byte_perm(w[e >> 2], 0x4B000000u, 0x7650u | (e & 3))),
-                     8388736.0f);
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t lo = __byte_perm(w[q], 0x64646464u, 0x5140u);   // bytes 0, 1
+    const uint32_t hi = __byte_perm(w[q], 0x64646464u, 0x7362u);   // bytes 2, 3
+    const float2 f0 = __half22float2(__hsub2(*reinterpret_cast<const __half2 *>(&lo), bias));
+    const float2 f1 = __half22float2(__hsub2(*reinterpret_cast<const __half2 *>(&hi), bias));
+    c[4 * q] = f0.x;
+    c[4 * q + 1] = f0.y;
+    c[4 * q + 2] = f1.x;
+    c[4 * q + 3] = f1.y;
+  }
 }
 // 16 int4 codes (two's complement nibbles, even column low) -> exact floats.
 __device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
