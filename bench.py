@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every batch x state-format point of the 48-layer sweep (one GPU)")
     return ap.parse_args()
 
 
@@ -392,6 +394,71 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def run_sweep(args):
+    """Every point of the 48-layer throughput sweep on one GPU: batch in {1, 16, 64, 256,
+    1024} x {int8, mixed int8/int4 (25% of heads at 8 bits by decay), fp32 state}.  Each
+    point: `warmup` untimed steps, then `steps` timed steps (CUDA events around the whole
+    step loop).  Points whose 48-layer state fits in the 126 MB L2 are flagged."""
+    import torch
+    from bit_recurrent_state_lores_b200 import lores as L
+    from bit_recurrent_state_lores_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = measured_peak()
+    points = []
+    for variant in ("int8", "mixed", "fp32"):
+        for B in (1, 16, 64, 256, 1024):
+            a = argparse.Namespace(**vars(args))
+            a.batch, a.variant = B, variant
+            wl = workload(a)
+            layers = []
+            for layer in range(wl.layers):
+                wll = layer_workload(wl, layer)
+                bits = layer_bits(a, wl, layer)
+                hp = synth.head_params(wll)
+                h = L.lores_create(B, wl.H, wl.d_k, wl.d_v, delta=wl.delta, head_bits=bits,
+                                   seed=wll.seed << 8, device=0)
+                inp = synth.step_inputs(wll, 0, hp, device=dev)
+                layers.append((h, bits, inp, torch.empty(B, wl.H, wl.d_v, device=dev)))
+            sptr = torch.cuda.current_stream(dev).cuda_stream
+
+            def step(t):
+                for (h, _, (q, k, v, al, be), o) in layers:
+                    L.lores_decode_step(h, q, k, v, al, be, o, t, sptr)
+
+            for t in range(args.warmup):
+                step(t)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            for t in range(args.steps):
+                step(args.warmup + t)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+            for (h, _, _, _) in layers:
+                assert L.lores_check_errors(h, sptr) == L.LORES_OK
+            step_bytes = sum(launch_bytes(wl, bits) for (_, bits, _, _) in layers)
+            state_bytes = sum(wl.B * sum(wl.d_v * wl.d_k * b // 8 for b in bits)
+                              for (_, bits, _, _) in layers)
+            gbs = step_bytes * args.steps / (ms / 1e3) / 1e9
+            points.append({"variant": variant, "batch": B,
+                           "value": wl.B * wl.H * wl.layers * args.steps / (ms / 1e3),
+                           "unit": UNIT, "ms_per_step": ms / args.steps,
+                           "algorithmic_GBps": gbs, "frac_of_peak": gbs / peak,
+                           "l2_resident": state_bytes < 126e6})
+            for (h, _, _, _) in layers:
+                L.lores_destroy(h)
+            del layers
+            torch.cuda.empty_cache()
+    return {"metric": METRIC, "sweep": points, "peak_GBps": peak, "peak_kind": peak_kind,
+            "steps": args.steps, "warmup": args.warmup,
+            "config": {"workload": "sweep-48-layers", "heads": 32, "d_k": 128, "d_v": 128,
+                       "delta": 1, "decay": "scalar per head", "group_size": 128,
+                       "rounding": "stochastic"}}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: same metric, timed on host cores."""
     if rank != 0:
@@ -424,6 +491,9 @@ def main():
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+    if args.sweep:
+        print(json.dumps(run_sweep(args)), flush=True)
         return
     import torch
     import torch.distributed as dist
