@@ -71,26 +71,32 @@ __host__ __device__ constexpr int full_rows(int dk, int bits) {
 }
 
 // -------------------------------------------------------------------------------------
-// producer (one lane of the warp): stage one unit's inputs into the warp's ring slot
+// producer (the whole warp): stage one unit's inputs into the warp's ring slot
 // -------------------------------------------------------------------------------------
+// Lane 0 announces the byte count on the slot's mbarrier; then lanes 0-5 each issue one
+// of the unit's bulk copies (codes, scales, k, q, v slice, per-column alpha) in parallel.
 template <int DK, bool DIAG>
 __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *tbl, int b, int ub,
                                            uint8_t *stage, uint64_t *bar) {
+  const int lane = threadIdx.x & 31;
   const UnitDesc d = tbl[ub];
   const long long tile = (long long)b * p.H + d.head;
   const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
   const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
   const unsigned vbytes = (unsigned)(d.nrows * 4);
   const unsigned vec = DK * 4;
-  const unsigned total = cbytes + sbytes + vbytes + 2 * vec + (DIAG ? vec : 0);
-  mbar_expect_tx(bar, total);
-  bulk_g2s(stage, p.codes + (long long)b * p.seq_bytes + d.code_off, cbytes, bar);
-  if (sbytes)
-    bulk_g2s(stage + p.st_scales, p.scales + (tile * p.d_v + d.row0) * p.ng, sbytes, bar);
-  bulk_g2s(stage + p.st_k, p.k + tile * DK, vec, bar);
-  bulk_g2s(stage + p.st_q, p.q + tile * DK, vec, bar);
-  bulk_g2s(stage + p.st_v, p.v + tile * p.d_v + d.row0, vbytes, bar);
-  if (DIAG) bulk_g2s(stage + p.st_a, p.alpha + tile * DK, vec, bar);
+  if (lane == 0) mbar_expect_tx(bar, cbytes + sbytes + vbytes + 2 * vec + (DIAG ? vec : 0));
+  __syncwarp();
+  const void *src = nullptr;
+  int dst = 0;
+  unsigned bytes = 0;
+  if (lane == 0) { src = p.codes + (long long)b * p.seq_bytes + d.code_off; dst = 0; bytes = cbytes; }
+  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; }
+  if (lane == 2) { src = p.k + tile * DK; dst = p.st_k; bytes = vec; }
+  if (lane == 3) { src = p.q + tile * DK; dst = p.st_q; bytes = vec; }
+  if (lane == 4) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
+  if (DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = vec; }
+  if (bytes) bulk_g2s(stage + dst, src, bytes, bar);
 }
 
 // -------------------------------------------------------------------------------------
@@ -144,6 +150,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
   const float kq = (float)kqd;
   const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
+  // shuffle distances of the group-max levels (0 beyond the group width: own value)
+  const int gd1 = 1 < lpg ? 1 : 0, gd2 = 2 < lpg ? 2 : 0, gd4 = 4 < lpg ? 4 : 0,
+            gd8 = 8 < lpg ? 8 : 0;
 
   uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
   float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
@@ -224,7 +233,8 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     } else {
       uint32_t words[4];
       float s_new;
-      gbad = requantize16_nb<LPR, BITS, SR>(x, lpg, cbase0 + kCtrPerPass * (uint32_t)n, words, s_new);
+      gbad = requantize16_nb<LPR, BITS, SR>(x, gd1, gd2, gd4, gd8,
+                                            cbase0 + kCtrPerPass * (uint32_t)n, words, s_new);
       if (active) {
         if (BITS == 8)
           __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
@@ -263,8 +273,16 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   float *go = p.o + tile * p.d_v + d.row0;
   for (int r = lane; r < d.nrows; r += 32) {
     float acc = 0.0f;
+    if (LPR >= 4) {
 #pragma unroll
-    for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
+      for (int l = 0; l < LPR; l += 4) {
+        const float4 v4 = *reinterpret_cast<const float4 *>(opart + r * LPR + l);
+        acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, v4.x), v4.y), v4.z), v4.w);
+      }
+    } else {
+#pragma unroll
+      for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
+    }
     go[r] = __fmaf_rn(ow[r], kq, acc);
   }
   __syncwarp();
@@ -280,16 +298,18 @@ __device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *
     compute_unit<DK, DIAG, DELTA, SR, BITS, false>(p, stage, b, d, alpha_s, beta, opart, ow);
 }
 
-// Position of a unit in (sequence b, unit index ub within the sequence), advanced by a
-// fixed stride without divisions.
+// Position of a unit: global unit u = ub * B + b (sequence b is the fast index, so a warp
+// striding through units visits the per-sequence unit table in order, and a table sorted
+// by bit width keeps each warp on one code path for long runs), advanced by a fixed
+// stride without divisions.
 struct UnitPos {
   int b, ub;
-  __device__ __forceinline__ void advance(int sb, int su, int ups) {
-    ub += su;
+  __device__ __forceinline__ void advance(int sb, int su, int B) {
     b += sb;
-    if (ub >= ups) {
-      ub -= ups;
-      ++b;
+    ub += su;
+    if (b >= B) {
+      b -= B;
+      ++ub;
     }
   }
 };
@@ -319,23 +339,26 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
   const long long first = (long long)blockIdx.x * kWarps + warp;
   if (first >= p.total_units) return;
   const long long stride = (long long)gridDim.x * kWarps;
-  const int sb = (int)(stride / ups), su = (int)(stride % ups);
-  UnitPos cur{(int)(first / ups), (int)(first % ups)};
+  const int B = p.B;
+  const int sb = (int)(stride % B), su = (int)(stride / B);
+  UnitPos cur{(int)(first % B), (int)(first / B)};
 
   if (lane == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
-    UnitPos q = cur;
-    for (int s = 0; s < kStages && q.b < p.B; ++s) {
-      issue_unit<DK, DIAG>(p, tbl, q.b, q.ub, stages + s * p.stage_bytes, &bars[s]);
-      q.advance(sb, su, ups);
-    }
   }
   __syncwarp();
+  {
+    UnitPos q = cur;
+    for (int s = 0; s < kStages && q.ub < ups; ++s) {
+      issue_unit<DK, DIAG>(p, tbl, q.b, q.ub, stages + s * p.stage_bytes, &bars[s]);
+      q.advance(sb, su, B);
+    }
+  }
   UnitPos nxt = cur;                                // the unit after `cur`
-  nxt.advance(sb, su, ups);
+  nxt.advance(sb, su, B);
   UnitPos fill = nxt;                               // the unit that refills the slot just used
-  fill.advance(sb, su, ups);
+  fill.advance(sb, su, B);
 
   // per-tile scalars of the current unit; the next unit's are loaded one unit ahead
   float alpha_cur = 0.0f, beta_cur;
@@ -345,11 +368,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
     if (!DIAG) alpha_cur = __ldg(p.alpha + t0);
   }
 
-  for (int n = 0; cur.b < p.B; ++n) {
+  for (int n = 0; cur.ub < ups; ++n) {
     const int s = n % kStages;
     uint8_t *stage = stages + s * p.stage_bytes;
     float alpha_nx = 0.0f, beta_nx = 0.0f;
-    if (nxt.b < p.B) {
+    if (nxt.ub < ups) {
       const long long tn = (long long)nxt.b * p.H + tbl[nxt.ub].head;
       beta_nx = __ldg(p.beta + tn);
       if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
@@ -359,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       // Give up: record it, let the other slot's copy (if any) land, and leave.
       if (lane == 0) {
         atomicOr(p.flag, kFlagTimeout);
-        if (nxt.b < p.B)
+        if (nxt.ub < ups)
           (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
       }
       __syncwarp();
@@ -373,13 +396,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
     else
       compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     // compute_any ends with __syncwarp: every lane is done reading this slot
-    if (lane == 0 && fill.b < p.B) {
+    if (fill.ub < ups) {
       fence_proxy_async();
       issue_unit<DK, DIAG>(p, tbl, fill.b, fill.ub, stage, &bars[s]);
     }
     cur = nxt;
-    nxt.advance(sb, su, ups);
-    fill.advance(sb, su, ups);
+    nxt.advance(sb, su, B);
+    fill.advance(sb, su, B);
     alpha_cur = alpha_nx;
     beta_cur = beta_nx;
   }
@@ -736,8 +759,12 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   };
   std::vector<UnitDesc> units;
   int ctas_per_sm = 1;
+  auto bits_rank = [](int b) { return b == 8 ? 0 : (b == 4 ? 1 : 2); };
   for (;;) {
     build_units(units);
+    std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
+      return bits_rank(x.bits) < bits_rank(y.bits);
+    });
     int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
     for (const UnitDesc &d : units) {
       cmax = std::max(cmax, d.nrows * row_bytes(dk, d.bits));

@@ -216,8 +216,9 @@ __device__ __forceinline__ float recip_nr(float m) {
 // scale written here are not meaningful.  cbase = tile key + golden * (n0 + 1) where
 // n0 is the quad index of the lane's first column (see the dither definition).
 template <int LPR, int BITS, bool SR>
-__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int lpg, uint32_t cbase,
-                                                uint32_t (&words)[4], float &s_out) {
+__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int gd1, int gd2, int gd4,
+                                                int gd8, uint32_t cbase, uint32_t (&words)[4],
+                                                float &s_out) {
   constexpr float r = (BITS == 8) ? 127.0f : 7.0f;
   constexpr float inv_r = (BITS == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
   float mq[4];
@@ -226,11 +227,11 @@ __device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int lpg, u
     mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[4 * c]), x[4 * c + 1]), x[4 * c + 2]),
                         x[4 * c + 3]);
   float m = max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
+  // group max over the lanes of the group: a level at or beyond the group width has
+  // shuffle distance 0 (the lane's own value)
+  const int dist[4] = {gd1, gd2, gd4, gd8};
 #pragma unroll
-  for (int st = 1; st < LPR; st <<= 1) {
-    const float mo = __shfl_xor_sync(kFull, m, st);
-    m = (st < lpg) ? max_nan(m, mo) : m;
-  }
+  for (int l = 0; (1 << l) < LPR; ++l) m = max_nan(m, __shfl_xor_sync(kFull, m, dist[l]));
   const bool gbad = !(m <= 0x1p100f);                    // inf, NaN or overflow
   const bool scaled = m >= 0x1p-100f && !gbad;           // below 2^-100: zero group
   const float y = recip_nr(scaled ? m : 1.0f);
