@@ -107,7 +107,7 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
 // The readout is reduced per warp: each lane leaves its share of S'q in opart, lane 0
 // of the row leaves w in ow, and after the rows each lane forms o for one row as
 // sum(opart) + w (k.q).
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL>
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL, bool GROW>
 __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow) {
@@ -117,10 +117,11 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   const int lane = threadIdx.x & 31;
   const int lir = lane % LPR, riw = lane / LPR;
   const int col0 = lir * 16;
-  const int lpg = p.G / 16;                               // lanes per scale group (power of 2)
-  const int g = lir / lpg;                                 // this lane's group in the row
+  // GROW: one scale per value row (G = d_k), known at compile time
+  const int lpg = GROW ? LPR : p.G / 16;                   // lanes per scale group (power of 2)
+  const int g = GROW ? 0 : lir / lpg;                      // this lane's group in the row
   const bool scale_writer = (lir & (lpg - 1)) == 0;
-  const int ng = p.ng;
+  const int ng = GROW ? 1 : p.ng;
   const long long tile = (long long)b * p.H + d.head;
 
   const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
@@ -170,6 +171,10 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     const int lr = n * RPW + riw;              // row inside the unit
     const bool active = FULL || lr < d.nrows;
     const int lrr = active ? lr : 0;           // keep shared loads in bounds
+    // dither words first: they depend only on the counter, so they fill the latency of
+    // the dot-product and group-max shuffles below
+    uint32_t hw[4] = {0u, 0u, 0u, 0u};
+    if (SR && BITS != 32) dither_words(cbase0 + kCtrPerPass * (uint32_t)n, hw);
 
     // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
     float sp[16];
@@ -233,8 +238,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     } else {
       uint32_t words[4];
       float s_new;
-      gbad = requantize16_nb<LPR, BITS, SR>(x, gd1, gd2, gd4, gd8,
-                                            cbase0 + kCtrPerPass * (uint32_t)n, words, s_new);
+      gbad = requantize16_nb<LPR, BITS, SR>(x, gd1, gd2, gd4, gd8, hw, words, s_new);
       if (active) {
         if (BITS == 8)
           __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
@@ -292,10 +296,14 @@ template <int DK, bool DIAG, bool DELTA, bool SR, int BITS>
 __device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *stage, int b,
                                             const UnitDesc &d, float alpha_s, float beta,
                                             float *opart, float *ow) {
-  if (d.nrows == full_rows(DK, BITS))
-    compute_unit<DK, DIAG, DELTA, SR, BITS, true>(p, stage, b, d, alpha_s, beta, opart, ow);
-  else
-    compute_unit<DK, DIAG, DELTA, SR, BITS, false>(p, stage, b, d, alpha_s, beta, opart, ow);
+  if (d.nrows == full_rows(DK, BITS)) {
+    if (p.G == DK)
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, true>(p, stage, b, d, alpha_s, beta, opart, ow);
+    else
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false>(p, stage, b, d, alpha_s, beta, opart, ow);
+  } else {
+    compute_unit<DK, DIAG, DELTA, SR, BITS, false, false>(p, stage, b, d, alpha_s, beta, opart, ow);
+  }
 }
 
 // Position of a unit: global unit u = ub * B + b (sequence b is the fast index, so a warp

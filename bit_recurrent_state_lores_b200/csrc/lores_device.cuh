@@ -215,10 +215,16 @@ __device__ __forceinline__ float recip_nr(float m) {
 // a bad group must then be zeroed by the caller (see zero_bad_rows); its codes and
 // scale written here are not meaningful.  cbase = tile key + golden * (n0 + 1) where
 // n0 is the quad index of the lane's first column (see the dither definition).
+// Dither words of one lane-row: four MurmurHash3 finalizer values of consecutive counters.
+__device__ __forceinline__ void dither_words(uint32_t cbase, uint32_t (&h)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
+}
+
 template <int LPR, int BITS, bool SR>
 __device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int gd1, int gd2, int gd4,
-                                                int gd8, uint32_t cbase, uint32_t (&words)[4],
-                                                float &s_out) {
+                                                int gd8, const uint32_t (&h)[4],
+                                                uint32_t (&words)[4], float &s_out) {
   constexpr float r = (BITS == 8) ? 127.0f : 7.0f;
   constexpr float inv_r = (BITS == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
   float mq[4];
@@ -239,9 +245,6 @@ __device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int gd1, i
   s_out = scaled ? __fmul_rn(m, inv_r) : 0.0f;
   uint32_t t[16];
   if (SR) {
-    uint32_t h[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float g = __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)));
