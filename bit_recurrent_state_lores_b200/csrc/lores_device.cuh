@@ -110,39 +110,43 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned by
 // -------------------------------------------------------------------------------------
 // code <-> float
 // -------------------------------------------------------------------------------------
+// Two fp16 halves of a word, each widened to fp32 and added to `bias` in one
+// mixed-precision add (fp16 operand, fp32 operand and result, round to nearest).
+__device__ __forceinline__ void halves_plus(uint32_t w, float bias, float &lo, float &hi) {
+  asm("{\n\t.reg .f16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %3;\n\t"
+      "add.rn.f32.f16 %1, h, %3;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w), "f"(bias));
+}
+
 // 16 int8 codes (two's complement) -> exact floats.  Bias to offset binary, drop pairs
-// of bytes into the mantissas of an fp16 pair (1024 + b: fp16 spacing is 1 there),
-// subtract 1024 + 128 from both halves (exact), widen each half to fp32.
+// of bytes into the mantissas of an fp16 pair (1024 + b: fp16 spacing is 1 there), and
+// add -(1024 + 128) to each half in fp32: the result is the code, exactly.
 __device__ __forceinline__ void unpack_i8(const uint4 &cw, float (&c)[16]) {
   const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
                          cw.w ^ 0x80808080u};
-  const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const uint32_t lo = __byte_perm(w[q], 0x64646464u, 0x5140u);   // bytes 0, 1
-    const uint32_t hi = __byte_perm(w[q], 0x64646464u, 0x7362u);   // bytes 2, 3
-    const float2 f0 = __half22float2(__hsub2(*reinterpret_cast<const __half2 *>(&lo), bias));
-    const float2 f1 = __half22float2(__hsub2(*reinterpret_cast<const __half2 *>(&hi), bias));
-    c[4 * q] = f0.x;
-    c[4 * q + 1] = f0.y;
-    c[4 * q + 2] = f1.x;
-    c[4 * q + 3] = f1.y;
+    halves_plus(__byte_perm(w[q], 0x64646464u, 0x5140u), -1152.0f, c[4 * q], c[4 * q + 1]);
+    halves_plus(__byte_perm(w[q], 0x64646464u, 0x7362u), -1152.0f, c[4 * q + 2], c[4 * q + 3]);
   }
 }
-// 16 int4 codes (two's complement nibbles, even column low) -> exact floats.
+// 16 int4 codes (two's complement nibbles, even column low) -> exact floats: nibbles to
+// offset-binary bytes (even columns in one word, odd in another), bytes into fp16 pairs
+// (columns 2p and 2p + 2 of the same parity), add -(1024 + 8) in fp32.
 __device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
   const uint32_t w[2] = {cw.x, cw.y};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t lo = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // even columns
-    const uint32_t hi = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // odd columns
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      c[8 * h + 2 * p] =
-          __fsub_rn(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650u | p)), 8388616.0f);
-      c[8 * h + 2 * p + 1] =
-          __fsub_rn(__uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650u | p)), 8388616.0f);
-    }
+    const uint32_t ev = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // columns 0, 2, 4, 6
+    const uint32_t od = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 1, 3, 5, 7
+    float *cc = c + 8 * h;
+    halves_plus(__byte_perm(ev, 0x64646464u, 0x5140u), -1032.0f, cc[0], cc[2]);
+    halves_plus(__byte_perm(ev, 0x64646464u, 0x7362u), -1032.0f, cc[4], cc[6]);
+    halves_plus(__byte_perm(od, 0x64646464u, 0x5140u), -1032.0f, cc[1], cc[3]);
+    halves_plus(__byte_perm(od, 0x64646464u, 0x7362u), -1032.0f, cc[5], cc[7]);
   }
 }
 // t holds 49152 + code + frac in fp32: its byte 1 is the code (two's complement).
