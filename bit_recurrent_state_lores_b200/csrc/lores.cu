@@ -35,9 +35,10 @@ struct __align__(16) UnitDesc {
   int32_t head;
   int32_t row0;
   int32_t nrows;
-  int32_t bits;          // 8, 4 or 32
+  int32_t bits;          // 4..8 (b-bit codes) or 32 (fp32 state)
   int64_t code_off;      // byte offset of row0 of this head inside one sequence's block
-  int64_t pad;
+  float r;               // largest code, 2^(bits-1) - 1
+  float inv_r;           // fl(1/r)
 };
 
 struct StepParams {
@@ -60,8 +61,12 @@ struct StepParams {
   int st_scales, st_k, st_q, st_v, st_a, stage_bytes;   // stage layout
 };
 
+// Storage of b-bit codes: 4-bit codes as nibbles, 5- to 8-bit codes one per byte.
+__host__ __device__ constexpr int storage_bits(int bits) {
+  return bits == 4 ? 4 : (bits == 32 ? 32 : 8);
+}
 // Bytes of one row of a tile with `bits`-bit entries.
-__host__ __device__ constexpr int row_bytes(int dk, int bits) { return dk * bits / 8; }
+__host__ __device__ constexpr int row_bytes(int dk, int bits) { return dk * storage_bits(bits) / 8; }
 
 // Rows of a full unit: 4 KB of state, a whole number of warp passes (32/(d_k/16) rows).
 __host__ __device__ constexpr int full_rows(int dk, int bits) {
@@ -238,7 +243,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     } else {
       uint32_t words[4];
       float s_new;
-      gbad = requantize16_nb<LPR, BITS, SR>(x, gd1, gd2, gd4, gd8, hw, words, s_new);
+      gbad = requantize16_nb<LPR, BITS, SR>(x, d.r, d.inv_r, gd1, gd2, gd4, gd8, hw, words, s_new);
       if (active) {
         if (BITS == 8)
           __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
@@ -397,12 +402,12 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       return;
     }
     const UnitDesc d = tbl[cur.ub];
-    if (d.bits == 8)
-      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
+    if (d.bits == 32)
+      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     else if (d.bits == 4)
       compute_any<DK, DIAG, DELTA, SR, 4>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     else
-      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
+      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
     // compute_any ends with __syncwarp: every lane is done reading this slot
     if (fill.ub < ups) {
       fence_proxy_async();
@@ -460,7 +465,7 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   const uint32_t n0 = (uint32_t)row * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
   uint32_t words[4];
   float s_new;
-  requantize16<LPR>(x, bits == 4 ? 4 : 8, lpg, lane, tkey, n0, p.stochastic, words, s_new);
+  requantize16<LPR>(x, bits == 32 ? 8 : bits, lpg, lane, tkey, n0, p.stochastic, words, s_new);
   if (!active) return;
   if (bits == 32) {
     float4 *dst = reinterpret_cast<float4 *>(tilecodes + (size_t)row * DK * 4) + lir * 4;
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
     for (int c = 0; c < 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
     return;
   }
-  if (bits == 8)
+  if (bits != 4)
     *reinterpret_cast<uint4 *>(tilecodes + (size_t)row * DK + lir * 16) =
         make_uint4(words[0], words[1], words[2], words[3]);
   else
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
     }
   } else {
     float cf[16];
-    if (bits == 8)
+    if (bits != 4)
       unpack_i8(*reinterpret_cast<const uint4 *>(tilecodes + (size_t)row * DK + lir * 16), cf);
     else
       unpack_i4(*reinterpret_cast<const uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8), cf);
@@ -675,7 +680,7 @@ const char *lores_status_string(lores_status s) {
 
 lores_status lores_assign_bits_by_decay(const float *mean_decay, int32_t H, float frac_high,
                                         int32_t bits_high, int32_t bits_low, int32_t *out_bits) {
-  auto okbits = [](int b) { return b == 4 || b == 8 || b == 32; };
+  auto okbits = [](int b) { return (b >= 4 && b <= 8) || b == 32; };
   if (!mean_decay || !out_bits || H < 1 || !(frac_high >= 0.0f && frac_high <= 1.0f) ||
       !okbits(bits_high) || !okbits(bits_low))
     return LORES_ERR_INVALID_ARG;
@@ -709,7 +714,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   if (c.head_bits)
     for (int h = 0; h < c.heads; ++h) {
       bits[h] = c.head_bits[h];
-      if (bits[h] != 8 && bits[h] != 4 && bits[h] != 32) return LORES_ERR_INVALID_ARG;
+      if (!((bits[h] >= 4 && bits[h] <= 8) || bits[h] == 32)) return LORES_ERR_INVALID_ARG;
     }
 
   DeviceGuard guard(c.device);
@@ -761,13 +766,15 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
         d.nrows = std::min(R, dv - r0);
         d.bits = b;
         d.code_off = h->head_off[hh] + (long long)r0 * row_bytes(dk, b);
+        d.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
+        d.inv_r = b == 32 ? 0.0f : 1.0f / d.r;
         u.push_back(d);
       }
     }
   };
   std::vector<UnitDesc> units;
   int ctas_per_sm = 1;
-  auto bits_rank = [](int b) { return b == 8 ? 0 : (b == 4 ? 1 : 2); };
+  auto bits_rank = [](int b) { return storage_bits(b) == 8 ? 0 : (b == 4 ? 1 : 2); };
   for (;;) {
     build_units(units);
     std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
@@ -1085,7 +1092,7 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
       (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
     return LORES_ERR_INVALID_ARG;
   for (int hh = 0; c.head_bits && hh < c.heads; ++hh)
-    if (c.head_bits[hh] != 8 && c.head_bits[hh] != 4 && c.head_bits[hh] != 32)
+    if (!((c.head_bits[hh] >= 4 && c.head_bits[hh] <= 8) || c.head_bits[hh] == 32))
       return LORES_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(scales) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
       (c.decay_diag ? !aligned16(alpha) : (reinterpret_cast<uintptr_t>(alpha) & 3u)) ||
@@ -1111,6 +1118,8 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
       d.nrows = std::min(R, dv - r0);
       d.bits = b;
       d.code_off = seq_bytes + (long long)r0 * row_bytes(dk, b);
+      d.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
+      d.inv_r = b == 32 ? 0.0f : 1.0f / d.r;
       cmax = std::max(cmax, d.nrows * row_bytes(dk, b));
       if (b != 32) smax = std::max(smax, d.nrows * ng * 4);
       vmax = std::max(vmax, d.nrows * 4);

@@ -225,12 +225,13 @@ __device__ __forceinline__ void dither_words(uint32_t cbase, uint32_t (&h)[4]) {
   for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
 }
 
+// r = 2^(b-1) - 1 of the unit's codes and inv_r = fl(1/r); BITS is the storage (8: one
+// byte per code, for 5- to 8-bit codes; 4: nibbles).
 template <int LPR, int BITS, bool SR>
-__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], int gd1, int gd2, int gd4,
-                                                int gd8, const uint32_t (&h)[4],
-                                                uint32_t (&words)[4], float &s_out) {
-  constexpr float r = (BITS == 8) ? 127.0f : 7.0f;
-  constexpr float inv_r = (BITS == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
+__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], float r, float inv_r,
+                                                int gd1, int gd2, int gd4, int gd8,
+                                                const uint32_t (&h)[4], uint32_t (&words)[4],
+                                                float &s_out) {
   float mq[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
@@ -272,8 +273,8 @@ template <int LPR>
 __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
                                              uint32_t tkey, uint32_t n0, int stochastic,
                                              uint32_t (&words)[4], float &s_out) {
-  const float r = (bits == 8) ? 127.0f : 7.0f;
-  const float inv_r = (bits == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   // fl(1/r)
+  const float r = (float)((1 << (bits - 1)) - 1);        // 2^(b-1) - 1
+  const float inv_r = __fdiv_rn(1.0f, r);                 // fl(1/r)
   float mq[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
@@ -315,7 +316,7 @@ __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int
 #pragma unroll
     for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, 49152.5f));
   }
-  if (bits == 8) {
+  if (bits != 4) {
     const uint4 w = pack_i8(t);
     words[0] = w.x; words[1] = w.y; words[2] = w.z; words[3] = w.w;
   } else {

@@ -64,7 +64,9 @@ typedef struct {
     int32_t group_size;     /* G: key entries per scale; 0 means d_k (one scale per row)     */
     int32_t delta;          /* 1: delta-rule correction (GDN, KDA); 0: none (Mamba-2)        */
     int32_t decay_diag;     /* 0: alpha is one scalar per (seq, head); 1: one per key column */
-    const int32_t *head_bits; /* host [H], each 8, 4 or 32 (fp32, unquantized); NULL: all 8 */
+    const int32_t *head_bits; /* host [H], each 4..8 (b-bit codes, r = 2^(b-1) - 1) or 32  */
+                              /* (fp32, unquantized); NULL: all 8.  4-bit codes are stored */
+                              /* as nibbles, 5- to 8-bit codes one per byte               */
     int32_t stochastic;     /* 1: stochastic rounding (LoReS); 0: round to nearest           */
     uint64_t seed;          /* key of the rounding dither                                    */
     int32_t device;         /* CUDA device ordinal                                           */
@@ -164,9 +166,9 @@ lores_status lores_dequant_state(lores_handle *h, float *out, void *stream);
 lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, void *stream);
 
 /* Copy the raw state out: codes (layout_.code_bytes bytes; per sequence the heads'
- * tiles back to back in head order; a tile is row-major [d_v][d_k] int8, or
- * [d_v][d_k/2] bytes of int4 with the even column in the low nibble, or
- * [d_v][d_k] fp32) and scales [B, H, d_v, n_groups] fp32.  Either pointer may be
+ * tiles back to back in head order; a tile is row-major [d_v][d_k] bytes of 5- to
+ * 8-bit codes (two's complement), or [d_v][d_k/2] bytes of 4-bit codes with the even
+ * column in the low nibble, or [d_v][d_k] fp32) and scales [B, H, d_v, n_groups] fp32.  Either pointer may be
  * host or device memory (unified addressing); either may be NULL to skip it.
  * Returns after the copies have finished on `stream`. */
 lores_status lores_export_codes(lores_handle *h, void *codes, float *scales, void *stream);
@@ -190,7 +192,7 @@ lores_status lores_check_errors(lores_handle *h, void *stream);
  * the largest mean decay (slowest to forget) get bits_high, the others bits_low;
  * equal decays go to the lower head index.  Host only; mean_decay and out_bits
  * are host arrays of H entries.  Errors: INVALID_ARG for NULL, H < 1, frac outside
- * [0, 1] or bits outside {4, 8, 32}. */
+ * [0, 1] or bits outside 4..8 and 32. */
 lores_status lores_assign_bits_by_decay(const float *mean_decay, int32_t H, float frac_high,
                                         int32_t bits_high, int32_t bits_low, int32_t *out_bits);
 

@@ -109,7 +109,7 @@ uint32_t lo_dither(uint32_t tile_key, int d_k, int i, int j)
 typedef struct {
     int d_k, d_v;      /* state is d_v x d_k (value rows, key columns)       */
     int group;         /* key entries per scale, divides d_k                 */
-    int bits;          /* 8, 4, or 32 (unquantized fp32 state)               */
+    int bits;          /* 4..8 (b-bit codes) or 32 (unquantized fp32 state)  */
     int delta;         /* 0 or 1: delta correction on/off                     */
     int diag;          /* 0: scalar decay; 1: decay per key column           */
     int stochastic;    /* 1: stochastic rounding; 0: round to nearest        */
@@ -117,12 +117,12 @@ typedef struct {
 
 static int code_max(int bits) { return (1 << (bits - 1)) - 1; }
 
-/* Read code (i, j) from a packed tile.  int8: one byte per code, two's
- * complement.  int4: two codes per byte, even column in the low nibble, odd
+/* Read code (i, j) from a packed tile.  5 to 8 bits: one byte per code, two's
+ * complement.  4 bits: two codes per byte, even column in the low nibble, odd
  * column in the high nibble, two's complement nibbles. */
 static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
 {
-    if (c->bits == 8)
+    if (c->bits != 4)
         return (int)(int8_t)codes[(size_t)i * c->d_k + j];
     uint8_t byte = codes[(size_t)i * (c->d_k / 2) + j / 2];
     int nib = (j % 2 == 0) ? (byte & 0xF) : (byte >> 4);
@@ -131,7 +131,7 @@ static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
 
 static void put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code)
 {
-    if (c->bits == 8) {
+    if (c->bits != 4) {
         codes[(size_t)i * c->d_k + j] = (uint8_t)(int8_t)code;
         return;
     }
@@ -200,7 +200,7 @@ static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_
                           uint8_t *codes, float *scales)
 {
     const int r = code_max(c->bits);
-    const float inv_r = (c->bits == 8) ? 0x1.020408p-7f : 0x1.24924ap-3f;   /* fl(1/r) */
+    const float inv_r = 1.0f / (float)r;                  /* fl(1/r), round to nearest */
     const float m_lo = 0x1p-100f, m_hi = 0x1p100f;
     const int ng = c->d_k / c->group;
     int bad = 0;

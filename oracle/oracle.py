@@ -86,7 +86,9 @@ class TileCfg:
     def code_bytes(self):
         if self.bits == 32:
             return self.d_v * self.d_k * 4
-        return self.d_v * self.d_k * self.bits // 8
+        if self.bits == 4:
+            return self.d_v * self.d_k // 2
+        return self.d_v * self.d_k          # 5 to 8 bits: one byte per code
 
     def zero_state(self):
         """(state, scales) of an all-zero tile."""

@@ -139,7 +139,7 @@ def compare_tile(cfg, gpu_state, gpu_scales, ref_state, ref_scales):
 def unpack_fast(cfg, codes):
     """Vectorised unpack for large tiles; checked against the oracle's unpack in tests."""
     b = np.asarray(codes, np.uint8)
-    if cfg.bits == 8:
+    if cfg.bits != 4:                       # 5- to 8-bit codes: one byte each
         return b.view(np.int8).reshape(cfg.d_v, cfg.d_k).astype(np.int32)
     lo = (b & 0xF).astype(np.int32)
     hi = (b >> 4).astype(np.int32)

@@ -39,7 +39,8 @@ def test_status_strings():
 @pytest.mark.parametrize("kw", [
     dict(batch=0), dict(heads=0), dict(d_k=48), dict(d_k=512), dict(d_v=6), dict(d_v=0),
     dict(d_v=8192), dict(group_size=8), dict(group_size=48), dict(delta=2), dict(decay_diag=3),
-    dict(stochastic=5), dict(head_bits=[8, 5]), dict(device=-1)])
+    dict(stochastic=5), dict(head_bits=[8, 3]), dict(head_bits=[9, 8]), dict(head_bits=[16, 8]),
+    dict(device=-1)])
 def test_create_rejects_bad_config_before_touching_cuda(kw):
     from bit_recurrent_state_lores_b200 import lores as L
     args = dict(batch=2, heads=2, d_k=64, d_v=16)
@@ -76,7 +77,8 @@ def test_policy_rejects_bad_arguments():
         with pytest.raises(L.LoresError):
             L.lores_assign_bits_by_decay(*args)
     with pytest.raises(L.LoresError):
-        L.lores_assign_bits_by_decay([0.5, 0.6], 0.5, bits_high=6)
+        L.lores_assign_bits_by_decay([0.5, 0.6], 0.5, bits_high=3)
+    assert L.lores_assign_bits_by_decay([0.5, 0.6], 0.5, bits_high=6, bits_low=4) == [4, 6]
 
 
 def test_fast_unpack_matches_oracle_unpack():

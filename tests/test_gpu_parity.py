@@ -123,6 +123,8 @@ SWEEP = [
     (256, 24, 256, "8", 1, 0, 1, 1, 2),
     (256, 40, 16, "mix", 1, 1, 1, 2, 3),
     (256, 16, 64, "4", 0, 0, 0, 2, 2),
+    (128, 64, 32, "b5678", 1, 1, 1, 2, 6),  # 5-, 6-, 7-bit codes (one byte each) with 8/4/32
+    (64, 36, 16, "b5678", 0, 0, 0, 2, 6),
 ]
 
 
@@ -132,6 +134,8 @@ def test_small_shapes_every_tile_every_step(d_k, d_v, G, bits, delta, diag, sr, 
                         group=G, decay="kda" if diag else "tau", outliers=min(2, d_v), seed=d_k + d_v)
     if bits == "mix":
         hb = [(8, 4, 32)[h % 3] for h in range(H)]
+    elif bits == "b5678":
+        hb = [(6, 5, 8, 4, 7, 32)[h % 6] for h in range(H)]
     else:
         hb = [int(bits)] * H
     tiles = [(b, h) for b in range(B) for h in range(H)]

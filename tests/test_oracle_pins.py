@@ -252,7 +252,8 @@ def test_quantized_step_matches_fp64_update(bits, group, delta, diag):
 
 
 @pytest.mark.parametrize("bits,group,sr", [(8, 128, 1), (8, 32, 1), (4, 128, 1), (4, 16, 1),
-                                            (8, 128, 0), (4, 32, 0)])
+                                            (8, 128, 0), (4, 32, 0), (6, 128, 1), (5, 32, 1),
+                                            (7, 64, 0), (6, 16, 0)])
 def test_absmax_quantizer_invariants(bits, group, sr):
     # Proposition 1's scale: s_G = max|S_G| / r, r = 2^(b-1) - 1, codes in [-r, r]
     d_k, d_v = 128, 64
@@ -277,11 +278,20 @@ def test_absmax_quantizer_invariants(bits, group, sr):
                 continue
             # s = m * fl(1/r): two roundings, so |s r / m - 1| <= 2^-24 + 2^-24 (+ tiny)
             assert s == np.float32(m * (np.float32(1) / np.float32(r)))
+            assert r == 2 ** (bits - 1) - 1                  # Proposition 1: r = 2^(b-1) - 1
             assert abs(float(s) * r / float(m) - 1.0) <= 2.0 ** -23 * (1 + 1e-6)
             assert np.abs(cs).max() == r            # the group's max code is r exactly
             err = np.abs(cs * np.float64(s) - xs)
             lim = (1.0 if sr else 0.5 + 2.0 ** -8) * float(s) * (1 + 1e-6)
             assert err.max() <= lim
+
+
+def test_int6_codes_one_byte_each():
+    # 5 to 7-bit codes are stored one per byte (two's complement), like int8
+    cfg = O.TileCfg(16, 2, bits=6)
+    ints = np.array([list(range(-31, -15)), list(range(16, 32))])
+    b = O.pack_codes(cfg, ints)
+    assert b.size == 32 and b.view(np.int8).reshape(2, 16).tolist() == ints.tolist()
 
 
 def test_int4_and_int8_packing_worked_example():
