@@ -113,6 +113,8 @@ typedef struct {
     int delta;         /* 0 or 1: delta correction on/off                     */
     int diag;          /* 0: scalar decay; 1: decay per key column           */
     int stochastic;    /* 1: stochastic rounding; 0: round to nearest        */
+    int axis;          /* 0: value-axis groups (scales [d_v][d_k/G]);
+                        * 1: key-axis (one scale per key column, scales [d_k]) */
 } lo_cfg;
 
 static int code_max(int bits) { return (1 << (bits - 1)) - 1; }
@@ -235,6 +237,47 @@ static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_
     return bad;
 }
 
+/* Key-axis requantization of a whole tile X (d_v x d_k): one scale per key column,
+ * s_j = m_j * fl(1/r) with m_j = max_i |X_ij| (Proposition 1's column range C_j).  A
+ * column with an entry that is inf, NaN or above 2^100 is stored as zero (scale 0,
+ * codes 0) and reported with return value 1; a column whose maximum is below 2^-100 is
+ * stored as zero. */
+static int requantize_tile_key(const lo_cfg *c, const float *X, uint32_t tile_key,
+                               uint8_t *codes, float *scales)
+{
+    const int r = code_max(c->bits);
+    const float inv_r = 1.0f / (float)r;
+    int flag = 0;
+    for (int j = 0; j < c->d_k; j++) {
+        int bad = 0;
+        float m = 0.0f;
+        for (int i = 0; i < c->d_v; i++) {
+            float a = X[(size_t)i * c->d_k + j];
+            if (!isfinite(a) || fabsf(a) > 0x1p100f)
+                bad = 1;
+            else if (fabsf(a) > m)
+                m = fabsf(a);
+        }
+        float inv = 0.0f, s = 0.0f;
+        if (!bad && m >= 0x1p-100f) {
+            inv = (float)r * lo_recip_nr(m);
+            s = m * inv_r;
+        }
+        flag |= bad;
+        scales[j] = s;
+        for (int i = 0; i < c->d_v; i++) {
+            int code = 0;
+            if (inv != 0.0f) {
+                float d = c->stochastic ? (float)lo_dither(tile_key, c->d_k, i, j) : 128.0f;
+                float t = fmaf(X[(size_t)i * c->d_k + j], inv, 49152.0f + d / 256.0f);
+                code = (int)floorf(t - 49152.0f);
+            }
+            put_code(c, codes, i, j, code);
+        }
+    }
+    return flag;
+}
+
 /* ------------------------------------------------------------------------ */
 /* One decode step of one (sequence, head) tile                             */
 /* ------------------------------------------------------------------------ */
@@ -253,6 +296,7 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
     const int dk = c->d_k, ng = dk / c->group;
     float *Sp = malloc(sizeof(float) * dk);   /* S_{t-1} diag(alpha), one row */
     float *x = malloc(sizeof(float) * dk);    /* S_t, one row                 */
+    float *X = (c->axis && c->bits != 32) ? malloc(sizeof(float) * dk * (size_t)c->d_v) : NULL;
     int flag = 0;
     for (int i = 0; i < c->d_v; i++) {
         /* dequantize and decay: entry (i, j) is c_ij * (s_ig * alpha_j) */
@@ -261,7 +305,7 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
             if (c->bits == 32) {
                 Sp[j] = ((float *)state)[(size_t)i * dk + j] * aj;
             } else {
-                float s = scales[(size_t)i * ng + j / c->group];
+                float s = c->axis ? scales[j] : scales[(size_t)i * ng + j / c->group];
                 Sp[j] = (float)get_code(c, (uint8_t *)state, i, j) * (s * aj);
             }
         }
@@ -290,9 +334,15 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
                     flag = 1;
                 ((float *)state)[(size_t)i * dk + j] = x[j];
             }
+        } else if (c->axis) {
+            memcpy(X + (size_t)i * dk, x, sizeof(float) * dk);   /* quantized after all rows */
         } else {
             flag |= requantize_row(c, x, i, tile_key, (uint8_t *)state, scales);
         }
+    }
+    if (X) {
+        flag |= requantize_tile_key(c, X, tile_key, (uint8_t *)state, scales);
+        free(X);
     }
     free(Sp);
     free(x);
@@ -304,6 +354,8 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
 int lo_tile_quantize(const lo_cfg *c, const float *S, uint8_t *codes, float *scales,
                      uint32_t tile_key)
 {
+    if (c->axis)
+        return requantize_tile_key(c, S, tile_key, codes, scales);
     int flag = 0;
     for (int i = 0; i < c->d_v; i++)
         flag |= requantize_row(c, S + (size_t)i * c->d_k, i, tile_key, codes, scales);
@@ -317,7 +369,8 @@ void lo_tile_dequant(const lo_cfg *c, const uint8_t *codes, const float *scales,
     for (int i = 0; i < c->d_v; i++)
         for (int j = 0; j < c->d_k; j++)
             S[(size_t)i * c->d_k + j] =
-                (float)get_code(c, codes, i, j) * scales[(size_t)i * ng + j / c->group];
+                (float)get_code(c, codes, i, j) *
+                (c->axis ? scales[j] : scales[(size_t)i * ng + j / c->group]);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -18,7 +18,8 @@ _lib = None
 
 class LoCfg(C.Structure):
     _fields_ = [("d_k", C.c_int), ("d_v", C.c_int), ("group", C.c_int), ("bits", C.c_int),
-                ("delta", C.c_int), ("diag", C.c_int), ("stochastic", C.c_int)]
+                ("delta", C.c_int), ("diag", C.c_int), ("stochastic", C.c_int),
+                ("axis", C.c_int)]
 
 
 def lib():
@@ -72,16 +73,21 @@ def _f32(a):
 class TileCfg:
     """Shape and recipe of one (sequence, head) tile."""
 
-    def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1):
+    def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1, axis=0):
         self.d_k, self.d_v = int(d_k), int(d_v)
         self.group = int(group if group else d_k)
         self.bits, self.delta, self.diag, self.stochastic = int(bits), int(delta), int(diag), int(stochastic)
+        self.axis = int(axis)
         self.c = LoCfg(self.d_k, self.d_v, self.group, self.bits, self.delta, self.diag,
-                       self.stochastic)
+                       self.stochastic, self.axis)
 
     @property
     def n_groups(self):
         return self.d_k // self.group
+
+    def scale_shape(self):
+        """value axis: [d_v, d_k/G]; key axis: [d_k] (one scale per key column)."""
+        return (self.d_k,) if self.axis else (self.d_v, self.n_groups)
 
     def code_bytes(self):
         if self.bits == 32:
@@ -94,8 +100,7 @@ class TileCfg:
         """(state, scales) of an all-zero tile."""
         if self.bits == 32:
             return np.zeros((self.d_v, self.d_k), np.float32), np.zeros((self.d_v, self.n_groups), np.float32)
-        return (np.zeros(self.code_bytes(), np.uint8),
-                np.zeros((self.d_v, self.n_groups), np.float32))
+        return (np.zeros(self.code_bytes(), np.uint8), np.zeros(self.scale_shape(), np.float32))
 
 
 # --- random bits ------------------------------------------------------------
@@ -172,7 +177,7 @@ def tile_step(cfg: TileCfg, state, scales, q, k, v, alpha, beta, tkey, want_x=Fa
 def tile_quantize(cfg: TileCfg, S, tkey):
     S = _f32(S)
     codes = np.zeros(cfg.code_bytes(), np.uint8)
-    scales = np.zeros((cfg.d_v, cfg.n_groups), np.float32)
+    scales = np.zeros(cfg.scale_shape(), np.float32)
     flag = lib().lo_tile_quantize(C.byref(cfg.c), _p(S), _p(codes), _p(scales), tkey)
     return codes, scales, int(flag)
 

@@ -516,3 +516,102 @@ def test_assign_bits_by_decay_worked_examples():
     assert (b[24:] == 8).all() and (b[:24] == 4).all()
     assert O.assign_bits_by_decay([0.3, 0.2], 0.0).tolist() == [4, 4]
     assert O.assign_bits_by_decay([0.3, 0.2], 1.0).tolist() == [8, 8]
+
+
+# --------------------------------------------------------------------------
+# Key-axis grouping (Scale Grouping paragraph; Proposition 1's column ranges)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,sr", [(8, 1), (8, 0), (4, 1), (6, 0)])
+def test_key_axis_quantizer_invariants(bits, sr):
+    # one scale per key column: s_j = C_j / r with C_j = max_i |S_ij|; each column's
+    # largest code is r; codes in [-r, r]
+    d_k, d_v = 64, 48
+    cfg = O.TileCfg(d_k, d_v, bits=bits, stochastic=sr, axis=1)
+    r = 2 ** (bits - 1) - 1
+    g = rng(70 + bits + sr)
+    X = (g.standard_normal((d_v, d_k)) * np.exp(g.uniform(-6, 6, (1, d_k)))).astype(np.float32)
+    X[:, 7] = 0.0                                     # an all-zero column
+    codes, scales, flag = O.tile_quantize(cfg, X, O.tile_key(O.step_key(4, 1), 2))
+    assert flag == 0 and scales.shape == (d_k,)
+    C_ = O.unpack_codes(cfg, codes)
+    assert C_.min() >= -r and C_.max() <= r
+    for j in range(d_k):
+        m = np.float32(np.abs(X[:, j]).max())
+        if m == 0:
+            assert scales[j] == 0 and not C_[:, j].any()
+            continue
+        assert scales[j] == np.float32(m * (np.float32(1) / np.float32(r)))
+        assert np.abs(C_[:, j]).max() == r
+        err = np.abs(C_[:, j] * np.float64(scales[j]) - X[:, j])
+        assert err.max() <= (1.0 if sr else 0.5 + 2.0 ** -8) * float(scales[j]) * (1 + 1e-6)
+
+
+def test_key_axis_quantized_step_matches_fp64_update():
+    d_k, d_v, r = 32, 16, 127
+    cfg = O.TileCfg(d_k, d_v, bits=8, delta=1, diag=1, axis=1)
+    g = rng(71)
+    ints = g.integers(-r, r + 1, (d_v, d_k))
+    codes = O.pack_codes(cfg, ints)
+    scales = g.uniform(0.01, 0.1, d_k).astype(np.float32)
+    q, k, v, alpha, beta = draw(1, d_k, d_v, 72, diag=True)
+    X = recur64(ints * scales.astype(np.float64)[None, :], alpha[0], k[0], v[0], beta[0], 1)
+    o, flag, x = O.tile_step(cfg, codes, scales, q[0], k[0], v[0], alpha[0], beta[0], 5,
+                             want_x=True)
+    assert flag == 0
+    np.testing.assert_allclose(x, X, rtol=0, atol=1e-5 * np.abs(X).max())
+    np.testing.assert_allclose(o, X @ q[0].astype(np.float64), rtol=0, atol=1e-5 * np.abs(X).max())
+    # and the stored state is the key-axis quantization of x
+    c2, s2, _ = O.tile_quantize(cfg, x, 5)
+    assert (c2 == codes).all() and (s2 == scales).all()
+
+
+def test_key_axis_nonfinite_column_is_zeroed_and_flagged():
+    cfg = O.TileCfg(32, 8, bits=8, axis=1)
+    X = rng(73).standard_normal((8, 32)).astype(np.float32)
+    X[3, 9] = np.nan
+    X[5, 20] = np.float32(2.0 ** 101)
+    codes, scales, flag = O.tile_quantize(cfg, X, 9)
+    C_ = O.unpack_codes(cfg, codes)
+    assert flag == 1
+    for j in (9, 20):
+        assert scales[j] == 0 and not C_[:, j].any()
+    keep = [j for j in range(32) if j not in (9, 20)]
+    assert (np.abs(C_[:, keep]).max(axis=0) == 127).all()
+
+
+def test_proposition1_key_axis_readout_error():
+    # RTN with one scale per key column: E[e_i^2] = sum_j q_j^2 C_j^2 / (12 r^2)
+    d_k, d_v, n = 128, 32, 400
+    cfg = O.TileCfg(d_k, d_v, bits=4, stochastic=0, axis=1)
+    g = rng(74)
+    num = 0.0
+    den = 0.0
+    for it in range(n):
+        S = (g.standard_normal((d_v, d_k)) * g.uniform(0.1, 10, (1, d_k))).astype(np.float32)
+        q = unit(g.standard_normal(d_k))
+        codes, sc, _ = O.tile_quantize(cfg, S, 0)
+        e = (O.tile_dequant(cfg, codes, sc).astype(np.float64) - S) @ q
+        Cj = np.abs(S).max(axis=0).astype(np.float64)
+        num += np.sum(e ** 2)
+        den += d_v * np.sum(q ** 2 * Cj ** 2) / (12 * 7 ** 2)
+    ratio = num / den
+    assert 0.9 < ratio < 1.1, ratio
+
+
+def test_value_axis_beats_key_axis_with_outlier_value_rows():
+    # Scale Grouping paragraph: value-axis grouping is preferred at INT8; with a few large
+    # value rows (outlier channels of v) a per-row scale keeps the other rows fine
+    d_k, d_v = 64, 64
+    g = rng(75)
+    errs = {0: 0.0, 1: 0.0}
+    for it in range(50):
+        S = g.standard_normal((d_v, d_k)).astype(np.float32)
+        S[g.choice(d_v, 4, replace=False)] *= 50.0
+        q = unit(g.standard_normal(d_k))
+        for axis in (0, 1):
+            cfg = O.TileCfg(d_k, d_v, bits=8, stochastic=1, axis=axis)
+            codes, sc, _ = O.tile_quantize(cfg, S, O.tile_key(O.step_key(it, 0), axis))
+            e = (O.tile_dequant(cfg, codes, sc).astype(np.float64) - S) @ q
+            errs[axis] += float(np.sum(e ** 2))
+    assert errs[0] < 0.5 * errs[1], errs
