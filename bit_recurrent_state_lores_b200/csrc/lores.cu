@@ -435,6 +435,7 @@ struct LoadParams {
   int H, d_v, ng, G;
   uint32_t step_key;
   int stochastic;
+  int axis;                     // 0: value-axis groups; 1: one scale per key column
 };
 
 template <int DK>
@@ -512,13 +513,275 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
       unpack_i8(*reinterpret_cast<const uint4 *>(tilecodes + (size_t)row * DK + lir * 16), cf);
     else
       unpack_i4(*reinterpret_cast<const uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8), cf);
-    const float s = p.scales[grr * p.ng + col0 / p.G];
+    if (p.axis) {
+      const float *sc = p.scales + tile * DK + col0;          // one scale per key column
 #pragma unroll
-    for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(cf[e], s);
+      for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(cf[e], sc[e]);
+    } else {
+      const float s = p.scales[grr * p.ng + col0 / p.G];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(cf[e], s);
+    }
   }
   float4 *dst = reinterpret_cast<float4 *>(out + grr * DK + col0);
 #pragma unroll
   for (int c = 0; c < 4; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+}
+
+// -------------------------------------------------------------------------------------
+// key-axis grouping (ablation comparator): one scale per key column of a tile
+// -------------------------------------------------------------------------------------
+// The column maximum couples all rows of a tile, so one CTA handles one whole tile:
+// pass 1 updates every row (x = S' + w k^T), keeps w and the readout shares, and
+// reduces per-column maxima; pass 2 recomputes x (the same fp32 operations) and writes
+// codes with the column scale.  Columns with an inf/NaN/overflow entry are stored as
+// zero and flagged; fp32 heads store x as in the value-axis path.
+struct KeyParams {
+  uint8_t *codes;
+  float *scales;                // [B][H][d_k]
+  const float *q, *k, *v, *alpha, *beta;
+  const float *S;               // load_state input [B][H][d_v][d_k], or null
+  float *o;
+  unsigned *flag;
+  const int32_t *head_bits;
+  const int64_t *head_off;
+  long long seq_bytes;
+  int H, d_v;
+  uint32_t step_key;
+  int delta, diag, stochastic;
+  // shared memory offsets
+  int sm_codes, sm_scales, sm_k, sm_q, sm_a, sm_v, sm_opart, sm_ow, sm_cm;
+};
+
+// Column maxima of the lane's 16 columns over the whole tile: reduce across the row groups
+// of the warp, then across warps through shared memory.
+template <int DK>
+__device__ __forceinline__ void column_max(float (&cm)[16], float *smcm) {
+  constexpr int LPR = DK / 16;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lir = lane % LPR, riw = lane / LPR;
+#pragma unroll
+  for (int st = LPR; st < 32; st <<= 1)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) cm[e] = max_nan(cm[e], __shfl_xor_sync(kFull, cm[e], st));
+  if (riw == 0)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) smcm[warp * DK + lir * 16 + e] = cm[e];
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float m = smcm[lir * 16 + e];
+    for (int w2 = 1; w2 < kWarps; ++w2) m = max_nan(m, smcm[w2 * DK + lir * 16 + e]);
+    cm[e] = m;
+  }
+}
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyParams p) {
+  constexpr int LPR = DK / 16, RPW = 32 / LPR;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lir = lane % LPR, riw = lane / LPR, col0 = lir * 16;
+  const long long tile = blockIdx.x;
+  const int head = (int)(tile % p.H);
+  const long long b = tile / p.H;
+  const int bits = __ldg(p.head_bits + head);
+  const int rb = row_bytes(DK, bits);
+  uint8_t *gcodes = p.codes + b * p.seq_bytes + __ldg(p.head_off + head);
+  const bool load = p.S != nullptr;            // load_state: x is given, no update
+
+  uint8_t *scodes = smem + p.sm_codes;
+  float *sscales = reinterpret_cast<float *>(smem + p.sm_scales);
+  float *sk = reinterpret_cast<float *>(smem + p.sm_k);
+  float *sq = reinterpret_cast<float *>(smem + p.sm_q);
+  float *sa = reinterpret_cast<float *>(smem + p.sm_a);
+  float *sv = reinterpret_cast<float *>(smem + p.sm_v);
+  float *opart = reinterpret_cast<float *>(smem + p.sm_opart);
+  float *ow = reinterpret_cast<float *>(smem + p.sm_ow);
+  float *smcm = reinterpret_cast<float *>(smem + p.sm_cm);
+
+  if (!load) {
+    if (threadIdx.x == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      const unsigned cb = (unsigned)(p.d_v * rb), sb = bits == 32 ? 0u : DK * 4u;
+      const unsigned vec = DK * 4, vb = (unsigned)(p.d_v * 4);
+      mbar_expect_tx(bar, cb + sb + 2 * vec + vb + (p.diag ? vec : 0u));
+      bulk_g2s(scodes, gcodes, cb, bar);
+      if (sb) bulk_g2s(sscales, p.scales + tile * DK, sb, bar);
+      bulk_g2s(sk, p.k + tile * DK, vec, bar);
+      bulk_g2s(sq, p.q + tile * DK, vec, bar);
+      bulk_g2s(sv, p.v + tile * p.d_v, vb, bar);
+      if (p.diag) bulk_g2s(sa, p.alpha + tile * DK, vec, bar);
+    }
+    __syncthreads();
+    if (!__syncthreads_and(mbar_wait_bounded(bar, 0))) {
+      if (threadIdx.x == 0) {
+        atomicOr(p.flag, kFlagTimeout);
+        (void)mbar_wait_bounded(bar, 0);       // let the copies land before the CTA exits
+      }
+      return;
+    }
+  }
+  float kk[16], qq[16], aj[16];
+  const float alpha_s = (load || p.diag) ? 1.0f : __ldg(p.alpha + tile);
+  const float beta = load ? 0.0f : __ldg(p.beta + tile);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    kk[e] = load ? 0.0f : sk[col0 + e];
+    qq[e] = load ? 0.0f : sq[col0 + e];
+    const float al = load ? 1.0f : (p.diag ? sa[col0 + e] : alpha_s);
+    // entry (i, j) of S_{t-1} diag(alpha) is c_ij * (s_j * alpha_j)
+    aj[e] = (bits == 32 || load) ? al : __fmul_rn(sscales[col0 + e], al);
+  }
+  const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
+
+  // x of one row for this lane's 16 columns (pass 1 and pass 2 compute it identically).
+  // `first` (pass 1) computes w with warp shuffles: every lane of the warp takes it, and
+  // only lanes of real rows (`write`) keep w and the readout share.
+  auto row_x = [&](int lr, bool write, bool first, float (&x)[16]) {
+    if (load) {
+      const float *src = p.S + (tile * p.d_v + lr) * DK + col0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[e] = src[e];
+      return;
+    }
+    float sp[16];
+    if (bits == 32) {
+      const float *srow = reinterpret_cast<const float *>(scodes + (size_t)lr * rb) + col0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(srow[e], aj[e]);
+    } else {
+      float cf[16];
+      if (bits == 4)
+        unpack_i4(*reinterpret_cast<const uint2 *>(scodes + (size_t)lr * rb + lir * 8), cf);
+      else
+        unpack_i8(*reinterpret_cast<const uint4 *>(scodes + (size_t)lr * rb + lir * 16), cf);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(cf[e], aj[e]);
+    }
+    float w;
+    if (first) {
+      if (p.delta) {
+        float u = dot16_c4(sp, kk);
+#pragma unroll
+        for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
+        w = __fmul_rn(beta, __fsub_rn(sv[lr], u));
+      } else {
+        w = __fmul_rn(beta, sv[lr]);
+      }
+      const float opv = dot16_c4(sp, qq);
+      if (write) {
+        opart[lr * LPR + lir] = opv;
+        if (lir == 0) ow[lr] = w;
+      }
+    } else {
+      w = ow[lr];
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(w, kk[e], sp[e]);
+  };
+
+  // ---- pass 1: update every row, column maxima --------------------------------------
+  float cm[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) cm[e] = 0.0f;
+  bool bad32 = false;
+  const int nbase = warp * RPW;
+  for (int base = nbase; base < p.d_v; base += kWarps * RPW) {
+    const int lr = base + riw;
+    const bool active = lr < p.d_v;
+    float x[16];
+    row_x(active ? lr : 0, active, !load, x);
+    if (!active) continue;
+    if (bits == 32) {
+      float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * rb) + lir * 4;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) bad32 |= !isfinite(x[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) cm[e] = max_abs_nan(cm[e], x[e]);
+    }
+  }
+  if (bits != 32) {
+    column_max<DK>(cm, smcm);
+    const float r = (float)((1 << (bits - 1)) - 1);
+    const float inv_r = __fdiv_rn(1.0f, r);
+    float inv[16];
+    unsigned badcols = 0;                        // bit e: column col0 + e is bad
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const bool bad = !(cm[e] <= 0x1p100f);
+      const bool scaled = !bad && cm[e] >= 0x1p-100f;
+      inv[e] = scaled ? __fmul_rn(r, recip_nr(cm[e])) : 0.0f;
+      const float s = scaled ? __fmul_rn(cm[e], inv_r) : 0.0f;
+      badcols |= (bad ? 1u : 0u) << e;
+      if (warp == 0 && riw == 0) p.scales[tile * DK + col0 + e] = s;
+    }
+    if (badcols && warp == 0 && riw == 0) atomicOr(p.flag, kFlagNonFinite);
+    // byte masks that clear the codes of bad columns
+    uint32_t keep[4];
+#pragma unroll
+    for (int qd = 0; qd < 4; ++qd) {
+      keep[qd] = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        keep[qd] |= ((badcols >> (4 * qd + e)) & 1u) ? 0u : (0xFFu << (8 * e));
+    }
+    // ---- pass 2: recompute x, write codes ------------------------------------------------
+    for (int base = nbase; base < p.d_v; base += kWarps * RPW) {
+      const int lr = base + riw;
+      const bool active = lr < p.d_v;
+      float x[16];
+      row_x(active ? lr : 0, false, false, x);
+      const uint32_t cbase = tkey + 0x9E3779B9u * ((uint32_t)lr * (uint32_t)(DK / 4) + (uint32_t)lir * 4u + 1u);
+      uint32_t h[4] = {0u, 0u, 0u, 0u};
+      if (p.stochastic) dither_words(cbase, h);
+      uint32_t t[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float g = p.stochastic
+                            ? __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)))
+                            : 49152.5f;
+        t[e] = __float_as_uint(__fmaf_rn(x[e], inv[e], g));
+      }
+      if (!active) continue;
+      if (bits == 4) {
+        uint2 w = pack_i4(t);
+        // nibble masks: column e of the lane sits in word e/8, nibble e%8
+        uint32_t k0 = 0, k1 = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (!((badcols >> e) & 1u)) (e < 8 ? k0 : k1) |= 0xFu << (4 * (e & 7));
+        w.x &= k0;
+        w.y &= k1;
+        *reinterpret_cast<uint2 *>(gcodes + (size_t)lr * rb + lir * 8) = w;
+      } else {
+        uint4 w = pack_i8(t);
+        w.x &= keep[0]; w.y &= keep[1]; w.z &= keep[2]; w.w &= keep[3];
+        *reinterpret_cast<uint4 *>(gcodes + (size_t)lr * rb + lir * 16) = w;
+      }
+    }
+  } else if (__any_sync(kFull, bad32) && bad32) {
+    atomicOr(p.flag, kFlagNonFinite);
+  }
+  if (load) return;
+  // ---- readout: o_i = sum of the lane shares + w_i (k.q) --------------------------------
+  __syncthreads();
+  double kqd = 0.0;
+  for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sq[j], kqd);
+#pragma unroll
+  for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
+  const float kq = (float)kqd;
+  float *go = p.o + tile * p.d_v;
+  for (int r = threadIdx.x; r < p.d_v; r += kThreads) {
+    float acc = 0.0f;
+    for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
+    go[r] = __fmaf_rn(ow[r], kq, acc);
+  }
 }
 
 // -------------------------------------------------------------------------------------
@@ -559,6 +822,17 @@ static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
     case 64: return pick_step<64>(diag, delta, sr);
     case 128: return pick_step<128>(diag, delta, sr);
     case 256: return pick_step<256>(diag, delta, sr);
+  }
+  return nullptr;
+}
+using KeyFn = void (*)(const KeyParams);
+static KeyFn key_kernel_for(int dk) {
+  switch (dk) {
+    case 16: return decode_step_key_kernel<16>;
+    case 32: return decode_step_key_kernel<32>;
+    case 64: return decode_step_key_kernel<64>;
+    case 128: return decode_step_key_kernel<128>;
+    case 256: return decode_step_key_kernel<256>;
   }
   return nullptr;
 }
@@ -604,6 +878,11 @@ struct lores_handle {
   int smem = 0;
   StepParams sp{};
   StepFn step_fn = nullptr;
+  // key-axis grouping
+  int axis = 0;
+  KeyParams kp{};
+  KeyFn key_fn = nullptr;
+  int key_smem = 0;
   // staging for lores_decode_step_host
   float *stage_in = nullptr;
   float *stage_o = nullptr;
@@ -645,6 +924,12 @@ void free_all(lores_handle *h) {
   cudaFree(h->stage_o);
 }
 
+long long scale_count_of(const lores_handle *h) {
+  const lores_config &c = h->cfg;
+  return h->axis ? (long long)c.batch * c.heads * c.d_k
+                 : (long long)c.batch * c.heads * c.d_v * h->ng;
+}
+
 LoadParams load_params(const lores_handle *h) {
   LoadParams p{};
   p.codes = h->codes;
@@ -658,6 +943,7 @@ LoadParams load_params(const lores_handle *h) {
   p.ng = h->ng;
   p.G = h->G;
   p.stochastic = h->cfg.stochastic;
+  p.axis = h->axis;
   return p;
 }
 
@@ -710,6 +996,8 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
       (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
     return LORES_ERR_INVALID_ARG;
+  if (c.scale_axis != 0 && c.scale_axis != 1) return LORES_ERR_INVALID_ARG;
+  if (c.scale_axis == 1 && G != dk) return LORES_ERR_INVALID_ARG;   // one scale per column
   std::vector<int32_t> bits(c.heads, 8);
   if (c.head_bits)
     for (int h = 0; h < c.heads; ++h) {
@@ -733,6 +1021,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->bits = bits;
   h->G = G;
   h->ng = dk / G;
+  h->axis = c.scale_axis;
   h->head_off.resize(c.heads);
   long long off = 0;
   for (int hh = 0; hh < c.heads; ++hh) {
@@ -835,7 +1124,38 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->step_fn = fn;
 
   const long long code_bytes = (long long)c.batch * h->seq_bytes;
-  const long long scale_count = (long long)c.batch * c.heads * dv * h->ng;
+  const long long scale_count = scale_count_of(h);
+  if (h->axis) {
+    // key-axis kernel: one CTA per tile, the whole tile in shared memory
+    int rbmax = 0;
+    for (int hh = 0; hh < c.heads; ++hh) rbmax = std::max(rbmax, row_bytes(dk, bits[hh]));
+    auto up128 = [](int x) { return (x + 127) & ~127; };
+    KeyParams &kp = h->kp;
+    int off = 128;
+    kp.sm_codes = off; off += up128(dv * rbmax);
+    kp.sm_scales = off; off += up128(dk * 4);
+    kp.sm_k = off; off += up128(dk * 4);
+    kp.sm_q = off; off += up128(dk * 4);
+    kp.sm_a = off; off += up128(dk * 4);
+    kp.sm_v = off; off += up128(dv * 4);
+    kp.sm_opart = off; off += up128(dv * (dk / 16) * 4);
+    kp.sm_ow = off; off += up128(dv * 4);
+    kp.sm_cm = off; off += up128(kWarps * dk * 4);
+    h->key_smem = off;
+    h->key_fn = key_kernel_for(dk);
+    cudaFuncAttributes fa;
+    if (off > 200 * 1024) {
+      delete h;
+      return LORES_ERR_UNSUPPORTED;                 // tile too large for one CTA
+    }
+    if (cudaFuncGetAttributes(&fa, h->key_fn) != cudaSuccess ||
+        (fa.maxDynamicSharedSizeBytes < off &&
+         cudaFuncSetAttribute(h->key_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, off) !=
+             cudaSuccess)) {
+      delete h;
+      return LORES_ERR_CUDA;
+    }
+  }
   cudaError_t e = cudaSuccess;
   if (e == cudaSuccess) e = cudaMalloc(&h->codes, (size_t)code_bytes);
   if (e == cudaSuccess) e = cudaMalloc(&h->scales, (size_t)scale_count * 4);
@@ -873,6 +1193,18 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   p.ng = h->ng;
   p.G = G;
   p.units_per_seq = h->units_per_seq;
+  KeyParams &kp = h->kp;
+  kp.codes = h->codes;
+  kp.scales = h->scales;
+  kp.flag = h->flag;
+  kp.head_bits = h->d_bits;
+  kp.head_off = h->d_head_off;
+  kp.seq_bytes = h->seq_bytes;
+  kp.H = c.heads;
+  kp.d_v = dv;
+  kp.delta = c.delta;
+  kp.diag = c.decay_diag;
+  kp.stochastic = c.stochastic;
   *out = h;
   return LORES_OK;
 }
@@ -895,6 +1227,20 @@ lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, 
     return LORES_ERR_INVALID_ARG;
   DeviceGuard guard(h->cfg.device);
   if (!guard.ok) return LORES_ERR_CUDA;
+  if (h->axis) {
+    KeyParams kp = h->kp;
+    kp.q = q;
+    kp.k = k;
+    kp.v = v;
+    kp.alpha = alpha;
+    kp.beta = beta;
+    kp.o = o;
+    kp.S = nullptr;
+    kp.step_key = step_key_of(h->cfg.seed, step);
+    const unsigned tiles = (unsigned)((long long)h->cfg.batch * h->cfg.heads);
+    h->key_fn<<<tiles, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
+    return cuda_status(cudaGetLastError());
+  }
   StepParams p = h->sp;
   p.q = q;
   p.k = k;
@@ -955,6 +1301,14 @@ lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, vo
   if (!h || !S || !aligned16(S)) return LORES_ERR_INVALID_ARG;
   DeviceGuard guard(h->cfg.device);
   if (!guard.ok) return LORES_ERR_CUDA;
+  if (h->axis) {
+    KeyParams kp = h->kp;
+    kp.S = S;
+    kp.step_key = step_key_of(h->cfg.seed, step);
+    const unsigned tiles = (unsigned)((long long)h->cfg.batch * h->cfg.heads);
+    h->key_fn<<<tiles, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
+    return cuda_status(cudaGetLastError());
+  }
   LoadParams p = load_params(h);
   p.S = S;
   p.step_key = step_key_of(h->cfg.seed, step);
@@ -974,9 +1328,7 @@ lores_status lores_export_codes(lores_handle *h, void *codes, float *scales, voi
   if (codes)
     e = cudaMemcpyAsync(codes, h->codes, (size_t)h->cfg.batch * h->seq_bytes, cudaMemcpyDefault, s);
   if (e == cudaSuccess && scales)
-    e = cudaMemcpyAsync(scales, h->scales,
-                        (size_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng * 4,
-                        cudaMemcpyDefault, s);
+    e = cudaMemcpyAsync(scales, h->scales, (size_t)scale_count_of(h) * 4, cudaMemcpyDefault, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e);
 }
@@ -990,9 +1342,7 @@ lores_status lores_load_codes(lores_handle *h, const void *codes, const float *s
   cudaError_t e =
       cudaMemcpyAsync(h->codes, codes, (size_t)h->cfg.batch * h->seq_bytes, cudaMemcpyDefault, s);
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(h->scales, scales,
-                        (size_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng * 4,
-                        cudaMemcpyDefault, s);
+    e = cudaMemcpyAsync(h->scales, scales, (size_t)scale_count_of(h) * 4, cudaMemcpyDefault, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e);
 }
@@ -1001,8 +1351,8 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
   if (!h || !out) return LORES_ERR_INVALID_ARG;
   out->code_bytes = (int64_t)h->cfg.batch * h->seq_bytes;
   out->seq_code_bytes = h->seq_bytes;
-  out->scale_count = (int64_t)h->cfg.batch * h->cfg.heads * h->cfg.d_v * h->ng;
-  out->n_groups = h->ng;
+  out->scale_count = scale_count_of(h);
+  out->n_groups = h->axis ? 0 : h->ng;
   out->units_per_step = (int32_t)((long long)h->cfg.batch * h->units_per_seq);
   out->grid = h->grid;
   out->smem_bytes = h->smem;
@@ -1091,6 +1441,7 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
       (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
     return LORES_ERR_INVALID_ARG;
+  if (c.scale_axis != 0) return LORES_ERR_UNSUPPORTED;          // value-axis groups only
   for (int hh = 0; c.head_bits && hh < c.heads; ++hh)
     if (!((c.head_bits[hh] >= 4 && c.head_bits[hh] <= 8) || c.head_bits[hh] == 32))
       return LORES_ERR_INVALID_ARG;

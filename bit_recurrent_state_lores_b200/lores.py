@@ -31,7 +31,8 @@ class lores_config(C.Structure):
     _fields_ = [("batch", C.c_int32), ("heads", C.c_int32), ("d_k", C.c_int32),
                 ("d_v", C.c_int32), ("group_size", C.c_int32), ("delta", C.c_int32),
                 ("decay_diag", C.c_int32), ("head_bits", C.POINTER(C.c_int32)),
-                ("stochastic", C.c_int32), ("seed", C.c_uint64), ("device", C.c_int32)]
+                ("stochastic", C.c_int32), ("seed", C.c_uint64), ("device", C.c_int32),
+                ("scale_axis", C.c_int32)]
 
 
 class lores_layout(C.Structure):
@@ -102,14 +103,14 @@ def lores_status_string(status):
 
 
 def lores_create(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                 stochastic=1, seed=0, device=0):
+                 stochastic=1, seed=0, device=0, scale_axis=0):
     """Returns an opaque handle (int)."""
     hb = None
     if head_bits is not None:
         arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
         hb = C.cast(arr, C.POINTER(C.c_int32))
     cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
-                       seed & (2**64 - 1), device)
+                       seed & (2**64 - 1), device, scale_axis)
     out = C.c_void_p()
     _check(_lib.lores_create(C.byref(cfg), C.byref(out)), "lores_create")
     return out.value
@@ -142,7 +143,7 @@ def lores_decode_step_noalloc(cfg, codes, scales, q, k, v, alpha, beta, o, step,
 
 
 def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                stochastic=1, seed=0, device=0):
+                stochastic=1, seed=0, device=0, scale_axis=0):
     """A lores_config; the head_bits array is kept alive on the returned object."""
     hb = None
     arr = None
@@ -150,7 +151,7 @@ def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, hea
         arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
         hb = C.cast(arr, C.POINTER(C.c_int32))
     cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
-                       seed & (2**64 - 1), device)
+                       seed & (2**64 - 1), device, scale_axis)
     cfg._head_bits_keepalive = arr
     return cfg
 

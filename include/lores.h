@@ -70,14 +70,20 @@ typedef struct {
     int32_t stochastic;     /* 1: stochastic rounding (LoReS); 0: round to nearest           */
     uint64_t seed;          /* key of the rounding dither                                    */
     int32_t device;         /* CUDA device ordinal                                           */
+    int32_t scale_axis;     /* 0: value-axis groups (LoReS: one scale per value row, or per  */
+                            /* G key entries of a row); 1: key axis, one scale per key       */
+                            /* column of a tile (the comparator of the Scale Grouping        */
+                            /* paragraph; needs G = d_k; a whole tile is processed by one    */
+                            /* CTA, so d_v * d_k is limited by shared memory)                 */
 } lores_config;
 
 /* Sizes of the handle's state, for export/import buffers. */
 typedef struct {
     int64_t code_bytes;        /* bytes of the whole code pool = batch * seq_code_bytes      */
     int64_t seq_code_bytes;    /* bytes of one sequence: all heads' tiles back to back       */
-    int64_t scale_count;       /* fp32 scales: batch * heads * d_v * n_groups                */
-    int32_t n_groups;          /* d_k / G                                                    */
+    int64_t scale_count;       /* fp32 scales: batch * heads * d_v * n_groups (value axis)   */
+                               /* or batch * heads * d_k (key axis)                          */
+    int32_t n_groups;          /* d_k / G scales per value row; 0 in key-axis mode           */
     int32_t units_per_step;    /* work units (sequence, head, row block) of one step         */
     int32_t grid;              /* CTAs of the decode kernel                                  */
     int32_t smem_bytes;        /* dynamic shared memory per CTA of the decode kernel         */
@@ -149,8 +155,9 @@ lores_status lores_decode_step_host(lores_handle *h, const float *q, const float
  * no ordering between them) race on it.  The first call on each device looks up the
  * array's device address; make that first call before any stream capture.
  * Asynchronous on `stream` (the table upload from host memory may wait for the
- * stream's earlier work).  Errors: INVALID_ARG (shapes, NULL or misaligned pointers),
- * UNSUPPORTED (too many units, device ordinal >= 64), CUDA. */
+ * stream's earlier work).  Value-axis groups only.  Errors: INVALID_ARG (shapes, NULL
+ * or misaligned pointers), UNSUPPORTED (too many units, key-axis scales, device
+ * ordinal >= 64), CUDA. */
 lores_status lores_decode_step_noalloc(const lores_config *cfg, void *codes, float *scales,
                                        const float *q, const float *k, const float *v,
                                        const float *alpha, const float *beta, float *o,

@@ -99,7 +99,7 @@ class TileCfg:
     def zero_state(self):
         """(state, scales) of an all-zero tile."""
         if self.bits == 32:
-            return np.zeros((self.d_v, self.d_k), np.float32), np.zeros((self.d_v, self.n_groups), np.float32)
+            return np.zeros((self.d_v, self.d_k), np.float32), np.zeros(self.scale_shape(), np.float32)
         return (np.zeros(self.code_bytes(), np.uint8), np.zeros(self.scale_shape(), np.float32))
 
 

@@ -26,12 +26,15 @@ def mixed_bits(wl, hp):
 class GpuRun:
     """One handle of the library holding the state of one layer for a batch."""
 
-    def __init__(self, wl, head_bits, seed, stochastic=1, device=0):
+    def __init__(self, wl, head_bits, seed, stochastic=1, device=0, axis=0):
         L = lib()
-        self.wl, self.bits, self.seed = wl, list(head_bits), seed
-        self.h = L.lores_create(wl.B, wl.H, wl.d_k, wl.d_v, group_size=wl.group or 0,
+        self.wl, self.bits, self.seed, self.axis = wl, list(head_bits), seed, axis
+        self.stochastic = stochastic
+        self.h = L.lores_create(wl.B, wl.H, wl.d_k, wl.d_v,
+                                group_size=wl.d_k if axis else (wl.group or 0),
                                 delta=wl.delta, decay_diag=wl.diag, head_bits=head_bits,
-                                stochastic=stochastic, seed=seed, device=device)
+                                stochastic=stochastic, seed=seed, device=device,
+                                scale_axis=axis)
         self.layout, self.head_off = L.lores_get_layout(self.h, wl.H)
         self.o = torch.empty(wl.B, wl.H, wl.d_v, device="cuda", dtype=torch.float32)
 
@@ -45,8 +48,8 @@ class GpuRun:
         codes = torch.empty(self.layout.code_bytes, dtype=torch.uint8)
         scales = torch.empty(self.layout.scale_count, dtype=torch.float32)
         lib().lores_export_codes(self.h, codes, scales)
-        return (codes.numpy().reshape(wl.B, -1),
-                scales.numpy().reshape(wl.B, wl.H, wl.d_v, self.layout.n_groups))
+        shape = (wl.B, wl.H, wl.d_k) if self.axis else (wl.B, wl.H, wl.d_v, self.layout.n_groups)
+        return codes.numpy().reshape(wl.B, -1), scales.numpy().reshape(shape)
 
     def load(self, codes, scales):
         lib().lores_load_codes(self.h, np.ascontiguousarray(codes), np.ascontiguousarray(scales))
@@ -64,7 +67,7 @@ class GpuRun:
     def tile(self, codes, scales, b, hh):
         """(state, scales) of tile (b, hh) from an export, in the oracle's layout."""
         wl, bits = self.wl, self.bits[hh]
-        cfg = tile_cfg(wl, bits)
+        cfg = tile_cfg(wl, bits, axis=self.axis)
         off = self.head_off[hh]
         raw = codes[b, off:off + cfg.code_bytes()].copy()
         if bits == 32:
@@ -77,9 +80,9 @@ class GpuRun:
             self.h = None
 
 
-def tile_cfg(wl, bits, stochastic=1):
-    return O.TileCfg(wl.d_k, wl.d_v, group=wl.G, bits=bits, delta=wl.delta, diag=wl.diag,
-                     stochastic=stochastic)
+def tile_cfg(wl, bits, stochastic=1, axis=0):
+    return O.TileCfg(wl.d_k, wl.d_v, group=wl.d_k if axis else wl.G, bits=bits,
+                     delta=wl.delta, diag=wl.diag, stochastic=stochastic, axis=axis)
 
 
 def host_tile_inputs(inputs, tiles):
@@ -98,9 +101,9 @@ def host_tile_inputs(inputs, tiles):
 class OracleTiles:
     """The oracle's own trajectory for a few (b, h) tiles of a workload."""
 
-    def __init__(self, wl, head_bits, seed, tiles, stochastic=1):
+    def __init__(self, wl, head_bits, seed, tiles, stochastic=1, axis=0):
         self.wl, self.bits, self.seed, self.tiles = wl, list(head_bits), seed, list(tiles)
-        self.cfg = {t: tile_cfg(wl, self.bits[t[1]], stochastic) for t in self.tiles}
+        self.cfg = {t: tile_cfg(wl, self.bits[t[1]], stochastic, axis) for t in self.tiles}
         self.state = {t: self.cfg[t].zero_state() for t in self.tiles}
 
     def load(self, t, state, scales):
@@ -131,8 +134,12 @@ def compare_tile(cfg, gpu_state, gpu_scales, ref_state, ref_scales):
     cg = O.unpack_codes(cfg, gpu_state) if cfg.d_v * cfg.d_k <= 4096 else unpack_fast(cfg, gpu_state)
     cr = O.unpack_codes(cfg, ref_state) if cfg.d_v * cfg.d_k <= 4096 else unpack_fast(cfg, ref_state)
     d = np.abs(cg - cr)
-    Sg = cg * np.repeat(gpu_scales.astype(np.float64), cfg.group, axis=1)
-    Sr = cr * np.repeat(ref_scales.astype(np.float64), cfg.group, axis=1)
+    if cfg.axis:                                   # one scale per key column
+        Sg = cg * gpu_scales.astype(np.float64)[None, :]
+        Sr = cr * ref_scales.astype(np.float64)[None, :]
+    else:
+        Sg = cg * np.repeat(gpu_scales.astype(np.float64), cfg.group, axis=1)
+        Sr = cr * np.repeat(ref_scales.astype(np.float64), cfg.group, axis=1)
     return int((d != 0).sum()), int(d.max()), rel_l2(Sg, Sr), bool((gpu_scales == ref_scales).all())
 
 
