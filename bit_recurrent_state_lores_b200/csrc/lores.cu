@@ -133,18 +133,19 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
   const float *sq = reinterpret_cast<const float *>(stage + p.st_q);
   const float *sv = reinterpret_cast<const float *>(stage + p.st_v);
   const float *ss = reinterpret_cast<const float *>(stage + p.st_scales);
-  float kk[16], qq[16], aa[16];
+  // element pair e holds columns (col0 + 2e, col0 + 2e + 1)
+  float2 kk[8], qq[8], aa[8];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     const float4 k4 = *reinterpret_cast<const float4 *>(sk + col0 + 4 * c);
     const float4 q4 = *reinterpret_cast<const float4 *>(sq + col0 + 4 * c);
-    kk[4 * c] = k4.x; kk[4 * c + 1] = k4.y; kk[4 * c + 2] = k4.z; kk[4 * c + 3] = k4.w;
-    qq[4 * c] = q4.x; qq[4 * c + 1] = q4.y; qq[4 * c + 2] = q4.z; qq[4 * c + 3] = q4.w;
+    kk[2 * c] = make_float2(k4.x, k4.y); kk[2 * c + 1] = make_float2(k4.z, k4.w);
+    qq[2 * c] = make_float2(q4.x, q4.y); qq[2 * c + 1] = make_float2(q4.z, q4.w);
     if (DIAG) {
       const float4 a4 =
           *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(stage + p.st_a) +
                                             col0 + 4 * c);
-      aa[4 * c] = a4.x; aa[4 * c + 1] = a4.y; aa[4 * c + 2] = a4.z; aa[4 * c + 3] = a4.w;
+      aa[2 * c] = make_float2(a4.x, a4.y); aa[2 * c + 1] = make_float2(a4.z, a4.w);
     }
   }
   // k.q in double (strided columns, warp butterfly): the readout is o = S'q + w (k.q),
@@ -182,46 +183,47 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     if (SR && BITS != 32) dither_words(cbase0 + kCtrPerPass * (uint32_t)n, hw);
 
     // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
-    float sp[16];
+    float2 sp[8];
     if (BITS == 32) {
       const float *srow = reinterpret_cast<const float *>(stage + (size_t)lrr * RB) + col0;
+      const float2 as = dup2(alpha_s);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float4 s4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
-        const float sv4[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          sp[4 * c + e] = __fmul_rn(sv4[e], DIAG ? aa[4 * c + e] : alpha_s);
+        sp[2 * c] = __fmul2_rn(make_float2(s4.x, s4.y), DIAG ? aa[2 * c] : as);
+        sp[2 * c + 1] = __fmul2_rn(make_float2(s4.z, s4.w), DIAG ? aa[2 * c + 1] : as);
       }
     } else {
-      float cf[16];
+      float2 cf[8];
       if (BITS == 8)
-        unpack_i8(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
+        unpack_i8_2(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
       else
-        unpack_i4(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
+        unpack_i4_2(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
       const float s_in = ss[lrr * ng + g];
-      const float a_row = __fmul_rn(s_in, alpha_s);
+      const float2 s2 = dup2(s_in);
+      const float2 a_row = dup2(__fmul_rn(s_in, alpha_s));
 #pragma unroll
-      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(cf[e], DIAG ? __fmul_rn(s_in, aa[e]) : a_row);
+      for (int e = 0; e < 8; ++e) sp[e] = __fmul2_rn(cf[e], DIAG ? __fmul2_rn(s2, aa[e]) : a_row);
     }
 
     // ---- write: w = beta (v - delta (S'k)), x = S' + w k^T ----------------------------
     const float vr = sv[lrr];
     float w;
     if (DELTA) {
-      float u = dot16_c4(sp, kk);
+      float u = dot16_p(sp, kk);
 #pragma unroll
       for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
       w = __fmul_rn(beta, __fsub_rn(vr, u));
     } else {
       w = __fmul_rn(beta, vr);
     }
-    float x[16];
+    float2 x[8];
+    const float2 w2 = dup2(w);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(w, kk[e], sp[e]);
+    for (int e = 0; e < 8; ++e) x[e] = __ffma2_rn(w2, kk[e], sp[e]);
 
     // ---- readout share: this lane's part of S'q ----------------------------------------
-    const float opv = dot16_c4(sp, qq);
+    const float opv = dot16_p(sp, qq);
     if (active) {
       opart[lr * LPR + lir] = opv;
       if (lir == 0) ow[lr] = w;
@@ -232,13 +234,13 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t 
     if (BITS == 32) {
       float m = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) m = max_abs_nan(m, x[e]);
+      for (int e = 0; e < 8; ++e) m = max_abs_nan(max_abs_nan(m, x[e].x), x[e].y);
       gbad = !(m <= 3.402823466e38f);
       if (active) {
         float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          __stcs(dst + c, make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]));
+          __stcs(dst + c, make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y));
       }
     } else {
       uint32_t words[4];
@@ -664,14 +666,14 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
     float w;
     if (first) {
       if (p.delta) {
-        float u = dot16_c4(sp, kk);
+        float u = dot16_b(sp, kk);
 #pragma unroll
         for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
         w = __fmul_rn(beta, __fsub_rn(sv[lr], u));
       } else {
         w = __fmul_rn(beta, sv[lr]);
       }
-      const float opv = dot16_c4(sp, qq);
+      const float opv = dot16_b(sp, qq);
       if (write) {
         opart[lr * LPR + lir] = opv;
         if (lir == 0) ow[lr] = w;

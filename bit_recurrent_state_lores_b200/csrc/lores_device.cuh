@@ -3,8 +3,10 @@
 // Arithmetic of one state row, shared by the decode kernel and the state loader.
 // The element order and every fp32 rounding follow the state format definition:
 //   entry of S_{t-1} diag(alpha):   c_ij * (s_ig * alpha_j)
-//   u_i = (S'k)_i:                  4-column fma chains, combined pairwise with the nearest
-//                                   partner first (distance 1, 2, 4, ... in chunks)
+//   u_i = (S'k)_i:                  per 16-column block, four fma chains (half h, column
+//                                   parity p: columns 8h + p + 2m), summed as
+//                                   (c00 + c10) + (c01 + c11); block sums combined
+//                                   pairwise, nearest partner first (distance 1, 2, ...)
 //   w_i = beta (v_i - u_i)  [delta] or beta v_i;   x_ij = fma(w_i, k_j, S'_ij)
 //   requantize per group:           m = max|x|; y = Newton reciprocal of m; inv = r * y;
 //                                   s = m * fl(1/r); t = fma(x, inv, 49152 + d/256);
@@ -149,6 +151,38 @@ __device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
     halves_plus(__byte_perm(od, 0x64646464u, 0x7362u), -1032.0f, cc[5], cc[7]);
   }
 }
+// Paired forms: element pair e of a lane holds its columns (2e, 2e + 1), so packed
+// fp32x2 instructions (two independent fp32 operations, each rounded to nearest) work
+// on natural neighbours.
+__device__ __forceinline__ void unpack_i8_2(const uint4 &cw, float2 (&c)[8]) {
+  const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
+                         cw.w ^ 0x80808080u};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    halves_plus(__byte_perm(w[q], 0x64646464u, 0x5140u), -1152.0f, c[2 * q].x, c[2 * q].y);
+    halves_plus(__byte_perm(w[q], 0x64646464u, 0x7362u), -1152.0f, c[2 * q + 1].x,
+                c[2 * q + 1].y);
+  }
+}
+// int4: the low (even column) and high (odd column) nibbles of a byte are interleaved
+// into neighbouring bytes first, then dropped into fp16 pairs.
+__device__ __forceinline__ void unpack_i4_2(const uint2 &cw, float2 (&c)[8]) {
+  const uint32_t w[2] = {cw.x, cw.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t ev = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // columns 0, 2, 4, 6
+    const uint32_t od = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 1, 3, 5, 7
+    const uint32_t x0 = __byte_perm(ev, od, 0x5140u);                 // columns 0, 1, 2, 3
+    const uint32_t x1 = __byte_perm(ev, od, 0x7362u);                 // columns 4, 5, 6, 7
+    float2 *cc = c + 4 * h;
+    halves_plus(__byte_perm(x0, 0x64646464u, 0x5140u), -1032.0f, cc[0].x, cc[0].y);
+    halves_plus(__byte_perm(x0, 0x64646464u, 0x7362u), -1032.0f, cc[1].x, cc[1].y);
+    halves_plus(__byte_perm(x1, 0x64646464u, 0x5140u), -1032.0f, cc[2].x, cc[2].y);
+    halves_plus(__byte_perm(x1, 0x64646464u, 0x7362u), -1032.0f, cc[3].x, cc[3].y);
+  }
+}
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+
 // t holds 49152 + code + frac in fp32: its byte 1 is the code (two's complement).
 __device__ __forceinline__ uint4 pack_i8(const uint32_t (&t)[16]) {
   uint32_t w[4];
@@ -178,18 +212,32 @@ __device__ __forceinline__ uint2 pack_i4(const uint32_t (&t)[16]) {
 // -------------------------------------------------------------------------------------
 // reductions over the lane's 16 entries
 // -------------------------------------------------------------------------------------
-// sum_e a_e b_e over the lane's 16 columns in the fixed order: four 4-column fma chains,
-// then (c0 + c1) + (c2 + c3).  Chunk c of the lane is columns 4c .. 4c+3.
-__device__ __forceinline__ float dot16_c4(const float (&a)[16], const float (&b)[16]) {
-  float p[4];
+// sum_e a_e b_e over the lane's 16 columns in the fixed order: four fma chains from zero,
+// chain (h, p) over columns 8h + p + 2m, m = 0..3 ascending (h: half of the 16, p: column
+// parity); the lane's sum is (chain(0,0) + chain(1,0)) + (chain(0,1) + chain(1,1)).
+// Paired form: chains (h, 0) and (h, 1) run side by side in one packed fma.
+__device__ __forceinline__ float dot16_p(const float2 (&a)[8], const float2 (&b)[8]) {
+  float2 lo = make_float2(0.0f, 0.0f), hi = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    float acc = 0.0f;
+  for (int e = 0; e < 4; ++e) lo = __ffma2_rn(a[e], b[e], lo);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc = __fmaf_rn(a[4 * c + e], b[4 * c + e], acc);
-    p[c] = acc;
-  }
-  return __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
+  for (int e = 4; e < 8; ++e) hi = __ffma2_rn(a[e], b[e], hi);
+  const float2 s = __fadd2_rn(lo, hi);
+  return __fadd_rn(s.x, s.y);
+}
+// The same order with scalar operations.
+__device__ __forceinline__ float dot16_b(const float (&a)[16], const float (&b)[16]) {
+  float ch[2][2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc = __fmaf_rn(a[8 * h + p + 2 * m], b[8 * h + p + 2 * m], acc);
+      ch[h][p] = acc;
+    }
+  return __fadd_rn(__fadd_rn(ch[0][0], ch[1][0]), __fadd_rn(ch[0][1], ch[1][1]));
 }
 
 // Newton-Raphson reciprocal of m in [2^-100, 2^100]: seed by reflecting the exponent
@@ -228,15 +276,15 @@ __device__ __forceinline__ void dither_words(uint32_t cbase, uint32_t (&h)[4]) {
 // r = 2^(b-1) - 1 of the unit's codes and inv_r = fl(1/r); BITS is the storage (8: one
 // byte per code, for 5- to 8-bit codes; 4: nibbles).
 template <int LPR, int BITS, bool SR>
-__device__ __forceinline__ bool requantize16_nb(const float (&x)[16], float r, float inv_r,
+__device__ __forceinline__ bool requantize16_nb(const float2 (&x)[8], float r, float inv_r,
                                                 int gd1, int gd2, int gd4, int gd8,
                                                 const uint32_t (&h)[4], uint32_t (&words)[4],
                                                 float &s_out) {
   float mq[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
-    mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[4 * c]), x[4 * c + 1]), x[4 * c + 2]),
-                        x[4 * c + 3]);
+    mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[2 * c].x), x[2 * c].y), x[2 * c + 1].x),
+                        x[2 * c + 1].y);
   float m = max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
   // group max over the lanes of the group: a level at or beyond the group width has
   // shuffle distance 0 (the lane's own value)
@@ -246,18 +294,20 @@ __device__ __forceinline__ bool requantize16_nb(const float (&x)[16], float r, f
   const bool gbad = !(m <= 0x1p100f);                    // inf, NaN or overflow
   const bool scaled = m >= 0x1p-100f && !gbad;           // below 2^-100: zero group
   const float y = recip_nr(scaled ? m : 1.0f);
-  const float inv = scaled ? __fmul_rn(r, y) : 0.0f;
+  const float2 inv = dup2(scaled ? __fmul_rn(r, y) : 0.0f);
   s_out = scaled ? __fmul_rn(m, inv_r) : 0.0f;
   uint32_t t[16];
-  if (SR) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float g = __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)));
-      t[e] = __float_as_uint(__fmaf_rn(x[e], inv, g));
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, 49152.5f));
+  for (int e = 0; e < 8; ++e) {
+    // addend 49152 + d/256 with d = byte (j mod 4) of the quad's hash word
+    const float2 g =
+        SR ? make_float2(
+                 __uint_as_float(__byte_perm(h[e >> 1], 0x47400000u, 0x7650u | ((2 * e) & 3))),
+                 __uint_as_float(__byte_perm(h[e >> 1], 0x47400000u, 0x7650u | ((2 * e + 1) & 3))))
+           : dup2(49152.5f);
+    const float2 tt = __ffma2_rn(x[e], inv, g);
+    t[2 * e] = __float_as_uint(tt.x);
+    t[2 * e + 1] = __float_as_uint(tt.y);
   }
   if (BITS == 8) {
     const uint4 w = pack_i8(t);

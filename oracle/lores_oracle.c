@@ -25,8 +25,9 @@
  *     in fp32, w in fp32) evaluated exactly, i.e. before requantization and before
  *     the fp32 rounding of the stored entries.
  *   - Products and sums are fp32 with the association written below; the
- *     dot product S'k uses a fixed order (4-column sequential chunks, then a
- *     pairwise combine of the chunk sums, nearest partners first) so that two
+ *     dot product S'k uses a fixed order (16-column blocks, four interleaved
+ *     sequential chains per block by half and column parity, then a pairwise
+ *     combine of the block sums, nearest partners first) so that two
  *     implementations that follow it agree bit for bit.  The readout is summed
  *     in double.
  *   - Scale and its inverse: s = m * fl(1/r); inv = r * y, where y ~ 1/m comes
@@ -152,23 +153,33 @@ void lo_put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code) { put_
 /* Fixed-order dot product                                                  */
 /* ------------------------------------------------------------------------ */
 
-/* sum_j a_j b_j for n = 4*C, C a power of two <= 64: each chunk of 4
- * consecutive terms is a sequential fma chain from zero; the C chunk sums are
- * then combined pairwise, partner at distance 1, then 2, 4, ..., C/2. */
-float lo_dot_c4(const float *a, const float *b, int n)
+/* sum_j a_j b_j for n = 16*L, L a power of two <= 16.  The row is cut into L
+ * blocks of 16 consecutive columns.  In block l, chain (h, p) (h = 0, 1 the
+ * half of the block, p = 0, 1 the column parity) is a sequential fma chain from
+ * zero over columns 16l + 8h + p + 2m, m = 0..3 ascending; the block sum is
+ * (chain(0,0) + chain(1,0)) + (chain(0,1) + chain(1,1)).  The L block sums are
+ * then combined pairwise, partner at distance 1, then 2, 4, ..., L/2. */
+float lo_dot_b16(const float *a, const float *b, int n)
 {
-    float p[64], nxt[64];
-    int C = n / 4;
-    for (int c = 0; c < C; c++) {
-        float acc = 0.0f;
-        for (int e = 0; e < 4; e++)
-            acc = fmaf(a[4 * c + e], b[4 * c + e], acc);
-        p[c] = acc;
+    float p[16], nxt[16];
+    int L = n / 16;
+    for (int l = 0; l < L; l++) {
+        float ch[2][2];
+        for (int h = 0; h < 2; h++)
+            for (int par = 0; par < 2; par++) {
+                float acc = 0.0f;
+                for (int m = 0; m < 4; m++) {
+                    int j = 16 * l + 8 * h + par + 2 * m;
+                    acc = fmaf(a[j], b[j], acc);
+                }
+                ch[h][par] = acc;
+            }
+        p[l] = (ch[0][0] + ch[1][0]) + (ch[0][1] + ch[1][1]);
     }
-    for (int stride = 1; stride < C; stride *= 2) {
-        for (int l = 0; l < C; l++)
+    for (int stride = 1; stride < L; stride *= 2) {
+        for (int l = 0; l < L; l++)
             nxt[l] = p[l] + p[l ^ stride];
-        memcpy(p, nxt, sizeof(float) * C);
+        memcpy(p, nxt, sizeof(float) * L);
     }
     return p[0];
 }
@@ -312,7 +323,7 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
         /* write: w_i = beta (v_i - delta u_i), u_i = (S' k)_i */
         float w;
         if (c->delta) {
-            float u = lo_dot_c4(Sp, k, dk);
+            float u = lo_dot_b16(Sp, k, dk);
             w = beta * (v[i] - u);
         } else {
             w = beta * v[i];

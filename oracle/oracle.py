@@ -37,8 +37,8 @@ def lib():
         L.lo_tile_key.argtypes = [C.c_uint32, C.c_uint32]
         L.lo_dither.restype = C.c_uint32
         L.lo_dither.argtypes = [C.c_uint32, C.c_int, C.c_int, C.c_int]
-        L.lo_dot_c4.restype = C.c_float
-        L.lo_dot_c4.argtypes = [C.c_void_p, C.c_void_p, C.c_int]
+        L.lo_dot_b16.restype = C.c_float
+        L.lo_dot_b16.argtypes = [C.c_void_p, C.c_void_p, C.c_int]
         L.lo_recip_nr.restype = C.c_float
         L.lo_recip_nr.argtypes = [C.c_float]
         L.lo_get_code.restype = C.c_int
@@ -125,9 +125,9 @@ def dither(tkey, d_k, i, j):
     return int(lib().lo_dither(tkey, d_k, i, j))
 
 
-def dot_c4(a, b):
+def dot_b16(a, b):
     a, b = _f32(a), _f32(b)
-    return float(lib().lo_dot_c4(_p(a), _p(b), a.size))
+    return float(lib().lo_dot_b16(_p(a), _p(b), a.size))
 
 
 def recip_nr(m):

@@ -118,7 +118,7 @@ def test_dot_exact_on_integers():
     for n in (16, 32, 64, 128, 256):
         a = g.integers(-50, 50, n).astype(np.float32)
         b = g.integers(-50, 50, n).astype(np.float32)
-        assert O.dot_c4(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
+        assert O.dot_b16(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
 
 
 def test_dot_error_bound():
@@ -130,18 +130,38 @@ def test_dot_error_bound():
         exact = sum(Fraction(float(x)) * Fraction(float(y)) for x, y in zip(a, b))
         u = 2.0 ** -24
         bound = n * u / (1 - n * u) * float(np.sum(np.abs(a.astype(np.float64) * b)))
-        assert abs(float(Fraction(O.dot_c4(a, b)) - exact)) <= bound
+        assert abs(float(Fraction(O.dot_b16(a, b)) - exact)) <= bound
 
 
 def test_dot_combine_order_worked_example():
-    # Chunk sums p = [1, 2^24, 1, -2^24] (one nonzero term per 4-column chunk).
+    # Block sums p = [1, 2^24, 1, -2^24] (one nonzero term per 16-column block).
     # Nearest partner first: [p0+p1, p2+p3] = [2^24 (the 1 is lost: tie to even),
     # 1 - 2^24 (exact)], then 2^24 + (1 - 2^24) = 1.  (Left to right would give 0;
     # the far partner first would give [p0+p2, p1+p3] = [2, 0] -> 2.)
-    a = np.zeros(16, np.float32)
+    a = np.zeros(64, np.float32)
+    b = np.ones(64, np.float32)
+    a[0], a[16], a[32], a[48] = 1.0, 2.0 ** 24, 1.0, -(2.0 ** 24)
+    assert O.dot_b16(a, b) == 1.0
+
+
+def test_dot_block_chains_worked_examples():
     b = np.ones(16, np.float32)
-    a[0], a[4], a[8], a[12] = 1.0, 2.0 ** 24, 1.0, -(2.0 ** 24)
-    assert O.dot_c4(a, b) == 1.0
+    # Chains by half and parity: c00 = col 0, c10 = col 8, c01 = col 1, c11 = col 9.
+    # (c00 + c10) + (c01 + c11) = (1 + 2^24 -> 2^24) + (1 - 2^24) = 1; pairing by
+    # parity first, (c00 + c01) + (c10 + c11), would give 2 + 0 = 2.
+    a = np.zeros(16, np.float32)
+    a[0], a[8], a[1], a[9] = 1.0, 2.0 ** 24, 1.0, -(2.0 ** 24)
+    assert O.dot_b16(a, b) == 1.0
+    # Columns 1 and 3 share chain (0, 1), away from column 0: 2^24 + (1 + 1) = 2^24 + 2
+    # exactly; one chain over columns 0..3 would lose both ones (2^24 + 1 -> 2^24).
+    a = np.zeros(16, np.float32)
+    a[0], a[1], a[3] = 2.0 ** 24, 1.0, 1.0
+    assert O.dot_b16(a, b) == 2.0 ** 24 + 2
+    # Inside a chain the order is ascending: 2^24 at column 0 absorbs the ones at
+    # columns 2 and 4 one at a time (ties to even); descending would give 2^24 + 2.
+    a = np.zeros(16, np.float32)
+    a[0], a[2], a[4] = 2.0 ** 24, 1.0, 1.0
+    assert O.dot_b16(a, b) == 2.0 ** 24
 
 
 def test_newton_reciprocal_error_bound():
