@@ -97,7 +97,7 @@ def launch_bytes(wl, bits):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("lores.cu", "lores_device.cuh"):
+    for f in ("lores.cu", "lores_mt.cu", "lores_step.cuh", "lores_device.cuh"):
         h.update(open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

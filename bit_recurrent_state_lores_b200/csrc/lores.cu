@@ -27,401 +27,9 @@
 
 #include "lores.h"
 #include "lores_device.cuh"
+#include "lores_step.cuh"
 
 namespace lores {
-
-// One work unit: a block of rows of one (sequence, head) tile, processed by one warp.
-struct __align__(16) UnitDesc {
-  int32_t head;
-  int32_t row0;
-  int32_t nrows;
-  int32_t bits;          // 4..8 (b-bit codes) or 32 (fp32 state)
-  int64_t code_off;      // byte offset of row0 of this head inside one sequence's block
-  float r;               // largest code, 2^(bits-1) - 1
-  float inv_r;           // fl(1/r)
-};
-
-struct StepParams {
-  uint8_t *codes;        // [B][seq_bytes]
-  float *scales;         // [B][H][d_v][ng]
-  const float *q, *k, *v, *alpha, *beta;
-  float *o;
-  unsigned *flag;
-  const UnitDesc *units; // [units_per_seq]
-  long long seq_bytes;
-  long long total_units;
-  int B, H, d_v, ng, G, units_per_seq;
-  uint32_t step_key;
-  // shared memory layout: [unit table][warp 0 area][warp 1 area]...; a warp area is
-  // [2 mbarriers | pad to 64][readout partials][row w][stage 0][stage 1]
-  int table_bytes;       // bytes of the unit table copy (0: read the table from global)
-  int warp_bytes;        // bytes of one warp area
-  int opart_floats;      // readout partials per warp (max rows * lanes per row)
-  int ow_floats;         // row w per warp (max rows)
-  int st_scales, st_k, st_q, st_v, st_a, stage_bytes;   // stage layout
-};
-
-// Storage of b-bit codes: 4-bit codes as nibbles, 5- to 8-bit codes one per byte.
-__host__ __device__ constexpr int storage_bits(int bits) {
-  return bits == 4 ? 4 : (bits == 32 ? 32 : 8);
-}
-// Bytes of one row of a tile with `bits`-bit entries.
-__host__ __device__ constexpr int row_bytes(int dk, int bits) { return dk * storage_bits(bits) / 8; }
-
-// Rows of a full unit: 4 KB of state, a whole number of warp passes (32/(d_k/16) rows).
-__host__ __device__ constexpr int full_rows(int dk, int bits) {
-  return (4096 / row_bytes(dk, bits)) < (32 / (dk / 16))
-             ? (32 / (dk / 16))
-             : (4096 / row_bytes(dk, bits)) - (4096 / row_bytes(dk, bits)) % (32 / (dk / 16));
-}
-
-// -------------------------------------------------------------------------------------
-// producer (the whole warp): stage one unit's inputs into the warp's ring slot
-// -------------------------------------------------------------------------------------
-// Lane 0 announces the byte count on the slot's mbarrier; then lanes 0-5 each issue one
-// of the unit's bulk copies (codes, scales, k, q, v slice, per-column alpha) in parallel.
-template <int DK, bool DIAG>
-__device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *tbl, int b, int ub,
-                                           uint8_t *stage, uint64_t *bar) {
-  const int lane = threadIdx.x & 31;
-  const UnitDesc d = tbl[ub];
-  const long long tile = (long long)b * p.H + d.head;
-  const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
-  const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
-  const unsigned vbytes = (unsigned)(d.nrows * 4);
-  const unsigned vec = DK * 4;
-  if (lane == 0) mbar_expect_tx(bar, cbytes + sbytes + vbytes + 2 * vec + (DIAG ? vec : 0));
-  __syncwarp();
-  const void *src = nullptr;
-  int dst = 0;
-  unsigned bytes = 0;
-  if (lane == 0) { src = p.codes + (long long)b * p.seq_bytes + d.code_off; dst = 0; bytes = cbytes; }
-  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; }
-  if (lane == 2) { src = p.k + tile * DK; dst = p.st_k; bytes = vec; }
-  if (lane == 3) { src = p.q + tile * DK; dst = p.st_q; bytes = vec; }
-  if (lane == 4) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
-  if (DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = vec; }
-  if (bytes) bulk_g2s(stage + dst, src, bytes, bar);
-}
-
-// -------------------------------------------------------------------------------------
-// consumer (the whole warp): rows [row0, row0 + nrows) of one tile from a stage
-// -------------------------------------------------------------------------------------
-// Lane layout: LPR = d_k/16 lanes own a row, 16 consecutive columns each; a warp pass
-// covers RPW = 32/LPR rows.  FULL: every pass is complete (nrows % RPW == 0).
-// The readout is reduced per warp: each lane leaves its share of S'q in opart, lane 0
-// of the row leaves w in ow, and after the rows each lane forms o for one row as
-// sum(opart) + w (k.q).
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL, bool GROW>
-__device__ __forceinline__ void compute_unit(const StepParams &p, const uint8_t *stage, int b,
-                                             const UnitDesc &d, float alpha_s, float beta,
-                                             float *opart, float *ow) {
-  constexpr int LPR = DK / 16;            // lanes per row
-  constexpr int RPW = 32 / LPR;           // rows per warp pass
-  constexpr int RB = DK * BITS / 8;       // bytes per row
-  const int lane = threadIdx.x & 31;
-  const int lir = lane % LPR, riw = lane / LPR;
-  const int col0 = lir * 16;
-  // GROW: one scale per value row (G = d_k), known at compile time
-  const int lpg = GROW ? LPR : p.G / 16;                   // lanes per scale group (power of 2)
-  const int g = GROW ? 0 : lir / lpg;                      // this lane's group in the row
-  const bool scale_writer = (lir & (lpg - 1)) == 0;
-  const int ng = GROW ? 1 : p.ng;
-  const long long tile = (long long)b * p.H + d.head;
-
-  const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
-  const float *sq = reinterpret_cast<const float *>(stage + p.st_q);
-  const float *sv = reinterpret_cast<const float *>(stage + p.st_v);
-  const float *ss = reinterpret_cast<const float *>(stage + p.st_scales);
-  // element pair e holds columns (col0 + 2e, col0 + 2e + 1)
-  float2 kk[8], qq[8], aa[8];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float4 k4 = *reinterpret_cast<const float4 *>(sk + col0 + 4 * c);
-    const float4 q4 = *reinterpret_cast<const float4 *>(sq + col0 + 4 * c);
-    kk[2 * c] = make_float2(k4.x, k4.y); kk[2 * c + 1] = make_float2(k4.z, k4.w);
-    qq[2 * c] = make_float2(q4.x, q4.y); qq[2 * c + 1] = make_float2(q4.z, q4.w);
-    if (DIAG) {
-      const float4 a4 =
-          *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(stage + p.st_a) +
-                                            col0 + 4 * c);
-      aa[2 * c] = make_float2(a4.x, a4.y); aa[2 * c + 1] = make_float2(a4.z, a4.w);
-    }
-  }
-  // k.q in double (strided columns, warp butterfly): the readout is o = S'q + w (k.q),
-  // which keeps the step-0 readout (S' = 0) exact even for nearly orthogonal k and q.
-  double kqd = 0.0;
-#pragma unroll
-  for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sq[j], kqd);
-#pragma unroll
-  for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
-  const float kq = (float)kqd;
-  const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
-  // shuffle distances of the group-max levels (0 beyond the group width: own value)
-  const int gd1 = 1 < lpg ? 1 : 0, gd2 = 2 < lpg ? 2 : 0, gd4 = 4 < lpg ? 4 : 0,
-            gd8 = 8 < lpg ? 8 : 0;
-
-  uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
-  float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
-  constexpr int kFullPasses = full_rows(DK, BITS) / RPW;
-  const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
-  // dither counter of the lane's first quad in pass 0: n0 = (row0 + riw) d_k/4 + 4 lir;
-  // each pass moves RPW rows, i.e. RPW d_k/4 quads
-  const uint32_t cbase0 =
-      tkey + 0x9E3779B9u * ((uint32_t)(d.row0 + riw) * (uint32_t)(DK / 4) + (uint32_t)lir * 4u + 1u);
-  constexpr uint32_t kCtrPerPass = 0x9E3779B9u * (uint32_t)(RPW * DK / 4);
-  uint32_t badmask = 0;                        // bit n: this lane's group was bad in pass n
-
-#pragma unroll(FULL ? 4 : 1)
-  for (int n = 0; n < npass; ++n) {
-    const int lr = n * RPW + riw;              // row inside the unit
-    const bool active = FULL || lr < d.nrows;
-    const int lrr = active ? lr : 0;           // keep shared loads in bounds
-    // dither words first: they depend only on the counter, so they fill the latency of
-    // the dot-product and group-max shuffles below
-    uint32_t hw[4] = {0u, 0u, 0u, 0u};
-    if (SR && BITS != 32) dither_words(cbase0 + kCtrPerPass * (uint32_t)n, hw);
-
-    // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
-    float2 sp[8];
-    if (BITS == 32) {
-      const float *srow = reinterpret_cast<const float *>(stage + (size_t)lrr * RB) + col0;
-      const float2 as = dup2(alpha_s);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float4 s4 = *reinterpret_cast<const float4 *>(srow + 4 * c);
-        sp[2 * c] = __fmul2_rn(make_float2(s4.x, s4.y), DIAG ? aa[2 * c] : as);
-        sp[2 * c + 1] = __fmul2_rn(make_float2(s4.z, s4.w), DIAG ? aa[2 * c + 1] : as);
-      }
-    } else {
-      float2 cf[8];
-      if (BITS == 8)
-        unpack_i8_2(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
-      else
-        unpack_i4_2(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
-      const float s_in = ss[lrr * ng + g];
-      const float2 s2 = dup2(s_in);
-      const float2 a_row = dup2(__fmul_rn(s_in, alpha_s));
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sp[e] = __fmul2_rn(cf[e], DIAG ? __fmul2_rn(s2, aa[e]) : a_row);
-    }
-
-    // ---- write: w = beta (v - delta (S'k)), x = S' + w k^T ----------------------------
-    const float vr = sv[lrr];
-    float w;
-    if (DELTA) {
-      float u = dot16_p(sp, kk);
-#pragma unroll
-      for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
-      w = __fmul_rn(beta, __fsub_rn(vr, u));
-    } else {
-      w = __fmul_rn(beta, vr);
-    }
-    float2 x[8];
-    const float2 w2 = dup2(w);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = __ffma2_rn(w2, kk[e], sp[e]);
-
-    // ---- readout share: this lane's part of S'q ----------------------------------------
-    const float opv = dot16_p(sp, qq);
-    if (active) {
-      opart[lr * LPR + lir] = opv;
-      if (lir == 0) ow[lr] = w;
-    }
-
-    // ---- requantize and store (bad rows are fixed up after the passes) ------------------
-    bool gbad;
-    if (BITS == 32) {
-      float m = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m = max_abs_nan(max_abs_nan(m, x[e].x), x[e].y);
-      gbad = !(m <= 3.402823466e38f);
-      if (active) {
-        float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          __stcs(dst + c, make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y));
-      }
-    } else {
-      uint32_t words[4];
-      float s_new;
-      gbad = requantize16_nb<LPR, BITS, SR>(x, d.r, d.inv_r, gd1, gd2, gd4, gd8, hw, words, s_new);
-      if (active) {
-        if (BITS == 8)
-          __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
-                 make_uint4(words[0], words[1], words[2], words[3]));
-        else
-          __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8),
-                 make_uint2(words[0], words[1]));
-        if (scale_writer) gscales[lr * ng + g] = s_new;
-      }
-    }
-    badmask |= (gbad && active ? 1u : 0u) << n;
-  }
-
-  // ---- rare: rows with a non-finite (or overflowing) entry -----------------------------
-  // A row is bad if any of its groups is; quantized rows are stored as zero.  The lane
-  // that wrote a word rewrites it, so no ordering between lanes is needed.
-  if (__any_sync(kFull, badmask != 0u)) {
-    const unsigned rowmask = (LPR == 32 ? kFull : ((1u << LPR) - 1u)) << (riw * LPR);
-    for (int n = 0; n < npass; ++n) {
-      const unsigned bal = __ballot_sync(kFull, (badmask >> n) & 1u);
-      const int lr = n * RPW + riw;
-      if ((bal & rowmask) == 0u || !(FULL || lr < d.nrows)) continue;
-      if (BITS != 32) {
-        if (BITS == 8)
-          __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16), make_uint4(0, 0, 0, 0));
-        else
-          __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8), make_uint2(0, 0));
-        if (scale_writer) gscales[lr * ng + g] = 0.0f;
-      }
-      if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
-    }
-  }
-
-  // ---- readout: o_i = sum of the row's lane shares + w_i (k.q) -------------------------
-  __syncwarp();
-  float *go = p.o + tile * p.d_v + d.row0;
-  for (int r = lane; r < d.nrows; r += 32) {
-    float acc = 0.0f;
-    if (LPR >= 4) {
-#pragma unroll
-      for (int l = 0; l < LPR; l += 4) {
-        const float4 v4 = *reinterpret_cast<const float4 *>(opart + r * LPR + l);
-        acc = __fadd_rn(__fadd_rn(__fadd_rn(__fadd_rn(acc, v4.x), v4.y), v4.z), v4.w);
-      }
-    } else {
-#pragma unroll
-      for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
-    }
-    go[r] = __fmaf_rn(ow[r], kq, acc);
-  }
-  __syncwarp();
-}
-
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS>
-__device__ __forceinline__ void compute_any(const StepParams &p, const uint8_t *stage, int b,
-                                            const UnitDesc &d, float alpha_s, float beta,
-                                            float *opart, float *ow) {
-  if (d.nrows == full_rows(DK, BITS)) {
-    if (p.G == DK)
-      compute_unit<DK, DIAG, DELTA, SR, BITS, true, true>(p, stage, b, d, alpha_s, beta, opart, ow);
-    else
-      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false>(p, stage, b, d, alpha_s, beta, opart, ow);
-  } else {
-    compute_unit<DK, DIAG, DELTA, SR, BITS, false, false>(p, stage, b, d, alpha_s, beta, opart, ow);
-  }
-}
-
-// Position of a unit: global unit u = ub * B + b (sequence b is the fast index, so a warp
-// striding through units visits the per-sequence unit table in order, and a table sorted
-// by bit width keeps each warp on one code path for long runs), advanced by a fixed
-// stride without divisions.
-struct UnitPos {
-  int b, ub;
-  __device__ __forceinline__ void advance(int sb, int su, int B) {
-    b += sb;
-    ub += su;
-    if (b >= B) {
-      b -= B;
-      ++ub;
-    }
-  }
-};
-
-// Persistent kernel: every warp runs its own pipeline over units gw, gw + W, gw + 2W, ...
-// (gw = global warp index, W = warps in the grid), with a 2-slot ring of bulk copies
-// whose producer is the warp's lane 0.  Warps never wait on one another.
-template <int DK, bool DIAG, bool DELTA, bool SR>
-__global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  UnitDesc *stbl = reinterpret_cast<UnitDesc *>(smem);
-  uint8_t *wa = smem + p.table_bytes + warp * p.warp_bytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(wa);
-  float *opart = reinterpret_cast<float *>(wa + 64);
-  float *ow = opart + p.opart_floats;
-  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
-
-  const UnitDesc *tbl = p.units;
-  const int ups = p.units_per_seq;
-  if (p.table_bytes) {
-    for (int i = threadIdx.x; i < ups; i += kThreads) stbl[i] = p.units[i];
-    tbl = stbl;
-  }
-  __syncthreads();                                  // the only CTA-wide barrier
-
-  const long long first = (long long)blockIdx.x * kWarps + warp;
-  if (first >= p.total_units) return;
-  const long long stride = (long long)gridDim.x * kWarps;
-  const int B = p.B;
-  const int sb = (int)(stride % B), su = (int)(stride / B);
-  UnitPos cur{(int)(first % B), (int)(first / B)};
-
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-  {
-    UnitPos q = cur;
-    for (int s = 0; s < kStages && q.ub < ups; ++s) {
-      issue_unit<DK, DIAG>(p, tbl, q.b, q.ub, stages + s * p.stage_bytes, &bars[s]);
-      q.advance(sb, su, B);
-    }
-  }
-  UnitPos nxt = cur;                                // the unit after `cur`
-  nxt.advance(sb, su, B);
-  UnitPos fill = nxt;                               // the unit that refills the slot just used
-  fill.advance(sb, su, B);
-
-  // per-tile scalars of the current unit; the next unit's are loaded one unit ahead
-  float alpha_cur = 0.0f, beta_cur;
-  {
-    const long long t0 = (long long)cur.b * p.H + tbl[cur.ub].head;
-    beta_cur = __ldg(p.beta + t0);
-    if (!DIAG) alpha_cur = __ldg(p.alpha + t0);
-  }
-
-  for (int n = 0; cur.ub < ups; ++n) {
-    const int s = n % kStages;
-    uint8_t *stage = stages + s * p.stage_bytes;
-    float alpha_nx = 0.0f, beta_nx = 0.0f;
-    if (nxt.ub < ups) {
-      const long long tn = (long long)nxt.b * p.H + tbl[nxt.ub].head;
-      beta_nx = __ldg(p.beta + tn);
-      if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
-    }
-    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1));
-    if (!__all_sync(kFull, ok)) {
-      // Give up: record it, let the other slot's copy (if any) land, and leave.
-      if (lane == 0) {
-        atomicOr(p.flag, kFlagTimeout);
-        if (nxt.ub < ups)
-          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
-      }
-      __syncwarp();
-      return;
-    }
-    const UnitDesc d = tbl[cur.ub];
-    if (d.bits == 32)
-      compute_any<DK, DIAG, DELTA, SR, 32>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
-    else if (d.bits == 4)
-      compute_any<DK, DIAG, DELTA, SR, 4>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
-    else
-      compute_any<DK, DIAG, DELTA, SR, 8>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow);
-    // compute_any ends with __syncwarp: every lane is done reading this slot
-    if (fill.ub < ups) {
-      fence_proxy_async();
-      issue_unit<DK, DIAG>(p, tbl, fill.b, fill.ub, stage, &bars[s]);
-    }
-    cur = nxt;
-    nxt.advance(sb, su, B);
-    fill.advance(sb, su, B);
-    alpha_cur = alpha_nx;
-    beta_cur = beta_nx;
-  }
-}
 
 // -------------------------------------------------------------------------------------
 // state loader: quantize an fp32 state [B][H][d_v][d_k] with the step's quantizer
@@ -803,29 +411,11 @@ static uint32_t step_key_of(uint64_t seed, uint64_t step) {
   return (uint32_t)(k ^ (k >> 32));
 }
 
-using StepFn = void (*)(const StepParams);
 using LoadFn = void (*)(const LoadParams);
 using DequantFn = void (*)(const LoadParams, float *);
 
-template <int DK, bool SR>
-static StepFn pick_step(bool diag, bool delta) {
-  if (diag)
-    return delta ? decode_step_kernel<DK, true, true, SR> : decode_step_kernel<DK, true, false, SR>;
-  return delta ? decode_step_kernel<DK, false, true, SR> : decode_step_kernel<DK, false, false, SR>;
-}
-template <int DK>
-static StepFn pick_step(bool diag, bool delta, bool sr) {
-  return sr ? pick_step<DK, true>(diag, delta) : pick_step<DK, false>(diag, delta);
-}
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
-  switch (dk) {
-    case 16: return pick_step<16>(diag, delta, sr);
-    case 32: return pick_step<32>(diag, delta, sr);
-    case 64: return pick_step<64>(diag, delta, sr);
-    case 128: return pick_step<128>(diag, delta, sr);
-    case 256: return pick_step<256>(diag, delta, sr);
-  }
-  return nullptr;
+  return pick_step_any<false>(dk, diag, delta, sr);
 }
 using KeyFn = void (*)(const KeyParams);
 static KeyFn key_kernel_for(int dk) {
@@ -880,6 +470,7 @@ struct lores_handle {
   int smem = 0;
   StepParams sp{};
   StepFn step_fn = nullptr;
+  StepFn mt_fn = nullptr;                // multi-token kernel of the same configuration
   // key-axis grouping
   int axis = 0;
   KeyParams kp{};
@@ -1124,6 +715,18 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   }
   h->units_per_seq = (int)units.size();
   h->step_fn = fn;
+  h->mt_fn = mt_step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, h->mt_fn) != cudaSuccess ||
+        (fa.maxDynamicSharedSizeBytes < h->smem &&
+         cudaFuncSetAttribute(h->mt_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, h->smem) !=
+             cudaSuccess)) {
+      delete h;
+      return LORES_ERR_CUDA;
+    }
+  }
+  h->sp.T = 1;
 
   const long long code_bytes = (long long)c.batch * h->seq_bytes;
   const long long scale_count = scale_count_of(h);
@@ -1252,6 +855,49 @@ lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, 
   p.o = o;
   p.step_key = step_key_of(h->cfg.seed, step);
   h->step_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+lores_status lores_decode_steps(lores_handle *h, int32_t T, const float *q, const float *k,
+                                const float *v, const float *alpha, const float *beta, float *o,
+                                uint64_t step0, void *stream) {
+  if (!h || T < 1 || !q || !k || !v || !alpha || !beta || !o) return LORES_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (h->cfg.decay_diag ? !aligned16(alpha) : (reinterpret_cast<uintptr_t>(alpha) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(o) & 3u))
+    return LORES_ERR_INVALID_ARG;
+  const lores_config &c = h->cfg;
+  const long long bh = (long long)c.batch * c.heads;
+  const long long tok_qk = bh * c.d_k, tok_v = bh * c.d_v, tok_b = bh;
+  const long long tok_a = c.decay_diag ? bh * c.d_k : bh;
+  if (T == 1 || h->axis) {
+    // one token, or key-axis groups (a tile per CTA): one step launch per token
+    for (int t = 0; t < T; ++t) {
+      const lores_status st =
+          lores_decode_step(h, q + t * tok_qk, k + t * tok_qk, v + t * tok_v, alpha + t * tok_a,
+                            beta + t * tok_b, o + t * tok_v, step0 + (uint64_t)t, stream);
+      if (st != LORES_OK) return st;
+    }
+    return LORES_OK;
+  }
+  DeviceGuard guard(c.device);
+  if (!guard.ok) return LORES_ERR_CUDA;
+  StepParams p = h->sp;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.T = T;
+  p.tok_qk = tok_qk;
+  p.tok_v = tok_v;
+  p.tok_a = tok_a;
+  p.tok_b = tok_b;
+  p.tok_o = tok_v;
+  p.seed = c.seed;
+  p.step0 = step0;
+  h->mt_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -1538,6 +1184,7 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   p.ng = ng;
   p.G = G;
   p.units_per_seq = nunits;
+  p.T = 1;
   p.step_key = step_key_of(c.seed, step);
   const long long ctas = (p.total_units + kWarps - 1) / kWarps;
   const int grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * sms);

@@ -52,6 +52,7 @@ def _load():
         "lores_destroy": (I32, [P]),
         "lores_decode_step": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_host": (I32, [P, P, P, P, P, P, P, U64, P]),
+        "lores_decode_steps": (I32, [P, I32, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_noalloc": (I32, [C.POINTER(lores_config), P, P, P, P, P, P, P, P, U64,
                                             P, P]),
         "lores_dequant_state": (I32, [P, P, P]),
@@ -124,6 +125,13 @@ def lores_decode_step(h, q, k, v, alpha, beta, o, step, stream=None):
     _check(_lib.lores_decode_step(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                   _ptr(o), step & (2**64 - 1), _stream(stream)),
            "lores_decode_step")
+
+
+def lores_decode_steps(h, T, q, k, v, alpha, beta, o, step0, stream=None):
+    """T consecutive tokens in one call; inputs token-major [T, B, H, ...]."""
+    _check(_lib.lores_decode_steps(h, int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                   _ptr(o), step0 & (2**64 - 1), _stream(stream)),
+           "lores_decode_steps")
 
 
 def lores_decode_step_host(h, q, k, v, alpha, beta, o, step, stream=None):

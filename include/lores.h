@@ -117,6 +117,22 @@ lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, 
                                const float *alpha, const float *beta, float *o,
                                uint64_t step, void *stream);
 
+/* T consecutive decode steps in one call (a chunk of tokens of each sequence: the
+ * decode side of a prefill -> decode handoff, or several tokens per scheduling step).
+ * Token t in [0, T) reads q + t*B*H*d_k, k + t*B*H*d_k, v + t*B*H*d_v, alpha + t*B*H
+ * (or + t*B*H*d_k with decay_diag), beta + t*B*H, writes o + t*B*H*d_v, and uses the
+ * dither of step step0 + t: the result (state, scales, every o_t, flags) is bit for
+ * bit that of T calls of lores_decode_step with steps step0 .. step0+T-1.  Inputs are
+ * token-major [T, B, H, ...] with the per-token layouts of lores_decode_step.  The
+ * recurrence (General recurrence form) is applied token by token with requantization
+ * after every token (Key properties item 3); the state stays on chip between tokens
+ * and is read from and written to HBM once per call.  Key-axis handles run one step
+ * launch per token.  Errors: INVALID_ARG (T < 1, NULL or misaligned pointers), CUDA.
+ * Asynchronous on `stream`. */
+lores_status lores_decode_steps(lores_handle *h, int32_t T, const float *q, const float *k,
+                                const float *v, const float *alpha, const float *beta,
+                                float *o, uint64_t step0, void *stream);
+
 /* The same step with HOST buffers of the same shapes (pinned or pageable).  The
  * call copies the inputs to device staging buffers owned by the handle (allocated
  * on first use), runs the step, copies o back, and returns after `stream` has
