@@ -116,34 +116,55 @@ typedef struct {
     int stochastic;    /* 1: stochastic rounding; 0: round to nearest        */
     int axis;          /* 0: value-axis groups (scales [d_v][d_k/G]);
                         * 1: key-axis (one scale per key column, scales [d_k]) */
+    const int *group_bits; /* NULL, or bits (4..8) of each of the d_k/G key groups:
+                            * per-channel precision (value axis only; bits unused) */
 } lo_cfg;
 
 static int code_max(int bits) { return (1 << (bits - 1)) - 1; }
+
+/* Bits of key group g, and its storage: 4-bit codes as nibbles, 5 to 8 bits in bytes. */
+static int group_bits_of(const lo_cfg *c, int g) { return c->group_bits ? c->group_bits[g] : c->bits; }
+static int storage_of(int bits) { return bits == 4 ? 4 : 8; }
+
+/* A quantized row stores its key groups back to back, group g in
+ * G * storage(bits_g) / 8 bytes (with equal bits: the plain row-major layout). */
+static size_t group_offset(const lo_cfg *c, int g)
+{
+    size_t off = 0;
+    for (int h = 0; h < g; h++)
+        off += (size_t)c->group * storage_of(group_bits_of(c, h)) / 8;
+    return off;
+}
+static size_t quant_row_bytes(const lo_cfg *c) { return group_offset(c, c->d_k / c->group); }
 
 /* Read code (i, j) from a packed tile.  5 to 8 bits: one byte per code, two's
  * complement.  4 bits: two codes per byte, even column in the low nibble, odd
  * column in the high nibble, two's complement nibbles. */
 static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
 {
-    if (c->bits != 4)
-        return (int)(int8_t)codes[(size_t)i * c->d_k + j];
-    uint8_t byte = codes[(size_t)i * (c->d_k / 2) + j / 2];
-    int nib = (j % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    int g = j / c->group, jj = j - g * c->group;
+    const uint8_t *grp = codes + (size_t)i * quant_row_bytes(c) + group_offset(c, g);
+    if (group_bits_of(c, g) != 4)
+        return (int)(int8_t)grp[jj];
+    uint8_t byte = grp[jj / 2];
+    int nib = (jj % 2 == 0) ? (byte & 0xF) : (byte >> 4);
     return nib >= 8 ? nib - 16 : nib;
 }
 
 static void put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code)
 {
-    if (c->bits != 4) {
-        codes[(size_t)i * c->d_k + j] = (uint8_t)(int8_t)code;
+    int g = j / c->group, jj = j - g * c->group;
+    uint8_t *grp = codes + (size_t)i * quant_row_bytes(c) + group_offset(c, g);
+    if (group_bits_of(c, g) != 4) {
+        grp[jj] = (uint8_t)(int8_t)code;
         return;
     }
-    size_t at = (size_t)i * (c->d_k / 2) + j / 2;
+    size_t at = (size_t)jj / 2;
     uint8_t nib = (uint8_t)(code & 0xF);
-    if (j % 2 == 0)
-        codes[at] = (uint8_t)((codes[at] & 0xF0) | nib);
+    if (jj % 2 == 0)
+        grp[at] = (uint8_t)((grp[at] & 0xF0) | nib);
     else
-        codes[at] = (uint8_t)((codes[at] & 0x0F) | (nib << 4));
+        grp[at] = (uint8_t)((grp[at] & 0x0F) | (nib << 4));
 }
 
 int lo_get_code(const lo_cfg *c, const uint8_t *codes, int i, int j) { return get_code(c, codes, i, j); }
@@ -207,13 +228,12 @@ float lo_recip_nr(float m)
 /* ------------------------------------------------------------------------ */
 
 /* x: the updated fp32 row (d_k entries).  Writes the row's codes and its
- * d_k/G scales.  A row that holds a non-finite entry (or one above 2^100) is
- * stored as zero (scales 0, codes 0) and reported with return value 1. */
+ * d_k/G scales; group g uses r = 2^(b_g - 1) - 1 of its own bit width.  A row
+ * that holds a non-finite entry (or one above 2^100) is stored as zero (scales
+ * 0, codes 0) and reported with return value 1. */
 static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_key,
                           uint8_t *codes, float *scales)
 {
-    const int r = code_max(c->bits);
-    const float inv_r = 1.0f / (float)r;                  /* fl(1/r), round to nearest */
     const float m_lo = 0x1p-100f, m_hi = 0x1p100f;
     const int ng = c->d_k / c->group;
     int bad = 0;
@@ -225,6 +245,8 @@ static int requantize_row(const lo_cfg *c, const float *x, int i, uint32_t tile_
             if (fabsf(x[j]) > m_hi)
                 bad = 1;                  /* overflow: treated like a non-finite row */
     for (int g = 0; g < ng; g++) {
+        const int r = code_max(group_bits_of(c, g));
+        const float inv_r = 1.0f / (float)r;              /* fl(1/r), round to nearest */
         float m = 0.0f;
         for (int j = g * c->group; j < (g + 1) * c->group; j++)
             if (fabsf(x[j]) > m)

@@ -19,7 +19,7 @@ _lib = None
 class LoCfg(C.Structure):
     _fields_ = [("d_k", C.c_int), ("d_v", C.c_int), ("group", C.c_int), ("bits", C.c_int),
                 ("delta", C.c_int), ("diag", C.c_int), ("stochastic", C.c_int),
-                ("axis", C.c_int)]
+                ("axis", C.c_int), ("group_bits", C.c_void_p)]
 
 
 def lib():
@@ -73,13 +73,22 @@ def _f32(a):
 class TileCfg:
     """Shape and recipe of one (sequence, head) tile."""
 
-    def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1, axis=0):
+    def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1, axis=0,
+                 group_bits=None):
         self.d_k, self.d_v = int(d_k), int(d_v)
         self.group = int(group if group else d_k)
         self.bits, self.delta, self.diag, self.stochastic = int(bits), int(delta), int(diag), int(stochastic)
         self.axis = int(axis)
+        # per-channel precision: bits of each key group (the `bits` field is then unused)
+        self.group_bits = None
+        gb = None
+        if group_bits is not None:
+            self.group_bits = np.ascontiguousarray(group_bits, dtype=np.int32)
+            assert self.group_bits.shape == (self.d_k // self.group,) and not self.axis
+            self.bits = 0
+            gb = self.group_bits.ctypes.data_as(C.c_void_p)
         self.c = LoCfg(self.d_k, self.d_v, self.group, self.bits, self.delta, self.diag,
-                       self.stochastic, self.axis)
+                       self.stochastic, self.axis, gb)
 
     @property
     def n_groups(self):
@@ -89,7 +98,15 @@ class TileCfg:
         """value axis: [d_v, d_k/G]; key axis: [d_k] (one scale per key column)."""
         return (self.d_k,) if self.axis else (self.d_v, self.n_groups)
 
+    def row_bytes(self):
+        """Bytes of one quantized row: key groups back to back, each G * storage / 8."""
+        if self.group_bits is not None:
+            return sum(self.group * (4 if b == 4 else 8) // 8 for b in self.group_bits)
+        return self.code_bytes() // self.d_v
+
     def code_bytes(self):
+        if self.group_bits is not None:
+            return self.d_v * self.row_bytes()
         if self.bits == 32:
             return self.d_v * self.d_k * 4
         if self.bits == 4:

@@ -635,3 +635,98 @@ def test_value_axis_beats_key_axis_with_outlier_value_rows():
             e = (O.tile_dequant(cfg, codes, sc).astype(np.float64) - S) @ q
             errs[axis] += float(np.sum(e ** 2))
     assert errs[0] < 0.5 * errs[1], errs
+
+
+# --------------------------------------------------------------------------
+# Per-channel precision: a bit width per key group (the abstract's decay-based
+# mixed precision across channels; value-axis scale groups of G columns)
+# --------------------------------------------------------------------------
+
+def test_group_bits_layout_worked_example():
+    # d_k = 32, G = 16, groups at 8 and 4 bits: a row is 16 code bytes then 8 nibble bytes
+    cfg = O.TileCfg(32, 1, group=16, group_bits=[8, 4])
+    assert cfg.row_bytes() == 24 and cfg.code_bytes() == 24
+    ints = np.array([[j - 10 for j in range(16)] + [1, -1, 7, -7, 0, 3, -3, 2, 5, -5, 6, -6, 4, -4, 1, 0]])
+    b = O.pack_codes(cfg, ints)
+    assert b[:16].view(np.int8).tolist() == list(range(-10, 6))
+    # the int4 group packs like a 16-column int4 row (same worked bytes as the plain layout)
+    assert b[16] == 0xF1 and b[17] == 0x97 and b[18] == 0x30 and b[19] == 0x2D
+    assert (O.unpack_codes(cfg, b) == ints).all()
+    # the other order: the nibble group first
+    cfg2 = O.TileCfg(32, 1, group=16, group_bits=[4, 8])
+    ints2 = np.concatenate([ints[:, 16:], ints[:, :16]], axis=1)
+    b2 = O.pack_codes(cfg2, ints2)
+    assert b2[:4].tolist() == [0xF1, 0x97, 0x30, 0x2D] and b2[8:].view(np.int8).tolist() == list(range(-10, 6))
+
+
+@pytest.mark.parametrize("bits", [4, 5, 6, 8])
+def test_uniform_group_bits_equal_plain_bits(bits):
+    # every group at the same width gives exactly the plain layout and the same step
+    d_k, d_v, G = 64, 8, 16
+    plain = O.TileCfg(d_k, d_v, group=G, bits=bits, delta=1, diag=1)
+    grp = O.TileCfg(d_k, d_v, group=G, group_bits=[bits] * (d_k // G), delta=1, diag=1)
+    assert plain.code_bytes() == grp.code_bytes()
+    g = rng(70 + bits)
+    S = g.standard_normal((d_v, d_k)).astype(np.float32)
+    tk = O.tile_key(O.step_key(5, 1), 2)
+    c1, s1, _ = O.tile_quantize(plain, S, tk)
+    c2, s2, _ = O.tile_quantize(grp, S, tk)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+    q, k, v, alpha, beta = draw(1, d_k, d_v, 71, diag=True)
+    o1, f1, _ = O.tile_step(plain, c1, s1, q[0], k[0], v[0], alpha[0], beta[0], tk)
+    o2, f2, _ = O.tile_step(grp, c2, s2, q[0], k[0], v[0], alpha[0], beta[0], tk)
+    assert np.array_equal(c1, c2) and np.array_equal(s1, s2) and np.array_equal(o1, o2)
+
+
+@pytest.mark.parametrize("sr", [1, 0])
+def test_group_bits_quantizer_invariants(sr):
+    # each group follows Proposition 1 with its own r = 2^(b_g - 1) - 1
+    d_k, d_v, G = 64, 32, 16
+    gb = [8, 4, 6, 5]
+    cfg = O.TileCfg(d_k, d_v, group=G, group_bits=gb, stochastic=sr)
+    g = rng(73 + sr)
+    X = (g.standard_normal((d_v, d_k)) * np.exp(g.uniform(-6, 6, (d_v, 1)))).astype(np.float32)
+    X[2, 16:32] = 0.0                            # an all-zero int4 group
+    codes, scales, flag = O.tile_quantize(cfg, X, O.tile_key(O.step_key(3, 9), 4))
+    assert flag == 0
+    C_ = O.unpack_codes(cfg, codes)
+    for gi, b in enumerate(gb):
+        r = (1 << (b - 1)) - 1
+        for i in range(d_v):
+            xs = X[i, gi * G:(gi + 1) * G]
+            cs = C_[i, gi * G:(gi + 1) * G]
+            m = np.float32(np.abs(xs).max())
+            s = scales[i, gi]
+            assert np.abs(cs).max() <= r
+            if m == 0:
+                assert s == 0 and not cs.any()
+                continue
+            assert s == np.float32(m * (np.float32(1) / np.float32(r)))
+            assert np.abs(cs).max() == r
+            err = np.abs(cs * np.float64(s) - xs)
+            assert err.max() <= (1.0 if sr else 0.5 + 2.0 ** -8) * float(s) * (1 + 1e-6)
+    # the dequantized tile is code times its group's scale
+    D = O.tile_dequant(cfg, codes, scales)
+    assert np.array_equal(D, (C_ * np.repeat(scales, G, axis=1)).astype(np.float32))
+
+
+def test_group_bits_step_matches_fp64_update():
+    d_k, d_v, G = 32, 12, 16
+    gb = [4, 8]
+    cfg = O.TileCfg(d_k, d_v, group=G, group_bits=gb, delta=1, diag=1)
+    g = rng(75)
+    ints = np.concatenate([g.integers(-7, 8, (d_v, 16)), g.integers(-127, 128, (d_v, 16))], axis=1)
+    codes = O.pack_codes(cfg, ints)
+    scales = g.uniform(0.01, 0.1, (d_v, 2)).astype(np.float32)
+    q, k, v, alpha, beta = draw(1, d_k, d_v, 76, diag=True)
+    S_hat = ints * np.repeat(scales.astype(np.float64), G, axis=1)
+    X = recur64(S_hat, alpha[0], k[0], v[0], beta[0], 1)
+    o, flag, x = O.tile_step(cfg, codes, scales, q[0], k[0], v[0], alpha[0], beta[0],
+                             O.tile_key(O.step_key(1, 2), 3), want_x=True)
+    assert flag == 0
+    np.testing.assert_allclose(x, X, rtol=0, atol=1e-5 * np.abs(X).max())
+    np.testing.assert_allclose(o, X @ q[0].astype(np.float64), rtol=0, atol=1e-5 * np.abs(X).max())
+    # requantized: every entry within one step of its group's new scale
+    C_ = O.unpack_codes(cfg, codes)
+    err = np.abs(C_ * np.repeat(scales.astype(np.float64), G, axis=1) - x)
+    assert (err <= np.repeat(scales.astype(np.float64), G, axis=1) * (1 + 1e-6)).all()
