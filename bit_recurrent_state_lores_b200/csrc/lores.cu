@@ -38,7 +38,7 @@ struct LoadParams {
   const float *S;
   uint8_t *codes;
   float *scales;
-  const int32_t *head_bits;     // device [H]
+  const LaneFmt *fmt;           // device [H][d_k/16]
   const int64_t *head_off;      // device [H]
   long long seq_bytes;
   long long rows;               // B * H * d_v
@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   const long long b = tile / p.H;
   // Rows of one warp may belong to different tiles (and bit widths): every lane runs the
   // quantizer (it shuffles across the warp) and each lane stores per its own row.
-  const int bits = __ldg(p.head_bits + head);
+  const LaneFmt f = p.fmt[head * (DK / 16) + lir];
+  const int bits = f.bits;
   float x[16];
   const float *src = p.S + grr * DK + col0;
 #pragma unroll
@@ -78,18 +79,18 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   float s_new;
   requantize16<LPR>(x, bits == 32 ? 8 : bits, lpg, lane, tkey, n0, p.stochastic, words, s_new);
   if (!active) return;
+  uint8_t *dst = tilecodes + (size_t)row * f.rowb + f.off;
   if (bits == 32) {
-    float4 *dst = reinterpret_cast<float4 *>(tilecodes + (size_t)row * DK * 4) + lir * 4;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+    for (int c = 0; c < 4; ++c)
+      reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
     return;
   }
+  // lane blocks are 8-byte aligned (16 with one width per head)
   if (bits != 4)
-    *reinterpret_cast<uint4 *>(tilecodes + (size_t)row * DK + lir * 16) =
-        make_uint4(words[0], words[1], words[2], words[3]);
+    st16_a8(dst, make_uint4(words[0], words[1], words[2], words[3]));
   else
-    *reinterpret_cast<uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8) =
-        make_uint2(words[0], words[1]);
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
   if (lir % lpg == 0) p.scales[grr * p.ng + g] = s_new;
 }
 
@@ -107,11 +108,12 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
   const long long tile = grr / p.d_v;
   const int head = (int)(tile % p.H);
   const long long b = tile / p.H;
-  const int bits = p.head_bits[head];
-  const uint8_t *tilecodes = p.codes + b * p.seq_bytes + p.head_off[head];
+  const LaneFmt f = p.fmt[head * (DK / 16) + lir];
+  const int bits = f.bits;
+  const uint8_t *lanecodes = p.codes + b * p.seq_bytes + p.head_off[head] + (size_t)row * f.rowb + f.off;
   float y[16];
   if (bits == 32) {
-    const float4 *src = reinterpret_cast<const float4 *>(tilecodes + (size_t)row * DK * 4) + lir * 4;
+    const float4 *src = reinterpret_cast<const float4 *>(lanecodes);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const float4 f = src[c];
@@ -120,9 +122,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
   } else {
     float cf[16];
     if (bits != 4)
-      unpack_i8(*reinterpret_cast<const uint4 *>(tilecodes + (size_t)row * DK + lir * 16), cf);
+      unpack_i8(ld16_a8(lanecodes), cf);          // lane blocks are 8-byte aligned
     else
-      unpack_i4(*reinterpret_cast<const uint2 *>(tilecodes + (size_t)row * (DK / 2) + lir * 8), cf);
+      unpack_i4(*reinterpret_cast<const uint2 *>(lanecodes), cf);
     if (p.axis) {
       const float *sc = p.scales + tile * DK + col0;          // one scale per key column
 #pragma unroll
@@ -465,6 +467,9 @@ struct lores_handle {
   UnitDesc *units = nullptr;
   int32_t *d_bits = nullptr;
   int64_t *d_head_off = nullptr;
+  LaneFmt *d_fmt = nullptr;        // [H][d_k/16]
+  std::vector<LaneFmt> fmt;
+  std::vector<int32_t> rowb;       // [H] bytes of one row
   int units_per_seq = 0;
   int grid = 0;
   int smem = 0;
@@ -513,6 +518,7 @@ void free_all(lores_handle *h) {
   cudaFree(h->units);
   cudaFree(h->d_bits);
   cudaFree(h->d_head_off);
+  cudaFree(h->d_fmt);
   cudaFree(h->stage_in);
   cudaFree(h->stage_o);
 }
@@ -527,7 +533,7 @@ LoadParams load_params(const lores_handle *h) {
   LoadParams p{};
   p.codes = h->codes;
   p.scales = h->scales;
-  p.head_bits = h->d_bits;
+  p.fmt = h->d_fmt;
   p.head_off = h->d_head_off;
   p.seq_bytes = h->seq_bytes;
   p.rows = (long long)h->cfg.batch * h->cfg.heads * h->cfg.d_v;
@@ -597,6 +603,26 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       bits[h] = c.head_bits[h];
       if (!((bits[h] >= 4 && bits[h] <= 8) || bits[h] == 32)) return LORES_ERR_INVALID_ARG;
     }
+  // per-channel precision: a width per (head, key group); a head whose groups all share
+  // one width is an ordinary head of that width, any other head is "mixed" (bits 0)
+  const int ngr = dk / G;
+  std::vector<int32_t> gbits((size_t)c.heads * ngr);
+  if (c.group_bits) {
+    if (c.head_bits || c.scale_axis) return LORES_ERR_INVALID_ARG;
+    for (int h = 0; h < c.heads; ++h) {
+      for (int g = 0; g < ngr; ++g) {
+        const int b = c.group_bits[(size_t)h * ngr + g];
+        if (b < 4 || b > 8) return LORES_ERR_INVALID_ARG;
+        gbits[(size_t)h * ngr + g] = b;
+      }
+      bits[h] = gbits[(size_t)h * ngr];
+      for (int g = 1; g < ngr; ++g)
+        if (gbits[(size_t)h * ngr + g] != bits[h]) bits[h] = 0;
+    }
+  } else {
+    for (int h = 0; h < c.heads; ++h)
+      for (int g = 0; g < ngr; ++g) gbits[(size_t)h * ngr + g] = bits[h];
+  }
 
   DeviceGuard guard(c.device);
   if (!guard.ok) {
@@ -610,16 +636,35 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   lores_handle *h = new (std::nothrow) lores_handle();
   if (!h) return LORES_ERR_OOM;
   h->cfg = c;
-  h->cfg.head_bits = nullptr;           // the caller's array is not kept
+  h->cfg.head_bits = nullptr;           // the caller's arrays are not kept
+  h->cfg.group_bits = nullptr;
   h->bits = bits;
   h->G = G;
   h->ng = dk / G;
   h->axis = c.scale_axis;
+  // row layout: key groups back to back, group g in G * storage(b_g) / 8 bytes; the lane
+  // table gives each 16-column block its width, offset, r and fl(1/r)
   h->head_off.resize(c.heads);
+  h->rowb.assign(c.heads, 0);
+  h->fmt.resize((size_t)c.heads * (dk / 16));
   long long off = 0;
   for (int hh = 0; hh < c.heads; ++hh) {
+    int goff = 0;
+    for (int g = 0; g < ngr; ++g) {
+      const int b = bits[hh] == 32 ? 32 : gbits[(size_t)hh * ngr + g];
+      for (int lb = g * G / 16; lb < (g + 1) * G / 16; ++lb) {
+        LaneFmt &f = h->fmt[(size_t)hh * (dk / 16) + lb];
+        f.bits = (int16_t)b;
+        f.off = goff + (lb * 16 - g * G) * storage_bits(b) / 8;
+        f.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
+        f.inv_r = b == 32 ? 0.0f : 1.0f / f.r;
+      }
+      goff += G * storage_bits(b) / 8;
+    }
+    h->rowb[hh] = goff;
+    for (int lb = 0; lb < dk / 16; ++lb) h->fmt[(size_t)hh * (dk / 16) + lb].rowb = (int16_t)goff;
     h->head_off[hh] = off;
-    off += (long long)dv * row_bytes(dk, bits[hh]);
+    off += (long long)dv * goff;
   }
   h->seq_bytes = off;
 
@@ -628,15 +673,20 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   // d_v allows; the last unit of a head takes the remainder.  Small batches split
   // units further (down to one pass) until every warp of one wave has work.
   const int LPR = dk / 16, rpw = 32 / LPR;
-  auto rows_for = [&](int b) { return std::min(full_rows(dk, b), dv); };
+  // rows of a full unit: 4 KB of state, a whole number of warp passes (full_rows for a
+  // head of one width)
+  auto rows_for = [&](int rb) {
+    const int n = 4096 / rb;
+    return std::min(n < rpw ? rpw : n - n % rpw, dv);
+  };
   StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
-  const int R8 = rows_for(8), R4 = rows_for(4), R32 = rows_for(32);
   int split = 1;
   auto build_units = [&](std::vector<UnitDesc> &u) {
     u.clear();
     for (int hh = 0; hh < c.heads; ++hh) {
       const int b = bits[hh];
-      int R = b == 8 ? R8 : (b == 4 ? R4 : R32);
+      const int rb = h->rowb[hh];
+      int R = rows_for(rb);
       int Rs = R / split;
       Rs -= Rs % std::min(rpw, R);
       Rs -= Rs % 4;
@@ -646,17 +696,18 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
         d.head = hh;
         d.row0 = r0;
         d.nrows = std::min(R, dv - r0);
-        d.bits = b;
-        d.code_off = h->head_off[hh] + (long long)r0 * row_bytes(dk, b);
-        d.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
-        d.inv_r = b == 32 ? 0.0f : 1.0f / d.r;
+        d.bits = (int16_t)b;
+        d.rowb = (int16_t)rb;
+        d.code_off = h->head_off[hh] + (long long)r0 * rb;
+        d.r = (b == 32 || b == 0) ? 0.0f : (float)((1 << (b - 1)) - 1);
+        d.inv_r = (b == 32 || b == 0) ? 0.0f : 1.0f / d.r;
         u.push_back(d);
       }
     }
   };
   std::vector<UnitDesc> units;
   int ctas_per_sm = 1;
-  auto bits_rank = [](int b) { return storage_bits(b) == 8 ? 0 : (b == 4 ? 1 : 2); };
+  auto bits_rank = [](int b) { return b == 0 ? 3 : (storage_bits(b) == 8 ? 0 : (b == 4 ? 1 : 2)); };
   for (;;) {
     build_units(units);
     std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
@@ -664,7 +715,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     });
     int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
     for (const UnitDesc &d : units) {
-      cmax = std::max(cmax, d.nrows * row_bytes(dk, d.bits));
+      cmax = std::max(cmax, d.nrows * (int)d.rowb);
       if (d.bits != 32) smax = std::max(smax, d.nrows * h->ng * 4);
       vmax = std::max(vmax, d.nrows * 4);
       maxrows = std::max(maxrows, d.nrows);
@@ -768,6 +819,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   if (e == cudaSuccess) e = cudaMalloc(&h->units, units.size() * sizeof(UnitDesc));
   if (e == cudaSuccess) e = cudaMalloc(&h->d_bits, c.heads * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMalloc(&h->d_head_off, c.heads * sizeof(int64_t));
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_fmt, h->fmt.size() * sizeof(LaneFmt));
   if (e == cudaSuccess) e = cudaMemset(h->codes, 0, (size_t)code_bytes);
   if (e == cudaSuccess) e = cudaMemset(h->scales, 0, (size_t)scale_count * 4);
   if (e == cudaSuccess) e = cudaMemset(h->flag, 0, 16);
@@ -778,6 +830,8 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   if (e == cudaSuccess)
     e = cudaMemcpy(h->d_head_off, h->head_off.data(), c.heads * sizeof(int64_t),
                    cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->d_fmt, h->fmt.data(), h->fmt.size() * sizeof(LaneFmt), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     const lores_status st = cuda_status(e);
     free_all(h);
@@ -798,6 +852,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   p.ng = h->ng;
   p.G = G;
   p.units_per_seq = h->units_per_seq;
+  p.fmt = h->d_fmt;
   KeyParams &kp = h->kp;
   kp.codes = h->codes;
   kp.scales = h->scales;
@@ -1089,7 +1144,8 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
       (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
     return LORES_ERR_INVALID_ARG;
-  if (c.scale_axis != 0) return LORES_ERR_UNSUPPORTED;          // value-axis groups only
+  if (c.scale_axis != 0 || c.group_bits) return LORES_ERR_UNSUPPORTED;   // per-head widths,
+                                                                          // value-axis groups
   for (int hh = 0; c.head_bits && hh < c.heads; ++hh)
     if (!((c.head_bits[hh] >= 4 && c.head_bits[hh] <= 8) || c.head_bits[hh] == 32))
       return LORES_ERR_INVALID_ARG;
@@ -1115,7 +1171,8 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
       d.head = hh;
       d.row0 = r0;
       d.nrows = std::min(R, dv - r0);
-      d.bits = b;
+      d.bits = (int16_t)b;
+      d.rowb = (int16_t)row_bytes(dk, b);
       d.code_off = seq_bytes + (long long)r0 * row_bytes(dk, b);
       d.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
       d.inv_r = b == 32 ? 0.0f : 1.0f / d.r;

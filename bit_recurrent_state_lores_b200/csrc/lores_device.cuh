@@ -109,6 +109,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned by
       : "memory");
 }
 
+// 16 code bytes at an address that is only 8-byte aligned (rows of per-channel
+// precision heads: key groups of 8 and 16 bytes back to back), as two 8-byte accesses.
+__device__ __forceinline__ uint4 ld16_a8(const uint8_t *p) {
+  const uint2 a = *reinterpret_cast<const uint2 *>(p);
+  const uint2 b = *reinterpret_cast<const uint2 *>(p + 8);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st16_a8(uint8_t *p, uint4 w) {
+  *reinterpret_cast<uint2 *>(p) = make_uint2(w.x, w.y);
+  *reinterpret_cast<uint2 *>(p + 8) = make_uint2(w.z, w.w);
+}
+
 // -------------------------------------------------------------------------------------
 // code <-> float
 // -------------------------------------------------------------------------------------
@@ -256,50 +268,55 @@ __device__ __forceinline__ float recip_nr(float m) {
 // -------------------------------------------------------------------------------------
 // requantize one lane's 16 entries of a value row
 // -------------------------------------------------------------------------------------
-// LPR lanes hold one row (16 consecutive columns each); LPG = G/16 lanes share a group.
-// Returns the row's "non-finite" verdict (same on all lanes of the row): a row with an
-// entry that is inf, NaN or above 2^100 is stored as zero.  Writes the lane's packed
-// codes into `words` (int8: 4 words, int4: 2 words) and the lane's group scale into
-// `s_out`.  `bits` (8 or 4) may differ between rows of one warp; every lane of the warp
-// must call this function together (it shuffles and votes across the warp).
-// Requantize one lane's 16 entries without any branch or vote: returns this lane's
-// group verdict (true: an entry of the group is inf, NaN or above 2^100).  A row with
-// a bad group must then be zeroed by the caller (see zero_bad_rows); its codes and
-// scale written here are not meaningful.  cbase = tile key + golden * (n0 + 1) where
-// n0 is the quad index of the lane's first column (see the dither definition).
-// Dither words of one lane-row: four MurmurHash3 finalizer values of consecutive counters.
+// Dither words of one lane-row: four MurmurHash3 finalizer values of consecutive
+// counters; cbase = tile key + golden * (n0 + 1), n0 the quad index of the lane's first
+// column (see the dither definition).
 __device__ __forceinline__ void dither_words(uint32_t cbase, uint32_t (&h)[4]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
 }
 
-// r = 2^(b-1) - 1 of the unit's codes and inv_r = fl(1/r); BITS is the storage (8: one
-// byte per code, for 5- to 8-bit codes; 4: nibbles).
-template <int LPR, int BITS, bool SR>
-__device__ __forceinline__ bool requantize16_nb(const float2 (&x)[8], float r, float inv_r,
-                                                int gd1, int gd2, int gd4, int gd8,
-                                                const uint32_t (&h)[4], uint32_t (&words)[4],
-                                                float &s_out) {
+// Largest |x| over one lane's 16 entries (NaN if any entry is NaN).
+__device__ __forceinline__ float chunk_absmax(const float2 (&x)[8]) {
   float mq[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c)
     mq[c] = max_abs_nan(max_abs_nan(max_abs_nan(fabsf(x[2 * c].x), x[2 * c].y), x[2 * c + 1].x),
                         x[2 * c + 1].y);
-  float m = max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
-  // group max over the lanes of the group: a level at or beyond the group width has
-  // shuffle distance 0 (the lane's own value)
+  return max_nan(max_nan(mq[0], mq[1]), max_nan(mq[2], mq[3]));
+}
+
+// Group maximum over the lanes of the group: a level at or beyond the group width has
+// shuffle distance 0 (the lane's own value).  Every lane of the warp must take part.
+template <int LPR>
+__device__ __forceinline__ float group_absmax(float m, int gd1, int gd2, int gd4, int gd8) {
   const int dist[4] = {gd1, gd2, gd4, gd8};
 #pragma unroll
   for (int l = 0; (1 << l) < LPR; ++l) m = max_nan(m, __shfl_xor_sync(kFull, m, dist[l]));
-  const bool gbad = !(m <= 0x1p100f);                    // inf, NaN or overflow
-  const bool scaled = m >= 0x1p-100f && !gbad;           // below 2^-100: zero group
+  return m;
+}
+
+// Scale and inverse of a group with largest |x| = m; returns the group's "bad" verdict
+// (an entry is inf, NaN or above 2^100).  Below 2^-100 the group is stored as zero.
+__device__ __forceinline__ bool group_scale(float m, float r, float inv_r, float2 &inv, float &s) {
+  const bool gbad = !(m <= 0x1p100f);
+  const bool scaled = m >= 0x1p-100f && !gbad;
   const float y = recip_nr(scaled ? m : 1.0f);
-  const float2 inv = dup2(scaled ? __fmul_rn(r, y) : 0.0f);
-  s_out = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+  inv = dup2(scaled ? __fmul_rn(r, y) : 0.0f);
+  s = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+  return gbad;
+}
+
+// Codes of a lane's 16 entries: t = fma(x, inv, 49152 + d/256) (d = byte j mod 4 of the
+// quad's hash word; 128 for round to nearest), packed from byte 1 of t.  BITS is the
+// storage: 8 (one byte per code, 5- to 8-bit codes; 4 words) or 4 (nibbles; 2 words).
+// No cross-lane operation: lanes may take different widths.
+template <int BITS, bool SR>
+__device__ __forceinline__ void quantize16(const float2 (&x)[8], float2 inv, const uint32_t (&h)[4],
+                                           uint32_t (&words)[4]) {
   uint32_t t[16];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    // addend 49152 + d/256 with d = byte (j mod 4) of the quad's hash word
     const float2 g =
         SR ? make_float2(
                  __uint_as_float(__byte_perm(h[e >> 1], 0x47400000u, 0x7650u | ((2 * e) & 3))),
@@ -316,9 +333,30 @@ __device__ __forceinline__ bool requantize16_nb(const float2 (&x)[8], float r, f
     const uint2 w = pack_i4(t);
     words[0] = w.x; words[1] = w.y; words[2] = 0u; words[3] = 0u;
   }
+}
+
+// Requantize one lane's 16 entries of a value row (a scale group spans G/16 lanes):
+// returns this lane's group verdict (true: an entry of the group is inf, NaN or above
+// 2^100; the caller then zeroes the row).  r = 2^(b-1) - 1 and inv_r = fl(1/r).
+template <int LPR, int BITS, bool SR>
+__device__ __forceinline__ bool requantize16_nb(const float2 (&x)[8], float r, float inv_r,
+                                                int gd1, int gd2, int gd4, int gd8,
+                                                const uint32_t (&h)[4], uint32_t (&words)[4],
+                                                float &s_out) {
+  const float m = group_absmax<LPR>(chunk_absmax(x), gd1, gd2, gd4, gd8);
+  float2 inv;
+  const bool gbad = group_scale(m, r, inv_r, inv, s_out);
+  quantize16<BITS, SR>(x, inv, h, words);
   return gbad;
 }
 
+// Requantizer of the state loader: LPR lanes hold one row (16 consecutive columns
+// each); lpg = G/16 lanes share a group.  Returns the row's "non-finite" verdict (same
+// on all lanes of the row): a row with an entry that is inf, NaN or above 2^100 is
+// stored as zero.  Writes the lane's packed codes into `words` (8-bit storage: 4 words,
+// int4: 2 words) and the lane's group scale into `s_out`.  `bits` may differ between
+// lanes of one warp; every lane of the warp must call this function together (it
+// shuffles and votes across the warp).
 template <int LPR>
 __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
                                              uint32_t tkey, uint32_t n0, int stochastic,

@@ -19,10 +19,24 @@ struct __align__(16) UnitDesc {
   int32_t head;
   int32_t row0;
   int32_t nrows;
-  int32_t bits;          // 4..8 (b-bit codes) or 32 (fp32 state)
+  int16_t bits;          // 4..8 (b-bit codes), 32 (fp32 state), or 0: a bit width per key
+                         // group (per-channel precision; the lane table has the layout)
+  int16_t rowb;          // bytes of one row of the head
   int64_t code_off;      // byte offset of row0 of this head inside one sequence's block
-  float r;               // largest code, 2^(bits-1) - 1
+  float r;               // largest code, 2^(bits-1) - 1 (bits 4..8)
   float inv_r;           // fl(1/r)
+};
+
+// Layout of the 16 columns a lane owns, per (head, 16-column block): the block's bit
+// width (its key group's), its byte offset inside a row, r and fl(1/r), and the head's
+// row bytes.  Rows store their key groups back to back, group g in G * storage(b_g) / 8
+// bytes (4-bit codes as nibbles, 5 to 8 bits one byte each, fp32 heads 4 bytes).
+struct __align__(16) LaneFmt {
+  float r;
+  float inv_r;
+  int32_t off;
+  int16_t bits;
+  int16_t rowb;
 };
 
 struct StepParams {
@@ -32,6 +46,7 @@ struct StepParams {
   float *o;
   unsigned *flag;
   const UnitDesc *units; // [units_per_seq]
+  const LaneFmt *fmt;    // [H][d_k/16]
   long long seq_bytes;
   long long total_units;
   int B, H, d_v, ng, G, units_per_seq;
@@ -90,7 +105,7 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
   const int lane = threadIdx.x & 31;
   const UnitDesc d = tbl[ub];
   const long long tile = (long long)b * p.H + d.head;
-  const unsigned cbytes = (unsigned)(d.nrows * row_bytes(DK, d.bits));
+  const unsigned cbytes = (unsigned)(d.nrows * d.rowb);
   const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
   const unsigned vbytes = (unsigned)(d.nrows * 4);
   const unsigned vec = DK * 4;
@@ -127,10 +142,22 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
                                              float *opart, float *ow, int t) {
   constexpr int LPR = DK / 16;            // lanes per row
   constexpr int RPW = 32 / LPR;           // rows per warp pass
-  constexpr int RB = DK * BITS / 8;       // bytes per row
   const int lane = threadIdx.x & 31;
   const int lir = lane % LPR, riw = lane / LPR;
   const int col0 = lir * 16;
+  // BITS = 0: a bit width per key group; the lane's width, offset and r come from the
+  // lane table (lanes of a warp may differ; cross-lane steps stay convergent)
+  const int RB = BITS == 0 ? (int)d.rowb : DK * BITS / 8;   // bytes per row
+  int lsb = BITS, loff = lir * 2 * BITS;                    // lane storage bits, byte offset
+  float rq = d.r, rq_inv = d.inv_r;
+  if (BITS == 0) {
+    const LaneFmt f = p.fmt[d.head * (DK / 16) + lir];
+    lsb = f.bits == 4 ? 4 : 8;
+    loff = f.off;
+    rq = f.r;
+    rq_inv = f.inv_r;
+  }
+  const bool w8 = BITS == 8 || (BITS == 0 && lsb == 8);     // byte codes (else nibbles)
   // GROW: one scale per value row (G = d_k), known at compile time
   const int lpg = GROW ? LPR : p.G / 16;                   // lanes per scale group (power of 2)
   const int g = GROW ? 0 : lir / lpg;                      // this lane's group in the row
@@ -209,10 +236,12 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       }
     } else {
       float2 cf[8];
-      if (BITS == 8)
-        unpack_i8_2(*reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + lir * 16), cf);
+      if (w8)
+        unpack_i8_2(BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
+                              : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff),
+                    cf);
       else
-        unpack_i4_2(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + lir * 8), cf);
+        unpack_i4_2(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + loff), cf);
       const float s_in = ss[lrr * ng + g];
       const float2 s2 = dup2(s_in);
       const float2 a_row = dup2(__fmul_rn(s_in, alpha_s));
@@ -266,21 +295,38 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     } else {
       uint32_t words[4];
       float s_new;
-      gbad = requantize16_nb<LPR, BITS, SR>(x, d.r, d.inv_r, gd1, gd2, gd4, gd8, hw, words, s_new);
+      if (BITS == 0) {
+        // group scale with every lane, then each lane packs at its own width
+        const float m = group_absmax<LPR>(chunk_absmax(x), gd1, gd2, gd4, gd8);
+        float2 inv;
+        gbad = group_scale(m, rq, rq_inv, inv, s_new);
+        if (w8)
+          quantize16<8, SR>(x, inv, hw, words);
+        else
+          quantize16<4, SR>(x, inv, hw, words);
+      } else {
+        gbad = requantize16_nb<LPR, BITS, SR>(x, rq, rq_inv, gd1, gd2, gd4, gd8, hw, words, s_new);
+      }
       if (active) {
         if (to_stage) {
-          if (BITS == 8)
-            *reinterpret_cast<uint4 *>(stage + (size_t)lr * RB + lir * 16) =
+          if (w8 && BITS == 0)
+            st16_a8(stage + (size_t)lr * RB + loff, make_uint4(words[0], words[1], words[2], words[3]));
+          else if (w8)
+            *reinterpret_cast<uint4 *>(stage + (size_t)lr * RB + loff) =
                 make_uint4(words[0], words[1], words[2], words[3]);
           else
-            *reinterpret_cast<uint2 *>(stage + (size_t)lr * RB + lir * 8) = make_uint2(words[0], words[1]);
+            *reinterpret_cast<uint2 *>(stage + (size_t)lr * RB + loff) = make_uint2(words[0], words[1]);
           if (scale_writer) ss[lr * ng + g] = s_new;
         } else {
-          if (BITS == 8)
-            __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16),
+          if (w8 && BITS == 0) {
+            uint2 *dst = reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + loff);
+            __stcs(dst, make_uint2(words[0], words[1]));
+            __stcs(dst + 1, make_uint2(words[2], words[3]));
+          } else if (w8) {
+            __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + loff),
                    make_uint4(words[0], words[1], words[2], words[3]));
-          else
-            __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8),
+          } else
+            __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + loff),
                    make_uint2(words[0], words[1]));
           if (scale_writer) gscales[lr * ng + g] = s_new;
         }
@@ -299,11 +345,11 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       const int lr = n * RPW + riw;
       if ((bal & rowmask) == 0u || !(FULL || lr < d.nrows)) continue;
       if (BITS != 32) {
-        uint8_t *dst = (to_stage ? stage : gcodes) + (size_t)lr * RB;
-        if (BITS == 8)
-          *reinterpret_cast<uint4 *>(dst + lir * 16) = make_uint4(0, 0, 0, 0);
+        uint8_t *dst = (to_stage ? stage : gcodes) + (size_t)lr * RB + loff;
+        if (w8)
+          st16_a8(dst, make_uint4(0, 0, 0, 0));
         else
-          *reinterpret_cast<uint2 *>(dst + lir * 8) = make_uint2(0, 0);
+          *reinterpret_cast<uint2 *>(dst) = make_uint2(0, 0);
         if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
       }
       if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
@@ -334,7 +380,7 @@ template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool MT>
 __device__ __forceinline__ void compute_any(const StepParams &p, uint8_t *stage, int b,
                                             const UnitDesc &d, float alpha_s, float beta,
                                             float *opart, float *ow, int t) {
-  if (d.nrows == full_rows(DK, BITS)) {
+  if (BITS != 0 && d.nrows == full_rows(DK, BITS)) {
     if (p.G == DK)
       compute_unit<DK, DIAG, DELTA, SR, BITS, true, true, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
@@ -350,6 +396,8 @@ __device__ __forceinline__ void compute_bits(const StepParams &p, uint8_t *stage
                                              float *opart, float *ow, int t) {
   if (d.bits == 32)
     compute_any<DK, DIAG, DELTA, SR, 32, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  else if (d.bits == 0)
+    compute_any<DK, DIAG, DELTA, SR, 0, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else if (d.bits == 4)
     compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else

@@ -32,7 +32,7 @@ class lores_config(C.Structure):
                 ("d_v", C.c_int32), ("group_size", C.c_int32), ("delta", C.c_int32),
                 ("decay_diag", C.c_int32), ("head_bits", C.POINTER(C.c_int32)),
                 ("stochastic", C.c_int32), ("seed", C.c_uint64), ("device", C.c_int32),
-                ("scale_axis", C.c_int32)]
+                ("scale_axis", C.c_int32), ("group_bits", C.POINTER(C.c_int32))]
 
 
 class lores_layout(C.Structure):
@@ -104,14 +104,10 @@ def lores_status_string(status):
 
 
 def lores_create(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                 stochastic=1, seed=0, device=0, scale_axis=0):
-    """Returns an opaque handle (int)."""
-    hb = None
-    if head_bits is not None:
-        arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
-        hb = C.cast(arr, C.POINTER(C.c_int32))
-    cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
-                       seed & (2**64 - 1), device, scale_axis)
+                 stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None):
+    """Returns an opaque handle (int).  group_bits: None or [H][d_k/G] bits per key group."""
+    cfg = make_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, head_bits,
+                      stochastic, seed, device, scale_axis, group_bits)
     out = C.c_void_p()
     _check(_lib.lores_create(C.byref(cfg), C.byref(out)), "lores_create")
     return out.value
@@ -151,16 +147,20 @@ def lores_decode_step_noalloc(cfg, codes, scales, q, k, v, alpha, beta, o, step,
 
 
 def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                stochastic=1, seed=0, device=0, scale_axis=0):
-    """A lores_config; the head_bits array is kept alive on the returned object."""
-    hb = None
-    arr = None
+                stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None):
+    """A lores_config; the bit arrays are kept alive on the returned object."""
+    hb = gb = None
+    arr = garr = None
     if head_bits is not None:
         arr = (C.c_int32 * heads)(*[int(b) for b in head_bits])
         hb = C.cast(arr, C.POINTER(C.c_int32))
+    if group_bits is not None:
+        flat = [int(b) for row in group_bits for b in row]
+        garr = (C.c_int32 * len(flat))(*flat)
+        gb = C.cast(garr, C.POINTER(C.c_int32))
     cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
-                       seed & (2**64 - 1), device, scale_axis)
-    cfg._head_bits_keepalive = arr
+                       seed & (2**64 - 1), device, scale_axis, gb)
+    cfg._keepalive = (arr, garr)
     return cfg
 
 

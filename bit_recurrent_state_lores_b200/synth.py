@@ -52,7 +52,7 @@ class Workload:
     bits: int = 8                        # uniform bits when mixed_frac is None
     mixed_frac: Optional[float] = None   # fraction of heads kept at 8 bits
     warmup: int = 0                      # fp32 warmup steps before quantizing
-    decay: str = "tau"                   # "softplus_normal" | "tau" | "kda"
+    decay: str = "tau"                   # "softplus_normal" | "tau" | "kda" | "kda_channel"
     tau_max: float = 1000.0
     beta_kind: str = "sigmoid"           # "sigmoid" | "softplus_clip"
     outliers: int = 0                    # value channels per head scaled x8
@@ -83,27 +83,37 @@ def workload(name, **over):
     return replace(WORKLOADS[name], **over)
 
 
-def _kda_mu(H):
-    """mu_h with E[exp(-softplus(mu_h + Z))] = m_h, 1 - m_h log-spaced 0.5 .. 1e-4."""
+def _solve_mu(targets):
+    """mu with E[exp(-softplus(mu + Z))] = m for each target m (Z ~ N(0, 1)): 64-point
+    Gauss-Hermite quadrature and bisection, elementwise over an array of targets."""
     z, w = np.polynomial.hermite.hermgauss(64)
     z = z * np.sqrt(2.0)
     w = w / np.sqrt(np.pi)
+    targets = np.asarray(targets, np.float64)
+    lo = np.full(targets.shape, -40.0)
+    hi = np.full(targets.shape, 40.0)             # the mean decay falls as mu rises
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        md = np.sum(w / (1.0 + np.exp(mid[..., None] + z)), axis=-1)
+        up = md > targets
+        lo = np.where(up, mid, lo)
+        hi = np.where(up, hi, mid)
+    return 0.5 * (lo + hi)
 
-    def mean_decay(mu):
-        return float(np.sum(w / (1.0 + np.exp(mu + z))))
 
+def _kda_mu(H):
+    """mu_h with E[exp(-softplus(mu_h + Z))] = m_h, 1 - m_h log-spaced 0.5 .. 1e-4."""
     targets = 1.0 - np.logspace(np.log10(0.5), np.log10(1e-4), H)
-    mus = []
-    for m in targets:
-        lo, hi = -40.0, 40.0          # mean_decay falls as mu rises
-        for _ in range(200):
-            mid = 0.5 * (lo + hi)
-            if mean_decay(mid) > m:
-                lo = mid
-            else:
-                hi = mid
-        mus.append(0.5 * (lo + hi))
-    return np.array(mus), targets
+    return _solve_mu(targets), targets
+
+
+def _kda_channel_mu(H, d_k, g):
+    """Per-channel decay means: in every head the d_k key channels span 1 - m log-spaced
+    0.5 .. 1e-4 in a seeded random order, so the slow channels of a head are scattered
+    over its key groups."""
+    base = 1.0 - np.logspace(np.log10(0.5), np.log10(1e-4), d_k)
+    targets = np.stack([base[torch.randperm(d_k, generator=g).numpy()] for _ in range(H)])
+    return _solve_mu(targets), targets
 
 
 def head_params(wl: Workload, layer: int = 0):
@@ -121,6 +131,11 @@ def head_params(wl: Workload, layer: int = 0):
         mu, target = _kda_mu(wl.H)
         out["mu"] = torch.tensor(mu, dtype=torch.float32)
         out["mean_decay"] = target.astype(np.float32)
+    elif wl.decay == "kda_channel":
+        mu, target = _kda_channel_mu(wl.H, wl.d_k, g)
+        out["mu"] = torch.tensor(mu, dtype=torch.float32)                  # [H, d_k]
+        out["mean_decay_channel"] = target.astype(np.float32)              # [H, d_k]
+        out["mean_decay"] = target.mean(axis=1).astype(np.float32)
     else:  # softplus_normal: E[exp(-softplus(Z))] = E[sigmoid(-Z)] = 1/2 for every head
         out["mean_decay"] = np.full(wl.H, 0.5, np.float32)
     if wl.outliers:
@@ -168,7 +183,8 @@ def step_inputs(wl: Workload, step: int, hp=None, device="cpu", layer: int = 0, 
     elif wl.decay == "tau":
         alpha = hp["alpha_h"].to(device)[None].expand(B, H).contiguous()
     else:
-        y = torch.randn(B, H, dk, **kw) + hp["mu"].to(device)[None, :, None]
+        mu = hp["mu"].to(device)
+        y = torch.randn(B, H, dk, **kw) + (mu[None, :, None] if mu.dim() == 1 else mu[None])
         alpha = torch.exp(-torch.nn.functional.softplus(y))
     return (q.contiguous(), k.contiguous(), v.contiguous(), alpha.contiguous(),
             beta.contiguous())

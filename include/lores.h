@@ -75,6 +75,13 @@ typedef struct {
                             /* column of a tile (the comparator of the Scale Grouping        */
                             /* paragraph; needs G = d_k; a whole tile is processed by one    */
                             /* CTA, so d_v * d_k is limited by shared memory)                 */
+    const int32_t *group_bits; /* NULL, or host [H][d_k/G] bits (4..8) of every key group of   */
+                            /* every head: per-channel precision (the abstract's decay-based  */
+                            /* mixed precision over channels).  A row stores its key groups   */
+                            /* back to back, group g in G*storage(b_g)/8 bytes (4 bits as     */
+                            /* nibbles, 5..8 bits one byte per code); each group is scaled    */
+                            /* with its own r = 2^(b_g-1)-1.  Needs head_bits = NULL and      */
+                            /* scale_axis = 0; not taken by lores_decode_step_noalloc.        */
 } lores_config;
 
 /* Sizes of the handle's state, for export/import buffers. */

@@ -40,7 +40,10 @@ def test_status_strings():
     dict(batch=0), dict(heads=0), dict(d_k=48), dict(d_k=512), dict(d_v=6), dict(d_v=0),
     dict(d_v=8192), dict(group_size=8), dict(group_size=48), dict(delta=2), dict(decay_diag=3),
     dict(stochastic=5), dict(head_bits=[8, 3]), dict(head_bits=[9, 8]), dict(head_bits=[16, 8]),
-    dict(device=-1), dict(scale_axis=2), dict(scale_axis=-1), dict(scale_axis=1, group_size=16)])
+    dict(device=-1), dict(scale_axis=2), dict(scale_axis=-1), dict(scale_axis=1, group_size=16),
+    dict(group_size=32, group_bits=[[8, 4], [4, 4]], head_bits=[8, 8]),
+    dict(group_size=32, group_bits=[[8, 3], [4, 4]]), dict(group_size=32, group_bits=[[8, 9], [4, 4]]),
+    dict(scale_axis=1, group_size=64, group_bits=[[8], [8]])])
 def test_create_rejects_bad_config_before_touching_cuda(kw):
     from bit_recurrent_state_lores_b200 import lores as L
     args = dict(batch=2, heads=2, d_k=64, d_v=16)
@@ -48,6 +51,15 @@ def test_create_rejects_bad_config_before_touching_cuda(kw):
     with pytest.raises(L.LoresError) as e:
         L.lores_create(**args)
     assert e.value.status == L.LORES_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_group_bits_before_touching_cuda():
+    import ctypes as C
+    from bit_recurrent_state_lores_b200 import lores as L
+    cfg = L.make_config(1, 1, 64, 64, group_size=32, group_bits=[[8, 4]])
+    a = 0x10000
+    assert L.raw_library().lores_decode_step_noalloc(C.byref(cfg), a, a, a, a, a, a, a, a, 0,
+                                                     None, None) == L.LORES_ERR_UNSUPPORTED
 
 
 def test_noalloc_rejects_key_axis_before_touching_cuda():

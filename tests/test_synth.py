@@ -62,3 +62,19 @@ def test_mamba2_beta_clipped():
     wl = synth.workload("mamba2", B=8)
     _, _, _, _, b = synth.step_inputs(wl, 0)
     assert b.min() >= 1e-6 and b.max() <= 2 - 1e-6
+
+
+def test_kda_channel_mean_decay_targets():
+    # per-channel decays: each head's channels span 1 - m = 0.5 .. 1e-4 in a seeded order
+    wl = synth.Workload("kdac", B=64, H=3, d_k=32, d_v=16, steps=1, diag=1, decay="kda_channel",
+                        seed=5)
+    hp = synth.head_params(wl)
+    target = hp["mean_decay_channel"]
+    assert target.shape == (3, 32) and hp["mu"].shape == (3, 32)
+    for h in range(3):
+        assert np.allclose(np.sort(1 - target[h].astype(np.float64)),
+                           np.sort(np.logspace(np.log10(0.5), -4, 32)), rtol=0, atol=1e-7)
+    assert not np.array_equal(target[0], target[1])          # orders differ per head
+    alphas = torch.stack([synth.step_inputs(wl, t, hp)[3] for t in range(200)])
+    mean = alphas.double().mean(dim=(0, 1)).numpy()           # [H, d_k]
+    assert np.allclose(mean, target, atol=6e-3)
