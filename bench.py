@@ -97,7 +97,7 @@ def launch_bytes(wl, bits):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("lores.cu", "lores_mt.cu", "lores_step.cuh", "lores_device.cuh"):
+    for f in ("lores_step.cuh", "lores_device.cuh"):       # the decode-step kernel's source
         h.update(open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -437,6 +437,24 @@ def run_sweep(args):
             e1.record()
             torch.cuda.synchronize(dev)
             ms = e0.elapsed_time(e1)
+            # the same steps replayed from one CUDA graph (the 48 launches and the device
+            # step counter's advance captured once)
+            dstep = torch.tensor([args.warmup + args.steps], dtype=torch.int64, device=dev)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                cs = torch.cuda.current_stream(dev).cuda_stream
+                for (h, _, (q, k, v, al, be), o) in layers:
+                    L.lores_decode_step_dev(h, q, k, v, al, be, o, dstep, cs)
+                L.lores_advance_step(dstep, 1, cs)
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            e0.record()
+            for t in range(args.steps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            gms = e0.elapsed_time(e1)
+            del graph
             for (h, _, _, _) in layers:
                 assert L.lores_check_errors(h, sptr) == L.LORES_OK
             step_bytes = sum(launch_bytes(wl, bits) for (_, bits, _, _) in layers)
@@ -447,6 +465,8 @@ def run_sweep(args):
                            "value": wl.B * wl.H * wl.layers * args.steps / (ms / 1e3),
                            "unit": UNIT, "ms_per_step": ms / args.steps,
                            "algorithmic_GBps": gbs, "frac_of_peak": gbs / peak,
+                           "graph_ms_per_step": gms / args.steps,
+                           "graph_value": wl.B * wl.H * wl.layers * args.steps / (gms / 1e3),
                            "l2_resident": state_bytes < 126e6})
             for (h, _, _, _) in layers:
                 L.lores_destroy(h)

@@ -160,6 +160,8 @@ struct KeyParams {
   long long seq_bytes;
   int H, d_v;
   uint32_t step_key;
+  uint64_t seed;
+  const uint64_t *step_dev;     // step in device memory (CUDA-graph replay), or null
   int delta, diag, stochastic;
   // shared memory offsets
   int sm_codes, sm_scales, sm_k, sm_q, sm_a, sm_v, sm_opart, sm_ow, sm_cm;
@@ -247,7 +249,8 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
     // entry (i, j) of S_{t-1} diag(alpha) is c_ij * (s_j * alpha_j)
     aj[e] = (bits == 32 || load) ? al : __fmul_rn(sscales[col0 + e], al);
   }
-  const uint32_t tkey = tile_key(p.step_key, (uint32_t)tile);
+  const uint32_t tkey =
+      tile_key(p.step_dev ? step_key_dev(p.seed, *p.step_dev) : p.step_key, (uint32_t)tile);
 
   // x of one row for this lane's 16 columns (pass 1 and pass 2 compute it identically).
   // `first` (pass 1) computes w with warp shuffles: every lane of the warp takes it, and
@@ -396,6 +399,10 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
   }
 }
 
+// Adds n to a device step counter (one thread; captured into a CUDA graph together with
+// the steps that read the counter).
+__global__ void advance_step_kernel(uint64_t *step, uint64_t n) { *step += n; }
+
 // -------------------------------------------------------------------------------------
 // host side
 // -------------------------------------------------------------------------------------
@@ -455,6 +462,9 @@ static DequantFn dequant_kernel_for(int dk) {
 
 using namespace lores;
 
+constexpr int kGuardBytes = 256;
+constexpr unsigned char kGuardByte = 0xA5;
+
 struct lores_handle {
   lores_config cfg;
   std::vector<int32_t> bits;       // [H]
@@ -512,8 +522,8 @@ lores_status cuda_status(cudaError_t e) {
 }
 
 void free_all(lores_handle *h) {
-  cudaFree(h->codes);
-  cudaFree(h->scales);
+  if (h->codes) cudaFree(h->codes - kGuardBytes);
+  if (h->scales) cudaFree(reinterpret_cast<uint8_t *>(h->scales) - kGuardBytes);
   cudaFree(h->flag);
   cudaFree(h->units);
   cudaFree(h->d_bits);
@@ -559,6 +569,7 @@ const char *lores_status_string(lores_status s) {
     case LORES_ERR_NONFINITE: return "non-finite state";
     case LORES_ERR_UNSUPPORTED: return "unsupported configuration";
     case LORES_ERR_TIMEOUT: return "kernel wait timed out";
+    case LORES_ERR_CORRUPT: return "memory around the state was overwritten";
   }
   return "unknown status";
 }
@@ -813,8 +824,19 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     }
   }
   cudaError_t e = cudaSuccess;
-  if (e == cudaSuccess) e = cudaMalloc(&h->codes, (size_t)code_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&h->scales, (size_t)scale_count * 4);
+  // guard bands of kGuardBytes before and after the code pool and the scales, filled
+  // with kGuardByte and verified by lores_check_errors: a write outside the state shows
+  // up as LORES_ERR_CORRUPT
+  uint8_t *cbase = nullptr, *sbase = nullptr;
+  if (e == cudaSuccess) e = cudaMalloc(&cbase, (size_t)code_bytes + 2 * kGuardBytes);
+  if (e == cudaSuccess) h->codes = cbase + kGuardBytes;
+  if (e == cudaSuccess) e = cudaMalloc(&sbase, (size_t)scale_count * 4 + 2 * kGuardBytes);
+  if (e == cudaSuccess) h->scales = reinterpret_cast<float *>(sbase + kGuardBytes);
+  if (e == cudaSuccess) e = cudaMemset(cbase, kGuardByte, kGuardBytes);
+  if (e == cudaSuccess) e = cudaMemset(cbase + kGuardBytes + code_bytes, kGuardByte, kGuardBytes);
+  if (e == cudaSuccess) e = cudaMemset(sbase, kGuardByte, kGuardBytes);
+  if (e == cudaSuccess)
+    e = cudaMemset(sbase + kGuardBytes + scale_count * 4, kGuardByte, kGuardBytes);
   if (e == cudaSuccess) e = cudaMalloc(&h->flag, 16);
   if (e == cudaSuccess) e = cudaMalloc(&h->units, units.size() * sizeof(UnitDesc));
   if (e == cudaSuccess) e = cudaMalloc(&h->d_bits, c.heads * sizeof(int32_t));
@@ -865,6 +887,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   kp.delta = c.delta;
   kp.diag = c.decay_diag;
   kp.stochastic = c.stochastic;
+  kp.seed = c.seed;
   *out = h;
   return LORES_OK;
 }
@@ -877,9 +900,32 @@ lores_status lores_destroy(lores_handle *h) {
   return LORES_OK;
 }
 
+static lores_status launch_step(lores_handle *h, const float *q, const float *k, const float *v,
+                                const float *alpha, const float *beta, float *o, uint64_t step,
+                                const uint64_t *step_dev, void *stream);
+
 lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, const float *v,
                                const float *alpha, const float *beta, float *o, uint64_t step,
                                void *stream) {
+  return launch_step(h, q, k, v, alpha, beta, o, step, nullptr, stream);
+}
+
+lores_status lores_decode_step_dev(lores_handle *h, const float *q, const float *k, const float *v,
+                                   const float *alpha, const float *beta, float *o,
+                                   const uint64_t *step, void *stream) {
+  if (!step || (reinterpret_cast<uintptr_t>(step) & 7u)) return LORES_ERR_INVALID_ARG;
+  return launch_step(h, q, k, v, alpha, beta, o, 0, step, stream);
+}
+
+lores_status lores_advance_step(uint64_t *step, uint64_t n, void *stream) {
+  if (!step || (reinterpret_cast<uintptr_t>(step) & 7u)) return LORES_ERR_INVALID_ARG;
+  advance_step_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(step, n);
+  return cuda_status(cudaGetLastError());
+}
+
+static lores_status launch_step(lores_handle *h, const float *q, const float *k, const float *v,
+                                const float *alpha, const float *beta, float *o, uint64_t step,
+                                const uint64_t *step_dev, void *stream) {
   if (!h || !q || !k || !v || !alpha || !beta || !o) return LORES_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
       (h->cfg.decay_diag ? !aligned16(alpha) : (reinterpret_cast<uintptr_t>(alpha) & 3u)) ||
@@ -897,6 +943,7 @@ lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, 
     kp.o = o;
     kp.S = nullptr;
     kp.step_key = step_key_of(h->cfg.seed, step);
+    kp.step_dev = step_dev;
     const unsigned tiles = (unsigned)((long long)h->cfg.batch * h->cfg.heads);
     h->key_fn<<<tiles, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
     return cuda_status(cudaGetLastError());
@@ -909,6 +956,8 @@ lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, 
   p.beta = beta;
   p.o = o;
   p.step_key = step_key_of(h->cfg.seed, step);
+  p.seed = h->cfg.seed;
+  p.step_dev = step_dev;
   h->step_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
   return cuda_status(cudaGetLastError());
 }
@@ -1059,6 +1108,8 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
   out->units_per_step = (int32_t)((long long)h->cfg.batch * h->units_per_seq);
   out->grid = h->grid;
   out->smem_bytes = h->smem;
+  out->codes_dev = h->codes;
+  out->scales_dev = h->scales;
   if (head_offsets)
     for (int hh = 0; hh < h->cfg.heads; ++hh) head_offsets[hh] = h->head_off[hh];
   return LORES_OK;
@@ -1075,6 +1126,18 @@ lores_status lores_check_errors(lores_handle *h, void *stream) {
   if (e == cudaSuccess) e = cudaMemset(h->flag, 0, sizeof(unsigned));
   if (e != cudaSuccess) return cuda_status(e);
   if (f & kFlagTimeout) return LORES_ERR_TIMEOUT;
+  // guard bands around the state
+  const long long cb = (long long)h->cfg.batch * h->seq_bytes, sb = scale_count_of(h) * 4;
+  const uint8_t *bands[4] = {h->codes - kGuardBytes, h->codes + cb,
+                             reinterpret_cast<const uint8_t *>(h->scales) - kGuardBytes,
+                             reinterpret_cast<const uint8_t *>(h->scales) + sb};
+  for (const uint8_t *band : bands) {
+    uint8_t host[kGuardBytes];
+    e = cudaMemcpy(host, band, kGuardBytes, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    for (int i = 0; i < kGuardBytes; ++i)
+      if (host[i] != kGuardByte) return LORES_ERR_CORRUPT;
+  }
   if (f & kFlagNonFinite) return LORES_ERR_NONFINITE;
   return LORES_OK;
 }

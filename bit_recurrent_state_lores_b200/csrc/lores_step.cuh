@@ -63,6 +63,8 @@ struct StepParams {
   int T;
   long long tok_qk, tok_v, tok_a, tok_b, tok_o;
   uint64_t seed, step0;
+  // single steps replayed from a captured CUDA graph read the step from device memory
+  const uint64_t *step_dev;
 };
 
 // Step key of the dither: SplitMix64 (Steele, Lea & Flood 2014; Vigna's constants) of the
@@ -196,8 +198,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
 #pragma unroll
   for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
   const float kq = (float)kqd;
-  const uint32_t tkey =
-      tile_key(MT ? step_key_dev(p.seed, p.step0 + (uint64_t)t) : p.step_key, (uint32_t)tile);
+  const uint32_t skey = MT ? step_key_dev(p.seed, p.step0 + (uint64_t)t)
+                           : (p.step_dev ? step_key_dev(p.seed, *p.step_dev) : p.step_key);
+  const uint32_t tkey = tile_key(skey, (uint32_t)tile);
   // shuffle distances of the group-max levels (0 beyond the group width: own value)
   const int gd1 = 1 < lpg ? 1 : 0, gd2 = 2 < lpg ? 2 : 0, gd4 = 4 < lpg ? 4 : 0,
             gd8 = 8 < lpg ? 8 : 0;

@@ -19,6 +19,7 @@ LORES_ERR_CUDA = 3
 LORES_ERR_NONFINITE = 4
 LORES_ERR_UNSUPPORTED = 5
 LORES_ERR_TIMEOUT = 6
+LORES_ERR_CORRUPT = 7
 
 
 class LoresError(RuntimeError):
@@ -38,7 +39,8 @@ class lores_config(C.Structure):
 class lores_layout(C.Structure):
     _fields_ = [("code_bytes", C.c_int64), ("seq_code_bytes", C.c_int64),
                 ("scale_count", C.c_int64), ("n_groups", C.c_int32),
-                ("units_per_step", C.c_int32), ("grid", C.c_int32), ("smem_bytes", C.c_int32)]
+                ("units_per_step", C.c_int32), ("grid", C.c_int32), ("smem_bytes", C.c_int32),
+                ("codes_dev", C.c_void_p), ("scales_dev", C.c_void_p)]
 
 
 def _load():
@@ -53,6 +55,8 @@ def _load():
         "lores_decode_step": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_host": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_steps": (I32, [P, I32, P, P, P, P, P, P, U64, P]),
+        "lores_decode_step_dev": (I32, [P, P, P, P, P, P, P, P, P]),
+        "lores_advance_step": (I32, [P, U64, P]),
         "lores_decode_step_noalloc": (I32, [C.POINTER(lores_config), P, P, P, P, P, P, P, P, U64,
                                             P, P]),
         "lores_dequant_state": (I32, [P, P, P]),
@@ -121,6 +125,18 @@ def lores_decode_step(h, q, k, v, alpha, beta, o, step, stream=None):
     _check(_lib.lores_decode_step(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                   _ptr(o), step & (2**64 - 1), _stream(stream)),
            "lores_decode_step")
+
+
+def lores_decode_step_dev(h, q, k, v, alpha, beta, o, step, stream=None):
+    """The step with its counter in device memory (`step`: int64 tensor of one element)."""
+    _check(_lib.lores_decode_step_dev(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                      _ptr(o), _ptr(step), _stream(stream)),
+           "lores_decode_step_dev")
+
+
+def lores_advance_step(step, n=1, stream=None):
+    _check(_lib.lores_advance_step(_ptr(step), n & (2**64 - 1), _stream(stream)),
+           "lores_advance_step")
 
 
 def lores_decode_steps(h, T, q, k, v, alpha, beta, o, step0, stream=None):
@@ -193,10 +209,10 @@ def lores_get_layout(h, heads=None):
 
 
 def lores_check_errors(h, stream=None):
-    """Returns the status (LORES_OK, LORES_ERR_NONFINITE or LORES_ERR_TIMEOUT); raises
-    on other failures."""
+    """Returns the status (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT or
+    LORES_ERR_CORRUPT); raises on other failures."""
     st = _lib.lores_check_errors(h, _stream(stream))
-    if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT):
+    if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT, LORES_ERR_CORRUPT):
         raise LoresError(st, "lores_check_errors")
     return st
 

@@ -50,7 +50,8 @@ typedef enum {
     LORES_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed                 */
     LORES_ERR_NONFINITE = 4,     /* a state row became non-finite (inf or NaN)            */
     LORES_ERR_UNSUPPORTED = 5,   /* well-formed but not supported (bits, d_k, device)     */
-    LORES_ERR_TIMEOUT = 6        /* a kernel gave up waiting on its own copies            */
+    LORES_ERR_TIMEOUT = 6,       /* a kernel gave up waiting on its own copies            */
+    LORES_ERR_CORRUPT = 7        /* the guard bands around the state were overwritten      */
 } lores_status;
 
 typedef struct lores_handle lores_handle;
@@ -84,7 +85,7 @@ typedef struct {
                             /* scale_axis = 0; not taken by lores_decode_step_noalloc.        */
 } lores_config;
 
-/* Sizes of the handle's state, for export/import buffers. */
+/* Sizes of the handle's state, for export/import buffers, and its device buffers. */
 typedef struct {
     int64_t code_bytes;        /* bytes of the whole code pool = batch * seq_code_bytes      */
     int64_t seq_code_bytes;    /* bytes of one sequence: all heads' tiles back to back       */
@@ -94,6 +95,10 @@ typedef struct {
     int32_t units_per_step;    /* work units (sequence, head, row block) of one step         */
     int32_t grid;              /* CTAs of the decode kernel                                  */
     int32_t smem_bytes;        /* dynamic shared memory per CTA of the decode kernel         */
+    void *codes_dev;           /* the handle's code pool and scales in device memory (owned  */
+    float *scales_dev;         /* by the handle, valid until lores_destroy): for zero-copy    */
+                               /* readers; writes through them must stay inside code_bytes   */
+                               /* and scale_count * 4 bytes                                   */
 } lores_layout;
 
 /* Create a handle: validate `cfg`, allocate the code pool, the scales and the
@@ -123,6 +128,20 @@ lores_status lores_destroy(lores_handle *h);
 lores_status lores_decode_step(lores_handle *h, const float *q, const float *k, const float *v,
                                const float *alpha, const float *beta, float *o,
                                uint64_t step, void *stream);
+
+/* The decode step with its step counter in DEVICE memory (`step`: a uint64_t, 8-byte
+ * aligned, read when the kernel runs), so that a sequence of steps captured once into a
+ * CUDA graph replays with a fresh dither each time; lores_advance_step moves the counter
+ * on the device (also capturable).  Otherwise identical to lores_decode_step: with
+ * *step = t the result equals lores_decode_step(..., t, ...) bit for bit.  Launch-only
+ * (no host synchronisation, no allocation), hence legal inside stream capture.
+ * Errors: INVALID_ARG (as lores_decode_step; NULL or misaligned `step`), CUDA. */
+lores_status lores_decode_step_dev(lores_handle *h, const float *q, const float *k,
+                                   const float *v, const float *alpha, const float *beta,
+                                   float *o, const uint64_t *step, void *stream);
+
+/* *step += n on the device, ordered on `stream`.  Errors: INVALID_ARG, CUDA. */
+lores_status lores_advance_step(uint64_t *step, uint64_t n, void *stream);
 
 /* T consecutive decode steps in one call (a chunk of tokens of each sequence: the
  * decode side of a prefill -> decode handoff, or several tokens per scheduling step).
@@ -212,9 +231,12 @@ lores_status lores_load_codes(lores_handle *h, const void *codes, const float *s
  * byte offsets of each head's tile inside one sequence's block. */
 lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t *head_offsets);
 
-/* Wait for `stream`, then read and clear the handle's sticky device flag.
+/* Wait for `stream`, then read and clear the handle's sticky device flag and verify
+ * the 256-byte guard bands written around the code pool and the scales at creation.
  * Returns LORES_ERR_TIMEOUT if a kernel gave up waiting on its own copies (its
- * outputs for that call are incomplete), else LORES_ERR_NONFINITE if any row
+ * outputs for that call are incomplete), else LORES_ERR_CORRUPT if a guard band was
+ * overwritten (a write outside the state: a library defect, or a caller's write
+ * through a pointer derived from the state), else LORES_ERR_NONFINITE if any row
  * became non-finite since the last check, else LORES_OK. */
 lores_status lores_check_errors(lores_handle *h, void *stream);
 

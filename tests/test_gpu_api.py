@@ -180,3 +180,28 @@ def test_many_handles_with_different_shared_memory_needs():
     for r in runs:
         assert r.check() == lib().LORES_OK
         r.close()
+
+
+def test_guard_bands_report_writes_outside_the_state():
+    # host-side fault injection: write one byte just past the code pool and one just
+    # before the scales (inside the guard bands the library allocates around them)
+    L = lib()
+    wl = small()
+    g = GpuRun(wl, [8, 4, 8], seed=1)
+    hp = synth.head_params(wl)
+    g.step(synth.step_inputs(wl, 0, hp, device="cuda"), 0)
+    assert g.check() == L.LORES_OK
+    from cuda.bindings import runtime as rt
+    lay = g.layout
+    torch.cuda.synchronize()
+    (err,) = rt.cudaMemset(lay.codes_dev + lay.code_bytes, 0x11, 1)
+    assert err == rt.cudaError_t.cudaSuccess
+    assert rt.cudaDeviceSynchronize()[0] == rt.cudaError_t.cudaSuccess
+    assert g.check() == L.LORES_ERR_CORRUPT
+    assert "overwritten" in L.lores_status_string(L.LORES_ERR_CORRUPT)
+    g.close()
+    g = GpuRun(wl, [8, 4, 8], seed=1)
+    (err,) = rt.cudaMemset(g.layout.scales_dev - 1, 0x11, 1)
+    assert err == rt.cudaError_t.cudaSuccess
+    assert g.check() == L.LORES_ERR_CORRUPT
+    g.close()
