@@ -253,3 +253,57 @@ def test_sweep_layers_in_bench_launch_configuration(variant):
         tiles = sample_tiles(wll, bits, 4, seed=layer)
         g = run_free(wll, bits, 77 + layer, tiles, steps, check_every=3)
         g.close()
+
+
+# ---------------------------------------------------------------------------------------
+# maximum sizes and degenerate inputs
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [[8], [4], [32], [6]])
+def test_largest_tile_every_step(bits):
+    # the largest tile the library takes: d_k = 256, d_v = 4096 (units split the rows)
+    wl = synth.Workload("max", B=1, H=1, d_k=256, d_v=4096, steps=3, delta=1, diag=1,
+                        group=64, decay="kda", outliers=4, seed=21)
+    g = run_free(wl, bits, seed=3, tiles=[(0, 0)], steps=3, exact=True)
+    g.close()
+
+
+def test_degenerate_inputs_match_oracle():
+    # alpha = 1 (no forgetting), beta = 0 (no write), k = q = 0 on some heads, a zero value
+    # row: every tile at every step equals the oracle, and nothing is flagged
+    wl = synth.Workload("degen", B=2, H=4, d_k=64, d_v=32, steps=4, delta=1, diag=0,
+                        group=32, decay="tau", outliers=0, seed=5)
+    bits = [8, 4, 6, 32]
+    hp = synth.head_params(wl)
+    g = GpuRun(wl, bits, seed=9)
+    tiles = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    ref = OracleTiles(wl, bits, 9, tiles)
+    for step in range(wl.steps):
+        q, k, v, a, b = [x.clone() for x in synth.step_inputs(wl, step, hp, device="cuda")]
+        a[:, 0] = 1.0                        # head 0: no decay
+        b[:, 1] = 0.0                        # head 1: no write (pure decay)
+        if step >= 2:
+            k[:, 2] = 0.0                    # head 2: k = q = 0 (decay only; readout 0)
+            q[:, 2] = 0.0
+        v[0, 3, 5] = 0.0
+        inp = (q, k, v, a, b)
+        o = g.step(inp, step).cpu().numpy()
+        oref, flags = ref.step(host_tile_inputs(inp, tiles), step)
+        codes, scales = g.export()
+        for t in tiles:
+            assert flags[t] == 0
+            assert rel_l2(o[t], oref[t]) <= 1e-5 or np.abs(o[t] - oref[t]).max() <= 1e-12
+            gs, gsc = g.tile(codes, scales, *t)
+            rs, rsc = ref.state[t]
+            if bits[t[1]] == 32:
+                assert np.array_equal(gs, rs)
+                continue
+            assert assert_parity(ref.cfg[t], gs, gsc, rs, rsc, f"{step} {t}") == 0
+            assert np.array_equal(gsc, rsc)
+    assert g.check() == lib_ok()
+    g.close()
+
+
+def lib_ok():
+    from bit_recurrent_state_lores_b200 import lores
+    return lores.LORES_OK
