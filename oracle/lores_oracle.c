@@ -118,6 +118,8 @@ typedef struct {
                         * 1: key-axis (one scale per key column, scales [d_k]) */
     const int *group_bits; /* NULL, or bits (4..8) of each of the d_k/G key groups:
                             * per-channel precision (value axis only; bits unused) */
+    int dense;         /* 1: 5- to 7-bit codes in bit planes (see dense_*); 0: one
+                        * byte per code.  Per-head bits only (group_bits NULL). */
 } lo_cfg;
 
 static int code_max(int bits) { return (1 << (bits - 1)) - 1; }
@@ -137,11 +139,87 @@ static size_t group_offset(const lo_cfg *c, int g)
 }
 static size_t quant_row_bytes(const lo_cfg *c) { return group_offset(c, c->d_k / c->group); }
 
+/* Dense b-bit codes, b = 5, 6, 7 (cfg.dense = 1).  A code c is stored in offset binary,
+ * u = c + 2^(b-1) in [1, 2^b - 1], split into bit planes laid out one row after another:
+ *   row = [4-bit plane: d_k/2 bytes][2-bit plane: d_k/4 bytes if b >= 6]
+ *         [1-bit plane: d_k/8 bytes if b is odd], padded to a multiple of 8 bytes.
+ * 4-bit plane: u & 15 of column j in byte j/2, low nibble for even j (the int4 layout).
+ * 2-bit plane: (u >> 4) & 3; the 16-column block l owns the 4 bytes at 4l; inside the
+ *   block, byte p (p = 0..3) holds column 8+2p in bits 0-1, column 9+2p in bits 2-3,
+ *   column 2p in bits 4-5 and column 2p+1 in bits 6-7.
+ * 1-bit plane: the top bit of u (bit 4 for b = 5, bit 6 for b = 7); block l owns the 2
+ *   bytes at 2l; byte 0 holds columns 0, 2, 4, 6 in bits 0-3 and columns 1, 3, 5, 7 in
+ *   bits 4-7, byte 1 likewise columns 8..15.
+ * (These positions let a lane that holds 16 columns rebuild each code's byte with a few
+ * shifts and masks per 4 codes.) */
+static int is_dense(const lo_cfg *c) { return c->dense && !c->group_bits && c->bits >= 5 && c->bits <= 7; }
+static size_t dense_row_bytes(const lo_cfg *c)
+{
+    size_t b = (size_t)c->d_k * c->bits / 8;
+    return (b + 7) / 8 * 8;
+}
+static size_t plane2_offset(const lo_cfg *c) { return (size_t)c->d_k / 2; }
+static size_t plane1_offset(const lo_cfg *c) { return (size_t)c->d_k / 2 + (c->bits >= 6 ? (size_t)c->d_k / 4 : 0); }
+/* byte and bit of column j's field in the 2-bit / 1-bit plane of a row */
+static void plane2_pos(int j, size_t *byte, int *bit)
+{
+    int l = j / 16, cc = j % 16, p = (cc % 8) / 2;
+    *byte = (size_t)4 * l + p;
+    *bit = cc < 8 ? (cc % 2 == 0 ? 4 : 6) : (cc % 2 == 0 ? 0 : 2);
+}
+static void plane1_pos(int j, size_t *byte, int *bit)
+{
+    int l = j / 16, cc = j % 16, half = cc / 8, k = cc % 8;
+    *byte = (size_t)2 * l + half;
+    *bit = (k % 2 == 0) ? k / 2 : 4 + k / 2;
+}
+static int dense_get(const lo_cfg *c, const uint8_t *codes, int i, int j)
+{
+    const uint8_t *row = codes + (size_t)i * dense_row_bytes(c);
+    uint8_t nb = row[j / 2];
+    int u = (j % 2 == 0) ? (nb & 0xF) : (nb >> 4);
+    size_t at;
+    int bit;
+    if (c->bits >= 6) {
+        plane2_pos(j, &at, &bit);
+        u |= ((row[plane2_offset(c) + at] >> bit) & 3) << 4;
+    }
+    if (c->bits % 2 == 1) {
+        plane1_pos(j, &at, &bit);
+        u |= ((row[plane1_offset(c) + at] >> bit) & 1) << (c->bits - 1);
+    }
+    return u - (1 << (c->bits - 1));
+}
+static void dense_put(const lo_cfg *c, uint8_t *codes, int i, int j, int code)
+{
+    uint8_t *row = codes + (size_t)i * dense_row_bytes(c);
+    int u = code + (1 << (c->bits - 1));
+    uint8_t *nb = &row[j / 2];
+    if (j % 2 == 0)
+        *nb = (uint8_t)((*nb & 0xF0) | (u & 0xF));
+    else
+        *nb = (uint8_t)((*nb & 0x0F) | ((u & 0xF) << 4));
+    size_t at;
+    int bit;
+    if (c->bits >= 6) {
+        plane2_pos(j, &at, &bit);
+        uint8_t *q = &row[plane2_offset(c) + at];
+        *q = (uint8_t)((*q & ~(3 << bit)) | (((u >> 4) & 3) << bit));
+    }
+    if (c->bits % 2 == 1) {
+        plane1_pos(j, &at, &bit);
+        uint8_t *q = &row[plane1_offset(c) + at];
+        *q = (uint8_t)((*q & ~(1 << bit)) | (((u >> (c->bits - 1)) & 1) << bit));
+    }
+}
+
 /* Read code (i, j) from a packed tile.  5 to 8 bits: one byte per code, two's
- * complement.  4 bits: two codes per byte, even column in the low nibble, odd
- * column in the high nibble, two's complement nibbles. */
+ * complement (or the dense planes above).  4 bits: two codes per byte, even column in
+ * the low nibble, odd column in the high nibble, two's complement nibbles. */
 static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
 {
+    if (is_dense(c))
+        return dense_get(c, codes, i, j);
     int g = j / c->group, jj = j - g * c->group;
     const uint8_t *grp = codes + (size_t)i * quant_row_bytes(c) + group_offset(c, g);
     if (group_bits_of(c, g) != 4)
@@ -153,6 +231,10 @@ static int get_code(const lo_cfg *c, const uint8_t *codes, int i, int j)
 
 static void put_code(const lo_cfg *c, uint8_t *codes, int i, int j, int code)
 {
+    if (is_dense(c)) {
+        dense_put(c, codes, i, j, code);
+        return;
+    }
     int g = j / c->group, jj = j - g * c->group;
     uint8_t *grp = codes + (size_t)i * quant_row_bytes(c) + group_offset(c, g);
     if (group_bits_of(c, g) != 4) {

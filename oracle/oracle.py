@@ -19,7 +19,7 @@ _lib = None
 class LoCfg(C.Structure):
     _fields_ = [("d_k", C.c_int), ("d_v", C.c_int), ("group", C.c_int), ("bits", C.c_int),
                 ("delta", C.c_int), ("diag", C.c_int), ("stochastic", C.c_int),
-                ("axis", C.c_int), ("group_bits", C.c_void_p)]
+                ("axis", C.c_int), ("group_bits", C.c_void_p), ("dense", C.c_int)]
 
 
 def lib():
@@ -74,7 +74,7 @@ class TileCfg:
     """Shape and recipe of one (sequence, head) tile."""
 
     def __init__(self, d_k, d_v, group=None, bits=8, delta=1, diag=0, stochastic=1, axis=0,
-                 group_bits=None):
+                 group_bits=None, dense=0):
         self.d_k, self.d_v = int(d_k), int(d_v)
         self.group = int(group if group else d_k)
         self.bits, self.delta, self.diag, self.stochastic = int(bits), int(delta), int(diag), int(stochastic)
@@ -87,8 +87,10 @@ class TileCfg:
             assert self.group_bits.shape == (self.d_k // self.group,) and not self.axis
             self.bits = 0
             gb = self.group_bits.ctypes.data_as(C.c_void_p)
+        # dense: 5- to 7-bit codes in bit planes instead of one byte each
+        self.dense = int(bool(dense) and group_bits is None and 5 <= self.bits <= 7)
         self.c = LoCfg(self.d_k, self.d_v, self.group, self.bits, self.delta, self.diag,
-                       self.stochastic, self.axis, gb)
+                       self.stochastic, self.axis, gb, self.dense)
 
     @property
     def n_groups(self):
@@ -107,6 +109,8 @@ class TileCfg:
     def code_bytes(self):
         if self.group_bits is not None:
             return self.d_v * self.row_bytes()
+        if self.dense:
+            return self.d_v * ((self.d_k * self.bits // 8 + 7) // 8 * 8)
         if self.bits == 32:
             return self.d_v * self.d_k * 4
         if self.bits == 4:

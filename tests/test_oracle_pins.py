@@ -730,3 +730,57 @@ def test_group_bits_step_matches_fp64_update():
     C_ = O.unpack_codes(cfg, codes)
     err = np.abs(C_ * np.repeat(scales.astype(np.float64), G, axis=1) - x)
     assert (err <= np.repeat(scales.astype(np.float64), G, axis=1) * (1 + 1e-6)).all()
+
+
+# --------------------------------------------------------------------------
+# Dense 5- to 7-bit codes: offset binary split into 4-, 2- and 1-bit planes
+# --------------------------------------------------------------------------
+
+def test_dense_layout_worked_examples():
+    # bytes written out by hand from the plane layout (16 columns, one row, padded to 16)
+    cases = {
+        6: ([-31, 31, 0, 1, -1, 15, -16, 16, 7, -7, 30, -30, 2, -2, 5, -5],
+            [0xF1, 0x10, 0xFF, 0x00, 0x97, 0x2E, 0xE2, 0xB5, 0xC6, 0xA3, 0x96, 0xD6, 0, 0, 0, 0]),
+        5: ([-15, 15, 0, 1, -1, 7, -8, 8, 3, -3, 14, -14, 2, -2, 5, -5],
+            [0xF1, 0x10, 0x7F, 0x88, 0xD3, 0x2E, 0xE2, 0xB5, 0xF2, 0x0F, 0, 0, 0, 0, 0, 0]),
+        7: ([-63, 63, 0, 1, -1, 31, -32, 32, 7, -7, 62, -62, 2, -2, 45, -45],
+            [0xF1, 0x10, 0xFF, 0x00, 0x97, 0x2E, 0xE2, 0x3D, 0xCC, 0x03, 0x7C, 0xA6, 0xF2, 0x0F,
+             0, 0]),
+    }
+    for bits, (ints, want) in cases.items():
+        cfg = O.TileCfg(16, 1, bits=bits, dense=1)
+        assert cfg.code_bytes() == 16
+        b = O.pack_codes(cfg, np.array([ints]))
+        assert b.tolist() == want, (bits, [hex(x) for x in b])
+        assert (O.unpack_codes(cfg, b) == np.array([ints])).all()
+
+
+@pytest.mark.parametrize("bits", [5, 6, 7])
+def test_dense_round_trip_and_row_sizes(bits):
+    r = (1 << (bits - 1)) - 1
+    for d_k, row in ((16, 16), (32, {5: 24, 6: 24, 7: 32}[bits]), (128, 16 * bits)):
+        cfg = O.TileCfg(d_k, 3, bits=bits, dense=1)
+        assert cfg.code_bytes() == 3 * row
+        ints = np.tile(np.arange(-r, r + 1), 3 * d_k)[:3 * d_k].reshape(3, d_k)
+        assert (O.unpack_codes(cfg, O.pack_codes(cfg, ints)) == ints).all()
+
+
+@pytest.mark.parametrize("bits", [5, 6, 7])
+def test_dense_codes_equal_byte_codes(bits):
+    # the layout does not change the arithmetic: the same state, step and dither give the
+    # same codes and scales in either layout
+    d_k, d_v, G = 64, 12, 32
+    dense = O.TileCfg(d_k, d_v, group=G, bits=bits, dense=1, delta=1, diag=1)
+    plain = O.TileCfg(d_k, d_v, group=G, bits=bits, delta=1, diag=1)
+    g = rng(90 + bits)
+    S = (g.standard_normal((d_v, d_k)) * np.exp(g.uniform(-3, 3, (d_v, 1)))).astype(np.float32)
+    tk = O.tile_key(O.step_key(8, 2), 5)
+    cd, sd, _ = O.tile_quantize(dense, S, tk)
+    cp, sp, _ = O.tile_quantize(plain, S, tk)
+    assert np.array_equal(sd, sp)
+    assert np.array_equal(O.unpack_codes(dense, cd), O.unpack_codes(plain, cp))
+    q, k, v, alpha, beta = draw(1, d_k, d_v, 91, diag=True)
+    od, _, _ = O.tile_step(dense, cd, sd, q[0], k[0], v[0], alpha[0], beta[0], tk)
+    op, _, _ = O.tile_step(plain, cp, sp, q[0], k[0], v[0], alpha[0], beta[0], tk)
+    assert np.array_equal(od, op) and np.array_equal(sd, sp)
+    assert np.array_equal(O.unpack_codes(dense, cd), O.unpack_codes(plain, cp))
