@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--formats", action="store_true",
+                    help="launch time of one layer's step for every state format and mode "
+                         "(batch --batch, 32 heads, 128 x 128), one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="time every batch x state-format point of the 48-layer sweep (one GPU)")
     return ap.parse_args()
@@ -479,6 +482,74 @@ def run_sweep(args):
                        "rounding": "stochastic"}}
 
 
+def run_formats(args):
+    """One layer (batch args.batch, 32 heads, 128 x 128, GDN-style inputs of step 0): the mean
+    launch time of the decode step over `steps` launches after `warmup`, for every state
+    format and mode the library has, with the algorithmic bytes of one launch.  Per-channel
+    rows use 32-column groups with 8 bits on a quarter of the (head, group) pairs."""
+    import torch
+    from bit_recurrent_state_lores_b200 import lores as L
+    from bit_recurrent_state_lores_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = measured_peak()
+    B, H, dk, dv = args.batch, 32, 128, 128
+    mix = [8 if h % 4 == 0 else 4 for h in range(H)]
+    chan = [[8 if (h + g) % 4 == 0 else 4 for g in range(4)] for h in range(H)]
+    cases = [
+        ("int8", dict(bits=[8] * H)), ("int8 round-to-nearest", dict(bits=[8] * H, sr=0)),
+        ("int8 delta=0", dict(bits=[8] * H, delta=0)), ("int4", dict(bits=[4] * H)),
+        ("mixed 25% int8 / int4 heads", dict(bits=mix)), ("fp32 reference state", dict(bits=[32] * H)),
+        ("int6 one byte per code", dict(bits=[6] * H)), ("int6 dense planes", dict(bits=[6] * H, dense=1)),
+        ("int5 dense planes", dict(bits=[5] * H, dense=1)), ("int7 dense planes", dict(bits=[7] * H, dense=1)),
+        ("per-channel 8/4 bits, G = 32", dict(group_bits=chan, G=32)),
+        ("key-axis scales, int8", dict(bits=[8] * H, axis=1)),
+        ("key-axis scales, int4", dict(bits=[4] * H, axis=1)),
+        ("int8, 8 tokens per call (per token)", dict(bits=[8] * H, tokens=8)),
+    ]
+    wl = synth.workload("sweep", B=B)
+    hp = synth.head_params(wl)
+    inp = synth.step_inputs(wl, 0, hp, device=dev)
+    o = torch.empty(B, H, dv, device=dev)
+    out = []
+    for name, c in cases:
+        gb = c.get("group_bits")
+        h = L.lores_create(B, H, dk, dv, group_size=c.get("G", 0), delta=c.get("delta", 1),
+                           head_bits=None if gb else c["bits"], stochastic=c.get("sr", 1),
+                           seed=1, scale_axis=c.get("axis", 0), group_bits=gb,
+                           dense_codes=c.get("dense", 0))
+        lay, _ = L.lores_get_layout(h, H)
+        T = c.get("tokens", 1)
+        if T > 1:
+            st = [torch.stack([x] * T).contiguous() for x in inp]
+            oo = torch.empty(T, B, H, dv, device=dev)
+            call = lambda t: L.lores_decode_steps(h, T, *st, oo, t * T)
+        else:
+            call = lambda t: L.lores_decode_step(h, *inp, o, t)
+        for t in range(args.warmup):
+            call(t)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for t in range(args.steps):
+            call(args.warmup + t)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / args.steps / T
+        assert L.lores_check_errors(h) == L.LORES_OK
+        # algorithmic bytes per token: state read + written once per call, inputs per token
+        vec = B * H * (2 * dk * 4 + 2 * dv * 4 + 8)  # q, k, v, alpha, beta read; o written
+        state = 2 * (lay.code_bytes + lay.scale_count * 4)
+        nbytes = state / T + vec
+        out.append({"format": name, "us_per_token": us, "state_bytes": lay.code_bytes + lay.scale_count * 4,
+                    "algorithmic_GBps": nbytes / us / 1e3, "frac_of_peak": nbytes / us / 1e3 / peak})
+        L.lores_destroy(h)
+    return {"metric": "decode-step launch time per token by state format", "batch": B,
+            "heads": H, "d_k": dk, "d_v": dv, "steps": args.steps, "warmup": args.warmup,
+            "peak_GBps": peak, "peak_kind": peak_kind, "formats": out}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: same metric, timed on host cores."""
     if rank != 0:
@@ -514,6 +585,9 @@ def main():
         return
     if args.sweep:
         print(json.dumps(run_sweep(args)), flush=True)
+        return
+    if args.formats:
+        print(json.dumps(run_formats(args)), flush=True)
         return
     import torch
     import torch.distributed as dist

@@ -77,8 +77,18 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   const uint32_t n0 = (uint32_t)row * (uint32_t)(DK / 4) + (uint32_t)lir * 4u;
   uint32_t words[4];
   float s_new;
-  requantize16<LPR>(x, bits == 32 ? 8 : bits, lpg, lane, tkey, n0, p.stochastic, words, s_new);
+  requantize16<LPR>(x, bits == 32 ? 8 : bits, lpg, lane, tkey, n0, p.stochastic, words, s_new,
+                    f.store);
   if (!active) return;
+  if (f.store >= 5 && f.store <= 7) {                 // dense bit planes
+    const DenseLane dl{words[0], words[1], words[2], words[3]};
+    uint8_t *rowp = tilecodes + (size_t)row * f.rowb;
+    if (f.store == 5) st_dense<5>(rowp, DK, lir, dl);
+    else if (f.store == 6) st_dense<6>(rowp, DK, lir, dl);
+    else st_dense<7>(rowp, DK, lir, dl);
+    if (lir % lpg == 0) p.scales[grr * p.ng + g] = s_new;
+    return;
+  }
   uint8_t *dst = tilecodes + (size_t)row * f.rowb + f.off;
   if (bits == 32) {
 #pragma unroll
@@ -121,10 +131,19 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
     }
   } else {
     float cf[16];
-    if (bits != 4)
+    if (f.store >= 5 && f.store <= 7) {               // dense bit planes
+      const uint8_t *rowp = lanecodes - f.off;
+      float2 c2[8];
+      if (f.store == 5) unpack_dense<5>(ld_dense<5>(rowp, DK, lir), c2);
+      else if (f.store == 6) unpack_dense<6>(ld_dense<6>(rowp, DK, lir), c2);
+      else unpack_dense<7>(ld_dense<7>(rowp, DK, lir), c2);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { cf[2 * e] = c2[e].x; cf[2 * e + 1] = c2[e].y; }
+    } else if (bits != 4) {
       unpack_i8(ld16_a8(lanecodes), cf);          // lane blocks are 8-byte aligned
-    else
+    } else {
       unpack_i4(*reinterpret_cast<const uint2 *>(lanecodes), cf);
+    }
     if (p.axis) {
       const float *sc = p.scales + tile * DK + col0;          // one scale per key column
 #pragma unroll
@@ -480,6 +499,7 @@ struct lores_handle {
   LaneFmt *d_fmt = nullptr;        // [H][d_k/16]
   std::vector<LaneFmt> fmt;
   std::vector<int32_t> rowb;       // [H] bytes of one row
+  std::vector<int32_t> store;      // [H] storage class (see UnitDesc::store)
   int units_per_seq = 0;
   int grid = 0;
   int smem = 0;
@@ -618,6 +638,8 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   // one width is an ordinary head of that width, any other head is "mixed" (bits 0)
   const int ngr = dk / G;
   std::vector<int32_t> gbits((size_t)c.heads * ngr);
+  if (c.dense_codes != 0 && c.dense_codes != 1) return LORES_ERR_INVALID_ARG;
+  if (c.dense_codes && (c.group_bits || c.scale_axis)) return LORES_ERR_INVALID_ARG;
   if (c.group_bits) {
     if (c.head_bits || c.scale_axis) return LORES_ERR_INVALID_ARG;
     for (int h = 0; h < c.heads; ++h) {
@@ -655,23 +677,29 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->axis = c.scale_axis;
   // row layout: key groups back to back, group g in G * storage(b_g) / 8 bytes; the lane
   // table gives each 16-column block its width, offset, r and fl(1/r)
+  // dense_codes: heads of 5 to 7 bits store their codes in bit planes (storage class b)
   h->head_off.resize(c.heads);
   h->rowb.assign(c.heads, 0);
+  h->store.assign(c.heads, 8);
   h->fmt.resize((size_t)c.heads * (dk / 16));
   long long off = 0;
   for (int hh = 0; hh < c.heads; ++hh) {
+    const bool dense = c.dense_codes && bits[hh] >= 5 && bits[hh] <= 7;
+    h->store[hh] = bits[hh] == 0 ? 0 : (dense ? bits[hh] : storage_bits(bits[hh]));
     int goff = 0;
     for (int g = 0; g < ngr; ++g) {
       const int b = bits[hh] == 32 ? 32 : gbits[(size_t)hh * ngr + g];
       for (int lb = g * G / 16; lb < (g + 1) * G / 16; ++lb) {
         LaneFmt &f = h->fmt[(size_t)hh * (dk / 16) + lb];
-        f.bits = (int16_t)b;
-        f.off = goff + (lb * 16 - g * G) * storage_bits(b) / 8;
+        f.bits = (int8_t)b;
+        f.store = (int8_t)(dense ? b : storage_bits(b));
+        f.off = dense ? 8 * lb : goff + (lb * 16 - g * G) * storage_bits(b) / 8;
         f.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
         f.inv_r = b == 32 ? 0.0f : 1.0f / f.r;
       }
       goff += G * storage_bits(b) / 8;
     }
+    if (dense) goff = store_row_bytes(dk, bits[hh]);
     h->rowb[hh] = goff;
     for (int lb = 0; lb < dk / 16; ++lb) h->fmt[(size_t)hh * (dk / 16) + lb].rowb = (int16_t)goff;
     h->head_off[hh] = off;
@@ -705,10 +733,11 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       for (int r0 = 0; r0 < dv; r0 += R) {
         UnitDesc d{};
         d.head = hh;
-        d.row0 = r0;
-        d.nrows = std::min(R, dv - r0);
+        d.row0 = (int16_t)r0;
+        d.nrows = (int16_t)std::min(R, dv - r0);
         d.bits = (int16_t)b;
         d.rowb = (int16_t)rb;
+        d.store = (int16_t)h->store[hh];
         d.code_off = h->head_off[hh] + (long long)r0 * rb;
         d.r = (b == 32 || b == 0) ? 0.0f : (float)((1 << (b - 1)) - 1);
         d.inv_r = (b == 32 || b == 0) ? 0.0f : 1.0f / d.r;
@@ -718,18 +747,20 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   };
   std::vector<UnitDesc> units;
   int ctas_per_sm = 1;
-  auto bits_rank = [](int b) { return b == 0 ? 3 : (storage_bits(b) == 8 ? 0 : (b == 4 ? 1 : 2)); };
+  auto bits_rank = [](const UnitDesc &u) {
+    return u.store == 8 ? 0 : (u.store == 4 ? 1 : (u.store == 32 ? 2 : 3 + u.store));
+  };
   for (;;) {
     build_units(units);
     std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
-      return bits_rank(x.bits) < bits_rank(y.bits);
+      return bits_rank(x) < bits_rank(y);
     });
     int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
     for (const UnitDesc &d : units) {
       cmax = std::max(cmax, d.nrows * (int)d.rowb);
       if (d.bits != 32) smax = std::max(smax, d.nrows * h->ng * 4);
       vmax = std::max(vmax, d.nrows * 4);
-      maxrows = std::max(maxrows, d.nrows);
+      maxrows = std::max(maxrows, (int)d.nrows);
     }
     auto up16 = [](int x) { return (x + 15) & ~15; };
     const int stage = up16(cmax) + up16(smax) + up16(vmax) + 2 * dk * 4 +
@@ -1207,7 +1238,8 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   if ((c.delta != 0 && c.delta != 1) || (c.decay_diag != 0 && c.decay_diag != 1) ||
       (c.stochastic != 0 && c.stochastic != 1) || c.device < 0)
     return LORES_ERR_INVALID_ARG;
-  if (c.scale_axis != 0 || c.group_bits) return LORES_ERR_UNSUPPORTED;   // per-head widths,
+  if (c.scale_axis != 0 || c.group_bits || c.dense_codes)
+    return LORES_ERR_UNSUPPORTED;                       // per-head byte/nibble codes,
                                                                           // value-axis groups
   for (int hh = 0; c.head_bits && hh < c.heads; ++hh)
     if (!((c.head_bits[hh] >= 4 && c.head_bits[hh] <= 8) || c.head_bits[hh] == 32))
@@ -1226,23 +1258,24 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   const int ng = dk / G, LPR = dk / 16;
   for (int hh = 0; hh < c.heads; ++hh) {
     const int b = c.head_bits ? c.head_bits[hh] : 8;
-    const int R = std::min(full_rows(dk, b), dv);
+    const int R = std::min(full_rows(dk, storage_bits(b)), dv);
     for (int r0 = 0; r0 < dv; r0 += R) {
       if (nunits == kNoAllocMaxUnits) return LORES_ERR_UNSUPPORTED;   // beyond the fixed table
       UnitDesc &d = units[nunits++];
       d = UnitDesc{};
       d.head = hh;
-      d.row0 = r0;
-      d.nrows = std::min(R, dv - r0);
+      d.row0 = (int16_t)r0;
+      d.nrows = (int16_t)std::min(R, dv - r0);
       d.bits = (int16_t)b;
       d.rowb = (int16_t)row_bytes(dk, b);
+      d.store = (int16_t)storage_bits(b);
       d.code_off = seq_bytes + (long long)r0 * row_bytes(dk, b);
       d.r = b == 32 ? 0.0f : (float)((1 << (b - 1)) - 1);
       d.inv_r = b == 32 ? 0.0f : 1.0f / d.r;
       cmax = std::max(cmax, d.nrows * row_bytes(dk, b));
       if (b != 32) smax = std::max(smax, d.nrows * ng * 4);
       vmax = std::max(vmax, d.nrows * 4);
-      maxrows = std::max(maxrows, d.nrows);
+      maxrows = std::max(maxrows, (int)d.nrows);
     }
     seq_bytes += (long long)dv * row_bytes(dk, b);
   }

@@ -221,6 +221,103 @@ __device__ __forceinline__ uint2 pack_i4(const uint32_t (&t)[16]) {
   return make_uint2(w[0], w[1]);
 }
 
+// Dense 5- to 7-bit codes (B = 5, 6, 7): offset binary u = c + 2^(B-1) split into a 4-bit
+// plane (the int4 nibble layout), a 2-bit plane (B >= 6) and a 1-bit plane (B odd).  A
+// lane's 16 columns own 8 nibble bytes, one 2-bit word and one 16-bit 1-bit word:
+//   2-bit word, byte p: column 8+2p in bits 0-1, 9+2p in 2-3, 2p in 4-5, 2p+1 in 6-7;
+//   1-bit word: columns 0,2,4,6 in bits 0-3, 1,3,5,7 in 4-7, 8..14 even in 8-11, odd in 12-15.
+// E0/O0/E1/O1 below are the offset-binary bytes of the even/odd columns of the two halves.
+struct DenseLane {
+  uint32_t nib0, nib1, p2, p1;
+};
+
+// Bit `s` of each byte of w, gathered into bits 0-3 (byte p -> bit p).
+template <int S>
+__device__ __forceinline__ uint32_t gather_bit4(uint32_t w) {
+  return (((w >> S) & 0x01010101u) * 0x01020408u) >> 24;
+}
+// Bits 0-3 of q spread to bit S of bytes 0-3 (bit p -> byte p).
+template <int S>
+__device__ __forceinline__ uint32_t spread_bit4(uint32_t q) {
+  return (((q & 0xFu) * 0x00204081u) & 0x01010101u) << S;
+}
+
+// t[e] = 49152 + u_e + fraction (byte 1 of t is u).
+template <int B>
+__device__ __forceinline__ DenseLane pack_dense(const uint32_t (&t)[16]) {
+  auto gather = [&](int a) {                 // byte 1 of t[a], t[a+2], t[a+4], t[a+6]
+    const uint32_t lo = __byte_perm(t[a], t[a + 2], 0x0051u);
+    const uint32_t hi = __byte_perm(t[a + 4], t[a + 6], 0x0051u);
+    return __byte_perm(lo, hi, 0x5410u);
+  };
+  const uint32_t E0 = gather(0), O0 = gather(1), E1 = gather(8), O1 = gather(9);
+  DenseLane d;
+  d.nib0 = (E0 & 0x0F0F0F0Fu) | ((O0 << 4) & 0xF0F0F0F0u);
+  d.nib1 = (E1 & 0x0F0F0F0Fu) | ((O1 << 4) & 0xF0F0F0F0u);
+  d.p2 = 0u;
+  d.p1 = 0u;
+  if (B >= 6) {
+    const uint32_t m = 0x30303030u;
+    d.p2 = (E0 & m) | ((O0 & m) << 2) | ((E1 & m) >> 4) | ((O1 & m) >> 2);
+  }
+  if (B & 1)
+    d.p1 = gather_bit4<B - 1>(E0) | (gather_bit4<B - 1>(O0) << 4) |
+           (gather_bit4<B - 1>(E1) << 8) | (gather_bit4<B - 1>(O1) << 12);
+  return d;
+}
+
+// 16 dense codes -> exact floats in column pairs: rebuild the offset-binary bytes, drop
+// them into fp16 pairs (1024 + u), add -(1024 + 2^(B-1)) in fp32.
+template <int B>
+__device__ __forceinline__ void unpack_dense(const DenseLane &d, float2 (&c)[8]) {
+  uint32_t E0 = d.nib0 & 0x0F0F0F0Fu, O0 = (d.nib0 >> 4) & 0x0F0F0F0Fu;
+  uint32_t E1 = d.nib1 & 0x0F0F0F0Fu, O1 = (d.nib1 >> 4) & 0x0F0F0F0Fu;
+  if (B >= 6) {
+    const uint32_t m = 0x30303030u;
+    E0 |= d.p2 & m;
+    O0 |= (d.p2 >> 2) & m;
+    E1 |= (d.p2 << 4) & m;
+    O1 |= (d.p2 << 2) & m;
+  }
+  if (B & 1) {
+    E0 |= spread_bit4<B - 1>(d.p1);
+    O0 |= spread_bit4<B - 1>(d.p1 >> 4);
+    E1 |= spread_bit4<B - 1>(d.p1 >> 8);
+    O1 |= spread_bit4<B - 1>(d.p1 >> 12);
+  }
+  constexpr float bias = -(1024.0f + (float)(1 << (B - 1)));
+  const uint32_t x[4] = {__byte_perm(E0, O0, 0x5140u), __byte_perm(E0, O0, 0x7362u),
+                         __byte_perm(E1, O1, 0x5140u), __byte_perm(E1, O1, 0x7362u)};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    halves_plus(__byte_perm(x[q], 0x64646464u, 0x5140u), bias, c[2 * q].x, c[2 * q].y);
+    halves_plus(__byte_perm(x[q], 0x64646464u, 0x7362u), bias, c[2 * q + 1].x, c[2 * q + 1].y);
+  }
+}
+
+// Byte offsets of a lane's dense parts inside a row of d_k columns (lane = 16-column block).
+__host__ __device__ constexpr int dense_p2_off(int dk, int lb) { return dk / 2 + 4 * lb; }
+__host__ __device__ constexpr int dense_p1_off(int dk, int b, int lb) {
+  return dk / 2 + (b >= 6 ? dk / 4 : 0) + 2 * lb;
+}
+// Load / store a lane's dense parts from a row (8-, 4- and 2-byte aligned accesses).
+template <int B>
+__device__ __forceinline__ DenseLane ld_dense(const uint8_t *row, int dk, int lb) {
+  DenseLane d;
+  const uint2 n = *reinterpret_cast<const uint2 *>(row + 8 * lb);
+  d.nib0 = n.x;
+  d.nib1 = n.y;
+  d.p2 = B >= 6 ? *reinterpret_cast<const uint32_t *>(row + dense_p2_off(dk, lb)) : 0u;
+  d.p1 = (B & 1) ? *reinterpret_cast<const uint16_t *>(row + dense_p1_off(dk, B, lb)) : 0u;
+  return d;
+}
+template <int B>
+__device__ __forceinline__ void st_dense(uint8_t *row, int dk, int lb, const DenseLane &d) {
+  *reinterpret_cast<uint2 *>(row + 8 * lb) = make_uint2(d.nib0, d.nib1);
+  if (B >= 6) *reinterpret_cast<uint32_t *>(row + dense_p2_off(dk, lb)) = d.p2;
+  if (B & 1) *reinterpret_cast<uint16_t *>(row + dense_p1_off(dk, B, lb)) = (uint16_t)d.p1;
+}
+
 // -------------------------------------------------------------------------------------
 // reductions over the lane's 16 entries
 // -------------------------------------------------------------------------------------
@@ -335,6 +432,26 @@ __device__ __forceinline__ void quantize16(const float2 (&x)[8], float2 inv, con
   }
 }
 
+// Dense codes of a lane's 16 entries: t = fma(x, inv, 49152 + 2^(B-1) + d/256), so byte 1
+// of t is the offset-binary u; then the planes.
+template <int B, bool SR>
+__device__ __forceinline__ DenseLane quantize16_dense(const float2 (&x)[8], float2 inv,
+                                                      const uint32_t (&h)[4]) {
+  constexpr uint32_t K = 0x47400000u | ((uint32_t)(1 << (B - 1)) << 8);
+  uint32_t t[16];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float2 g =
+        SR ? make_float2(__uint_as_float(__byte_perm(h[e >> 1], K, 0x7650u | ((2 * e) & 3))),
+                         __uint_as_float(__byte_perm(h[e >> 1], K, 0x7650u | ((2 * e + 1) & 3))))
+           : dup2(__uint_as_float(K | 0x80u));
+    const float2 tt = __ffma2_rn(x[e], inv, g);
+    t[2 * e] = __float_as_uint(tt.x);
+    t[2 * e + 1] = __float_as_uint(tt.y);
+  }
+  return pack_dense<B>(t);
+}
+
 // Requantize one lane's 16 entries of a value row (a scale group spans G/16 lanes):
 // returns this lane's group verdict (true: an entry of the group is inf, NaN or above
 // 2^100; the caller then zeroes the row).  r = 2^(b-1) - 1 and inv_r = fl(1/r).
@@ -360,7 +477,10 @@ __device__ __forceinline__ bool requantize16_nb(const float2 (&x)[8], float r, f
 template <int LPR>
 __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int lpg, int lane,
                                              uint32_t tkey, uint32_t n0, int stochastic,
-                                             uint32_t (&words)[4], float &s_out) {
+                                             uint32_t (&words)[4], float &s_out, int store = 0) {
+  // store 5..7: dense planes (words = nibble word 0, nibble word 1, 2-bit word, 1-bit word)
+  const bool dense = store >= 5 && store <= 7;
+  const uint32_t kbase = 0x47400000u | (dense ? (1u << (bits - 1)) << 8 : 0u);
   const float r = (float)((1 << (bits - 1)) - 1);        // 2^(b-1) - 1
   const float inv_r = __fdiv_rn(1.0f, r);                 // fl(1/r)
   float mq[4];
@@ -397,14 +517,18 @@ __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int
     for (int q = 0; q < 4; ++q) h[q] = fmix32(tkey + 0x9E3779B9u * (n0 + q + 1u));
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float g = __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)));
+      const float g = __uint_as_float(__byte_perm(h[e >> 2], kbase, 0x7650u | (e & 3)));
       t[e] = __float_as_uint(__fmaf_rn(x[e], inv, g));
     }
   } else {
+    const float g = __uint_as_float(kbase | 0x80u);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, 49152.5f));
+    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fmaf_rn(x[e], inv, g));
   }
-  if (bits != 4) {
+  if (dense) {
+    const DenseLane d = store == 5 ? pack_dense<5>(t) : (store == 6 ? pack_dense<6>(t) : pack_dense<7>(t));
+    words[0] = d.nib0; words[1] = d.nib1; words[2] = d.p2; words[3] = d.p1;
+  } else if (bits != 4) {
     const uint4 w = pack_i8(t);
     words[0] = w.x; words[1] = w.y; words[2] = w.z; words[3] = w.w;
   } else {

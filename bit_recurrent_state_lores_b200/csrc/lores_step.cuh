@@ -17,11 +17,14 @@ namespace lores {
 // One work unit: a block of rows of one (sequence, head) tile, processed by one warp.
 struct __align__(16) UnitDesc {
   int32_t head;
-  int32_t row0;
-  int32_t nrows;
+  int16_t row0;
+  int16_t nrows;
   int16_t bits;          // 4..8 (b-bit codes), 32 (fp32 state), or 0: a bit width per key
                          // group (per-channel precision; the lane table has the layout)
   int16_t rowb;          // bytes of one row of the head
+  int16_t store;         // storage: 4 nibbles, 8 one byte per code, 32 fp32, 5..7 dense
+                         // bit planes, 0 per-lane (lane table)
+  int16_t pad;
   int64_t code_off;      // byte offset of row0 of this head inside one sequence's block
   float r;               // largest code, 2^(bits-1) - 1 (bits 4..8)
   float inv_r;           // fl(1/r)
@@ -35,7 +38,8 @@ struct __align__(16) LaneFmt {
   float r;
   float inv_r;
   int32_t off;
-  int16_t bits;
+  int8_t bits;
+  int8_t store;          // as UnitDesc::store (dense lanes: off is the nibble part's)
   int16_t rowb;
 };
 
@@ -84,14 +88,22 @@ __device__ __forceinline__ uint32_t step_key_dev(uint64_t seed, uint64_t step) {
 __host__ __device__ constexpr int storage_bits(int bits) {
   return bits == 4 ? 4 : (bits == 32 ? 32 : 8);
 }
-// Bytes of one row of a tile with `bits`-bit entries.
+// Bytes of one row of a tile with `bits`-bit entries stored one byte per code (5..8),
+// as nibbles (4) or fp32 (32).
 __host__ __device__ constexpr int row_bytes(int dk, int bits) { return dk * storage_bits(bits) / 8; }
+// Bytes of one row for a storage class: 4, 8, 32 as above; 5..7 dense bit planes, the
+// row padded to a multiple of 8 bytes.
+__host__ __device__ constexpr int store_row_bytes(int dk, int store) {
+  return (store >= 5 && store <= 7) ? (dk * store / 8 + 7) / 8 * 8 : dk * store / 8;
+}
 
 // Rows of a full unit: 4 KB of state, a whole number of warp passes (32/(d_k/16) rows).
-__host__ __device__ constexpr int full_rows(int dk, int bits) {
-  return (4096 / row_bytes(dk, bits)) < (32 / (dk / 16))
+// (store: the storage class, see UnitDesc::store)
+__host__ __device__ constexpr int full_rows(int dk, int store) {
+  return (4096 / store_row_bytes(dk, store)) < (32 / (dk / 16))
              ? (32 / (dk / 16))
-             : (4096 / row_bytes(dk, bits)) - (4096 / row_bytes(dk, bits)) % (32 / (dk / 16));
+             : (4096 / store_row_bytes(dk, store)) -
+                   (4096 / store_row_bytes(dk, store)) % (32 / (dk / 16));
 }
 
 // -------------------------------------------------------------------------------------
@@ -149,7 +161,8 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
   const int col0 = lir * 16;
   // BITS = 0: a bit width per key group; the lane's width, offset and r come from the
   // lane table (lanes of a warp may differ; cross-lane steps stay convergent)
-  const int RB = BITS == 0 ? (int)d.rowb : DK * BITS / 8;   // bytes per row
+  constexpr bool DENSE = BITS >= 5 && BITS <= 7;            // dense bit planes
+  const int RB = BITS == 0 ? (int)d.rowb : store_row_bytes(DK, BITS);   // bytes per row
   int lsb = BITS, loff = lir * 2 * BITS;                    // lane storage bits, byte offset
   float rq = d.r, rq_inv = d.inv_r;
   if (BITS == 0) {
@@ -207,7 +220,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
 
   uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
   float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
-  constexpr int kFullPasses = full_rows(DK, BITS) / RPW;
+  constexpr int kFullPasses = full_rows(DK, BITS == 0 ? 8 : BITS) / RPW;   // FULL: BITS != 0
   const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
   // dither counter of the lane's first quad in pass 0: n0 = (row0 + riw) d_k/4 + 4 lir;
   // each pass moves RPW rows, i.e. RPW d_k/4 quads
@@ -239,7 +252,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       }
     } else {
       float2 cf[8];
-      if (w8)
+      if (DENSE)
+        unpack_dense<DENSE ? BITS : 5>(ld_dense<DENSE ? BITS : 5>(stage + (size_t)lrr * RB, DK, lir), cf);
+      else if (w8)
         unpack_i8_2(BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
                               : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff),
                     cf);
@@ -298,7 +313,17 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     } else {
       uint32_t words[4];
       float s_new;
-      if (BITS == 0) {
+      if (DENSE) {
+        constexpr int DB = DENSE ? BITS : 5;
+        const float m = group_absmax<LPR>(chunk_absmax(x), gd1, gd2, gd4, gd8);
+        float2 inv;
+        gbad = group_scale(m, rq, rq_inv, inv, s_new);
+        const DenseLane dl = quantize16_dense<DB, SR>(x, inv, hw);
+        if (active) {
+          st_dense<DB>((to_stage ? stage : gcodes) + (size_t)lr * RB, DK, lir, dl);
+          if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = s_new;
+        }
+      } else if (BITS == 0) {
         // group scale with every lane, then each lane packs at its own width
         const float m = group_absmax<LPR>(chunk_absmax(x), gd1, gd2, gd4, gd8);
         float2 inv;
@@ -310,7 +335,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       } else {
         gbad = requantize16_nb<LPR, BITS, SR>(x, rq, rq_inv, gd1, gd2, gd4, gd8, hw, words, s_new);
       }
-      if (active) {
+      if (!DENSE && active) {
         if (to_stage) {
           if (w8 && BITS == 0)
             st16_a8(stage + (size_t)lr * RB + loff, make_uint4(words[0], words[1], words[2], words[3]));
@@ -347,7 +372,11 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       const unsigned bal = __ballot_sync(kFull, (badmask >> n) & 1u);
       const int lr = n * RPW + riw;
       if ((bal & rowmask) == 0u || !(FULL || lr < d.nrows)) continue;
-      if (BITS != 32) {
+      if (DENSE) {
+        st_dense<DENSE ? BITS : 5>((to_stage ? stage : gcodes) + (size_t)lr * RB, DK, lir,
+                                   DenseLane{0u, 0u, 0u, 0u});
+        if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
+      } else if (BITS != 32) {
         uint8_t *dst = (to_stage ? stage : gcodes) + (size_t)lr * RB + loff;
         if (w8)
           st16_a8(dst, make_uint4(0, 0, 0, 0));
@@ -397,11 +426,17 @@ template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
 __device__ __forceinline__ void compute_bits(const StepParams &p, uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow, int t) {
-  if (d.bits == 32)
+  if (d.store == 32)
     compute_any<DK, DIAG, DELTA, SR, 32, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.bits == 0)
+  else if (d.store == 0)
     compute_any<DK, DIAG, DELTA, SR, 0, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.bits == 4)
+  else if (d.store == 6)
+    compute_any<DK, DIAG, DELTA, SR, 6, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  else if (d.store == 5)
+    compute_any<DK, DIAG, DELTA, SR, 5, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  else if (d.store == 7)
+    compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  else if (d.store == 4)
     compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else
     compute_any<DK, DIAG, DELTA, SR, 8, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);

@@ -33,7 +33,8 @@ class lores_config(C.Structure):
                 ("d_v", C.c_int32), ("group_size", C.c_int32), ("delta", C.c_int32),
                 ("decay_diag", C.c_int32), ("head_bits", C.POINTER(C.c_int32)),
                 ("stochastic", C.c_int32), ("seed", C.c_uint64), ("device", C.c_int32),
-                ("scale_axis", C.c_int32), ("group_bits", C.POINTER(C.c_int32))]
+                ("scale_axis", C.c_int32), ("group_bits", C.POINTER(C.c_int32)),
+                ("dense_codes", C.c_int32)]
 
 
 class lores_layout(C.Structure):
@@ -108,10 +109,11 @@ def lores_status_string(status):
 
 
 def lores_create(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                 stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None):
-    """Returns an opaque handle (int).  group_bits: None or [H][d_k/G] bits per key group."""
+                 stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None, dense_codes=0):
+    """Returns an opaque handle (int).  group_bits: None or [H][d_k/G] bits per key group;
+    dense_codes: 5- to 7-bit codes in bit planes instead of one byte each."""
     cfg = make_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, head_bits,
-                      stochastic, seed, device, scale_axis, group_bits)
+                      stochastic, seed, device, scale_axis, group_bits, dense_codes)
     out = C.c_void_p()
     _check(_lib.lores_create(C.byref(cfg), C.byref(out)), "lores_create")
     return out.value
@@ -163,7 +165,7 @@ def lores_decode_step_noalloc(cfg, codes, scales, q, k, v, alpha, beta, o, step,
 
 
 def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, head_bits=None,
-                stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None):
+                stochastic=1, seed=0, device=0, scale_axis=0, group_bits=None, dense_codes=0):
     """A lores_config; the bit arrays are kept alive on the returned object."""
     hb = gb = None
     arr = garr = None
@@ -175,7 +177,7 @@ def make_config(batch, heads, d_k, d_v, group_size=0, delta=1, decay_diag=0, hea
         garr = (C.c_int32 * len(flat))(*flat)
         gb = C.cast(garr, C.POINTER(C.c_int32))
     cfg = lores_config(batch, heads, d_k, d_v, group_size, delta, decay_diag, hb, stochastic,
-                       seed & (2**64 - 1), device, scale_axis, gb)
+                       seed & (2**64 - 1), device, scale_axis, gb, dense_codes)
     cfg._keepalive = (arr, garr)
     return cfg
 

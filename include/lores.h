@@ -83,6 +83,13 @@ typedef struct {
                             /* nibbles, 5..8 bits one byte per code); each group is scaled    */
                             /* with its own r = 2^(b_g-1)-1.  Needs head_bits = NULL and      */
                             /* scale_axis = 0; not taken by lores_decode_step_noalloc.        */
+    int32_t dense_codes;    /* 0: 5- to 7-bit codes one per byte (two's complement);         */
+                            /* 1: dense, b bits per code: offset binary u = c + 2^(b-1) in    */
+                            /* bit planes per row, [4-bit plane d_k/2 B][2-bit plane d_k/4 B  */
+                            /* if b >= 6][1-bit plane d_k/8 B if b odd], padded to 8 bytes    */
+                            /* (plane bit order in the oracle and csrc/lores_device.cuh).     */
+                            /* Per-head bits only (group_bits NULL, scale_axis 0); not taken  */
+                            /* by lores_decode_step_noalloc.                                   */
 } lores_config;
 
 /* Sizes of the handle's state, for export/import buffers, and its device buffers. */

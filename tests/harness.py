@@ -26,19 +26,21 @@ def mixed_bits(wl, hp):
 class GpuRun:
     """One handle of the library holding the state of one layer for a batch."""
 
-    def __init__(self, wl, head_bits, seed, stochastic=1, device=0, axis=0, group_bits=None):
+    def __init__(self, wl, head_bits, seed, stochastic=1, device=0, axis=0, group_bits=None,
+                 dense=0):
         """group_bits: None, or per head a list of the key groups' bit widths (then
         head_bits only names the heads' nominal widths for the oracle configs)."""
         L = lib()
         self.wl, self.bits, self.seed, self.axis = wl, list(head_bits), seed, axis
         self.stochastic = stochastic
         self.group_bits = group_bits
+        self.dense = dense
         self.h = L.lores_create(wl.B, wl.H, wl.d_k, wl.d_v,
                                 group_size=wl.d_k if axis else (wl.group or 0),
                                 delta=wl.delta, decay_diag=wl.diag,
                                 head_bits=None if group_bits is not None else head_bits,
                                 stochastic=stochastic, seed=seed, device=device,
-                                scale_axis=axis, group_bits=group_bits)
+                                scale_axis=axis, group_bits=group_bits, dense_codes=dense)
         self.layout, self.head_off = L.lores_get_layout(self.h, wl.H)
         self.o = torch.empty(wl.B, wl.H, wl.d_v, device="cuda", dtype=torch.float32)
 
@@ -72,7 +74,8 @@ class GpuRun:
         """(state, scales) of tile (b, hh) from an export, in the oracle's layout."""
         wl, bits = self.wl, self.bits[hh]
         cfg = tile_cfg(wl, bits, axis=self.axis,
-                       group_bits=None if self.group_bits is None else self.group_bits[hh])
+                       group_bits=None if self.group_bits is None else self.group_bits[hh],
+                       dense=self.dense)
         off = self.head_off[hh]
         raw = codes[b, off:off + cfg.code_bytes()].copy()
         if bits == 32:
@@ -85,10 +88,10 @@ class GpuRun:
             self.h = None
 
 
-def tile_cfg(wl, bits, stochastic=1, axis=0, group_bits=None):
+def tile_cfg(wl, bits, stochastic=1, axis=0, group_bits=None, dense=0):
     return O.TileCfg(wl.d_k, wl.d_v, group=wl.d_k if axis else wl.G, bits=bits,
                      delta=wl.delta, diag=wl.diag, stochastic=stochastic, axis=axis,
-                     group_bits=group_bits)
+                     group_bits=group_bits, dense=dense)
 
 
 def host_tile_inputs(inputs, tiles):
@@ -107,10 +110,11 @@ def host_tile_inputs(inputs, tiles):
 class OracleTiles:
     """The oracle's own trajectory for a few (b, h) tiles of a workload."""
 
-    def __init__(self, wl, head_bits, seed, tiles, stochastic=1, axis=0, group_bits=None):
+    def __init__(self, wl, head_bits, seed, tiles, stochastic=1, axis=0, group_bits=None,
+                 dense=0):
         self.wl, self.bits, self.seed, self.tiles = wl, list(head_bits), seed, list(tiles)
         self.cfg = {t: tile_cfg(wl, self.bits[t[1]], stochastic, axis,
-                                None if group_bits is None else group_bits[t[1]])
+                                None if group_bits is None else group_bits[t[1]], dense)
                     for t in self.tiles}
         self.state = {t: self.cfg[t].zero_state() for t in self.tiles}
 
@@ -139,7 +143,7 @@ def compare_tile(cfg, gpu_state, gpu_scales, ref_state, ref_scales):
     """Returns (n_diff_codes, max_abs_code_diff, dequant_rel_l2, scales_equal)."""
     if cfg.bits == 32:
         return 0, 0, rel_l2(gpu_state, ref_state), True
-    small = cfg.d_v * cfg.d_k <= 4096 or cfg.group_bits is not None
+    small = cfg.d_v * cfg.d_k <= 4096 or cfg.group_bits is not None or cfg.dense
     cg = O.unpack_codes(cfg, gpu_state) if small else unpack_fast(cfg, gpu_state)
     cr = O.unpack_codes(cfg, ref_state) if small else unpack_fast(cfg, ref_state)
     d = np.abs(cg - cr)

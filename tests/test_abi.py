@@ -43,7 +43,9 @@ def test_status_strings():
     dict(device=-1), dict(scale_axis=2), dict(scale_axis=-1), dict(scale_axis=1, group_size=16),
     dict(group_size=32, group_bits=[[8, 4], [4, 4]], head_bits=[8, 8]),
     dict(group_size=32, group_bits=[[8, 3], [4, 4]]), dict(group_size=32, group_bits=[[8, 9], [4, 4]]),
-    dict(scale_axis=1, group_size=64, group_bits=[[8], [8]])])
+    dict(scale_axis=1, group_size=64, group_bits=[[8], [8]]), dict(dense_codes=2),
+    dict(dense_codes=1, group_size=32, group_bits=[[6, 6], [6, 6]]),
+    dict(dense_codes=1, scale_axis=1, head_bits=[6, 6])])
 def test_create_rejects_bad_config_before_touching_cuda(kw):
     from bit_recurrent_state_lores_b200 import lores as L
     args = dict(batch=2, heads=2, d_k=64, d_v=16)
@@ -57,6 +59,15 @@ def test_noalloc_rejects_group_bits_before_touching_cuda():
     import ctypes as C
     from bit_recurrent_state_lores_b200 import lores as L
     cfg = L.make_config(1, 1, 64, 64, group_size=32, group_bits=[[8, 4]])
+    a = 0x10000
+    assert L.raw_library().lores_decode_step_noalloc(C.byref(cfg), a, a, a, a, a, a, a, a, 0,
+                                                     None, None) == L.LORES_ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_dense_codes_before_touching_cuda():
+    import ctypes as C
+    from bit_recurrent_state_lores_b200 import lores as L
+    cfg = L.make_config(1, 1, 64, 64, head_bits=[6], dense_codes=1)
     a = 0x10000
     assert L.raw_library().lores_decode_step_noalloc(C.byref(cfg), a, a, a, a, a, a, a, a, 0,
                                                      None, None) == L.LORES_ERR_UNSUPPORTED
