@@ -1036,9 +1036,26 @@ lores_status lores_decode_steps(lores_handle *h, int32_t T, const float *q, cons
   return cuda_status(cudaGetLastError());
 }
 
+static lores_status step_host(lores_handle *h, const float *q, const float *k, const float *v,
+                              const float *alpha, const float *beta, float *o, uint64_t step,
+                              void *stream, bool wait);
+
 lores_status lores_decode_step_host(lores_handle *h, const float *q, const float *k,
                                     const float *v, const float *alpha, const float *beta,
                                     float *o, uint64_t step, void *stream) {
+  return step_host(h, q, k, v, alpha, beta, o, step, stream, true);
+}
+
+lores_status lores_decode_step_host_async(lores_handle *h, const float *q, const float *k,
+                                          const float *v, const float *alpha,
+                                          const float *beta, float *o, uint64_t step,
+                                          void *stream) {
+  return step_host(h, q, k, v, alpha, beta, o, step, stream, false);
+}
+
+static lores_status step_host(lores_handle *h, const float *q, const float *k, const float *v,
+                              const float *alpha, const float *beta, float *o, uint64_t step,
+                              void *stream, bool wait) {
   if (!h || !q || !k || !v || !alpha || !beta || !o) return LORES_ERR_INVALID_ARG;
   DeviceGuard guard(h->cfg.device);
   if (!guard.ok) return LORES_ERR_CUDA;
@@ -1065,7 +1082,7 @@ lores_status lores_decode_step_host(lores_handle *h, const float *q, const float
       lores_decode_step(h, d + oq, d + ok_, d + ov, d + oa, d + ob, h->stage_o, step, stream);
   if (st != LORES_OK) return st;
   e = cudaMemcpyAsync(o, h->stage_o, nv * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && wait) e = cudaStreamSynchronize(s);
   return cuda_status(e);
 }
 

@@ -55,6 +55,7 @@ def _load():
         "lores_destroy": (I32, [P]),
         "lores_decode_step": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_host": (I32, [P, P, P, P, P, P, P, U64, P]),
+        "lores_decode_step_host_async": (I32, [P, P, P, P, P, P, P, U64, P]),
         "lores_decode_steps": (I32, [P, I32, P, P, P, P, P, P, U64, P]),
         "lores_decode_step_dev": (I32, [P, P, P, P, P, P, P, P, P]),
         "lores_advance_step": (I32, [P, U64, P]),
@@ -146,6 +147,14 @@ def lores_decode_steps(h, T, q, k, v, alpha, beta, o, step0, stream=None):
     _check(_lib.lores_decode_steps(h, int(T), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                    _ptr(o), step0 & (2**64 - 1), _stream(stream)),
            "lores_decode_steps")
+
+
+def lores_decode_step_host_async(h, q, k, v, alpha, beta, o, step, stream=None):
+    """Host-buffer step, enqueued only (pinned buffers; o valid when the stream gets there)."""
+    _check(_lib.lores_decode_step_host_async(h, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                             _ptr(beta), _ptr(o), step & (2**64 - 1),
+                                             _stream(stream)),
+           "lores_decode_step_host_async")
 
 
 def lores_decode_step_host(h, q, k, v, alpha, beta, o, step, stream=None):

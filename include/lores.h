@@ -174,6 +174,16 @@ lores_status lores_decode_step_host(lores_handle *h, const float *q, const float
                                     const float *v, const float *alpha, const float *beta,
                                     float *o, uint64_t step, void *stream);
 
+/* lores_decode_step_host without the final wait: the copies and the step are only
+ * enqueued on `stream` (o is valid once the stream reaches the call).  For true overlap
+ * the host buffers must be pinned (page-locked); they must stay untouched until then.
+ * Steps of different handles on different streams overlap one handle's host<->device
+ * copies with another handle's kernel.  Errors: as lores_decode_step_host. */
+lores_status lores_decode_step_host_async(lores_handle *h, const float *q, const float *k,
+                                          const float *v, const float *alpha,
+                                          const float *beta, float *o, uint64_t step,
+                                          void *stream);
+
 /* The decode step for callers that must not let this library allocate device memory:
  * for example a serving engine that hands out every buffer from its own pre-planned
  * pool (a cudaMalloc inside a step can stall the device and fragment that pool), or an

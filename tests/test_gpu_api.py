@@ -138,8 +138,22 @@ def test_host_buffer_step_equals_device_step():
         torch.cuda.synchronize()
         assert torch.equal(o_h, d.o.cpu())
     assert all(np.array_equal(x, y) for x, y in zip(d.export(), hst.export()))
-    d.close()
-    hst.close()
+    # the enqueue-only variant on two streams (pinned buffers) gives the same steps
+    a1 = GpuRun(wl, bits, seed=5)
+    a2 = GpuRun(wl, bits, seed=5)
+    lanes = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for t in range(3):
+        inp = synth.step_inputs(wl, t, hp, device="cuda")
+        host = [x.cpu().pin_memory() for x in inp]
+        outs = [torch.empty(wl.B, wl.H, wl.d_v).pin_memory() for _ in range(2)]
+        for r, ls, oh in zip((a1, a2), lanes, outs):
+            L.lores_decode_step_host_async(r.h, *host, oh, t, ls.cuda_stream)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1])
+    assert all(np.array_equal(x, y) for x, y in zip(d.export(), a1.export()))
+    assert all(np.array_equal(x, y) for x, y in zip(d.export(), a2.export()))
+    for r in (d, hst, a1, a2):
+        r.close()
 
 
 def test_load_state_and_dequant_match_oracle_on_every_tile():
