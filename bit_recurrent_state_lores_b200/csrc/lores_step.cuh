@@ -221,7 +221,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
   uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
   float *gscales = p.scales + (tile * p.d_v + d.row0) * ng;
   constexpr int kFullPasses = full_rows(DK, BITS == 0 ? 8 : BITS) / RPW;   // FULL: BITS != 0
-  const int npass = FULL ? kFullPasses : (d.nrows + RPW - 1) / RPW;
+  // FULL: every pass complete; the pass count is a compile-time constant except for
+  // mixed-width rows (BITS = 0), whose unit sizes follow each head's row bytes
+  const int npass = FULL ? (BITS == 0 ? d.nrows / RPW : kFullPasses) : (d.nrows + RPW - 1) / RPW;
   // dither counter of the lane's first quad in pass 0: n0 = (row0 + riw) d_k/4 + 4 lir;
   // each pass moves RPW rows, i.e. RPW d_k/4 quads
   const uint32_t cbase0 =
@@ -229,7 +231,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
   constexpr uint32_t kCtrPerPass = 0x9E3779B9u * (uint32_t)(RPW * DK / 4);
   uint32_t badmask = 0;                        // bit n: this lane's group was bad in pass n
 
-#pragma unroll(FULL ? 4 : 1)
+#pragma unroll(FULL ? (BITS == 0 ? 2 : 4) : 1)
   for (int n = 0; n < npass; ++n) {
     const int lr = n * RPW + riw;              // row inside the unit
     const bool active = FULL || lr < d.nrows;
@@ -412,7 +414,13 @@ template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool MT>
 __device__ __forceinline__ void compute_any(const StepParams &p, uint8_t *stage, int b,
                                             const UnitDesc &d, float alpha_s, float beta,
                                             float *opart, float *ow, int t) {
-  if (BITS != 0 && d.nrows == full_rows(DK, BITS)) {
+  if (BITS == 0) {
+    constexpr int RPW = 32 / (DK / 16);
+    if (d.nrows % RPW == 0)
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    else
+      compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  } else if (d.nrows == full_rows(DK, BITS)) {
     if (p.G == DK)
       compute_unit<DK, DIAG, DELTA, SR, BITS, true, true, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
