@@ -2,6 +2,10 @@
 
     python -m bit_recurrent_state_lores_b200.build [--verbose]
 
+csrc/lores.cu (host side, loader, dequantizer, key-axis kernels) and 20 compilations of
+csrc/lores_inst.cu (one decode-step kernel family per key width x single/multi-token x
+plain/extended storage) build in parallel, one nvcc process per CPU core, then link.
+
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
 rounding-sensitive operation is written with explicit round-to-nearest intrinsics
 and fma contraction is disabled as a second guard.
@@ -9,48 +13,58 @@ and fma contraction is disabled as a second guard.
 import os
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "lores.cu")
-DEPS = [SRC, os.path.join(PKG, "csrc", "lores_device.cuh"), os.path.join(ROOT, "include", "lores.h")]
+CSRC = os.path.join(PKG, "csrc")
+SRC = os.path.join(CSRC, "lores.cu")
+INST = os.path.join(CSRC, "lores_inst.cu")
+DEPS = [SRC, INST, os.path.join(CSRC, "lores_step.cuh"), os.path.join(CSRC, "lores_device.cuh"),
+        os.path.join(ROOT, "include", "lores.h")]
 LIB = os.path.join(PKG, "liblores.so")
 NVCC = os.environ.get("NVCC", "nvcc")
-
-
-SRCS = [SRC, os.path.join(PKG, "csrc", "lores_mt.cu")]
-DEPS += SRCS[1:] + [os.path.join(PKG, "csrc", "lores_step.cuh")]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-         "-fmad=false", "-Xcompiler", "-fPIC"]
+         "-fmad=false", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
+KEY_WIDTHS = (16, 32, 64, 128, 256)
 
 
-def nvcc_cmd(out=LIB, verbose=False):
-    """One-shot command line (both translation units in one nvcc call)."""
-    cmd = [NVCC] + FLAGS + ["-shared", "-I", os.path.join(ROOT, "include"), "-o", out] + SRCS
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    return cmd
+def units():
+    """(source, extra flags, object name) of every compilation."""
+    out = [(SRC, [], "lores.o")]
+    for dk in KEY_WIDTHS:
+        for mt in (0, 1):
+            for ext in (0, 1):
+                out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],
+                            f"lores_inst_{dk}_{mt}_{ext}.o"))
+    return out
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the translation units in parallel, then link the shared library."""
+def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
+    """Compile every unit (up to `jobs` at a time, default: the CPU count), then link."""
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in DEPS)):
         return LIB
-    objs, procs = [], []
-    for src in SRCS:
-        obj = os.path.join(PKG, "csrc", os.path.basename(src)[:-3] + ".o")
-        cmd = [NVCC] + FLAGS + (["-Xptxas=-v"] if verbose else []) + [
-            "-I", os.path.join(ROOT, "include"), "-c", "-o", obj, src]
-        procs.append(subprocess.Popen(cmd))
-        objs.append(obj)
-    codes = [pr.wait() for pr in procs]
-    if any(codes):
-        raise subprocess.CalledProcessError(max(codes), "nvcc")
-    subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB]
-                   + objs, check=True)
-    for obj in objs:
-        os.remove(obj)
+    jobs = jobs or max(1, os.cpu_count() or 1)
+    with tempfile.TemporaryDirectory(prefix="lores_build_") as tmp:
+        pending = list(units())
+        running, objs = [], []
+        while pending or running:
+            while pending and len(running) < jobs:
+                src, extra, name = pending.pop(0)
+                obj = os.path.join(tmp, name)
+                cmd = [NVCC] + FLAGS + extra + (["-Xptxas=-v"] if verbose else []) + [
+                    "-c", "-o", obj, src]
+                running.append((subprocess.Popen(cmd), name))
+                objs.append(obj)
+            proc, name = running.pop(0)
+            if proc.wait() != 0:
+                for p, _ in running:
+                    p.wait()
+                raise subprocess.CalledProcessError(proc.returncode, f"nvcc ({name})")
+        subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o",
+                        LIB + ".tmp"] + objs, check=True)
+    os.replace(LIB + ".tmp", LIB)
     return LIB
 
 

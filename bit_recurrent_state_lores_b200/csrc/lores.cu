@@ -442,8 +442,26 @@ static uint32_t step_key_of(uint64_t seed, uint64_t step) {
 using LoadFn = void (*)(const LoadParams);
 using DequantFn = void (*)(const LoadParams, float *);
 
+// The decode-step kernel of a configuration: mt = multi-token, ext = extended storage.
+static StepFn kernel_for(int dk, bool mt, bool ext, bool diag, bool delta, bool sr) {
+#define LORES_PICK(dk_)                                                        \
+  case dk_:                                                                    \
+    return mt ? (ext ? step_kernels_##dk_##_1_1(diag, delta, sr)               \
+                     : step_kernels_##dk_##_1_0(diag, delta, sr))              \
+              : (ext ? step_kernels_##dk_##_0_1(diag, delta, sr)               \
+                     : step_kernels_##dk_##_0_0(diag, delta, sr));
+  switch (dk) {
+    LORES_PICK(16)
+    LORES_PICK(32)
+    LORES_PICK(64)
+    LORES_PICK(128)
+    LORES_PICK(256)
+  }
+#undef LORES_PICK
+  return nullptr;
+}
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
-  return pick_step_any<false>(dk, diag, delta, sr);
+  return kernel_for(dk, false, false, diag, delta, sr);
 }
 using KeyFn = void (*)(const KeyParams);
 static KeyFn key_kernel_for(int dk) {
@@ -718,7 +736,11 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     const int n = 4096 / rb;
     return std::min(n < rpw ? rpw : n - n % rpw, dv);
   };
-  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  // handles with dense or mixed-width heads take the extended kernel family
+  bool ext = false;
+  for (int hh = 0; hh < c.heads; ++hh)
+    ext |= !(h->store[hh] == 4 || h->store[hh] == 8 || h->store[hh] == 32);
+  StepFn fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
   int split = 1;
   auto build_units = [&](std::vector<UnitDesc> &u) {
     u.clear();
@@ -808,7 +830,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   }
   h->units_per_seq = (int)units.size();
   h->step_fn = fn;
-  h->mt_fn = mt_step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  h->mt_fn = kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
   {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, h->mt_fn) != cudaSuccess ||

@@ -429,25 +429,28 @@ __device__ __forceinline__ void compute_any(const StepParams &p, uint8_t *stage,
     compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   }
 }
-// One unit for one token: the unit's storage width picks the code path.
-template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
+// One unit for one token: the unit's storage class picks the code path.  EXT: the kernel
+// also carries the dense and per-lane paths (kept out of the plain kernel, whose code
+// stays smaller and faster for int8 / int4 / fp32 handles).
+template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, bool EXT>
 __device__ __forceinline__ void compute_bits(const StepParams &p, uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow, int t) {
   if (d.store == 32)
     compute_any<DK, DIAG, DELTA, SR, 32, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.store == 0)
+  else if (!EXT || d.store == 4 || d.store == 8) {
+    if (d.store == 4)
+      compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    else
+      compute_any<DK, DIAG, DELTA, SR, 8, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  } else if (d.store == 0)
     compute_any<DK, DIAG, DELTA, SR, 0, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else if (d.store == 6)
     compute_any<DK, DIAG, DELTA, SR, 6, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else if (d.store == 5)
     compute_any<DK, DIAG, DELTA, SR, 5, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.store == 7)
-    compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.store == 4)
-    compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   else
-    compute_any<DK, DIAG, DELTA, SR, 8, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
 }
 
 // Position of a unit: global unit u = ub * B + b (sequence b is the fast index, so a warp
@@ -469,7 +472,7 @@ struct UnitPos {
 // Persistent kernel: every warp runs its own pipeline over units gw, gw + W, gw + 2W, ...
 // (gw = global warp index, W = warps in the grid), with a 2-slot ring of bulk copies
 // whose producer is the warp's lane 0.  Warps never wait on one another.
-template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
+template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, bool EXT>
 __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -547,10 +550,10 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       for (int t = 0; t < p.T; ++t) {
         const float beta_t = __ldg(p.beta + t * p.tok_b + tile);
         const float alpha_t = DIAG ? 0.0f : __ldg(p.alpha + t * p.tok_a + tile);
-        compute_bits<DK, DIAG, DELTA, SR, MT>(p, stage, cur.b, d, alpha_t, beta_t, opart, ow, t);
+        compute_bits<DK, DIAG, DELTA, SR, MT, EXT>(p, stage, cur.b, d, alpha_t, beta_t, opart, ow, t);
       }
     } else {
-      compute_bits<DK, DIAG, DELTA, SR, MT>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow, 0);
+      compute_bits<DK, DIAG, DELTA, SR, MT, EXT>(p, stage, cur.b, d, alpha_cur, beta_cur, opart, ow, 0);
     }
     // compute_unit ends with __syncwarp: every lane is done reading this slot
     if (fill.ub < ups) {
@@ -567,25 +570,28 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
 
 using StepFn = void (*)(const StepParams);
 
-// Kernel pickers: MT = false is instantiated in lores.cu, MT = true in lores_mt.cu.
-template <int DK, bool SR, bool MT>
+// Kernel pickers: the plain single-token kernels are instantiated in lores.cu, the plain
+// multi-token ones in lores_mt.cu, and both extended families in lores_ext.cu.
+template <int DK, bool SR, bool MT, bool EXT>
 StepFn pick_step(bool diag, bool delta) {
   if (diag)
-    return delta ? decode_step_kernel<DK, true, true, SR, MT> : decode_step_kernel<DK, true, false, SR, MT>;
-  return delta ? decode_step_kernel<DK, false, true, SR, MT> : decode_step_kernel<DK, false, false, SR, MT>;
+    return delta ? decode_step_kernel<DK, true, true, SR, MT, EXT>
+                 : decode_step_kernel<DK, true, false, SR, MT, EXT>;
+  return delta ? decode_step_kernel<DK, false, true, SR, MT, EXT>
+               : decode_step_kernel<DK, false, false, SR, MT, EXT>;
 }
-template <bool MT>
-StepFn pick_step_any(int dk, bool diag, bool delta, bool sr) {
-  switch (dk) {
-    case 16: return sr ? pick_step<16, true, MT>(diag, delta) : pick_step<16, false, MT>(diag, delta);
-    case 32: return sr ? pick_step<32, true, MT>(diag, delta) : pick_step<32, false, MT>(diag, delta);
-    case 64: return sr ? pick_step<64, true, MT>(diag, delta) : pick_step<64, false, MT>(diag, delta);
-    case 128: return sr ? pick_step<128, true, MT>(diag, delta) : pick_step<128, false, MT>(diag, delta);
-    case 256: return sr ? pick_step<256, true, MT>(diag, delta) : pick_step<256, false, MT>(diag, delta);
-  }
-  return nullptr;
-}
-// Multi-token kernels (defined in lores_mt.cu).
-StepFn mt_step_kernel_for(int dk, bool diag, bool delta, bool sr);
+// One function per (key width, multi-token, extended) family, each defined in its own
+// compilation of lores_inst.cu; kernel_for picks among them.
+#define LORES_DECLARE_FAMILY(dk)                                   \
+  StepFn step_kernels_##dk##_0_0(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_1_0(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_0_1(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_1_1(bool diag, bool delta, bool sr);
+LORES_DECLARE_FAMILY(16)
+LORES_DECLARE_FAMILY(32)
+LORES_DECLARE_FAMILY(64)
+LORES_DECLARE_FAMILY(128)
+LORES_DECLARE_FAMILY(256)
+#undef LORES_DECLARE_FAMILY
 
 }  // namespace lores
