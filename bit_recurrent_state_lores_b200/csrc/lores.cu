@@ -499,6 +499,10 @@ static DequantFn dequant_kernel_for(int dk) {
 
 using namespace lores;
 
+static_assert(sizeof(UnitDesc) == 32, "unit table entries are 32 bytes (shared-memory copy, "
+                                      "allocation-free scratch)");
+static_assert(sizeof(LaneFmt) == 16, "lane table entries are 16 bytes");
+
 constexpr int kGuardBytes = 256;
 constexpr unsigned char kGuardByte = 0xA5;
 
