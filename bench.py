@@ -398,7 +398,8 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                         "kernel": "lores::decode_step_kernel<128,false,true>",
+                         "kernel": "decode_step_kernel<128, scalar decay, delta, stochastic "
+                                   "rounding, single token, plain>",
                          "bytes_per_launch": avg_bytes, "avg_launch_us": avg_launch_s * 1e6,
                          "frac_of_8TBps": achieved / 8000.0},
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clock_summary,
