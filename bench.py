@@ -492,6 +492,34 @@ def run_sweep(args):
                        "rounding": "stochastic"}}
 
 
+def oracle_rate(c, wl, hp, seconds):
+    """The oracle (one host core) on the same format: sequence 0's 32 tiles, step after
+    step until `seconds` elapse; (seq, head) updates per second."""
+    import numpy as np
+    from bit_recurrent_state_lores_b200 import synth
+    from oracle import oracle as O
+    H = wl.H
+    gb = c.get("group_bits")
+    cfgs = [O.TileCfg(wl.d_k, wl.d_v, group=wl.d_k if c.get("axis") else c.get("G", wl.d_k),
+                      bits=8 if gb else c["bits"][h], delta=c.get("delta", 1), diag=wl.diag,
+                      stochastic=c.get("sr", 1), axis=c.get("axis", 0),
+                      group_bits=gb[h] if gb else None, dense=c.get("dense", 0))
+            for h in range(H)]
+    states = [cf.zero_state() for cf in cfgs]
+    done, elapsed, t = 0, 0.0, 0
+    while elapsed < seconds or done == 0:
+        q, k, v, a, b = [x.numpy() for x in synth.step_inputs(synth.replace(wl, B=1), t, hp)]
+        sk = O.step_key(1, t)
+        t0 = time.perf_counter()
+        for h, cf in enumerate(cfgs):
+            st, sc = states[h]
+            O.tile_step(cf, st, sc, q[0, h], k[0, h], v[0, h], a[0, h], b[0, h], O.tile_key(sk, h))
+        elapsed += time.perf_counter() - t0
+        done += H
+        t += 1
+    return done / elapsed
+
+
 def run_formats(args):
     """One layer (batch args.batch, 32 heads, 128 x 128, GDN-style inputs of step 0): the mean
     launch time of the decode step over `steps` launches after `warmup`, for every state
@@ -552,10 +580,14 @@ def run_formats(args):
         vec = B * H * (2 * dk * 4 + 2 * dv * 4 + 8)  # q, k, v, alpha, beta read; o written
         state = 2 * (lay.code_bytes + lay.scale_count * 4)
         nbytes = state / T + vec
+        orate = oracle_rate(c, wl, hp, args.cpu_seconds / len(cases))
         out.append({"format": name, "us_per_token": us, "state_bytes": lay.code_bytes + lay.scale_count * 4,
-                    "algorithmic_GBps": nbytes / us / 1e3, "frac_of_peak": nbytes / us / 1e3 / peak})
+                    "algorithmic_GBps": nbytes / us / 1e3, "frac_of_peak": nbytes / us / 1e3 / peak,
+                    "state_updates_per_s": B * H / (us * 1e-6),
+                    "oracle_state_updates_per_s": orate})
         L.lores_destroy(h)
     return {"metric": "decode-step launch time per token by state format", "batch": B,
+            "oracle": "one host core, sequence 0's 32 tiles, %.1f s per format" % (args.cpu_seconds / len(cases)),
             "heads": H, "d_k": dk, "d_v": dv, "steps": args.steps, "warmup": args.warmup,
             "peak_GBps": peak, "peak_kind": peak_kind, "formats": out}
 
