@@ -69,6 +69,8 @@ KEY_SWEEP = [
     (128, 52, [8, 5, 4], 1, 0, 0, 2, 3),      # round to nearest
     (128, 128, [8, 7, 32], 1, 1, 1, 2, 3),
     (256, 64, [8, 4], 1, 0, 1, 2, 2),
+    (64, 512, [8, 4], 1, 1, 1, 2, 2),         # tall tile: the two-pass recompute kernel
+    (32, 4, [8, 4], 1, 0, 1, 3, 2),           # four rows
 ]
 
 
