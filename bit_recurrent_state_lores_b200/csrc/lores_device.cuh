@@ -334,6 +334,23 @@ __device__ __forceinline__ float dot16_p(const float2 (&a)[8], const float2 (&b)
   const float2 s = __fadd2_rn(lo, hi);
   return __fadd_rn(s.x, s.y);
 }
+// The same order from pairs with scalar fma chains (four independent chains; the fp32
+// state path issues these faster than the packed form).
+__device__ __forceinline__ float dot16_s(const float2 (&a)[8], const float2 (&b)[8]) {
+  float c00 = 0.0f, c01 = 0.0f, c10 = 0.0f, c11 = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    c00 = __fmaf_rn(a[e].x, b[e].x, c00);
+    c01 = __fmaf_rn(a[e].y, b[e].y, c01);
+  }
+#pragma unroll
+  for (int e = 4; e < 8; ++e) {
+    c10 = __fmaf_rn(a[e].x, b[e].x, c10);
+    c11 = __fmaf_rn(a[e].y, b[e].y, c11);
+  }
+  return __fadd_rn(__fadd_rn(c00, c10), __fadd_rn(c01, c11));
+}
+
 // The same order with scalar operations.
 __device__ __forceinline__ float dot16_b(const float (&a)[16], const float (&b)[16]) {
   float ch[2][2];

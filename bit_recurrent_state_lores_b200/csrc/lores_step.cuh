@@ -273,7 +273,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     const float vr = sv[lrr];
     float w;
     if (DELTA) {
-      float u = dot16_p(sp, kk);
+      float u = BITS == 32 ? dot16_s(sp, kk) : dot16_p(sp, kk);
 #pragma unroll
       for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
       w = __fmul_rn(beta, __fsub_rn(vr, u));
@@ -286,7 +286,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     for (int e = 0; e < 8; ++e) x[e] = __ffma2_rn(w2, kk[e], sp[e]);
 
     // ---- readout share: this lane's part of S'q ----------------------------------------
-    const float opv = dot16_p(sp, qq);
+    const float opv = BITS == 32 ? dot16_s(sp, qq) : dot16_p(sp, qq);
     if (active) {
       opart[lr * LPR + lir] = opv;
       if (lir == 0) ow[lr] = w;
