@@ -195,6 +195,41 @@ __device__ __forceinline__ void unpack_i4_2(const uint2 &cw, float2 (&c)[8]) {
 }
 __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
+// Offset-binary bytes (code + 128) of a lane's 16 columns, 4 columns per word in
+// column order -> exact floats in column pairs (the int8 path after its bias flip).
+__device__ __forceinline__ void unpack_ob_2(const uint32_t (&ob)[4], float2 (&c)[8]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    halves_plus(__byte_perm(ob[q], 0x64646464u, 0x5140u), -1152.0f, c[2 * q].x, c[2 * q].y);
+    halves_plus(__byte_perm(ob[q], 0x64646464u, 0x7362u), -1152.0f, c[2 * q + 1].x,
+                c[2 * q + 1].y);
+  }
+}
+// 16 int4 codes -> offset-binary bytes (code + 128): nibble n -> (n ^ 8) + 120, no carry
+// between bytes ((n ^ 8) <= 15), then even and odd columns interleaved into column order.
+__device__ __forceinline__ void widen_i4_ob(const uint2 &cw, uint32_t (&ob)[4]) {
+  const uint32_t w[2] = {cw.x, cw.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t ev = ((w[h] & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u;
+    const uint32_t od = (((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u;
+    ob[2 * h] = __byte_perm(ev, od, 0x5140u);       // columns 8h + 0..3
+    ob[2 * h + 1] = __byte_perm(ev, od, 0x7362u);   // columns 8h + 4..7
+  }
+}
+// Two's complement code bytes of 16 columns (|code| <= 7) -> int4 nibbles, even column low.
+__device__ __forceinline__ uint2 compact_i4(const uint4 &b) {
+  const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t e = __byte_perm(w[2 * h], w[2 * h + 1], 0x6420u);   // columns 0, 2, 4, 6
+    const uint32_t o = __byte_perm(w[2 * h], w[2 * h + 1], 0x7531u);   // columns 1, 3, 5, 7
+    out[h] = (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 // t holds 49152 + code + frac in fp32: its byte 1 is the code (two's complement).
 __device__ __forceinline__ uint4 pack_i8(const uint32_t (&t)[16]) {
   uint32_t w[4];
@@ -334,23 +369,6 @@ __device__ __forceinline__ float dot16_p(const float2 (&a)[8], const float2 (&b)
   const float2 s = __fadd2_rn(lo, hi);
   return __fadd_rn(s.x, s.y);
 }
-// The same order from pairs with scalar fma chains (four independent chains; the fp32
-// state path issues these faster than the packed form).
-__device__ __forceinline__ float dot16_s(const float2 (&a)[8], const float2 (&b)[8]) {
-  float c00 = 0.0f, c01 = 0.0f, c10 = 0.0f, c11 = 0.0f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    c00 = __fmaf_rn(a[e].x, b[e].x, c00);
-    c01 = __fmaf_rn(a[e].y, b[e].y, c01);
-  }
-#pragma unroll
-  for (int e = 4; e < 8; ++e) {
-    c10 = __fmaf_rn(a[e].x, b[e].x, c10);
-    c11 = __fmaf_rn(a[e].y, b[e].y, c11);
-  }
-  return __fadd_rn(__fadd_rn(c00, c10), __fadd_rn(c01, c11));
-}
-
 // The same order with scalar operations.
 __device__ __forceinline__ float dot16_b(const float (&a)[16], const float (&b)[16]) {
   float ch[2][2];

@@ -254,9 +254,22 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       }
     } else {
       float2 cf[8];
-      if (DENSE)
+      if (DENSE) {
         unpack_dense<DENSE ? BITS : 5>(ld_dense<DENSE ? BITS : 5>(stage + (size_t)lrr * RB, DK, lir), cf);
-      else if (w8)
+      } else if (BITS == 0) {
+        // per-lane widths: both kinds of lane bring their codes to offset-binary bytes,
+        // then take one conversion together
+        uint32_t ob[4];
+        const uint8_t *src = stage + (size_t)lrr * RB + loff;
+        if (w8) {
+          const uint4 cw = ld16_a8(src);
+          ob[0] = cw.x ^ 0x80808080u; ob[1] = cw.y ^ 0x80808080u;
+          ob[2] = cw.z ^ 0x80808080u; ob[3] = cw.w ^ 0x80808080u;
+        } else {
+          widen_i4_ob(*reinterpret_cast<const uint2 *>(src), ob);
+        }
+        unpack_ob_2(ob, cf);
+      } else if (w8)
         unpack_i8_2(BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
                               : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff),
                     cf);
@@ -273,7 +286,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     const float vr = sv[lrr];
     float w;
     if (DELTA) {
-      float u = BITS == 32 ? dot16_s(sp, kk) : dot16_p(sp, kk);
+      float u = dot16_p(sp, kk);
 #pragma unroll
       for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
       w = __fmul_rn(beta, __fsub_rn(vr, u));
@@ -286,7 +299,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     for (int e = 0; e < 8; ++e) x[e] = __ffma2_rn(w2, kk[e], sp[e]);
 
     // ---- readout share: this lane's part of S'q ----------------------------------------
-    const float opv = BITS == 32 ? dot16_s(sp, qq) : dot16_p(sp, qq);
+    const float opv = dot16_p(sp, qq);
     if (active) {
       opart[lr * LPR + lir] = opv;
       if (lir == 0) ow[lr] = w;
@@ -330,10 +343,12 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
         const float m = group_absmax<LPR>(chunk_absmax(x), gd1, gd2, gd4, gd8);
         float2 inv;
         gbad = group_scale(m, rq, rq_inv, inv, s_new);
-        if (w8)
-          quantize16<8, SR>(x, inv, hw, words);
-        else
-          quantize16<4, SR>(x, inv, hw, words);
+        quantize16<8, SR>(x, inv, hw, words);            // code bytes for every lane
+        if (!w8) {                                       // nibble lanes compact them
+          const uint2 nw = compact_i4(make_uint4(words[0], words[1], words[2], words[3]));
+          words[0] = nw.x;
+          words[1] = nw.y;
+        }
       } else {
         gbad = requantize16_nb<LPR, BITS, SR>(x, rq, rq_inv, gd1, gd2, gd4, gd8, hw, words, s_new);
       }
