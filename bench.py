@@ -99,9 +99,15 @@ def launch_bytes(wl, bits):
 
 
 def kernel_source_hash():
+    """Hash of the decode-step kernel's source (csrc/lores_step.cuh, csrc/lores_device.cuh)
+    with comments and blank space removed, so a change of wording leaves it unchanged."""
+    import re
     h = hashlib.sha256()
-    for f in ("lores_step.cuh", "lores_device.cuh"):       # the decode-step kernel's source
-        h.update(open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f), "rb").read())
+    for f in ("lores_step.cuh", "lores_device.cuh"):
+        src = open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,14 +7,11 @@
 // with S_{t-1} dequantized from int8/int4 codes and per-(value row, key block) fp32
 // scales, and S_t requantized with stochastic rounding, all in one pass over the state.
 //
-// Work decomposition.  Every value row of every (sequence, head) tile is independent.
-// A work unit is a block of rows of one tile; a persistent CTA (4 warps) walks its
-// share of units round robin.  For each unit one elected thread issues bulk async
-// copies (TMA, non-tensor form) of the unit's codes, scales, k, q, v (and per-column
-// alpha) into a 2-deep shared-memory ring, so the next unit streams in while the
-// current one is computed.  In a warp, d_k/16 lanes own one row, 16 consecutive
-// columns each; dot products and the group absmax reduce across those lanes with
-// shuffles.  Codes go back with 16-byte (int8) / 8-byte (int4) stores.
+// This file: the C ABI (handles, unit planning, launches), the state loader and
+// dequantizer, and the key-axis kernel.  The decode-step kernel (a persistent grid whose
+// warps stream row blocks of tiles through a bulk-copy ring, d_k/16 lanes per row) is in
+// lores_step.cuh, its row arithmetic in lores_device.cuh, and its instantiations in
+// lores_inst.cu.
 #include <cuda_runtime.h>
 
 #include <algorithm>

@@ -585,8 +585,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
 
 using StepFn = void (*)(const StepParams);
 
-// Kernel pickers: the plain single-token kernels are instantiated in lores.cu, the plain
-// multi-token ones in lores_mt.cu, and both extended families in lores_ext.cu.
+// Kernel pickers: every (key width, single/multi-token, plain/extended) family is
+// instantiated in its own compilation of lores_inst.cu.
 template <int DK, bool SR, bool MT, bool EXT>
 StepFn pick_step(bool diag, bool delta) {
   if (diag)
