@@ -2,9 +2,10 @@
 
     python -m bit_recurrent_state_lores_b200.build [--verbose]
 
-csrc/lores.cu (host side, loader, dequantizer, key-axis kernels) and 20 compilations of
-csrc/lores_inst.cu (one decode-step kernel family per key width x single/multi-token x
-plain/extended storage) build in parallel, one nvcc process per CPU core, then link.
+csrc/lores.cu (host side, loader, dequantizer) and 25 compilations of csrc/lores_inst.cu
+(one decode-step kernel family per key width x single/multi-token x plain/extended
+storage, and one key-axis family per key width) build in parallel, one nvcc process per
+CPU core, then link.
 
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
 rounding-sensitive operation is written with explicit round-to-nearest intrinsics
@@ -21,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 SRC = os.path.join(CSRC, "lores.cu")
 INST = os.path.join(CSRC, "lores_inst.cu")
 DEPS = [SRC, INST, os.path.join(CSRC, "lores_step.cuh"), os.path.join(CSRC, "lores_device.cuh"),
-        os.path.join(ROOT, "include", "lores.h")]
+        os.path.join(CSRC, "lores_key.cuh"), os.path.join(ROOT, "include", "lores.h")]
 LIB = os.path.join(PKG, "liblores.so")
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
@@ -32,6 +33,8 @@ KEY_WIDTHS = (16, 32, 64, 128, 256)
 def units():
     """(source, extra flags, object name) of every compilation."""
     out = [(SRC, [], "lores.o")]
+    for dk in KEY_WIDTHS:
+        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
     for dk in KEY_WIDTHS:
         for mt in (0, 1):
             for ext in (0, 1):

@@ -7,11 +7,11 @@
 // with S_{t-1} dequantized from int8/int4 codes and per-(value row, key block) fp32
 // scales, and S_t requantized with stochastic rounding, all in one pass over the state.
 //
-// This file: the C ABI (handles, unit planning, launches), the state loader and
-// dequantizer, and the key-axis kernel.  The decode-step kernel (a persistent grid whose
-// warps stream row blocks of tiles through a bulk-copy ring, d_k/16 lanes per row) is in
-// lores_step.cuh, its row arithmetic in lores_device.cuh, and its instantiations in
-// lores_inst.cu.
+// This file: the C ABI (handles, unit planning, launches), the state loader and the
+// dequantizer.  The decode-step kernel (a persistent grid whose warps stream row blocks
+// of tiles through a bulk-copy ring, d_k/16 lanes per row) is in lores_step.cuh, its row
+// arithmetic in lores_device.cuh, the key-axis variant in lores_key.cuh, and their
+// instantiations in lores_inst.cu.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -25,6 +25,7 @@
 #include "lores.h"
 #include "lores_device.cuh"
 #include "lores_step.cuh"
+#include "lores_key.cuh"
 
 namespace lores {
 
@@ -156,265 +157,6 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
   for (int c = 0; c < 4; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
 }
 
-// -------------------------------------------------------------------------------------
-// key-axis grouping (ablation comparator): one scale per key column of a tile
-// -------------------------------------------------------------------------------------
-// The column maximum couples all rows of a tile, so one CTA handles one whole tile:
-// pass 1 updates every row (x = S' + w k^T), keeps w and the readout shares, and
-// reduces per-column maxima; pass 2 recomputes x (the same fp32 operations) and writes
-// codes with the column scale.  Columns with an inf/NaN/overflow entry are stored as
-// zero and flagged; fp32 heads store x as in the value-axis path.
-struct KeyParams {
-  uint8_t *codes;
-  float *scales;                // [B][H][d_k]
-  const float *q, *k, *v, *alpha, *beta;
-  const float *S;               // load_state input [B][H][d_v][d_k], or null
-  float *o;
-  unsigned *flag;
-  const int32_t *head_bits;
-  const int64_t *head_off;
-  long long seq_bytes;
-  int H, d_v;
-  uint32_t step_key;
-  uint64_t seed;
-  const uint64_t *step_dev;     // step in device memory (CUDA-graph replay), or null
-  int delta, diag, stochastic;
-  // shared memory offsets
-  int sm_codes, sm_scales, sm_k, sm_q, sm_a, sm_v, sm_opart, sm_ow, sm_cm;
-};
-
-// Column maxima of the lane's 16 columns over the whole tile: reduce across the row groups
-// of the warp, then across warps through shared memory.
-template <int DK>
-__device__ __forceinline__ void column_max(float (&cm)[16], float *smcm) {
-  constexpr int LPR = DK / 16;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lir = lane % LPR, riw = lane / LPR;
-#pragma unroll
-  for (int st = LPR; st < 32; st <<= 1)
-#pragma unroll
-    for (int e = 0; e < 16; ++e) cm[e] = max_nan(cm[e], __shfl_xor_sync(kFull, cm[e], st));
-  if (riw == 0)
-#pragma unroll
-    for (int e = 0; e < 16; ++e) smcm[warp * DK + lir * 16 + e] = cm[e];
-  __syncthreads();
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    float m = smcm[lir * 16 + e];
-    for (int w2 = 1; w2 < kWarps; ++w2) m = max_nan(m, smcm[w2 * DK + lir * 16 + e]);
-    cm[e] = m;
-  }
-}
-
-template <int DK>
-__global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyParams p) {
-  constexpr int LPR = DK / 16, RPW = 32 / LPR;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lir = lane % LPR, riw = lane / LPR, col0 = lir * 16;
-  const long long tile = blockIdx.x;
-  const int head = (int)(tile % p.H);
-  const long long b = tile / p.H;
-  const int bits = __ldg(p.head_bits + head);
-  const int rb = row_bytes(DK, bits);
-  uint8_t *gcodes = p.codes + b * p.seq_bytes + __ldg(p.head_off + head);
-  const bool load = p.S != nullptr;            // load_state: x is given, no update
-
-  uint8_t *scodes = smem + p.sm_codes;
-  float *sscales = reinterpret_cast<float *>(smem + p.sm_scales);
-  float *sk = reinterpret_cast<float *>(smem + p.sm_k);
-  float *sq = reinterpret_cast<float *>(smem + p.sm_q);
-  float *sa = reinterpret_cast<float *>(smem + p.sm_a);
-  float *sv = reinterpret_cast<float *>(smem + p.sm_v);
-  float *opart = reinterpret_cast<float *>(smem + p.sm_opart);
-  float *ow = reinterpret_cast<float *>(smem + p.sm_ow);
-  float *smcm = reinterpret_cast<float *>(smem + p.sm_cm);
-
-  if (!load) {
-    if (threadIdx.x == 0) {
-      mbar_init(bar, 1);
-      fence_mbar_init();
-      const unsigned cb = (unsigned)(p.d_v * rb), sb = bits == 32 ? 0u : DK * 4u;
-      const unsigned vec = DK * 4, vb = (unsigned)(p.d_v * 4);
-      mbar_expect_tx(bar, cb + sb + 2 * vec + vb + (p.diag ? vec : 0u));
-      bulk_g2s(scodes, gcodes, cb, bar);
-      if (sb) bulk_g2s(sscales, p.scales + tile * DK, sb, bar);
-      bulk_g2s(sk, p.k + tile * DK, vec, bar);
-      bulk_g2s(sq, p.q + tile * DK, vec, bar);
-      bulk_g2s(sv, p.v + tile * p.d_v, vb, bar);
-      if (p.diag) bulk_g2s(sa, p.alpha + tile * DK, vec, bar);
-    }
-    __syncthreads();
-    if (!__syncthreads_and(mbar_wait_bounded(bar, 0))) {
-      if (threadIdx.x == 0) {
-        atomicOr(p.flag, kFlagTimeout);
-        (void)mbar_wait_bounded(bar, 0);       // let the copies land before the CTA exits
-      }
-      return;
-    }
-  }
-  float kk[16], qq[16], aj[16];
-  const float alpha_s = (load || p.diag) ? 1.0f : __ldg(p.alpha + tile);
-  const float beta = load ? 0.0f : __ldg(p.beta + tile);
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    kk[e] = load ? 0.0f : sk[col0 + e];
-    qq[e] = load ? 0.0f : sq[col0 + e];
-    const float al = load ? 1.0f : (p.diag ? sa[col0 + e] : alpha_s);
-    // entry (i, j) of S_{t-1} diag(alpha) is c_ij * (s_j * alpha_j)
-    aj[e] = (bits == 32 || load) ? al : __fmul_rn(sscales[col0 + e], al);
-  }
-  const uint32_t tkey =
-      tile_key(p.step_dev ? step_key_dev(p.seed, *p.step_dev) : p.step_key, (uint32_t)tile);
-
-  // x of one row for this lane's 16 columns (pass 1 and pass 2 compute it identically).
-  // `first` (pass 1) computes w with warp shuffles: every lane of the warp takes it, and
-  // only lanes of real rows (`write`) keep w and the readout share.
-  auto row_x = [&](int lr, bool write, bool first, float (&x)[16]) {
-    if (load) {
-      const float *src = p.S + (tile * p.d_v + lr) * DK + col0;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) x[e] = src[e];
-      return;
-    }
-    float sp[16];
-    if (bits == 32) {
-      const float *srow = reinterpret_cast<const float *>(scodes + (size_t)lr * rb) + col0;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(srow[e], aj[e]);
-    } else {
-      float cf[16];
-      if (bits == 4)
-        unpack_i4(*reinterpret_cast<const uint2 *>(scodes + (size_t)lr * rb + lir * 8), cf);
-      else
-        unpack_i8(*reinterpret_cast<const uint4 *>(scodes + (size_t)lr * rb + lir * 16), cf);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sp[e] = __fmul_rn(cf[e], aj[e]);
-    }
-    float w;
-    if (first) {
-      if (p.delta) {
-        float u = dot16_b(sp, kk);
-#pragma unroll
-        for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
-        w = __fmul_rn(beta, __fsub_rn(sv[lr], u));
-      } else {
-        w = __fmul_rn(beta, sv[lr]);
-      }
-      const float opv = dot16_b(sp, qq);
-      if (write) {
-        opart[lr * LPR + lir] = opv;
-        if (lir == 0) ow[lr] = w;
-      }
-    } else {
-      w = ow[lr];
-    }
-#pragma unroll
-    for (int e = 0; e < 16; ++e) x[e] = __fmaf_rn(w, kk[e], sp[e]);
-  };
-
-  // ---- pass 1: update every row, column maxima --------------------------------------
-  float cm[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) cm[e] = 0.0f;
-  bool bad32 = false;
-  const int nbase = warp * RPW;
-  for (int base = nbase; base < p.d_v; base += kWarps * RPW) {
-    const int lr = base + riw;
-    const bool active = lr < p.d_v;
-    float x[16];
-    row_x(active ? lr : 0, active, !load, x);
-    if (!active) continue;
-    if (bits == 32) {
-      float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * rb) + lir * 4;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) dst[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) bad32 |= !isfinite(x[e]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) cm[e] = max_abs_nan(cm[e], x[e]);
-    }
-  }
-  if (bits != 32) {
-    column_max<DK>(cm, smcm);
-    const float r = (float)((1 << (bits - 1)) - 1);
-    const float inv_r = __fdiv_rn(1.0f, r);
-    float inv[16];
-    unsigned badcols = 0;                        // bit e: column col0 + e is bad
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const bool bad = !(cm[e] <= 0x1p100f);
-      const bool scaled = !bad && cm[e] >= 0x1p-100f;
-      inv[e] = scaled ? __fmul_rn(r, recip_nr(cm[e])) : 0.0f;
-      const float s = scaled ? __fmul_rn(cm[e], inv_r) : 0.0f;
-      badcols |= (bad ? 1u : 0u) << e;
-      if (warp == 0 && riw == 0) p.scales[tile * DK + col0 + e] = s;
-    }
-    if (badcols && warp == 0 && riw == 0) atomicOr(p.flag, kFlagNonFinite);
-    // byte masks that clear the codes of bad columns
-    uint32_t keep[4];
-#pragma unroll
-    for (int qd = 0; qd < 4; ++qd) {
-      keep[qd] = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        keep[qd] |= ((badcols >> (4 * qd + e)) & 1u) ? 0u : (0xFFu << (8 * e));
-    }
-    // ---- pass 2: recompute x, write codes ------------------------------------------------
-    for (int base = nbase; base < p.d_v; base += kWarps * RPW) {
-      const int lr = base + riw;
-      const bool active = lr < p.d_v;
-      float x[16];
-      row_x(active ? lr : 0, false, false, x);
-      const uint32_t cbase = tkey + 0x9E3779B9u * ((uint32_t)lr * (uint32_t)(DK / 4) + (uint32_t)lir * 4u + 1u);
-      uint32_t h[4] = {0u, 0u, 0u, 0u};
-      if (p.stochastic) dither_words(cbase, h);
-      uint32_t t[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float g = p.stochastic
-                            ? __uint_as_float(__byte_perm(h[e >> 2], 0x47400000u, 0x7650u | (e & 3)))
-                            : 49152.5f;
-        t[e] = __float_as_uint(__fmaf_rn(x[e], inv[e], g));
-      }
-      if (!active) continue;
-      if (bits == 4) {
-        uint2 w = pack_i4(t);
-        // nibble masks: column e of the lane sits in word e/8, nibble e%8
-        uint32_t k0 = 0, k1 = 0;
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (!((badcols >> e) & 1u)) (e < 8 ? k0 : k1) |= 0xFu << (4 * (e & 7));
-        w.x &= k0;
-        w.y &= k1;
-        *reinterpret_cast<uint2 *>(gcodes + (size_t)lr * rb + lir * 8) = w;
-      } else {
-        uint4 w = pack_i8(t);
-        w.x &= keep[0]; w.y &= keep[1]; w.z &= keep[2]; w.w &= keep[3];
-        *reinterpret_cast<uint4 *>(gcodes + (size_t)lr * rb + lir * 16) = w;
-      }
-    }
-  } else if (__any_sync(kFull, bad32) && bad32) {
-    atomicOr(p.flag, kFlagNonFinite);
-  }
-  if (load) return;
-  // ---- readout: o_i = sum of the lane shares + w_i (k.q) --------------------------------
-  __syncthreads();
-  double kqd = 0.0;
-  for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sq[j], kqd);
-#pragma unroll
-  for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
-  const float kq = (float)kqd;
-  float *go = p.o + tile * p.d_v;
-  for (int r = threadIdx.x; r < p.d_v; r += kThreads) {
-    float acc = 0.0f;
-    for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
-    go[r] = __fmaf_rn(ow[r], kq, acc);
-  }
-}
-
 // Adds n to a device step counter (one thread; captured into a CUDA graph together with
 // the steps that read the counter).
 __global__ void advance_step_kernel(uint64_t *step, uint64_t n) { *step += n; }
@@ -460,14 +202,13 @@ static StepFn kernel_for(int dk, bool mt, bool ext, bool diag, bool delta, bool 
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
   return kernel_for(dk, false, false, diag, delta, sr);
 }
-using KeyFn = void (*)(const KeyParams);
-static KeyFn key_kernel_for(int dk) {
+static KeyFn key_kernel_for(int dk, bool sr, bool load) {
   switch (dk) {
-    case 16: return decode_step_key_kernel<16>;
-    case 32: return decode_step_key_kernel<32>;
-    case 64: return decode_step_key_kernel<64>;
-    case 128: return decode_step_key_kernel<128>;
-    case 256: return decode_step_key_kernel<256>;
+    case 16: return key_kernels_16(sr, load);
+    case 32: return key_kernels_32(sr, load);
+    case 64: return key_kernels_64(sr, load);
+    case 128: return key_kernels_128(sr, load);
+    case 256: return key_kernels_256(sr, load);
   }
   return nullptr;
 }
@@ -530,6 +271,9 @@ struct lores_handle {
   KeyParams kp{};
   KeyFn key_fn = nullptr;
   int key_smem = 0;
+  KeyFn key_load_fn = nullptr;           // the same kernel as the state loader
+  int key_grid = 0;                      // persistent grids of the two
+  int key_load_grid = 0;
   // staging for lores_decode_step_host
   float *stage_in = nullptr;
   float *stage_o = nullptr;
@@ -847,34 +591,52 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   const long long code_bytes = (long long)c.batch * h->seq_bytes;
   const long long scale_count = scale_count_of(h);
   if (h->axis) {
-    // key-axis kernel: one CTA per tile, the whole tile in shared memory
+    // key-axis kernel: a CTA holds one whole tile in shared memory at a time, and a second
+    // stage for its next tile where both fit
     int rbmax = 0;
     for (int hh = 0; hh < c.heads; ++hh) rbmax = std::max(rbmax, row_bytes(dk, bits[hh]));
     auto up128 = [](int x) { return (x + 127) & ~127; };
     KeyParams &kp = h->kp;
-    int off = 128;
-    kp.sm_codes = off; off += up128(dv * rbmax);
-    kp.sm_scales = off; off += up128(dk * 4);
-    kp.sm_k = off; off += up128(dk * 4);
-    kp.sm_q = off; off += up128(dk * 4);
-    kp.sm_a = off; off += up128(dk * 4);
-    kp.sm_v = off; off += up128(dv * 4);
+    int so = 0;                                     // offsets inside a stage
+    kp.sm_codes = so; so += up128(dv * rbmax);
+    kp.sm_scales = so; so += up128(dk * 4);
+    kp.sm_k = so; so += up128(dk * 4);
+    kp.sm_q = so; so += up128(dk * 4);
+    kp.sm_a = so; so += up128(dk * 4);
+    kp.sm_v = so; so += up128(dv * 4);
+    kp.stage_bytes = so;
+    int off = 128;                                  // two mbarriers
     kp.sm_opart = off; off += up128(dv * (dk / 16) * 4);
     kp.sm_ow = off; off += up128(dv * 4);
     kp.sm_cm = off; off += up128(kWarps * dk * 4);
-    h->key_smem = off;
-    h->key_fn = key_kernel_for(dk);
-    cudaFuncAttributes fa;
-    if (off > 200 * 1024) {
+    kp.stage0 = off;
+    const int limit = 200 * 1024;
+    if (off + so > limit) {
       delete h;
       return LORES_ERR_UNSUPPORTED;                 // tile too large for one CTA
     }
-    if (cudaFuncGetAttributes(&fa, h->key_fn) != cudaSuccess ||
-        (fa.maxDynamicSharedSizeBytes < off &&
-         cudaFuncSetAttribute(h->key_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, off) !=
-             cudaSuccess)) {
-      delete h;
-      return LORES_ERR_CUDA;
+    kp.nstage = off + 2 * so <= limit ? 2 : 1;
+    off += kp.nstage * so;
+    h->key_smem = off;
+    h->key_fn = key_kernel_for(dk, c.stochastic != 0, false);
+    h->key_load_fn = key_kernel_for(dk, c.stochastic != 0, true);
+    const long long tiles = (long long)c.batch * c.heads;
+    int *grids[2] = {&h->key_grid, &h->key_load_grid};
+    KeyFn fns[2] = {h->key_fn, h->key_load_fn};
+    for (int i = 0; i < 2; ++i) {
+      cudaFuncAttributes fa;
+      int per_sm = 0;
+      if (cudaFuncGetAttributes(&fa, fns[i]) != cudaSuccess ||
+          (fa.maxDynamicSharedSizeBytes < off &&
+           cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, off) !=
+               cudaSuccess) ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fns[i], kThreads, off) !=
+              cudaSuccess ||
+          per_sm < 1) {
+        delete h;
+        return LORES_ERR_CUDA;
+      }
+      *grids[i] = (int)std::min<long long>(tiles, (long long)per_sm * prop.multiProcessorCount);
     }
   }
   cudaError_t e = cudaSuccess;
@@ -936,6 +698,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   kp.head_bits = h->d_bits;
   kp.head_off = h->d_head_off;
   kp.seq_bytes = h->seq_bytes;
+  kp.tiles = (long long)c.batch * c.heads;
   kp.H = c.heads;
   kp.d_v = dv;
   kp.delta = c.delta;
@@ -998,8 +761,7 @@ static lores_status launch_step(lores_handle *h, const float *q, const float *k,
     kp.S = nullptr;
     kp.step_key = step_key_of(h->cfg.seed, step);
     kp.step_dev = step_dev;
-    const unsigned tiles = (unsigned)((long long)h->cfg.batch * h->cfg.heads);
-    h->key_fn<<<tiles, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
+    h->key_fn<<<h->key_grid, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
     return cuda_status(cudaGetLastError());
   }
   StepParams p = h->sp;
@@ -1128,8 +890,7 @@ lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, vo
     KeyParams kp = h->kp;
     kp.S = S;
     kp.step_key = step_key_of(h->cfg.seed, step);
-    const unsigned tiles = (unsigned)((long long)h->cfg.batch * h->cfg.heads);
-    h->key_fn<<<tiles, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
+    h->key_load_fn<<<h->key_load_grid, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
     return cuda_status(cudaGetLastError());
   }
   LoadParams p = load_params(h);

@@ -1,22 +1,39 @@
 // lores_inst.cu -- one family of decode-step kernels for one key width, compiled once per
-// (LORES_DK, LORES_MT, LORES_EXT) so that the families build in parallel:
-//   LORES_MT  = 1: multi-token steps (lores_decode_steps); 0: single-token steps
-//   LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
-// The function defined here returns the kernel for the decay/delta/rounding modes.
+// family so that the families build in parallel:
+//   -DLORES_DK=<d_k> -DLORES_MT=<0|1> -DLORES_EXT=<0|1>: the value-axis step kernels
+//     LORES_MT  = 1: multi-token steps (lores_decode_steps); 0: single-token steps
+//     LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
+//   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
+// The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
-
-#if !defined(LORES_DK) || !defined(LORES_MT) || !defined(LORES_EXT)
-#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1>"
-#endif
+#include "lores_key.cuh"
 
 #define LORES_CAT2(a, b, c, d) a##_##b##_##c##_##d
 #define LORES_CAT(a, b, c, d) LORES_CAT2(a, b, c, d)
+#define LORES_CAT1_2(a, b) a##_##b
+#define LORES_CAT1(a, b) LORES_CAT1_2(a, b)
 
 namespace lores {
 
+#if defined(LORES_KEY)
+#if !defined(LORES_DK)
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_KEY=1"
+#endif
+KeyFn LORES_CAT1(key_kernels, LORES_DK)(bool sr, bool load) {
+  if (load)
+    return sr ? decode_step_key_kernel<LORES_DK, true, true>
+              : decode_step_key_kernel<LORES_DK, false, true>;
+  return sr ? decode_step_key_kernel<LORES_DK, true, false>
+            : decode_step_key_kernel<LORES_DK, false, false>;
+}
+#else
+#if !defined(LORES_DK) || !defined(LORES_MT) || !defined(LORES_EXT)
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1>"
+#endif
 StepFn LORES_CAT(step_kernels, LORES_DK, LORES_MT, LORES_EXT)(bool diag, bool delta, bool sr) {
   return sr ? pick_step<LORES_DK, true, LORES_MT != 0, LORES_EXT != 0>(diag, delta)
             : pick_step<LORES_DK, false, LORES_MT != 0, LORES_EXT != 0>(diag, delta);
 }
+#endif
 
 }  // namespace lores
