@@ -2,9 +2,9 @@
 
     python -m bit_recurrent_state_lores_b200.build [--verbose]
 
-csrc/lores.cu (host side, loader, dequantizer) and 25 compilations of csrc/lores_inst.cu
-(one decode-step kernel family per key width x single/multi-token x plain/extended
-storage, and one key-axis family per key width) build in parallel, one nvcc process per
+csrc/lores.cu (host side, loader, dequantizer) and 35 compilations of csrc/lores_inst.cu
+(one decode-step kernel family per key width x single/multi-token x storage family --
+plain; dense and per-lane; per-lane only -- and one key-axis family per key width) build in parallel, one nvcc process per
 CPU core, then link.
 
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
@@ -37,7 +37,7 @@ def units():
         out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
     for dk in KEY_WIDTHS:
         for mt in (0, 1):
-            for ext in (0, 1):
+            for ext in (0, 1, 2):
                 out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],
                             f"lores_inst_{dk}_{mt}_{ext}.o"))
     return out

@@ -182,13 +182,18 @@ using LoadFn = void (*)(const LoadParams);
 using DequantFn = void (*)(const LoadParams, float *);
 
 // The decode-step kernel of a configuration: mt = multi-token, ext = extended storage.
-static StepFn kernel_for(int dk, bool mt, bool ext, bool diag, bool delta, bool sr) {
+// ext: 0 plain kernel, 1 with the dense and per-lane paths, 2 with the per-lane path only
+static StepFn kernel_for(int dk, bool mt, int ext, bool diag, bool delta, bool sr) {
+#define LORES_PICK_EXT(dk_, m_)                                                \
+  return ext == 2 ? step_kernels_##dk_##_##m_##_2(diag, delta, sr)             \
+                  : (ext == 1 ? step_kernels_##dk_##_##m_##_1(diag, delta, sr) \
+                              : step_kernels_##dk_##_##m_##_0(diag, delta, sr));
 #define LORES_PICK(dk_)                                                        \
   case dk_:                                                                    \
-    return mt ? (ext ? step_kernels_##dk_##_1_1(diag, delta, sr)               \
-                     : step_kernels_##dk_##_1_0(diag, delta, sr))              \
-              : (ext ? step_kernels_##dk_##_0_1(diag, delta, sr)               \
-                     : step_kernels_##dk_##_0_0(diag, delta, sr));
+    if (mt) {                                                                  \
+      LORES_PICK_EXT(dk_, 1)                                                   \
+    }                                                                          \
+    LORES_PICK_EXT(dk_, 0)
   switch (dk) {
     LORES_PICK(16)
     LORES_PICK(32)
@@ -197,10 +202,11 @@ static StepFn kernel_for(int dk, bool mt, bool ext, bool diag, bool delta, bool 
     LORES_PICK(256)
   }
 #undef LORES_PICK
+#undef LORES_PICK_EXT
   return nullptr;
 }
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
-  return kernel_for(dk, false, false, diag, delta, sr);
+  return kernel_for(dk, false, 0, diag, delta, sr);
 }
 static KeyFn key_kernel_for(int dk, bool sr, bool load) {
   switch (dk) {
@@ -481,10 +487,14 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     const int n = 4096 / rb;
     return std::min(n < rpw ? rpw : n - n % rpw, dv);
   };
-  // handles with dense or mixed-width heads take the extended kernel family
-  bool ext = false;
-  for (int hh = 0; hh < c.heads; ++hh)
-    ext |= !(h->store[hh] == 4 || h->store[hh] == 8 || h->store[hh] == 32);
+  // handles with dense heads take the kernel family with the dense and per-lane paths;
+  // handles with per-channel (mixed-width) rows and no dense heads the per-lane family
+  bool dense_heads = false, lane_heads = false;
+  for (int hh = 0; hh < c.heads; ++hh) {
+    dense_heads |= h->store[hh] >= 5 && h->store[hh] <= 7;
+    lane_heads |= h->store[hh] == 0;
+  }
+  const int ext = dense_heads ? 1 : (lane_heads ? 2 : 0);
   StepFn fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
   int split = 1;
   auto build_units = [&](std::vector<UnitDesc> &u) {

@@ -3,6 +3,7 @@
 //   -DLORES_DK=<d_k> -DLORES_MT=<0|1> -DLORES_EXT=<0|1>: the value-axis step kernels
 //     LORES_MT  = 1: multi-token steps (lores_decode_steps); 0: single-token steps
 //     LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
+//     LORES_EXT = 2: with the per-lane path only
 //   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
 // The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
@@ -28,11 +29,11 @@ KeyFn LORES_CAT1(key_kernels, LORES_DK)(bool sr, bool load) {
 }
 #else
 #if !defined(LORES_DK) || !defined(LORES_MT) || !defined(LORES_EXT)
-#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1>"
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1|2>"
 #endif
 StepFn LORES_CAT(step_kernels, LORES_DK, LORES_MT, LORES_EXT)(bool diag, bool delta, bool sr) {
-  return sr ? pick_step<LORES_DK, true, LORES_MT != 0, LORES_EXT != 0>(diag, delta)
-            : pick_step<LORES_DK, false, LORES_MT != 0, LORES_EXT != 0>(diag, delta);
+  return sr ? pick_step<LORES_DK, true, LORES_MT != 0, LORES_EXT>(diag, delta)
+            : pick_step<LORES_DK, false, LORES_MT != 0, LORES_EXT>(diag, delta);
 }
 #endif
 

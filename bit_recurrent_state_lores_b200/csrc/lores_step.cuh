@@ -444,28 +444,31 @@ __device__ __forceinline__ void compute_any(const StepParams &p, uint8_t *stage,
     compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   }
 }
-// One unit for one token: the unit's storage class picks the code path.  EXT: the kernel
-// also carries the dense and per-lane paths (kept out of the plain kernel, whose code
-// stays smaller and faster for int8 / int4 / fp32 handles).
-template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, bool EXT>
+// One unit for one token: the unit's storage class picks the code path.  EXT: 0 the plain
+// kernel (int8 / int4 / fp32 units only, the smallest code); 1 also the dense 5- to 7-bit
+// and per-lane (per-channel) paths; 2 the per-lane path without the dense ones, so a
+// handle with per-channel rows and no dense heads runs with fewer registers live.
+template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, int EXT>
 __device__ __forceinline__ void compute_bits(const StepParams &p, uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow, int t) {
   if (d.store == 32)
     compute_any<DK, DIAG, DELTA, SR, 32, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (!EXT || d.store == 4 || d.store == 8) {
+  else if (EXT == 0 || d.store == 4 || d.store == 8) {
     if (d.store == 4)
       compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
       compute_any<DK, DIAG, DELTA, SR, 8, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  } else if (d.store == 0)
+  } else if (d.store == 0) {
     compute_any<DK, DIAG, DELTA, SR, 0, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.store == 6)
-    compute_any<DK, DIAG, DELTA, SR, 6, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (d.store == 5)
-    compute_any<DK, DIAG, DELTA, SR, 5, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else
-    compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  } else if constexpr (EXT == 1) {
+    if (d.store == 6)
+      compute_any<DK, DIAG, DELTA, SR, 6, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    else if (d.store == 5)
+      compute_any<DK, DIAG, DELTA, SR, 5, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    else
+      compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  }
 }
 
 // Position of a unit: global unit u = ub * B + b (sequence b is the fast index, so a warp
@@ -487,7 +490,7 @@ struct UnitPos {
 // Persistent kernel: every warp runs its own pipeline over units gw, gw + W, gw + 2W, ...
 // (gw = global warp index, W = warps in the grid), with a 2-slot ring of bulk copies
 // whose producer is the warp's lane 0.  Warps never wait on one another.
-template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, bool EXT>
+template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, int EXT>
 __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -585,9 +588,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
 
 using StepFn = void (*)(const StepParams);
 
-// Kernel pickers: every (key width, single/multi-token, plain/extended) family is
-// instantiated in its own compilation of lores_inst.cu.
-template <int DK, bool SR, bool MT, bool EXT>
+// Kernel pickers: every (key width, single/multi-token, storage family) is instantiated
+// in its own compilation of lores_inst.cu.
+template <int DK, bool SR, bool MT, int EXT>
 StepFn pick_step(bool diag, bool delta) {
   if (diag)
     return delta ? decode_step_kernel<DK, true, true, SR, MT, EXT>
@@ -601,7 +604,9 @@ StepFn pick_step(bool diag, bool delta) {
   StepFn step_kernels_##dk##_0_0(bool diag, bool delta, bool sr);  \
   StepFn step_kernels_##dk##_1_0(bool diag, bool delta, bool sr);  \
   StepFn step_kernels_##dk##_0_1(bool diag, bool delta, bool sr);  \
-  StepFn step_kernels_##dk##_1_1(bool diag, bool delta, bool sr);
+  StepFn step_kernels_##dk##_1_1(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_0_2(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_1_2(bool diag, bool delta, bool sr);
 LORES_DECLARE_FAMILY(16)
 LORES_DECLARE_FAMILY(32)
 LORES_DECLARE_FAMILY(64)
