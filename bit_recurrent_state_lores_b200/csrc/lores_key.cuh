@@ -198,6 +198,22 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
     }
   }
 
+  if (!LOAD) {
+    // ---- readout of this warp's rows: o_i = the lane shares in lane order + w_i (k.q);
+    // the shares and w were written by this warp in pass 1, so no CTA barrier is needed
+    __syncwarp();
+    const float kq = (float)kqd;
+    float *go = p.o + tile * p.d_v;
+    for (int k = lane;; k += 32) {
+      const int r = (k / RPW) * (kWarps * RPW) + nbase + k % RPW;   // the warp's k-th row
+      if (r >= p.d_v) break;
+      float acc = 0.0f;
+#pragma unroll
+      for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
+      go[r] = __fmaf_rn(ow[r], kq, acc);
+    }
+    __syncwarp();
+  }
   if (STORE == 32) {
     if (__any_sync(kFull, bad32) && bad32) atomicOr(p.flag, kFlagNonFinite);
   } else {
@@ -274,18 +290,6 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
         w.x &= keep[0]; w.y &= keep[1]; w.z &= keep[2]; w.w &= keep[3];
         *reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16) = w;
       }
-    }
-  }
-  if (!LOAD) {
-    // ---- readout: o_i = sum of the lane shares + w_i (k.q) --------------------------------
-    __syncthreads();
-    const float kq = (float)kqd;
-    float *go = p.o + tile * p.d_v;
-    for (int r = threadIdx.x; r < p.d_v; r += kThreads) {
-      float acc = 0.0f;
-#pragma unroll
-      for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
-      go[r] = __fmaf_rn(ow[r], kq, acc);
     }
   }
 }
