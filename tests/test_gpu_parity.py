@@ -1,6 +1,6 @@
 """GPU <-> oracle parity through the C ABI, on the seeded synthetic workloads.
 
-Bounds (the acceptance bounds of this build): o_t and the dequantized state within
+Acceptance bounds: o_t and the dequantized state within
 rel-L2 1e-5; codes equal except at most 1e-4 of entries at +-1 (the arithmetic is
 specified down to the fp32 rounding of every step, so codes are expected to match
 exactly, and the small shapes assert that); packing and scale indexing bit-exact.
