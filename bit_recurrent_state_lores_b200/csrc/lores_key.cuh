@@ -313,6 +313,21 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
   }
   __syncthreads();
 
+  // the first tile's stage: every thread waits, then the CTA agrees it landed
+  if (!LOAD && blockIdx.x < p.tiles) {
+    const bool ok = mbar_wait_bounded(&bars[0], 0u);
+    if (!__syncthreads_and(ok)) {
+      if (threadIdx.x == 0) {
+        atomicOr(p.flag, kFlagTimeout);
+        // let every copy in flight land before the CTA exits
+        for (int s2 = 0; s2 < p.nstage; ++s2)
+          if (blockIdx.x + (long long)s2 * gridDim.x < p.tiles)
+            (void)mbar_wait_bounded(&bars[s2], 0u);
+      }
+      return;
+    }
+  }
+
   int n = 0;
   for (long long tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++n) {
     const int s = n % p.nstage;
@@ -320,31 +335,39 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
     const int bits = __ldg(p.head_bits + (int)(tile % p.H));
     const float alpha_s = (LOAD || p.diag) ? 1.0f : __ldg(p.alpha + tile);
     const float beta = LOAD ? 0.0f : __ldg(p.beta + tile);
-    if (!LOAD) {
-      const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / p.nstage) & 1));
-      if (!__syncthreads_and(ok)) {
-        if (threadIdx.x == 0) {
-          atomicOr(p.flag, kFlagTimeout);
-          // let every copy in flight land before the CTA exits
-          (void)mbar_wait_bounded(&bars[s], (unsigned)((n / p.nstage) & 1));
-          for (int s2 = 1; s2 < p.nstage; ++s2)
-            if (tile + (long long)s2 * gridDim.x < p.tiles)
-              (void)mbar_wait_bounded(&bars[(n + s2) % p.nstage],
-                                      (unsigned)(((n + s2) / p.nstage) & 1));
-        }
-        return;
-      }
-    }
     if (bits == 32)
       key_tile<DK, 32, SR, LOAD>(p, tile, bits, st, alpha_s, beta, skey, opart, ow, smcm);
     else if (bits == 4)
       key_tile<DK, 4, SR, LOAD>(p, tile, bits, st, alpha_s, beta, skey, opart, ow, smcm);
     else
       key_tile<DK, 8, SR, LOAD>(p, tile, bits, st, alpha_s, beta, skey, opart, ow, smcm);
-    // every thread is done with this stage, the readout shares and the column maxima
-    __syncthreads();
-    if (!LOAD && threadIdx.x == 0) {
-      const long long tn = tile + (long long)p.nstage * gridDim.x;
+    if (LOAD) {
+      __syncthreads();                         // the column maxima are reused next tile
+      continue;
+    }
+    const long long tnext = tile + gridDim.x;
+    const int snext = (n + 1) % p.nstage;
+    const unsigned pnext = (unsigned)(((n + 1) / p.nstage) & 1);
+    if (p.nstage == 1) {
+      // one stage: every thread is done with it before it is refilled with the next tile
+      __syncthreads();
+      if (threadIdx.x == 0 && tnext < p.tiles) {
+        fence_proxy_async();
+        issue_key_tile<DK>(p, tnext, st, &bars[0]);
+      }
+    }
+    // Wait for the next tile's stage; the barrier also says that every thread is done
+    // with this tile's stage and column maxima, so (two stages) it can be refilled.
+    const bool ok = tnext < p.tiles ? mbar_wait_bounded(&bars[snext], pnext) : true;
+    if (!__syncthreads_and(ok)) {
+      if (threadIdx.x == 0) {
+        atomicOr(p.flag, kFlagTimeout);
+        (void)mbar_wait_bounded(&bars[snext], pnext);   // the copy in flight lands first
+      }
+      return;
+    }
+    if (p.nstage == 2 && threadIdx.x == 0) {
+      const long long tn = tile + 2LL * gridDim.x;
       if (tn < p.tiles) {
         fence_proxy_async();
         issue_key_tile<DK>(p, tn, st, &bars[s]);

@@ -71,6 +71,7 @@ KEY_SWEEP = [
     (256, 64, [8, 4], 1, 0, 1, 2, 2),
     (64, 512, [8, 4], 1, 1, 1, 2, 2),         # tall tile: the two-pass recompute kernel
     (32, 4, [8, 4], 1, 0, 1, 3, 2),           # four rows
+    (128, 256, [32, 8], 1, 0, 1, 2, 2),       # 128 KB fp32 tile: one shared-memory stage
 ]
 
 
