@@ -31,15 +31,17 @@ KEY_WIDTHS = (16, 32, 64, 128, 256)
 
 
 def units():
-    """(source, extra flags, object name) of every compilation."""
-    out = [(SRC, [], "lores.o")]
-    for dk in KEY_WIDTHS:
-        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
-    for dk in KEY_WIDTHS:
-        for mt in (0, 1):
-            for ext in (0, 1, 2):
+    """(source, extra flags, object name) of every compilation, the slowest first (the
+    extended families), so the parallel build does not end on one long unit."""
+    out = []
+    for ext in (1, 2, 0):
+        for mt in (1, 0):
+            for dk in reversed(KEY_WIDTHS):
                 out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],
                             f"lores_inst_{dk}_{mt}_{ext}.o"))
+    for dk in KEY_WIDTHS:
+        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
+    out.append((SRC, [], "lores.o"))
     return out
 
 
