@@ -69,15 +69,20 @@ def workload(args):
     return synth.workload("sweep", B=args.batch, layers=args.layers)
 
 
-def layer_bits(args, wl, layer):
+def layer_bits(args, wl, layer, policy=None):
+    """Head bits of one layer.  Mixed precision: the 25 % slowest-decaying heads at 8 bits,
+    by `policy` (the library's lores_assign_bits_by_decay on the GPU arm; the oracle's own
+    copy of the rule on the CPU arm, which must not load the GPU library)."""
     from bit_recurrent_state_lores_b200 import synth
-    from bit_recurrent_state_lores_b200 import lores as L
     if args.variant == "int8":
         return [8] * wl.H
     if args.variant == "fp32":
         return [32] * wl.H
+    if policy is None:
+        from bit_recurrent_state_lores_b200 import lores as L
+        policy = L.lores_assign_bits_by_decay
     hp = synth.head_params(layer_workload(wl, layer))
-    return L.lores_assign_bits_by_decay(hp["mean_decay"], 0.25, 8, 4)
+    return [int(b) for b in policy(hp["mean_decay"], 0.25, 8, 4)]
 
 
 def layer_workload(wl, layer):
@@ -101,11 +106,12 @@ def launch_bytes(wl, bits):
 
 
 def kernel_source_hash():
-    """Hash of the decode-step kernel's source (csrc/lores_step.cuh, csrc/lores_device.cuh)
-    with comments and blank space removed, so a change of wording leaves it unchanged."""
+    """Hash of the decode-step kernels' source (csrc/lores_pair.cuh, csrc/lores_step.cuh,
+    csrc/lores_device.cuh) with comments and blank space removed, so a change of wording
+    leaves it unchanged."""
     import re
     h = hashlib.sha256()
-    for f in ("lores_step.cuh", "lores_device.cuh"):
+    for f in ("lores_pair.cuh", "lores_step.cuh", "lores_device.cuh"):
         src = open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f)).read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
         src = re.sub(r"//[^\n]*", " ", src)
@@ -195,6 +201,55 @@ class ClockSampler:
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------------------
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def time_oracle_all_cores(wl, variant_bits, seconds, steps=None):
+    """The oracle's decode step on every host core: the same C step (lo_tile_step) over the
+    (sequence, head) tiles of the sample in an OpenMP loop (oracle/lores_oracle_omp.c).
+    Sample: layer 0, enough sequences for at least four tiles per core, all heads, for
+    successive steps until `seconds` elapse (or `steps` steps).  Returns (rate in
+    state-updates/s, tiles done, elapsed s, threads used, description)."""
+    import numpy as np
+    from bit_recurrent_state_lores_b200 import synth
+    from oracle import oracle as O
+
+    cores = len(os.sched_getaffinity(0))
+    nb = max(1, (4 * cores + wl.H - 1) // wl.H)
+    wl0 = synth.replace(layer_workload(wl, 0), B=nb)
+    hp = synth.head_params(wl0)
+    cfgs = [O.TileCfg(wl0.d_k, wl0.d_v, group=wl0.G, bits=b, delta=wl0.delta, diag=wl0.diag)
+            for b in variant_bits]
+    n = nb * wl0.H
+    cfg_of = [i % wl0.H for i in range(n)]
+    states = [cfgs[c].zero_state() for c in cfg_of]
+    done, elapsed, t, used = 0, 0.0, 0, 1
+    while (steps is None and elapsed < seconds) or (steps is not None and t < steps):
+        q, k, v, a, b = [x.numpy() for x in synth.step_inputs(wl0, t, hp, device="cpu")]
+        sk = O.step_key(wl0.seed, t)
+        keys = [O.tile_key(sk, i) for i in range(n)]
+        t0 = time.perf_counter()
+        _, _, used = O.batch_step(cfgs, cfg_of, [st[0] for st in states], [st[1] for st in states],
+                                  q.reshape(n, -1), k.reshape(n, -1), v.reshape(n, -1),
+                                  a.reshape(n, -1), b.reshape(n), keys)
+        elapsed += time.perf_counter() - t0
+        done += n
+        t += 1
+    desc = (f"oracle decode step on {used} threads (OpenMP over tiles): layer 0, batch {nb}, "
+            f"{wl0.H} heads {wl0.d_v}x{wl0.d_k}, {t} steps ({done} (seq,head) updates, "
+            f"{elapsed:.1f} s)")
+    return done / elapsed, done, elapsed, used, desc
+
+
 def time_oracle(wl, variant_bits, seconds, steps=None):
     """Run the oracle's decode step on a bounded sample of the workload: tiles of layer 0,
     batch 1, all heads, for successive steps until `seconds` elapse (or `steps` steps).
@@ -223,10 +278,6 @@ def time_oracle(wl, variant_bits, seconds, steps=None):
     desc = (f"oracle decode step, single thread: layer 0, batch 1, {wl0.H} heads "
             f"{wl0.d_v}x{wl0.d_k}, {t} steps ({done} (seq,head) updates, {elapsed:.1f} s)")
     return done / elapsed, done, elapsed, desc
-
-
-def cpu_cores_used():
-    return 1
 
 
 # ---------------------------------------------------------------------------------------
@@ -415,9 +466,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            rate, done, el, desc = time_oracle(wl, layers[0][1], args.cpu_seconds)
-            cpu = {"value": rate, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
-                   "sample": desc}
+            cpu = cpu_baseline(wl, layers[0][1], args.cpu_seconds)
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
@@ -441,6 +490,16 @@ def run_ours(args, rank, world, local_rank):
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clock_summary,
         }
     return result
+
+
+def cpu_baseline(wl, bits, seconds):
+    """The oracle on the host: all cores (the reported value) and one core, half of
+    `seconds` each."""
+    rate, _, _, used, desc = time_oracle_all_cores(wl, bits, seconds / 2)
+    rate1, _, _, desc1 = time_oracle(wl, bits, seconds / 2)
+    return {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle", "sample": desc,
+            "cpu_model": cpu_model(), "affinity_cores": len(os.sched_getaffinity(0)),
+            "one_core": {"value": rate1, "unit": UNIT, "cores": 1, "sample": desc1}}
 
 
 def run_sweep(args):
@@ -629,15 +688,17 @@ def run_formats(args):
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: same metric, timed on host cores."""
+    """The oracle as the reference arm: same metric, timed on every host core (the oracle's
+    OpenMP tile loop); `warmup` untimed steps, then `steps` timed steps of the sample."""
     if rank != 0:
         return None
+    from oracle import oracle as O
     wl = workload(args)
-    bits = layer_bits(args, wl, 0)
+    bits = layer_bits(args, wl, 0, policy=O.assign_bits_by_decay)
     K = args.steps
-    per_step_budget = max(0.2, min(2.0, 120.0 / max(1, K + args.warmup)))
-    time_oracle(wl, bits, per_step_budget * args.warmup) if args.warmup else None
-    rate, done, el, desc = time_oracle(wl, bits, per_step_budget * K)
+    if args.warmup:
+        time_oracle_all_cores(wl, bits, 0.0, steps=args.warmup)
+    rate, done, el, used, desc = time_oracle_all_cores(wl, bits, 0.0, steps=K)
     return {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
@@ -645,8 +706,9 @@ def run_reference(args, rank, world):
         "config": {"workload": f"sweep-{args.variant}-b{wl.B}-L{wl.layers}",
                    "batch_per_gpu": wl.B, "heads": wl.H, "d_k": wl.d_k, "d_v": wl.d_v,
                    "layers": wl.layers},
-        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cpu_cores_used(),
-                         "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": desc, "cpu_model": cpu_model(),
+                         "affinity_cores": len(os.sched_getaffinity(0))},
         "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

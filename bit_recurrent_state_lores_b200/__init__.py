@@ -9,8 +9,12 @@ there is no CPU fallback.
 import importlib
 
 
+# submodules: `from bit_recurrent_state_lores_b200 import synth` must not load the library
+_SUBMODULES = ("synth", "build", "lores")
+
+
 def __getattr__(name):
-    if name.startswith("__"):
+    if name.startswith("__") or name in _SUBMODULES:
         raise AttributeError(name)
     mod = importlib.import_module(__name__ + ".lores")
     try:

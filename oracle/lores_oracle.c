@@ -464,6 +464,141 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
     return flag;
 }
 
+/* ------------------------------------------------------------------------ */
+/* The plain definition of the same step                                    */
+/* ------------------------------------------------------------------------ */
+
+/* One decode step written as the pages state it, with none of the evaluation
+ * choices above: every product and sum in double precision in plain order,
+ *   S'_ij = c_ij s_ig alpha_j,  u_i = sum_j S'_ij k_j,  w_i = beta (v_i - delta u_i),
+ *   x_ij = S'_ij + w_i k_j,     o_i = sum_j x_ij q_j,
+ * and the requantization of Proposition 1 and Proposition 3 with plain division:
+ * per group m = max |x|, the stored scale s = m / r rounded once to fp32, y = x r / m,
+ * code = floor(y + (d + 1/2) / 256) with the same dither byte d as the step above (an
+ * 8-bit uniform offset in (0, 1)), or floor(y + 1/2) for round to nearest, clamped to
+ * [-r, r].  The non-finite, overflow (above 2^100) and tiny (below 2^-100) rules are the
+ * step's.  Key-axis groups: m and the scale per key column over the tile.
+ * The evaluated step (lo_tile_step) must agree with this one within the parity bounds:
+ * its fixed fp32 dot order, Newton reciprocal and 1/256-grid quantizer are evaluation
+ * choices, not a different method.  Same arguments and results as lo_tile_step
+ * (x_out: x rounded to fp32). */
+static int quantize_group_plain(const lo_cfg *c, const double *x, int n, int stride, int bits,
+                                const uint32_t *dither, int *codes_out, float *s_out)
+{
+    const int r = code_max(bits);
+    double m = 0.0;
+    int bad = 0;
+    for (int a = 0; a < n; a++) {
+        double v = x[(size_t)a * stride];
+        if (!isfinite(v) || fabs(v) > 0x1p100)
+            bad = 1;
+        else if (fabs(v) > m)
+            m = fabs(v);
+    }
+    if (bad || m < 0x1p-100) {
+        for (int a = 0; a < n; a++)
+            codes_out[a] = 0;
+        *s_out = 0.0f;
+        return bad;
+    }
+    *s_out = (float)(m / (double)r);
+    for (int a = 0; a < n; a++) {
+        double y = x[(size_t)a * stride] * (double)r / m;
+        double u = c->stochastic ? ((double)dither[a] + 0.5) / 256.0 : 0.5;
+        int code = (int)floor(y + u);
+        if (code > r) code = r;
+        if (code < -r) code = -r;
+        codes_out[a] = code;
+    }
+    return 0;
+}
+
+int lo_tile_step_plain(const lo_cfg *c, void *state, float *scales,
+                       const float *q, const float *k, const float *v,
+                       const float *alpha, float beta, uint32_t tile_key,
+                       double *o_out, float *x_out)
+{
+    const int dk = c->d_k, dv = c->d_v, ng = dk / c->group;
+    double *X = malloc(sizeof(double) * (size_t)dk * dv);
+    double *Sp = malloc(sizeof(double) * dk);
+    uint32_t *dith = malloc(sizeof(uint32_t) * (dk > dv ? dk : dv));
+    int *cod = malloc(sizeof(int) * (dk > dv ? dk : dv));
+    int flag = 0;
+    for (int i = 0; i < dv; i++) {
+        for (int j = 0; j < dk; j++) {
+            double aj = c->diag ? alpha[j] : alpha[0];
+            if (c->bits == 32)
+                Sp[j] = (double)((float *)state)[(size_t)i * dk + j] * aj;
+            else {
+                double s = c->axis ? scales[j] : scales[(size_t)i * ng + j / c->group];
+                Sp[j] = (double)get_code(c, (uint8_t *)state, i, j) * s * aj;
+            }
+        }
+        double u = 0.0;
+        for (int j = 0; j < dk; j++)
+            u += Sp[j] * (double)k[j];
+        double w = (double)beta * ((double)v[i] - (c->delta ? u : 0.0));
+        double o = 0.0;
+        for (int j = 0; j < dk; j++) {
+            double xv = Sp[j] + w * (double)k[j];
+            X[(size_t)i * dk + j] = xv;
+            o += xv * (double)q[j];
+        }
+        o_out[i] = o;
+    }
+    if (x_out)
+        for (size_t e = 0; e < (size_t)dk * dv; e++)
+            x_out[e] = (float)X[e];
+    if (c->bits == 32) {
+        for (size_t e = 0; e < (size_t)dk * dv; e++) {
+            float f = (float)X[e];
+            if (!isfinite(f))
+                flag = 1;
+            ((float *)state)[e] = f;
+        }
+    } else if (c->axis) {
+        for (int j = 0; j < dk; j++) {
+            for (int i = 0; i < dv; i++)
+                dith[i] = lo_dither(tile_key, dk, i, j);
+            flag |= quantize_group_plain(c, X + j, dv, dk, c->bits, dith, cod, &scales[j]);
+            for (int i = 0; i < dv; i++)
+                put_code(c, (uint8_t *)state, i, j, cod[i]);
+        }
+    } else {
+        for (int i = 0; i < dv; i++) {
+            /* a row with any non-finite (or overflowing) entry is stored as zero */
+            int rowbad = 0;
+            for (int j = 0; j < dk; j++) {
+                double xv = X[(size_t)i * dk + j];
+                if (!isfinite(xv) || fabs(xv) > 0x1p100)
+                    rowbad = 1;
+            }
+            for (int g = 0; g < ng; g++) {
+                const int j0 = g * c->group;
+                for (int j = 0; j < c->group; j++)
+                    dith[j] = lo_dither(tile_key, dk, i, j0 + j);
+                float s;
+                quantize_group_plain(c, X + (size_t)i * dk + j0, c->group, 1,
+                                     group_bits_of(c, g), dith, cod, &s);
+                if (rowbad) {
+                    s = 0.0f;
+                    for (int j = 0; j < c->group; j++)
+                        cod[j] = 0;
+                }
+                scales[(size_t)i * ng + g] = s;
+                for (int j = 0; j < c->group; j++)
+                    put_code(c, (uint8_t *)state, i, j0 + j, cod[j]);
+            }
+            flag |= rowbad;
+        }
+    }
+    free(X);
+    free(Sp);
+    free(dith);
+    free(cod);
+    return flag;
+}
+
 /* Quantize an fp32 tile S (d_v x d_k) into codes and scales with the same
  * quantizer as the decode step.  Returns 1 if a row was non-finite. */
 int lo_tile_quantize(const lo_cfg *c, const float *S, uint8_t *codes, float *scales,

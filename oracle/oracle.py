@@ -49,6 +49,8 @@ def lib():
         L.lo_tile_step.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_void_p, C.c_void_p,
                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_float, C.c_uint32,
                                    C.c_void_p, C.c_void_p]
+        L.lo_tile_step_plain.restype = C.c_int
+        L.lo_tile_step_plain.argtypes = L.lo_tile_step.argtypes
         L.lo_tile_quantize.restype = C.c_int
         L.lo_tile_quantize.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_void_p, C.c_void_p,
                                        C.c_uint32]
@@ -195,6 +197,20 @@ def tile_step(cfg: TileCfg, state, scales, q, k, v, alpha, beta, tkey, want_x=Fa
     return o, int(flag), x
 
 
+def tile_step_plain(cfg: TileCfg, state, scales, q, k, v, alpha, beta, tkey, want_x=False):
+    """The plain definition of the same step (double precision, plain division and
+    floor; see lo_tile_step_plain).  Same arguments and results as tile_step."""
+    assert state.flags.c_contiguous and scales.flags.c_contiguous
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    alpha = _f32(np.atleast_1d(alpha))
+    o = np.empty(cfg.d_v, np.float64)
+    x = np.empty((cfg.d_v, cfg.d_k), np.float32) if want_x else None
+    flag = lib().lo_tile_step_plain(C.byref(cfg.c), _p(state), _p(scales), _p(q), _p(k), _p(v),
+                                    _p(alpha), float(np.float32(beta)), tkey, _p(o),
+                                    _p(x) if want_x else None)
+    return o, int(flag), x
+
+
 def tile_quantize(cfg: TileCfg, S, tkey):
     S = _f32(S)
     codes = np.zeros(cfg.code_bytes(), np.uint8)
@@ -209,6 +225,46 @@ def tile_dequant(cfg: TileCfg, codes, scales):
     S = np.empty((cfg.d_v, cfg.d_k), np.float32)
     lib().lo_tile_dequant(C.byref(cfg.c), _p(codes), _p(scales), _p(S))
     return S
+
+
+_lib_omp = None
+
+
+def lib_omp():
+    """The oracle built with its OpenMP tile loop (lores_oracle_omp.c)."""
+    global _lib_omp
+    if _lib_omp is None:
+        L = C.CDLL(_build.build_omp())
+        L.lo_batch_step.restype = C.c_int
+        L.lo_batch_step.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p,
+                                    C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                    C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
+                                    C.c_void_p, C.c_int]
+        _lib_omp = L
+    return _lib_omp
+
+
+def batch_step(cfgs, cfg_of, states, scales, q, k, v, alpha, beta, tile_keys, threads=0):
+    """One decode step of n tiles on all host cores: tile t is lo_tile_step with
+    cfgs[cfg_of[t]], states[t], scales[t] (in place) and row t of q, k, v [n, d], alpha
+    [n, 1 or d_k], beta [n], tile_keys [n].  Returns (o [n, d_v] float64, flags [n], the
+    number of threads used)."""
+    n = len(states)
+    d_k, d_v = cfgs[0].d_k, cfgs[0].d_v
+    q, k, v = _f32(q).reshape(n, d_k), _f32(k).reshape(n, d_k), _f32(v).reshape(n, d_v)
+    alpha = _f32(alpha).reshape(n, -1)
+    beta = _f32(beta).reshape(n)
+    keys = np.ascontiguousarray(tile_keys, dtype=np.uint32)
+    cfg_ptrs = (C.c_void_p * len(cfgs))(*[C.cast(C.pointer(c.c), C.c_void_p) for c in cfgs])
+    idx = np.ascontiguousarray(cfg_of, dtype=np.int32)
+    sp = (C.c_void_p * n)(*[st.ctypes.data for st in states])
+    scp = (C.c_void_p * n)(*[sc.ctypes.data for sc in scales])
+    o = np.empty((n, d_v), np.float64)
+    flags = np.zeros(n, np.int32)
+    used = lib_omp().lo_batch_step(cfg_ptrs, _p(idx), n, sp, scp, _p(q), _p(k), _p(v),
+                                   _p(alpha), _p(beta), _p(keys), d_k, d_v, alpha.shape[1],
+                                   _p(o), _p(flags), int(threads))
+    return o, flags, int(used)
 
 
 def assign_bits_by_decay(mean_decay, frac_high, bits_high=8, bits_low=4):

@@ -45,3 +45,26 @@ def test_tile_and_launch_bytes_of_the_default_workload():
     assert bench.tile_bytes(wl, 4) == 19464
     assert bench.tile_bytes(wl, 32) == 2 * 4 * codes + (3 * 128 + 2) * 4 + 128 * 4 == 133128
     assert bench.launch_bytes(wl, [8] * 32) == 256 * 32 * 35848 == 293666816
+
+
+def test_reference_arm_runs_the_oracle_without_the_gpu_library():
+    """The CPU arm times the oracle on all host cores and never loads liblores.so."""
+    import subprocess
+    code = (
+        "import sys, json, runpy, io, contextlib\n"
+        "sys.argv = ['bench.py', '--impl', 'reference', '--steps', '2', '--warmup', '1']\n"
+        "buf = io.StringIO()\n"
+        "with contextlib.redirect_stdout(buf):\n"
+        "    runpy.run_path('bench.py', run_name='__main__')\n"
+        "line = json.loads(buf.getvalue().strip().splitlines()[-1])\n"
+        "print(json.dumps({'line': line, 'loaded': 'bit_recurrent_state_lores_b200.lores' in sys.modules}))\n")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                         timeout=600, check=True).stdout
+    res = json.loads(out.strip().splitlines()[-1])
+    assert res["loaded"] is False
+    line = res["line"]
+    assert line["impl"] == "reference" and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["affinity_cores"] >= 1
+    assert cb["cpu_model"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
