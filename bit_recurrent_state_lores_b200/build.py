@@ -2,10 +2,10 @@
 
     python -m bit_recurrent_state_lores_b200.build [--verbose]
 
-csrc/lores.cu (host side, loader, dequantizer) and 35 compilations of csrc/lores_inst.cu
+csrc/lores.cu (host side, loader, dequantizer) and 40 compilations of csrc/lores_inst.cu
 (one decode-step kernel family per key width x single/multi-token x storage family --
-plain; dense and per-lane; per-lane only -- and one key-axis family per key width) build in parallel, one nvcc process per
-CPU core, then link.
+plain; dense and per-lane; per-lane only --, one two-rows-per-lane family and one key-axis
+family per key width) build in parallel, one nvcc process per CPU core, then link.
 
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
 rounding-sensitive operation is written with explicit round-to-nearest intrinsics
@@ -22,7 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 SRC = os.path.join(CSRC, "lores.cu")
 INST = os.path.join(CSRC, "lores_inst.cu")
 DEPS = [SRC, INST, os.path.join(CSRC, "lores_step.cuh"), os.path.join(CSRC, "lores_device.cuh"),
-        os.path.join(CSRC, "lores_key.cuh"), os.path.join(ROOT, "include", "lores.h")]
+        os.path.join(CSRC, "lores_key.cuh"), os.path.join(CSRC, "lores_pair.cuh"),
+        os.path.join(ROOT, "include", "lores.h")]
 LIB = os.path.join(PKG, "liblores.so")
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
@@ -39,6 +40,8 @@ def units():
             for dk in reversed(KEY_WIDTHS):
                 out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],
                             f"lores_inst_{dk}_{mt}_{ext}.o"))
+    for dk in reversed(KEY_WIDTHS):
+        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_PAIR=1"], f"lores_pair_{dk}.o"))
     for dk in KEY_WIDTHS:
         out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
     out.append((SRC, [], "lores.o"))

@@ -26,6 +26,7 @@
 #include "lores_device.cuh"
 #include "lores_step.cuh"
 #include "lores_key.cuh"
+#include "lores_pair.cuh"
 
 namespace lores {
 
@@ -203,6 +204,17 @@ static StepFn kernel_for(int dk, bool mt, int ext, bool diag, bool delta, bool s
   }
 #undef LORES_PICK
 #undef LORES_PICK_EXT
+  return nullptr;
+}
+// The two-rows-per-lane kernel (heads of one byte or one nibble per code, single token).
+static StepFn pair_kernel_for(int dk, bool diag, bool delta, bool sr, bool grow) {
+  switch (dk) {
+    case 16: return pair_kernels_16(diag, delta, sr, grow);
+    case 32: return pair_kernels_32(diag, delta, sr, grow);
+    case 64: return pair_kernels_64(diag, delta, sr, grow);
+    case 128: return pair_kernels_128(diag, delta, sr, grow);
+    case 256: return pair_kernels_256(diag, delta, sr, grow);
+  }
   return nullptr;
 }
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
@@ -495,7 +507,15 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     lane_heads |= h->store[hh] == 0;
   }
   const int ext = dense_heads ? 1 : (lane_heads ? 2 : 0);
-  StepFn fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
+  // heads that all store one byte or one nibble per code, cut into full units, take the
+  // two-rows-per-lane kernel; any other handle the general one
+  bool pair_heads = ext == 0;
+  for (int hh = 0; hh < c.heads; ++hh) pair_heads &= h->store[hh] == 8 || h->store[hh] == 4;
+  const StepFn general_fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
+  const StepFn pair_fn =
+      pair_heads ? pair_kernel_for(dk, c.decay_diag, c.delta, c.stochastic, G == dk) : nullptr;
+  StepFn fn = general_fn;
+  bool pair = false;
   int split = 1;
   auto build_units = [&](std::vector<UnitDesc> &u) {
     u.clear();
@@ -532,6 +552,10 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
       return bits_rank(x) < bits_rank(y);
     });
+    pair = pair_heads;
+    for (const UnitDesc &d : units)      // (storage 8 or 4 checked first: full_rows needs it)
+      pair = pair && (d.store == 8 || d.store == 4) && d.nrows == full_rows(dk, d.store);
+    fn = pair ? pair_fn : general_fn;
     int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
     for (const UnitDesc &d : units) {
       cmax = std::max(cmax, d.nrows * (int)d.rowb);
@@ -579,6 +603,28 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       h->sp.stage_bytes = stage;
       const long long ctas = (total + kWarps - 1) / kWarps;
       h->grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * prop.multiProcessorCount);
+      if (pair) {
+        // the table is sorted bytes first: class 0 = one byte per code, class 1 = nibbles;
+        // CTAs are split in proportion to the classes' state entries
+        int n8 = 0;
+        long long e8 = 0, e4 = 0;
+        for (const UnitDesc &d : units) {
+          if (d.store == 8) {
+            ++n8;
+            e8 += (long long)d.nrows * dk;
+          } else {
+            e4 += (long long)d.nrows * dk;
+          }
+        }
+        if (e8 > 0 && e4 > 0) h->grid = std::max(h->grid, 2);
+        long long c8 = (h->grid * e8 + (e8 + e4) / 2) / (e8 + e4);
+        if (e8 > 0 && e4 > 0) c8 = std::min<long long>(std::max<long long>(c8, 1), h->grid - 1);
+        h->sp.pair_lo[0] = 0;
+        h->sp.pair_hi[0] = n8;
+        h->sp.pair_lo[1] = n8;
+        h->sp.pair_hi[1] = (int)units.size();
+        h->sp.pair_ctas = (int)c8;
+      }
       break;
     }
     split *= 2;

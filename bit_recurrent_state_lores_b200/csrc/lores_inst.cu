@@ -5,9 +5,12 @@
 //     LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
 //     LORES_EXT = 2: with the per-lane path only
 //   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
+//   -DLORES_DK=<d_k> -DLORES_PAIR=1: the two-rows-per-lane step kernels (heads of one byte
+//     or one nibble per code, single-token steps)
 // The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
 #include "lores_key.cuh"
+#include "lores_pair.cuh"
 
 #define LORES_CAT2(a, b, c, d) a##_##b##_##c##_##d
 #define LORES_CAT(a, b, c, d) LORES_CAT2(a, b, c, d)
@@ -16,7 +19,16 @@
 
 namespace lores {
 
-#if defined(LORES_KEY)
+#if defined(LORES_PAIR)
+#if !defined(LORES_DK)
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_PAIR=1"
+#endif
+StepFn LORES_CAT1(pair_kernels, LORES_DK)(bool diag, bool delta, bool sr, bool grow) {
+  if (grow)
+    return sr ? pick_pair<LORES_DK, true, true>(diag, delta) : pick_pair<LORES_DK, false, true>(diag, delta);
+  return sr ? pick_pair<LORES_DK, true, false>(diag, delta) : pick_pair<LORES_DK, false, false>(diag, delta);
+}
+#elif defined(LORES_KEY)
 #if !defined(LORES_DK)
 #error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_KEY=1"
 #endif

@@ -69,6 +69,11 @@ struct StepParams {
   uint64_t seed, step0;
   // single steps replayed from a captured CUDA graph read the step from device memory
   const uint64_t *step_dev;
+  // two-rows-per-lane kernel (lores_pair.cuh): per-sequence table ranges of the heads
+  // stored one byte per code [pair_lo[0], pair_hi[0]) and one nibble per code
+  // [pair_lo[1], pair_hi[1]); CTAs [0, pair_ctas) take the first
+  int pair_lo[2], pair_hi[2];
+  int pair_ctas;
 };
 
 // Step key of the dither: SplitMix64 (Steele, Lea & Flood 2014; Vigna's constants) of the
