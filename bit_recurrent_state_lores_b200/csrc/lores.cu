@@ -284,6 +284,7 @@ struct lores_handle {
   StepParams sp{};
   StepFn step_fn = nullptr;
   StepFn mt_fn = nullptr;                // multi-token kernel of the same configuration
+  bool pair = false;                     // step_fn is the two-rows-per-lane kernel
   // key-axis grouping
   int axis = 0;
   KeyParams kp{};
@@ -631,6 +632,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   }
   h->units_per_seq = (int)units.size();
   h->step_fn = fn;
+  h->pair = pair;
   h->mt_fn = kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
   {
     cudaFuncAttributes fa;
@@ -737,6 +739,9 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   p.codes = h->codes;
   p.scales = h->scales;
   p.flag = h->flag;
+  p.wait_ns = kWaitNs;
+  p.fault_b = -1;
+  p.fault_ub = -1;
   p.units = h->units;
   p.seq_bytes = h->seq_bytes;
   p.total_units = (long long)c.batch * h->units_per_seq;
@@ -761,6 +766,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   kp.diag = c.decay_diag;
   kp.stochastic = c.stochastic;
   kp.seed = c.seed;
+  kp.wait_ns = kWaitNs;
   *out = h;
   return LORES_OK;
 }
@@ -998,8 +1004,22 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
   out->smem_bytes = h->smem;
   out->codes_dev = h->codes;
   out->scales_dev = h->scales;
+  out->step_kernel = h->axis ? 2 : (h->pair ? 1 : 0);
   if (head_offsets)
     for (int hh = 0; hh < h->cfg.heads; ++hh) head_offsets[hh] = h->head_off[hh];
+  return LORES_OK;
+}
+
+lores_status lores_set_fault_injection(lores_handle *h, int32_t seq, int32_t unit,
+                                       uint32_t wait_us) {
+  if (!h || seq < -1 || seq >= h->cfg.batch) return LORES_ERR_INVALID_ARG;
+  if (seq >= 0 && (unit < 0 || unit >= h->units_per_seq)) return LORES_ERR_INVALID_ARG;
+  if (seq >= 0 && h->axis) return LORES_ERR_UNSUPPORTED;
+  const unsigned long long ns = wait_us ? (unsigned long long)wait_us * 1000ull : kWaitNs;
+  h->sp.fault_b = seq;
+  h->sp.fault_ub = seq >= 0 ? unit : -1;
+  h->sp.wait_ns = ns;
+  h->kp.wait_ns = ns;
   return LORES_OK;
 }
 
@@ -1052,6 +1072,11 @@ constexpr int kNoAllocMaxDevices = 64;
 
 std::mutex g_noalloc_mutex;
 void *g_noalloc_scratch_ptr[kNoAllocMaxDevices] = {};
+// The work-unit table is planned in host memory of the library (not on the caller's stack,
+// which may be small in a worker thread); the lock is held from planning until the
+// upload from it has returned.
+UnitDesc g_noalloc_units[kNoAllocMaxUnits];
+std::mutex g_noalloc_plan_mutex;
 
 }  // namespace
 
@@ -1106,9 +1131,12 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
       (reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(o) & 3u))
     return LORES_ERR_INVALID_ARG;
 
-  // Work units of one sequence, planned on the stack: full units of ~4 KB of state, the
-  // last unit of each head takes the remainder (the same plan as a handle at full batch).
-  UnitDesc units[kNoAllocMaxUnits];
+  // Work units of one sequence: full units of ~4 KB of state, the last unit of each head
+  // takes the remainder (the same plan as a handle at full batch).  A pageable upload has
+  // copied the table out of host memory when cudaMemcpyAsync returns, so the lock can be
+  // released after it.
+  std::lock_guard<std::mutex> plan_lock(g_noalloc_plan_mutex);
+  UnitDesc *units = g_noalloc_units;
   int nunits = 0;
   long long seq_bytes = 0;
   int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
@@ -1195,6 +1223,9 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   p.G = G;
   p.units_per_seq = nunits;
   p.T = 1;
+  p.wait_ns = kWaitNs;
+  p.fault_b = -1;
+  p.fault_ub = -1;
   p.step_key = step_key_of(c.seed, step);
   const long long ctas = (p.total_units + kWarps - 1) / kWarps;
   const int grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * sms);

@@ -29,8 +29,11 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;
 
-// Bounded waits: every spin on an mbarrier gives up after this many polls.
+// Bounded waits: a wait on an mbarrier gives up after the launch's limit in nanoseconds of
+// GPU time (%globaltimer; kWaitNs unless a test sets a shorter one), and after kMaxPolls
+// polls in any case.
 constexpr unsigned kMaxPolls = 1u << 24;
+constexpr unsigned long long kWaitNs = 1000000000ull;   // one second
 
 // -------------------------------------------------------------------------------------
 // random bits (MurmurHash3 32-bit finalizer, Appleby)
@@ -93,10 +96,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait; returns false if the phase did not complete within kMaxPolls polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
-  for (unsigned n = 0; n < kMaxPolls; ++n)
-    if (mbar_try_wait(bar, parity)) return true;
+// GPU time in nanoseconds.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait; returns false if the phase did not complete within limit_ns nanoseconds
+// (the clock is read every 32 polls) or kMaxPolls polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity,
+                                                  unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (unsigned n = 0; n < kMaxPolls; n += 32) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
   return false;
 }
 // global -> shared bulk copy completing on `bar`; dst, src 16-byte aligned, bytes % 16 == 0.

@@ -37,6 +37,7 @@ struct KeyParams {
   uint64_t seed;
   const uint64_t *step_dev;     // step in device memory (CUDA-graph replay), or null
   int delta, diag, stochastic;
+  unsigned long long wait_ns;   // bounded waits give up after this much GPU time
   // shared memory: stage s starts at stage0 + s * stage_bytes and holds the tile's codes,
   // scales, k, q, alpha, v at the sm_* offsets inside it; opart, ow, cm are absolute
   int stage0, stage_bytes, nstage;
@@ -315,14 +316,14 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
 
   // the first tile's stage: every thread waits, then the CTA agrees it landed
   if (!LOAD && blockIdx.x < p.tiles) {
-    const bool ok = mbar_wait_bounded(&bars[0], 0u);
+    const bool ok = mbar_wait_bounded(&bars[0], 0u, p.wait_ns);
     if (!__syncthreads_and(ok)) {
       if (threadIdx.x == 0) {
         atomicOr(p.flag, kFlagTimeout);
         // let every copy in flight land before the CTA exits
         for (int s2 = 0; s2 < p.nstage; ++s2)
           if (blockIdx.x + (long long)s2 * gridDim.x < p.tiles)
-            (void)mbar_wait_bounded(&bars[s2], 0u);
+            (void)mbar_wait_bounded(&bars[s2], 0u, p.wait_ns);
       }
       return;
     }
@@ -358,11 +359,11 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
     }
     // Wait for the next tile's stage; the barrier also says that every thread is done
     // with this tile's stage and column maxima, so (two stages) it can be refilled.
-    const bool ok = tnext < p.tiles ? mbar_wait_bounded(&bars[snext], pnext) : true;
+    const bool ok = tnext < p.tiles ? mbar_wait_bounded(&bars[snext], pnext, p.wait_ns) : true;
     if (!__syncthreads_and(ok)) {
       if (threadIdx.x == 0) {
         atomicOr(p.flag, kFlagTimeout);
-        (void)mbar_wait_bounded(&bars[snext], pnext);   // the copy in flight lands first
+        (void)mbar_wait_bounded(&bars[snext], pnext, p.wait_ns);   // the copy in flight lands first
       }
       return;
     }

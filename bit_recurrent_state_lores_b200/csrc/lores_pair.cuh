@@ -46,10 +46,11 @@ struct PairTile {
 // unit that starts a new tile (vec), the tile's k, q and per-column alpha.  Lane 0
 // announces the byte count; lanes 0-5 issue one copy each.
 template <int DK, bool DIAG>
-__device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &d, int b, bool vec,
-                                           uint8_t *stage, uint64_t *bar) {
+__device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &d, int b, int ub,
+                                           bool vec, uint8_t *stage, uint64_t *bar) {
   const int lane = threadIdx.x & 31;
   const long long tile = (long long)b * p.H + d.head;
+  const bool withhold = b == p.fault_b && ub == p.fault_ub;   // failure-path test only
   const unsigned cbytes = (unsigned)(d.nrows * d.rowb);
   const unsigned sbytes = (unsigned)(d.nrows * p.ng * 4);
   const unsigned vbytes = (unsigned)(d.nrows * 4);
@@ -66,7 +67,7 @@ __device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &
   if (vec && lane == 3) { src = p.k + tile * DK; dst = p.st_k; bytes = kVec; }
   if (vec && lane == 4) { src = p.q + tile * DK; dst = p.st_q; bytes = kVec; }
   if (vec && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = kVec; }
-  if (bytes) bulk_g2s(stage + dst, src, bytes, bar);
+  if (bytes && !withhold) bulk_g2s(stage + dst, src, bytes, bar);
 }
 
 // 16 codes of one lane's row -> exact floats in column pairs.
@@ -319,7 +320,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
   for (int s = 0; s < kStages && s < count; ++s) {
     const UnitDesc d = tbl[fill.ub];
     const int tl = fill.b * H + d.head;
-    pair_issue<DK, DIAG>(p, d, fill.b, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
+    pair_issue<DK, DIAG>(p, d, fill.b, fill.ub, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
     ftile = tl;
     fill.next(lo, hi);
   }
@@ -347,13 +348,14 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
       beta_n = __ldg(p.beta + tn);
       if (!DIAG) alpha_n = __ldg(p.alpha + tn);
     }
-    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1));
+    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1), p.wait_ns);
     if (!__all_sync(kFull, ok)) {
       // Give up: record it, let the other slot's copy (if any) land, and leave.
       if (lane == 0) {
         atomicOr(p.flag, kFlagTimeout);
         if (n + 1 < count)
-          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
+          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1),
+                                  p.wait_ns);
       }
       __syncwarp();
       return;
@@ -396,7 +398,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
       fence_proxy_async();
       const UnitDesc dn = tbl[fill.ub];
       const int tf = fill.b * H + dn.head;
-      pair_issue<DK, DIAG>(p, dn, fill.b, tf != ftile, stage, &bars[s]);
+      pair_issue<DK, DIAG>(p, dn, fill.b, fill.ub, tf != ftile, stage, &bars[s]);
       ftile = tf;
       fill.next(lo, hi);
     }

@@ -74,6 +74,10 @@ struct StepParams {
   // [pair_lo[1], pair_hi[1]); CTAs [0, pair_ctas) take the first
   int pair_lo[2], pair_hi[2];
   int pair_ctas;
+  // bounded waits give up after wait_ns of GPU time; failure-path testing: the copies of
+  // unit fault_ub of sequence fault_b are withheld (fault_b = -1: none)
+  unsigned long long wait_ns;
+  int fault_b, fault_ub;
 };
 
 // Step key of the dither: SplitMix64 (Steele, Lea & Flood 2014; Vigna's constants) of the
@@ -124,6 +128,7 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
   const int lane = threadIdx.x & 31;
   const UnitDesc d = tbl[ub];
   const long long tile = (long long)b * p.H + d.head;
+  const bool withhold = b == p.fault_b && ub == p.fault_ub;   // failure-path test only
   const unsigned cbytes = (unsigned)(d.nrows * d.rowb);
   const unsigned sbytes = d.bits == 32 ? 0u : (unsigned)(d.nrows * p.ng * 4);
   const unsigned vbytes = (unsigned)(d.nrows * 4);
@@ -140,7 +145,7 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
   if (!MT && lane == 3) { src = p.q + tile * DK; dst = p.st_q; bytes = vec; }
   if (!MT && lane == 4) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
   if (!MT && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = vec; }
-  if (bytes) bulk_g2s(stage + dst, src, bytes, bar);
+  if (bytes && !withhold) bulk_g2s(stage + dst, src, bytes, bar);
 }
 
 // -------------------------------------------------------------------------------------
@@ -555,13 +560,14 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       beta_nx = __ldg(p.beta + tn);
       if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
     }
-    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1));
+    const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1), p.wait_ns);
     if (!__all_sync(kFull, ok)) {
       // Give up: record it, let the other slot's copy (if any) land, and leave.
       if (lane == 0) {
         atomicOr(p.flag, kFlagTimeout);
         if (nxt.ub < ups)
-          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1));
+          (void)mbar_wait_bounded(&bars[(n + 1) % kStages], (unsigned)(((n + 1) / kStages) & 1),
+                                  p.wait_ns);
       }
       __syncwarp();
       return;

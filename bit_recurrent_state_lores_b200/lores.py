@@ -41,7 +41,8 @@ class lores_layout(C.Structure):
     _fields_ = [("code_bytes", C.c_int64), ("seq_code_bytes", C.c_int64),
                 ("scale_count", C.c_int64), ("n_groups", C.c_int32),
                 ("units_per_step", C.c_int32), ("grid", C.c_int32), ("smem_bytes", C.c_int32),
-                ("codes_dev", C.c_void_p), ("scales_dev", C.c_void_p)]
+                ("codes_dev", C.c_void_p), ("scales_dev", C.c_void_p),
+                ("step_kernel", C.c_int32)]
 
 
 def _load():
@@ -67,6 +68,7 @@ def _load():
         "lores_load_codes": (I32, [P, P, P, P]),
         "lores_get_layout": (I32, [P, C.POINTER(lores_layout), P]),
         "lores_check_errors": (I32, [P, P]),
+        "lores_set_fault_injection": (I32, [P, I32, I32, C.c_uint32]),
         "lores_assign_bits_by_decay": (I32, [P, I32, F32, I32, I32, P]),
         "lores_status_string": (C.c_char_p, [I32]),
     }
@@ -226,6 +228,13 @@ def lores_check_errors(h, stream=None):
     if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT, LORES_ERR_CORRUPT):
         raise LoresError(st, "lores_check_errors")
     return st
+
+
+def lores_set_fault_injection(h, seq, unit=0, wait_us=0):
+    """Testing hook of the failure path: withhold the copies of unit `unit` of sequence
+    `seq` (-1: none) and bound every wait by `wait_us` microseconds (0: the default)."""
+    _check(_lib.lores_set_fault_injection(h, int(seq), int(unit), int(wait_us)),
+           "lores_set_fault_injection")
 
 
 def lores_assign_bits_by_decay(mean_decay, frac_high, bits_high=8, bits_low=4):

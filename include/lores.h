@@ -84,13 +84,24 @@ typedef struct {
                             /* with its own r = 2^(b_g-1)-1.  Needs head_bits = NULL and      */
                             /* scale_axis = 0; not taken by lores_decode_step_noalloc.        */
     int32_t dense_codes;    /* 0: 5- to 7-bit codes one per byte (two's complement);         */
-                            /* 1: dense, b bits per code: offset binary u = c + 2^(b-1) in    */
-                            /* bit planes per row, [4-bit plane d_k/2 B][2-bit plane d_k/4 B  */
-                            /* if b >= 6][1-bit plane d_k/8 B if b odd], padded to 8 bytes    */
-                            /* (plane bit order in the oracle and csrc/lores_device.cuh).     */
-                            /* Per-head bits only (group_bits NULL, scale_axis 0); not taken  */
-                            /* by lores_decode_step_noalloc.                                   */
+                            /* 1: dense, b bits per code (layout below).  Per-head bits only  */
+                            /* (group_bits NULL, scale_axis 0); not taken by                   */
+                            /* lores_decode_step_noalloc.                                      */
 } lores_config;
+
+/* Dense b-bit codes (dense_codes = 1, b = 5, 6, 7).  A code c is stored in offset binary,
+ * u = c + 2^(b-1) (1 .. 2^b - 1), split into bit planes laid out one after another in
+ * each row of the tile, the row padded to a multiple of 8 bytes:
+ *   4-bit plane, d_k/2 bytes: u & 15 of column j in byte j/2, the low nibble for even j;
+ *   2-bit plane, d_k/4 bytes (b >= 6): (u >> 4) & 3.  The 16-column block l (columns
+ *     16l .. 16l+15) owns bytes 4l .. 4l+3; with m = j - 16l, byte 4l + p (p = 0..3)
+ *     holds m = 8+2p in bits 0-1, m = 9+2p in bits 2-3, m = 2p in bits 4-5 and
+ *     m = 2p+1 in bits 6-7;
+ *   1-bit plane, d_k/8 bytes (b odd): bit b-1 of u.  Block l owns bytes 2l, 2l+1; byte
+ *     2l holds m = 0, 2, 4, 6 in bits 0-3 and m = 1, 3, 5, 7 in bits 4-7, byte 2l+1
+ *     likewise m = 8, 10, 12, 14 in bits 0-3 and m = 9, 11, 13, 15 in bits 4-7.
+ * (A 16-column block's fields sit so that one lane holding the block rebuilds its 16
+ * offset-binary bytes with a few shifts and masks per 4 codes.) */
 
 /* Sizes of the handle's state, for export/import buffers, and its device buffers. */
 typedef struct {
@@ -106,6 +117,9 @@ typedef struct {
     float *scales_dev;         /* by the handle, valid until lores_destroy): for zero-copy    */
                                /* readers; writes through them must stay inside code_bytes   */
                                /* and scale_count * 4 bytes                                   */
+    int32_t step_kernel;       /* single-token decode kernel: 1 two rows per lane (heads of   */
+                               /* one byte or one nibble per code, full row blocks), 0 the     */
+                               /* general one, 2 the key-axis one                              */
 } lores_layout;
 
 /* Create a handle: validate `cfg`, allocate the code pool, the scales and the
@@ -256,6 +270,22 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
  * through a pointer derived from the state), else LORES_ERR_NONFINITE if any row
  * became non-finite since the last check, else LORES_OK. */
 lores_status lores_check_errors(lores_handle *h, void *stream);
+
+/* Testing hook for the kernels' failure path (no counterpart on the pages).  Every
+ * wait of a decode kernel on its own bulk copies is bounded: it gives up after a limit of
+ * GPU time (one second by default), sets the handle's TIMEOUT flag, lets its other copy
+ * in flight land and leaves, so the call's outputs are incomplete but the GPU context
+ * stays usable.  This call makes that path run on purpose: on every later decode step of
+ * h, the bulk copies of work unit `unit` (0 .. units_per_step / batch - 1, see
+ * lores_get_layout) of sequence `seq` are announced to the unit's barrier but never
+ * issued, so the warp that owns the unit waits out the limit; and every bounded wait of
+ * the handle gives up after `wait_us` microseconds (0: the default).  Nothing is left in
+ * flight: the withheld unit has no copies.  seq = -1 withholds nothing (wait_us still
+ * sets the limit); lores_set_fault_injection(h, -1, 0, 0) restores normal operation.
+ * Errors: INVALID_ARG (NULL, seq outside -1 .. B-1, unit outside the table),
+ * UNSUPPORTED (withholding on a key-axis handle). */
+lores_status lores_set_fault_injection(lores_handle *h, int32_t seq, int32_t unit,
+                                       uint32_t wait_us);
 
 /* Decay-based mixed precision (Table 5 text): the round(frac_high * H) heads with
  * the largest mean decay (slowest to forget) get bits_high, the others bits_low;
