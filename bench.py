@@ -57,6 +57,10 @@ def parse():
                          "(batch --batch, 32 heads, 128 x 128), one JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="time every batch x state-format point of the 48-layer sweep (one GPU)")
+    ap.add_argument("--sweep-variants", default="int8,mixed,fp32",
+                    help="state formats of the sweep (comma list of int8, mixed, fp32)")
+    ap.add_argument("--sweep-batches", default="1,16,64,256,1024",
+                    help="batches of the sweep (comma list)")
     return ap.parse_args()
 
 
@@ -389,6 +393,10 @@ def run_ours(args, rank, world, local_rank):
         assert st == L.LORES_OK, L.lores_status_string(st)
 
     value = job_rate(world, wl.B, wl.H, wl.layers, K, ms)
+    kernel_label = {1: "decode_pair_kernel<128, scalar decay, delta, stochastic rounding, "
+                       "one scale per row> (two rows per lane)",
+                    0: "decode_step_kernel<128, scalar decay, delta, stochastic rounding, "
+                       "single token, plain>"}[L.lores_get_layout(layers[0][0], wl.H)[0].step_kernel]
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     avg_bytes = statistics.mean(bytes_per_launch)
     peak, peak_kind = measured_peak()
@@ -483,8 +491,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                         "kernel": "decode_step_kernel<128, scalar decay, delta, stochastic "
-                                   "rounding, single token, plain>",
+                         "kernel": kernel_label,
                          "bytes_per_launch": avg_bytes, "avg_launch_us": avg_launch_s * 1e6,
                          "frac_of_8TBps": achieved / 8000.0},
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clock_summary,
@@ -515,8 +522,8 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     peak, peak_kind = measured_peak()
     points = []
-    for variant in ("int8", "mixed", "fp32"):
-        for B in (1, 16, 64, 256, 1024):
+    for variant in args.sweep_variants.split(","):
+        for B in [int(x) for x in args.sweep_batches.split(",")]:
             a = argparse.Namespace(**vars(args))
             a.batch, a.variant = B, variant
             wl = workload(a)

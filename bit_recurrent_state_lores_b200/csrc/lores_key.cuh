@@ -46,10 +46,15 @@ struct KeyParams {
 
 using KeyFn = void (*)(const KeyParams);
 
-// Column maxima of the lane's 16 columns over the whole tile: reduce across the row groups
-// of the warp, then across warps through shared memory.
+// Scales and inverses of the tile's columns from the lanes' running maxima: reduce across
+// the row groups of each warp, then across warps through shared memory; then one thread
+// per column forms its maximum m, stores the column scale s = m fl(1/r) (0 below 2^-100 or
+// for a bad column) to gscales, raises NONFINITE for a bad column (inf, NaN or above
+// 2^100), and leaves in smcm[j] the inverse r y (y the Newton reciprocal of m), 0 for a
+// tiny column, or a NaN marker for a bad one.  Every thread of the CTA calls this together.
 template <int DK>
-__device__ __forceinline__ void column_max(float (&cm)[16], float *smcm) {
+__device__ __forceinline__ void column_inverses(float (&cm)[16], float *smcm, float r, float inv_r,
+                                                float *gscales, unsigned *flag) {
   constexpr int LPR = DK / 16;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int lir = lane % LPR, riw = lane / LPR;
@@ -61,12 +66,16 @@ __device__ __forceinline__ void column_max(float (&cm)[16], float *smcm) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) smcm[warp * DK + lir * 16 + e] = cm[e];
   __syncthreads();
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    float m = smcm[lir * 16 + e];
-    for (int w2 = 1; w2 < kWarps; ++w2) m = max_nan(m, smcm[w2 * DK + lir * 16 + e]);
-    cm[e] = m;
+  for (int j = threadIdx.x; j < DK; j += kThreads) {
+    float m = smcm[j];
+    for (int w2 = 1; w2 < kWarps; ++w2) m = max_nan(m, smcm[w2 * DK + j]);
+    const bool bad = !(m <= 0x1p100f);
+    const bool scaled = !bad && m >= 0x1p-100f;
+    gscales[j] = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+    if (bad) atomicOr(flag, kFlagNonFinite);
+    smcm[j] = bad ? __uint_as_float(0x7FC00000u) : (scaled ? __fmul_rn(r, recip_nr(m)) : 0.0f);
   }
+  __syncthreads();
 }
 
 // Bulk copies of tile t's codes, scales and vectors into one stage (one thread).
@@ -218,22 +227,24 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
   if (STORE == 32) {
     if (__any_sync(kFull, bad32) && bad32) atomicOr(p.flag, kFlagNonFinite);
   } else {
-    column_max<DK>(cm, smcm);
     const float r = (float)((1 << (bits - 1)) - 1);
     const float inv_r = __fdiv_rn(1.0f, r);
+    column_inverses<DK>(cm, smcm, r, inv_r, p.scales + tile * DK, p.flag);
     float2 inv[8];
     unsigned badcols = 0;                        // bit e: column col0 + e is bad
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const bool bad = !(cm[e] <= 0x1p100f);
-      const bool scaled = !bad && cm[e] >= 0x1p-100f;
-      const float ie = scaled ? __fmul_rn(r, recip_nr(cm[e])) : 0.0f;
-      if (e & 1) inv[e >> 1].y = ie; else inv[e >> 1].x = ie;
-      const float sc = scaled ? __fmul_rn(cm[e], inv_r) : 0.0f;
-      badcols |= (bad ? 1u : 0u) << e;
-      if (warp == 0 && riw == 0) p.scales[tile * DK + col0 + e] = sc;
+    for (int c = 0; c < 4; ++c) {
+      const float4 f = *reinterpret_cast<const float4 *>(smcm + col0 + 4 * c);
+      const float fe[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = 4 * c + u;
+        const bool bad = fe[u] != fe[u];        // the NaN marker of a bad column
+        const float ie = bad ? 0.0f : fe[u];
+        if (e & 1) inv[e >> 1].y = ie; else inv[e >> 1].x = ie;
+        badcols |= (bad ? 1u : 0u) << e;
+      }
     }
-    if (badcols && warp == 0 && riw == 0) atomicOr(p.flag, kFlagNonFinite);
     // masks that clear the codes of bad columns (bytes, or nibbles: column e of the
     // lane sits in word e/8, nibble e%8)
     uint32_t keep[4];
