@@ -307,3 +307,50 @@ def test_degenerate_inputs_match_oracle():
 def lib_ok():
     from bit_recurrent_state_lores_b200 import lores
     return lores.LORES_OK
+
+
+@pytest.mark.parametrize("name,B", [("gdn", 96), ("mamba2", 24), ("kda", 96)])
+def test_gpu_step_within_bounds_of_the_plain_definition(name, B):
+    """The GPU step against the oracle's plain-definition step (double precision, IEEE
+    division, floor of x r/m + (d + 1/2)/256), teacher-forced from the GPU's state on
+    sampled tiles over several steps: codes at +-1 on <= 1e-4 of the entries, the
+    dequantized state of entries with equal codes and the readout within rel-L2 1e-5.
+    (The bit-exact tests above compare with the evaluated step; this one ties the GPU
+    to the definition itself.)"""
+    wl = synth.workload(name, B=B)
+    hp = synth.head_params(wl)
+    bits = mixed_bits(wl, hp)
+    seed = 17
+    g = GpuRun(wl, bits, seed)
+    tiles = sample_tiles(wl, bits, 12, seed=3)
+    bi = torch.tensor([t[0] for t in tiles])
+    hi = torch.tensor([t[1] for t in tiles])
+    n_diff = n_total = 0
+    try:
+        for step in range(5):
+            codes, scales = g.export()
+            before = {t: g.tile(codes, scales, *t) for t in tiles}
+            inp = synth.step_inputs(wl, step, hp, device="cuda")
+            og = g.step(inp, step)[bi, hi].cpu().numpy()
+            codes, scales = g.export()
+            sk = O.step_key(seed, step)
+            for m, (t, (q, k, v, a, b)) in enumerate(zip(tiles, host_tile_inputs(inp, tiles))):
+                cfg = tile_cfg(wl, bits[t[1]])
+                st, sc = (x.copy() for x in before[t])
+                o, flag, _ = O.tile_step_plain(cfg, st, sc, q, k, v, a, b,
+                                               O.tile_key(sk, t[0] * wl.H + t[1]))
+                assert flag == 0
+                gs, gsc = g.tile(codes, scales, *t)
+                cg, cr = unpack_fast(cfg, gs), unpack_fast(cfg, st)
+                d = np.abs(cg - cr)
+                assert d.max() <= 1, (step, t)
+                n_diff += int((d != 0).sum())
+                n_total += d.size
+                same = d == 0
+                Sg = cg * np.repeat(gsc.astype(np.float64), cfg.group, axis=1) * same
+                Sr = cr * np.repeat(sc.astype(np.float64), cfg.group, axis=1) * same
+                assert rel_l2(Sg, Sr) <= 1e-5, (step, t)
+                assert rel_l2(og[m], o) <= 1e-5, (step, t)
+        assert n_diff <= 1e-4 * n_total, (n_diff, n_total)
+    finally:
+        g.close()
