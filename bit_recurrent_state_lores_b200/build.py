@@ -2,10 +2,11 @@
 
     python -m bit_recurrent_state_lores_b200.build [--verbose]
 
-csrc/lores.cu (host side, loader, dequantizer) and 40 compilations of csrc/lores_inst.cu
+csrc/lores.cu (host side, loader, dequantizer) and 45 compilations of csrc/lores_inst.cu
 (one decode-step kernel family per key width x single/multi-token x storage family --
-plain; dense and per-lane; per-lane only --, one two-rows-per-lane family and one key-axis
-family per key width) build in parallel, one nvcc process per CPU core, then link.
+plain; dense and per-lane; per-lane only --, one two-rows-per-lane family per key width x
+single/multi-token, and one key-axis family per key width) build in parallel, one nvcc
+process per CPU core, then link.
 
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
 rounding-sensitive operation is written with explicit round-to-nearest intrinsics
@@ -40,8 +41,10 @@ def units():
             for dk in reversed(KEY_WIDTHS):
                 out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],
                             f"lores_inst_{dk}_{mt}_{ext}.o"))
-    for dk in reversed(KEY_WIDTHS):
-        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_PAIR=1"], f"lores_pair_{dk}.o"))
+    for mt in (1, 0):
+        for dk in reversed(KEY_WIDTHS):
+            out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_PAIR=1", f"-DLORES_MT={mt}"],
+                        f"lores_pair_{dk}_{mt}.o"))
     for dk in KEY_WIDTHS:
         out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
     out.append((SRC, [], "lores.o"))

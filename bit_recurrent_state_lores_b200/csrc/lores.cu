@@ -207,14 +207,19 @@ static StepFn kernel_for(int dk, bool mt, int ext, bool diag, bool delta, bool s
   return nullptr;
 }
 // The two-rows-per-lane kernel (heads of one byte or one nibble per code, single token).
-static StepFn pair_kernel_for(int dk, bool diag, bool delta, bool sr, bool grow) {
+static StepFn pair_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr, bool grow) {
+#define LORES_PAIR_PICK(dk_)                                                      \
+  case dk_:                                                                       \
+    return mt ? pair_kernels_##dk_##_1(diag, delta, sr, grow)                     \
+              : pair_kernels_##dk_##_0(diag, delta, sr, grow);
   switch (dk) {
-    case 16: return pair_kernels_16(diag, delta, sr, grow);
-    case 32: return pair_kernels_32(diag, delta, sr, grow);
-    case 64: return pair_kernels_64(diag, delta, sr, grow);
-    case 128: return pair_kernels_128(diag, delta, sr, grow);
-    case 256: return pair_kernels_256(diag, delta, sr, grow);
+    LORES_PAIR_PICK(16)
+    LORES_PAIR_PICK(32)
+    LORES_PAIR_PICK(64)
+    LORES_PAIR_PICK(128)
+    LORES_PAIR_PICK(256)
   }
+#undef LORES_PAIR_PICK
   return nullptr;
 }
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
@@ -514,7 +519,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   for (int hh = 0; hh < c.heads; ++hh) pair_heads &= h->store[hh] == 8 || h->store[hh] == 4;
   const StepFn general_fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
   const StepFn pair_fn =
-      pair_heads ? pair_kernel_for(dk, c.decay_diag, c.delta, c.stochastic, G == dk) : nullptr;
+      pair_heads ? pair_kernel_for(dk, false, c.decay_diag, c.delta, c.stochastic, G == dk) : nullptr;
   StepFn fn = general_fn;
   bool pair = false;
   int split = 1;
@@ -633,7 +638,8 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->units_per_seq = (int)units.size();
   h->step_fn = fn;
   h->pair = pair;
-  h->mt_fn = kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
+  h->mt_fn = pair ? pair_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic, G == dk)
+                  : kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
   {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, h->mt_fn) != cudaSuccess ||

@@ -5,8 +5,8 @@
 //     LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
 //     LORES_EXT = 2: with the per-lane path only
 //   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
-//   -DLORES_DK=<d_k> -DLORES_PAIR=1: the two-rows-per-lane step kernels (heads of one byte
-//     or one nibble per code, single-token steps)
+//   -DLORES_DK=<d_k> -DLORES_PAIR=1 -DLORES_MT=<0|1>: the two-rows-per-lane step kernels
+//     (heads of one byte or one nibble per code), single- or multi-token
 // The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
 #include "lores_key.cuh"
@@ -16,6 +16,8 @@
 #define LORES_CAT(a, b, c, d) LORES_CAT2(a, b, c, d)
 #define LORES_CAT1_2(a, b) a##_##b
 #define LORES_CAT1(a, b) LORES_CAT1_2(a, b)
+#define LORES_CAT3_2(a, b, c) a##_##b##_##c
+#define LORES_CAT3(a, b, c) LORES_CAT3_2(a, b, c)
 
 namespace lores {
 
@@ -23,10 +25,16 @@ namespace lores {
 #if !defined(LORES_DK)
 #error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_PAIR=1"
 #endif
-StepFn LORES_CAT1(pair_kernels, LORES_DK)(bool diag, bool delta, bool sr, bool grow) {
+#if !defined(LORES_MT)
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_PAIR=1 -DLORES_MT=<0|1>"
+#endif
+StepFn LORES_CAT3(pair_kernels, LORES_DK, LORES_MT)(bool diag, bool delta, bool sr, bool grow) {
+  constexpr bool kMT = LORES_MT != 0;
   if (grow)
-    return sr ? pick_pair<LORES_DK, true, true>(diag, delta) : pick_pair<LORES_DK, false, true>(diag, delta);
-  return sr ? pick_pair<LORES_DK, true, false>(diag, delta) : pick_pair<LORES_DK, false, false>(diag, delta);
+    return sr ? pick_pair<LORES_DK, true, true, kMT>(diag, delta)
+              : pick_pair<LORES_DK, false, true, kMT>(diag, delta);
+  return sr ? pick_pair<LORES_DK, true, false, kMT>(diag, delta)
+            : pick_pair<LORES_DK, false, false, kMT>(diag, delta);
 }
 #elif defined(LORES_KEY)
 #if !defined(LORES_DK)

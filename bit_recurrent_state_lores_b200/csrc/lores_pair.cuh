@@ -15,8 +15,9 @@
 //    scalars (scale times decay, u and its shuffle sums, w, the reciprocal of the group
 //    maximum, the new scale) run as packed fp32x2 operations on the pair, and the two
 //    rows' dependency chains interleave.
-// Heads with fp32 state, dense bit planes or per-channel widths, multi-token calls and
-// key-axis scales stay on the kernels of lores_step.cuh and lores_key.cuh.
+// Multi-token calls (MT) keep each unit's codes and scales in its ring slot across the
+// tokens.  Heads with fp32 state, dense bit planes or per-channel widths and key-axis scales
+// stay on the kernels of lores_step.cuh and lores_key.cuh.
 #pragma once
 #include <cstdint>
 
@@ -45,15 +46,17 @@ struct PairTile {
 // Bulk copies of one unit into a ring slot: codes, scales and the v slice, and, for a
 // unit that starts a new tile (vec), the tile's k, q and per-column alpha.  Lane 0
 // announces the byte count; lanes 0-5 issue one copy each.
-template <int DK, bool DIAG>
+template <int DK, bool DIAG, bool MT>
 __device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &d, int b, int ub,
                                            bool vec, uint8_t *stage, uint64_t *bar) {
+  // multi-token calls stage codes and scales only; every token's vectors come from memory
+  vec = vec && !MT;
   const int lane = threadIdx.x & 31;
   const long long tile = (long long)b * p.H + d.head;
   const bool withhold = b == p.fault_b && ub == p.fault_ub;   // failure-path test only
   const unsigned cbytes = (unsigned)(d.nrows * d.rowb);
   const unsigned sbytes = (unsigned)(d.nrows * p.ng * 4);
-  const unsigned vbytes = (unsigned)(d.nrows * 4);
+  const unsigned vbytes = MT ? 0u : (unsigned)(d.nrows * 4);
   constexpr unsigned kVec = DK * 4;
   if (lane == 0)
     mbar_expect_tx(bar, cbytes + sbytes + vbytes + (vec ? (DIAG ? 3u : 2u) * kVec : 0u));
@@ -63,7 +66,7 @@ __device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &
   unsigned bytes = 0;
   if (lane == 0) { src = p.codes + (long long)b * p.seq_bytes + d.code_off; dst = 0; bytes = cbytes; }
   if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; }
-  if (lane == 2) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
+  if (!MT && lane == 2) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
   if (vec && lane == 3) { src = p.k + tile * DK; dst = p.st_k; bytes = kVec; }
   if (vec && lane == 4) { src = p.q + tile * DK; dst = p.st_q; bytes = kVec; }
   if (vec && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = kVec; }
@@ -79,11 +82,17 @@ __device__ __forceinline__ void pair_unpack(const uint8_t *src, float2 (&c)[8]) 
     unpack_i4_2(*reinterpret_cast<const uint2 *>(src), c);
 }
 template <int BITS>
-__device__ __forceinline__ void pair_store(uint8_t *dst, const uint32_t (&w)[4]) {
-  if (BITS == 8)
+__device__ __forceinline__ void pair_store(uint8_t *dst, const uint32_t (&w)[4], bool to_stage = false) {
+  if (to_stage) {                                 // shared memory: an ordinary store
+    if (BITS == 8)
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    else
+      *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+  } else if (BITS == 8) {
     __stcs(reinterpret_cast<uint4 *>(dst), make_uint4(w[0], w[1], w[2], w[3]));
-  else
+  } else {
     __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(w[0], w[1]));
+  }
 }
 
 // Scale and inverse of two groups at once (the rows' own groups) with largest |x| = m:
@@ -114,11 +123,14 @@ __device__ __forceinline__ void pair_scale(float2 m, float2 r, float2 inv_r, flo
 // LPR = d_k/16 lanes own a row, 16 consecutive columns each; a pass covers 2 RPW rows,
 // lane (riw, lir) taking rows 2 riw and 2 riw + 1 of the pass.  The pass count and every
 // shared- and global-memory offset inside the unit are compile-time constants from the
-// lane's base addresses.  GROW: one scale per value row (G = d_k).
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool GROW>
-__device__ __forceinline__ void pair_unit(const StepParams &p, const uint8_t *stage, int b,
+// lane's base addresses.  GROW: one scale per value row (G = d_k).  Multi-token calls (MT):
+// token tok reads its v from memory and writes o at tok * tok_o; tokens before the last
+// (to_stage) write the requantized rows and scales back into the slot, each lane the bytes
+// it read, a group's scale after the group's shuffles (so after its lanes have read it).
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool GROW, bool MT>
+__device__ __forceinline__ void pair_unit(const StepParams &p, uint8_t *stage, int b,
                                           const UnitDesc &d, const PairTile<DIAG> &t,
-                                          float *opart, float *ow) {
+                                          float *opart, float *ow, int tok, bool to_stage) {
   constexpr int LPR = DK / 16, RPW = 32 / LPR;
   constexpr int RB = DK * BITS / 8;                 // bytes of one row
   constexpr int LB = 2 * BITS;                      // bytes of one lane's 16 codes
@@ -133,12 +145,17 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, const uint8_t *st
   const int r0 = 2 * riw;                           // the lane's first row in pass 0
   const uint8_t *sc = stage + r0 * RB + lir * LB;
   const float *ssr = reinterpret_cast<const float *>(stage + p.st_scales) + r0 * ng + g;
-  const float *svr = reinterpret_cast<const float *>(stage + p.st_v) + r0;
   float *opr = opart + r0 * LPR + lir;
   float *owr = ow + r0;
   const long long tile = (long long)b * p.H + d.head;
-  uint8_t *gc = p.codes + (long long)b * p.seq_bytes + d.code_off + r0 * RB + lir * LB;
-  float *gs = p.scales + (tile * p.d_v + d.row0 + r0) * ng + g;
+  const float *svr = MT ? p.v + tok * p.tok_v + tile * p.d_v + d.row0 + r0
+                        : reinterpret_cast<const float *>(stage + p.st_v) + r0;
+  // where the requantized rows and scales go: the slot (a multi-token call's tokens before
+  // the last) or global memory
+  uint8_t *gc = to_stage ? stage + r0 * RB + lir * LB
+                         : p.codes + (long long)b * p.seq_bytes + d.code_off + r0 * RB + lir * LB;
+  float *gs = to_stage ? reinterpret_cast<float *>(stage + p.st_scales) + r0 * ng + g
+                       : p.scales + (tile * p.d_v + d.row0 + r0) * ng + g;
   const float2 r2 = dup2(d.r), inv_r2 = dup2(d.inv_r);
   // dither counter of the lane's first quad in its first row of pass 0; the second row
   // is d_k/4 quads further, the next pass 2 RPW rows further
@@ -221,8 +238,8 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, const uint8_t *st
     uint32_t wA[4], wB[4];
     quantize16<BITS, SR>(spA, dup2(inv2.x), hA, wA);
     quantize16<BITS, SR>(spB, dup2(inv2.y), hB, wB);
-    pair_store<BITS>(gc + oc, wA);
-    pair_store<BITS>(gc + oc + RB, wB);
+    pair_store<BITS>(gc + oc, wA, MT && to_stage);
+    pair_store<BITS>(gc + oc + RB, wB, MT && to_stage);
     if (scale_writer) {
       if (GROW) {
         *reinterpret_cast<float2 *>(gs + orow) = s2;
@@ -245,7 +262,7 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, const uint8_t *st
         const unsigned bal = __ballot_sync(kFull, (badmask >> (2 * n + h)) & 1u);
         if ((bal & rowmask) == 0u) continue;
         const uint32_t z[4] = {0u, 0u, 0u, 0u};
-        pair_store<BITS>(gc + n * 2 * RPW * RB + h * RB, z);
+        pair_store<BITS>(gc + n * 2 * RPW * RB + h * RB, z, MT && to_stage);
         if (scale_writer) gs[(n * 2 * RPW + h) * ng] = 0.0f;
         if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
       }
@@ -255,7 +272,7 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, const uint8_t *st
   // ---- readout: o_i = sum of the row's lane shares + w_i (k.q) -------------------------
   __syncwarp();
   constexpr int kRows = full_rows(DK, BITS);
-  float *go = p.o + tile * p.d_v + d.row0;
+  float *go = p.o + (MT ? tok * p.tok_o : 0ll) + tile * p.d_v + d.row0;
 #pragma unroll
   for (int r = lane; r < kRows; r += 32) {
     float acc = 0.0f;
@@ -291,7 +308,7 @@ struct PairPos {
 // warp gw of the W warps given to the class takes units [U gw / W, U (gw + 1) / W) in
 // (sequence, unit) order, through a 2-slot ring of bulk copies whose producer is the
 // warp itself.  Warps never wait on one another.
-template <int DK, bool DIAG, bool DELTA, bool SR, bool GROW, int BITS>
+template <int DK, bool DIAG, bool DELTA, bool SR, bool GROW, int BITS, bool MT>
 __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tbl, uint8_t *wa,
                                          int cta, int nctas, int lo, int hi) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -320,7 +337,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
   for (int s = 0; s < kStages && s < count; ++s) {
     const UnitDesc d = tbl[fill.ub];
     const int tl = fill.b * H + d.head;
-    pair_issue<DK, DIAG>(p, d, fill.b, fill.ub, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
+    pair_issue<DK, DIAG, MT>(p, d, fill.b, fill.ub, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
     ftile = tl;
     fill.next(lo, hi);
   }
@@ -330,8 +347,8 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
   int ctile = -1;                                   // tile whose vectors are in registers
   PairTile<DIAG> t;
   // beta and scalar alpha of the current unit's tile, and of the next unit's
-  float beta_c, alpha_c = 0.0f;
-  {
+  float beta_c = 0.0f, alpha_c = 0.0f;
+  if (!MT) {
     const int t0 = cur.b * H + tbl[cur.ub].head;
     beta_c = __ldg(p.beta + t0);
     if (!DIAG) alpha_c = __ldg(p.alpha + t0);
@@ -343,7 +360,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
     PairPos nx = cur;
     nx.next(lo, hi);
     float beta_n = 0.0f, alpha_n = 0.0f;
-    if (n + 1 < count) {
+    if (!MT && n + 1 < count) {
       const int tn = nx.b * H + tbl[nx.ub].head;
       beta_n = __ldg(p.beta + tn);
       if (!DIAG) alpha_n = __ldg(p.alpha + tn);
@@ -362,43 +379,78 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
     }
     const UnitDesc d = tbl[cur.ub];
     const int tl = cur.b * H + d.head;
-    if (tl != ctile) {
-      // a new tile: its vectors are in this slot
-      const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
+    if (MT) {
+      // every token of the unit in turn; the unit's rows stay in the slot in between
       const int col0 = (lane % (DK / 16)) * 16;
+      for (int tok = 0; tok < p.T; ++tok) {
+        const float *k = p.k + tok * p.tok_qk + (long long)tl * DK;
+        const float *q = p.q + tok * p.tok_qk + (long long)tl * DK;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(sk + col0 + 4 * c);
-        const float4 q4 = *reinterpret_cast<const float4 *>(sk + DK + col0 + 4 * c);   // q
-        t.kk[2 * c] = make_float2(k4.x, k4.y);
-        t.kk[2 * c + 1] = make_float2(k4.z, k4.w);
-        t.qq[2 * c] = make_float2(q4.x, q4.y);
-        t.qq[2 * c + 1] = make_float2(q4.z, q4.w);
-        if (DIAG) {
-          const float4 a4 = *reinterpret_cast<const float4 *>(sk + 2 * DK + col0 + 4 * c);
-          t.aa[2 * c] = make_float2(a4.x, a4.y);
-          t.aa[2 * c + 1] = make_float2(a4.z, a4.w);
+        for (int c = 0; c < 4; ++c) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4 *>(k + col0) + c);
+          const float4 q4 = __ldg(reinterpret_cast<const float4 *>(q + col0) + c);
+          t.kk[2 * c] = make_float2(k4.x, k4.y);
+          t.kk[2 * c + 1] = make_float2(k4.z, k4.w);
+          t.qq[2 * c] = make_float2(q4.x, q4.y);
+          t.qq[2 * c + 1] = make_float2(q4.z, q4.w);
+          if (DIAG) {
+            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(
+                                        p.alpha + tok * p.tok_a + (long long)tl * DK + col0) + c);
+            t.aa[2 * c] = make_float2(a4.x, a4.y);
+            t.aa[2 * c + 1] = make_float2(a4.z, a4.w);
+          }
         }
+        double kqd = 0.0;
+#pragma unroll
+        for (int j = lane; j < DK; j += 32) kqd = fma((double)__ldg(k + j), (double)__ldg(q + j), kqd);
+#pragma unroll
+        for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
+        t.kq = (float)kqd;
+        t.tkey = tile_key(step_key_dev(p.seed, p.step0 + (uint64_t)tok), (uint32_t)tl);
+        t.beta = __ldg(p.beta + tok * p.tok_b + tl);
+        t.alpha = DIAG ? 0.0f : __ldg(p.alpha + tok * p.tok_a + tl);
+        pair_unit<DK, DIAG, DELTA, SR, BITS, GROW, MT>(p, stage, cur.b, d, t, opart, ow, tok,
+                                                       tok + 1 < p.T);
       }
-      // k.q in double (strided columns, warp butterfly): the readout is S'q + w (k.q)
-      double kqd = 0.0;
+    } else {
+      if (tl != ctile) {
+        // a new tile: its vectors are in this slot
+        const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
+        const int col0 = (lane % (DK / 16)) * 16;
 #pragma unroll
-      for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sk[DK + j], kqd);
+        for (int c = 0; c < 4; ++c) {
+          const float4 k4 = *reinterpret_cast<const float4 *>(sk + col0 + 4 * c);
+          const float4 q4 = *reinterpret_cast<const float4 *>(sk + DK + col0 + 4 * c);   // q
+          t.kk[2 * c] = make_float2(k4.x, k4.y);
+          t.kk[2 * c + 1] = make_float2(k4.z, k4.w);
+          t.qq[2 * c] = make_float2(q4.x, q4.y);
+          t.qq[2 * c + 1] = make_float2(q4.z, q4.w);
+          if (DIAG) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(sk + 2 * DK + col0 + 4 * c);
+            t.aa[2 * c] = make_float2(a4.x, a4.y);
+            t.aa[2 * c + 1] = make_float2(a4.z, a4.w);
+          }
+        }
+        // k.q in double (strided columns, warp butterfly): the readout is S'q + w (k.q)
+        double kqd = 0.0;
 #pragma unroll
-      for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
-      t.kq = (float)kqd;
-      t.tkey = tile_key(skey, (uint32_t)tl);
-      ctile = tl;
+        for (int j = lane; j < DK; j += 32) kqd = fma((double)sk[j], (double)sk[DK + j], kqd);
+#pragma unroll
+        for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
+        t.kq = (float)kqd;
+        t.tkey = tile_key(skey, (uint32_t)tl);
+        ctile = tl;
+      }
+      t.beta = beta_c;
+      t.alpha = alpha_c;
+      pair_unit<DK, DIAG, DELTA, SR, BITS, GROW, MT>(p, stage, cur.b, d, t, opart, ow, 0, false);
     }
-    t.beta = beta_c;
-    t.alpha = alpha_c;
-    pair_unit<DK, DIAG, DELTA, SR, BITS, GROW>(p, stage, cur.b, d, t, opart, ow);
     // pair_unit ends with __syncwarp: every lane is done reading this slot
     if (n + kStages < count) {
       fence_proxy_async();
       const UnitDesc dn = tbl[fill.ub];
       const int tf = fill.b * H + dn.head;
-      pair_issue<DK, DIAG>(p, dn, fill.b, fill.ub, tf != ftile, stage, &bars[s]);
+      pair_issue<DK, DIAG, MT>(p, dn, fill.b, fill.ub, tf != ftile, stage, &bars[s]);
       ftile = tf;
       fill.next(lo, hi);
     }
@@ -412,7 +464,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
 // [pair_lo[0], pair_hi[0]) of every sequence) and one nibble per code ([pair_lo[1],
 // pair_hi[1])): CTAs [0, pair_ctas) take the first class, the others the second, so every
 // CTA runs one code path (the host splits the CTAs in proportion to the state entries).
-template <int DK, bool DIAG, bool DELTA, bool SR, bool GROW>
+template <int DK, bool DIAG, bool DELTA, bool SR, bool GROW, bool MT>
 __global__ void __launch_bounds__(kThreads, LORES_PAIR_MIN_CTAS) decode_pair_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -426,27 +478,33 @@ __global__ void __launch_bounds__(kThreads, LORES_PAIR_MIN_CTAS) decode_pair_ker
   __syncthreads();                                  // the only CTA-wide barrier
   const int cta = (int)blockIdx.x;
   if (cta < p.pair_ctas)
-    pair_run<DK, DIAG, DELTA, SR, GROW, 8>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
+    pair_run<DK, DIAG, DELTA, SR, GROW, 8, MT>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0],
+                                               p.pair_hi[0]);
   else
-    pair_run<DK, DIAG, DELTA, SR, GROW, 4>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
-                                           p.pair_lo[1], p.pair_hi[1]);
+    pair_run<DK, DIAG, DELTA, SR, GROW, 4, MT>(p, tbl, wa, cta - p.pair_ctas,
+                                               (int)gridDim.x - p.pair_ctas, p.pair_lo[1],
+                                               p.pair_hi[1]);
 }
 
-template <int DK, bool SR, bool GROW>
+template <int DK, bool SR, bool GROW, bool MT>
 StepFn pick_pair(bool diag, bool delta) {
   if (diag)
-    return delta ? decode_pair_kernel<DK, true, true, SR, GROW>
-                 : decode_pair_kernel<DK, true, false, SR, GROW>;
-  return delta ? decode_pair_kernel<DK, false, true, SR, GROW>
-               : decode_pair_kernel<DK, false, false, SR, GROW>;
+    return delta ? decode_pair_kernel<DK, true, true, SR, GROW, MT>
+                 : decode_pair_kernel<DK, true, false, SR, GROW, MT>;
+  return delta ? decode_pair_kernel<DK, false, true, SR, GROW, MT>
+               : decode_pair_kernel<DK, false, false, SR, GROW, MT>;
 }
 
-// One function per key width, each defined in its own compilation of lores_inst.cu.
-// grow: one scale per value row (G = d_k).
-StepFn pair_kernels_16(bool diag, bool delta, bool sr, bool grow);
-StepFn pair_kernels_32(bool diag, bool delta, bool sr, bool grow);
-StepFn pair_kernels_64(bool diag, bool delta, bool sr, bool grow);
-StepFn pair_kernels_128(bool diag, bool delta, bool sr, bool grow);
-StepFn pair_kernels_256(bool diag, bool delta, bool sr, bool grow);
+// One function per (key width, single / multi-token), each defined in its own compilation
+// of lores_inst.cu.  grow: one scale per value row (G = d_k).
+#define LORES_DECLARE_PAIR(dk)                                               \
+  StepFn pair_kernels_##dk##_0(bool diag, bool delta, bool sr, bool grow);  \
+  StepFn pair_kernels_##dk##_1(bool diag, bool delta, bool sr, bool grow);
+LORES_DECLARE_PAIR(16)
+LORES_DECLARE_PAIR(32)
+LORES_DECLARE_PAIR(64)
+LORES_DECLARE_PAIR(128)
+LORES_DECLARE_PAIR(256)
+#undef LORES_DECLARE_PAIR
 
 }  // namespace lores

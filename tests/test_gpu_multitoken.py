@@ -158,3 +158,17 @@ def test_gdn_shape_eight_tokens_per_call():
     a, b = run_pair(wl, [8] * 32, 8, chunks=2)
     a.close()
     b.close()
+
+
+@pytest.mark.parametrize("diag,delta,sr", [(1, 1, 1), (0, 0, 0)])
+def test_two_rows_per_lane_kernel_tokens_per_call(diag, delta, sr):
+    """Handles that step with the two-rows-per-lane kernel (byte and nibble heads in full
+    row blocks): T tokens per call equal T single-token calls bit for bit."""
+    bits = [8, 4, 8, 8, 4, 8, 4, 8]
+    wl = synth.Workload("mt-pair", B=72, H=len(bits), d_k=128, d_v=128, steps=8, delta=delta,
+                        diag=diag, group=128, decay="kda" if diag else "tau", outliers=2, seed=9)
+    a, b = run_pair(wl, bits, 4, stochastic=sr, chunks=2)
+    assert a.layout.step_kernel == 1 and b.layout.step_kernel == 1
+    assert a.check() == lib().LORES_OK
+    a.close()
+    b.close()

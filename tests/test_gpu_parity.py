@@ -354,3 +354,25 @@ def test_gpu_step_within_bounds_of_the_plain_definition(name, B):
         assert n_diff <= 1e-4 * n_total, (n_diff, n_total)
     finally:
         g.close()
+
+
+PAIR_WIDTHS = [
+    # d_k, d_v, bits, G, delta, diag, sr, B: handles large enough that every row block is
+    # full and the batch fills the GPU, so they step with the two-rows-per-lane kernel
+    (16, 512, [8, 4], 16, 1, 0, 1, 600),
+    (32, 256, [8, 4], 32, 1, 1, 1, 600),
+    (64, 128, [4, 8], 64, 0, 0, 0, 600),
+    (256, 64, [8, 4], 64, 1, 1, 1, 300),
+]
+
+
+@pytest.mark.parametrize("d_k,d_v,bits,G,delta,diag,sr,B", PAIR_WIDTHS)
+def test_two_rows_per_lane_kernel_every_key_width(d_k, d_v, bits, G, delta, diag, sr, B):
+    wl = synth.Workload("pair-width", B=B, H=len(bits), d_k=d_k, d_v=d_v, steps=4, delta=delta,
+                        diag=diag, group=G, decay="kda" if diag else "tau", outliers=2, seed=13)
+    tiles = sample_tiles(wl, bits, 8, seed=1)
+    g = run_free(wl, bits, 21, tiles, 4, stochastic=sr, exact=True)
+    try:
+        assert g.layout.step_kernel == 1
+    finally:
+        g.close()
