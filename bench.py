@@ -393,8 +393,10 @@ def run_ours(args, rank, world, local_rank):
         assert st == L.LORES_OK, L.lores_status_string(st)
 
     value = job_rate(world, wl.B, wl.H, wl.layers, K, ms)
-    kernel_label = {1: "decode_pair_kernel<128, scalar decay, delta, stochastic rounding, "
-                       "one scale per row> (two rows per lane)",
+    kernel_label = {3: "decode_mma_kernel<128, scalar decay, delta, stochastic rounding> "
+                       "(tensor-core contractions, one scale per row)",
+                    1: "decode_pair_kernel<128, scalar decay, delta, stochastic rounding, "
+                       "several scales per row> (two rows per lane)",
                     0: "decode_step_kernel<128, scalar decay, delta, stochastic rounding, "
                        "single token, plain>"}[L.lores_get_layout(layers[0][0], wl.H)[0].step_kernel]
     avg_launch_s = statistics.mean(launch_ms) / 1e3

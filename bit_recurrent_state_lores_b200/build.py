@@ -24,12 +24,14 @@ SRC = os.path.join(CSRC, "lores.cu")
 INST = os.path.join(CSRC, "lores_inst.cu")
 DEPS = [SRC, INST, os.path.join(CSRC, "lores_step.cuh"), os.path.join(CSRC, "lores_device.cuh"),
         os.path.join(CSRC, "lores_key.cuh"), os.path.join(CSRC, "lores_pair.cuh"),
+        os.path.join(CSRC, "lores_mma.cuh"),
         os.path.join(ROOT, "include", "lores.h")]
 LIB = os.path.join(PKG, "liblores.so")
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-fmad=false", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
 KEY_WIDTHS = (16, 32, 64, 128, 256)
+MMA_WIDTHS = (16, 32, 64, 128)       # key widths of the tensor-core kernel
 
 
 def units():
@@ -45,6 +47,8 @@ def units():
         for dk in reversed(KEY_WIDTHS):
             out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_PAIR=1", f"-DLORES_MT={mt}"],
                         f"lores_pair_{dk}_{mt}.o"))
+    for dk in MMA_WIDTHS:
+        out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_MMA=1"], f"lores_mma_{dk}.o"))
     for dk in KEY_WIDTHS:
         out.append((INST, [f"-DLORES_DK={dk}", "-DLORES_KEY=1"], f"lores_key_{dk}.o"))
     out.append((SRC, [], "lores.o"))

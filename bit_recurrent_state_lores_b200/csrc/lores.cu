@@ -27,6 +27,7 @@
 #include "lores_step.cuh"
 #include "lores_key.cuh"
 #include "lores_pair.cuh"
+#include "lores_mma.cuh"
 
 namespace lores {
 
@@ -206,12 +207,12 @@ static StepFn kernel_for(int dk, bool mt, int ext, bool diag, bool delta, bool s
 #undef LORES_PICK_EXT
   return nullptr;
 }
-// The two-rows-per-lane kernel (heads of one byte or one nibble per code, single token).
-static StepFn pair_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr, bool grow) {
+// The two-rows-per-lane kernel (heads of one byte or one nibble per code, several scales
+// per row).
+static StepFn pair_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr) {
 #define LORES_PAIR_PICK(dk_)                                                      \
   case dk_:                                                                       \
-    return mt ? pair_kernels_##dk_##_1(diag, delta, sr, grow)                     \
-              : pair_kernels_##dk_##_0(diag, delta, sr, grow);
+    return mt ? pair_kernels_##dk_##_1(diag, delta, sr) : pair_kernels_##dk_##_0(diag, delta, sr);
   switch (dk) {
     LORES_PAIR_PICK(16)
     LORES_PAIR_PICK(32)
@@ -220,6 +221,16 @@ static StepFn pair_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr, b
     LORES_PAIR_PICK(256)
   }
 #undef LORES_PAIR_PICK
+  return nullptr;
+}
+// The tensor-core kernel (heads of one byte or one nibble per code, one scale per row).
+static StepFn mma_kernel_for(int dk, bool diag, bool delta, bool sr) {
+  switch (dk) {
+    case 16: return mma_kernels_16(diag, delta, sr);
+    case 32: return mma_kernels_32(diag, delta, sr);
+    case 64: return mma_kernels_64(diag, delta, sr);
+    case 128: return mma_kernels_128(diag, delta, sr);
+  }
   return nullptr;
 }
 static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
@@ -290,6 +301,7 @@ struct lores_handle {
   StepFn step_fn = nullptr;
   StepFn mt_fn = nullptr;                // multi-token kernel of the same configuration
   bool pair = false;                     // step_fn is the two-rows-per-lane kernel
+  bool mma = false;                      // step_fn is the tensor-core kernel
   // key-axis grouping
   int axis = 0;
   KeyParams kp{};
@@ -513,13 +525,16 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     lane_heads |= h->store[hh] == 0;
   }
   const int ext = dense_heads ? 1 : (lane_heads ? 2 : 0);
-  // heads that all store one byte or one nibble per code, cut into full units, take the
-  // two-rows-per-lane kernel; any other handle the general one
+  // heads that all store one byte or one nibble per code take the tensor-core kernel with
+  // one scale per row (d_k up to 128), or else the two-rows-per-lane kernel when cut into
+  // full units; any other handle the general one
   bool pair_heads = ext == 0;
   for (int hh = 0; hh < c.heads; ++hh) pair_heads &= h->store[hh] == 8 || h->store[hh] == 4;
+  const bool mma = pair_heads && G == dk && dk <= 128;
   const StepFn general_fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
   const StepFn pair_fn =
-      pair_heads ? pair_kernel_for(dk, false, c.decay_diag, c.delta, c.stochastic, G == dk) : nullptr;
+      pair_heads && !mma ? pair_kernel_for(dk, false, c.decay_diag, c.delta, c.stochastic) : nullptr;
+  const StepFn mma_fn = mma ? mma_kernel_for(dk, c.decay_diag, c.delta, c.stochastic) : nullptr;
   StepFn fn = general_fn;
   bool pair = false;
   int split = 1;
@@ -558,10 +573,10 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     std::stable_sort(units.begin(), units.end(), [&](const UnitDesc &x, const UnitDesc &y) {
       return bits_rank(x) < bits_rank(y);
     });
-    pair = pair_heads;
+    pair = pair_heads && !mma;
     for (const UnitDesc &d : units)      // (storage 8 or 4 checked first: full_rows needs it)
       pair = pair && (d.store == 8 || d.store == 4) && d.nrows == full_rows(dk, d.store);
-    fn = pair ? pair_fn : general_fn;
+    fn = mma ? mma_fn : (pair ? pair_fn : general_fn);
     int cmax = 0, smax = 0, vmax = 0, maxrows = 0;
     for (const UnitDesc &d : units) {
       cmax = std::max(cmax, d.nrows * (int)d.rowb);
@@ -574,7 +589,9 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
                       (c.decay_diag ? dk * 4 : 0);
     const int opart_floats = ((maxrows * LPR + 31) / 32) * 32;     // 128-byte multiples
     const int ow_floats = ((maxrows + 31) / 32) * 32;
-    const int warp_bytes = ((64 + 4 * (opart_floats + ow_floats) + kStages * stage + 127) / 128) * 128;
+    const int plane_bytes = 16 * dk;     // digit planes (8 d_k), a tile's k and alpha (8 d_k)
+    const int warp_bytes =
+        ((64 + 4 * (opart_floats + ow_floats) + plane_bytes + kStages * stage + 127) / 128) * 128;
     const int table = (int)units.size() * (int)sizeof(UnitDesc) <= 16384
                           ? (((int)units.size() * (int)sizeof(UnitDesc) + 127) / 128) * 128 : 0;
     const int smem = table + kWarps * warp_bytes;
@@ -601,6 +618,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       h->sp.warp_bytes = warp_bytes;
       h->sp.opart_floats = opart_floats;
       h->sp.ow_floats = ow_floats;
+      h->sp.plane_bytes = plane_bytes;
       h->sp.st_scales = up16(cmax);
       h->sp.st_v = h->sp.st_scales + up16(smax);
       h->sp.st_k = h->sp.st_v + up16(vmax);
@@ -609,7 +627,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
       h->sp.stage_bytes = stage;
       const long long ctas = (total + kWarps - 1) / kWarps;
       h->grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * prop.multiProcessorCount);
-      if (pair) {
+      if (pair || mma) {
         // the table is sorted bytes first: class 0 = one byte per code, class 1 = nibbles;
         // CTAs are split in proportion to the classes' state entries
         int n8 = 0;
@@ -638,7 +656,9 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->units_per_seq = (int)units.size();
   h->step_fn = fn;
   h->pair = pair;
-  h->mt_fn = pair ? pair_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic, G == dk)
+  h->mma = mma;
+  // multi-token calls: the two-rows-per-lane kernel's form, or the general one
+  h->mt_fn = pair ? pair_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic)
                   : kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
   {
     cudaFuncAttributes fa;
@@ -1010,7 +1030,7 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
   out->smem_bytes = h->smem;
   out->codes_dev = h->codes;
   out->scales_dev = h->scales;
-  out->step_kernel = h->axis ? 2 : (h->pair ? 1 : 0);
+  out->step_kernel = h->axis ? 2 : (h->mma ? 3 : (h->pair ? 1 : 0));
   if (head_offsets)
     for (int hh = 0; hh < h->cfg.heads; ++hh) head_offsets[hh] = h->head_off[hh];
   return LORES_OK;
@@ -1188,7 +1208,9 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   const int stage = up16(cmax) + up16(smax) + up16(vmax) + 2 * dk * 4 + (c.decay_diag ? dk * 4 : 0);
   p.opart_floats = ((maxrows * LPR + 31) / 32) * 32;
   p.ow_floats = ((maxrows + 31) / 32) * 32;
-  p.warp_bytes = ((64 + 4 * (p.opart_floats + p.ow_floats) + kStages * stage + 127) / 128) * 128;
+  p.plane_bytes = 16 * dk;
+  p.warp_bytes =
+      ((64 + 4 * (p.opart_floats + p.ow_floats) + p.plane_bytes + kStages * stage + 127) / 128) * 128;
   p.table_bytes = nunits * (int)sizeof(UnitDesc) <= 16384
                       ? ((nunits * (int)sizeof(UnitDesc) + 127) / 128) * 128 : 0;
   p.st_scales = up16(cmax);

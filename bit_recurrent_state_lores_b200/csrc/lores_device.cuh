@@ -36,7 +36,8 @@ constexpr unsigned kMaxPolls = 1u << 24;
 constexpr unsigned long long kWaitNs = 1000000000ull;   // one second
 
 // -------------------------------------------------------------------------------------
-// random bits (MurmurHash3 32-bit finalizer, Appleby)
+// random bits: tile keys from the MurmurHash3 32-bit finalizer (Appleby), dither words
+// from multiply-fold rounds of a 16-column block's counter
 // -------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t fmix32(uint32_t h) {
   h ^= h >> 16;
@@ -50,6 +51,21 @@ __device__ __forceinline__ uint32_t fmix32(uint32_t h) {
 __device__ __forceinline__ uint32_t tile_key(uint32_t step_key, uint32_t tile_index) {
   return fmix32(step_key + 0x85EBCA77u * (tile_index + 1u));
 }
+
+// Multiply-fold: low and high halves of the 64-bit product, XORed (one wide multiply
+// and one XOR).
+__device__ __forceinline__ uint32_t mulfold(uint32_t a, uint32_t b) {
+  const unsigned long long p = (unsigned long long)a * b;
+  return (uint32_t)p ^ (uint32_t)(p >> 32);
+}
+// Dither of a 16-column block of a row: its counter c (tile key + golden * (4 block +
+// 1), block = row d_k/16 + column/16) is folded once; word q (columns 4q .. 4q + 3 of
+// the block, one byte each) folds that again with multiplier q.
+__device__ __forceinline__ uint32_t dither_mul(int q) {
+  return q == 0 ? 0x846CA68Bu : (q == 1 ? 0xCC9E2D51u : (q == 2 ? 0x1B873593u : 0xE6546B65u));
+}
+__device__ __forceinline__ uint32_t dither_block_key(uint32_t c) { return mulfold(c, 0x7FEB352Du); }
+__device__ __forceinline__ uint32_t dither_word(uint32_t bkey, int q) { return mulfold(bkey, dither_mul(q)); }
 
 // max(m, |x|) that propagates NaN (PTX max.NaN), so a group max is non-finite
 // exactly when some entry is.
@@ -141,43 +157,52 @@ __device__ __forceinline__ void st16_a8(uint8_t *p, uint4 w) {
 // -------------------------------------------------------------------------------------
 // code <-> float
 // -------------------------------------------------------------------------------------
-// Two fp16 halves of a word, each widened to fp32 and added to `bias` in one
-// mixed-precision add (fp16 operand, fp32 operand and result, round to nearest).
-__device__ __forceinline__ void halves_plus(uint32_t w, float bias, float &lo, float &hi) {
-  asm("{\n\t.reg .f16 l, h;\n\t"
-      "mov.b32 {l, h}, %2;\n\t"
-      "add.rn.f32.f16 %0, l, %3;\n\t"
-      "add.rn.f32.f16 %1, h, %3;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(w), "f"(bias));
+// Bytes -> exact floats: a byte b dropped into the low mantissa byte of 2^23 (bits
+// 0x4B0000bb) is the float 2^23 + b, exactly (the float spacing is 1 there); one packed
+// add of -(2^23 + offset) then gives b - offset, exactly, for two bytes at once.
+// byte_float(w, k): 2^23 + byte k of w.
+__device__ __forceinline__ float byte_float(uint32_t w, int k) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (uint32_t)k));
 }
+// (byte k of a, byte k of b) - offset as a float pair
+__device__ __forceinline__ float2 bytes_minus(uint32_t a, uint32_t b, int k, float2 off) {
+  return __fadd2_rn(make_float2(byte_float(a, k), byte_float(b, k)), off);
+}
+// (byte k, byte k + 1 of w) - offset
+__device__ __forceinline__ float2 byte_pair_minus(uint32_t w, int k, float2 off) {
+  return __fadd2_rn(make_float2(byte_float(w, k), byte_float(w, k + 1)), off);
+}
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+// -(2^23 + offset): the packed addend that turns 2^23 + b into b - offset
+__device__ __forceinline__ float2 byte_bias(int offset) { return dup2(-(8388608.0f + (float)offset)); }
 
-// 16 int8 codes (two's complement) -> exact floats.  Bias to offset binary, drop pairs
-// of bytes into the mantissas of an fp16 pair (1024 + b: fp16 spacing is 1 there), and
-// add -(1024 + 128) to each half in fp32: the result is the code, exactly.
+// 16 int8 codes (two's complement) -> exact floats: bias to offset binary (b = code +
+// 128), then b - 128.
 __device__ __forceinline__ void unpack_i8(const uint4 &cw, float (&c)[16]) {
   const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
                          cw.w ^ 0x80808080u};
+  const float2 off = byte_bias(128);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    halves_plus(__byte_perm(w[q], 0x64646464u, 0x5140u), -1152.0f, c[4 * q], c[4 * q + 1]);
-    halves_plus(__byte_perm(w[q], 0x64646464u, 0x7362u), -1152.0f, c[4 * q + 2], c[4 * q + 3]);
+    const float2 lo = byte_pair_minus(w[q], 0, off), hi = byte_pair_minus(w[q], 2, off);
+    c[4 * q] = lo.x; c[4 * q + 1] = lo.y; c[4 * q + 2] = hi.x; c[4 * q + 3] = hi.y;
   }
 }
 // 16 int4 codes (two's complement nibbles, even column low) -> exact floats: nibbles to
-// offset-binary bytes (even columns in one word, odd in another), bytes into fp16 pairs
-// (columns 2p and 2p + 2 of the same parity), add -(1024 + 8) in fp32.
+// offset-binary bytes (even columns in one word, odd in another), then b - 8.
 __device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
   const uint32_t w[2] = {cw.x, cw.y};
+  const float2 off = byte_bias(8);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint32_t ev = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // columns 0, 2, 4, 6
     const uint32_t od = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 1, 3, 5, 7
-    float *cc = c + 8 * h;
-    halves_plus(__byte_perm(ev, 0x64646464u, 0x5140u), -1032.0f, cc[0], cc[2]);
-    halves_plus(__byte_perm(ev, 0x64646464u, 0x7362u), -1032.0f, cc[4], cc[6]);
-    halves_plus(__byte_perm(od, 0x64646464u, 0x5140u), -1032.0f, cc[1], cc[3]);
-    halves_plus(__byte_perm(od, 0x64646464u, 0x7362u), -1032.0f, cc[5], cc[7]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 e = bytes_minus(ev, od, k, off);
+      c[8 * h + 2 * k] = e.x;
+      c[8 * h + 2 * k + 1] = e.y;
+    }
   }
 }
 // Paired forms: element pair e of a lane holds its columns (2e, 2e + 1), so packed
@@ -186,40 +211,34 @@ __device__ __forceinline__ void unpack_i4(const uint2 &cw, float (&c)[16]) {
 __device__ __forceinline__ void unpack_i8_2(const uint4 &cw, float2 (&c)[8]) {
   const uint32_t w[4] = {cw.x ^ 0x80808080u, cw.y ^ 0x80808080u, cw.z ^ 0x80808080u,
                          cw.w ^ 0x80808080u};
+  const float2 off = byte_bias(128);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    halves_plus(__byte_perm(w[q], 0x64646464u, 0x5140u), -1152.0f, c[2 * q].x, c[2 * q].y);
-    halves_plus(__byte_perm(w[q], 0x64646464u, 0x7362u), -1152.0f, c[2 * q + 1].x,
-                c[2 * q + 1].y);
+    c[2 * q] = byte_pair_minus(w[q], 0, off);
+    c[2 * q + 1] = byte_pair_minus(w[q], 2, off);
   }
 }
-// int4: the low (even column) and high (odd column) nibbles of a byte are interleaved
-// into neighbouring bytes first, then dropped into fp16 pairs.
+// int4: column 2k is the low nibble of byte k, column 2k + 1 its high nibble.
 __device__ __forceinline__ void unpack_i4_2(const uint2 &cw, float2 (&c)[8]) {
   const uint32_t w[2] = {cw.x, cw.y};
+  const float2 off = byte_bias(8);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const uint32_t ev = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // columns 0, 2, 4, 6
     const uint32_t od = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 1, 3, 5, 7
-    const uint32_t x0 = __byte_perm(ev, od, 0x5140u);                 // columns 0, 1, 2, 3
-    const uint32_t x1 = __byte_perm(ev, od, 0x7362u);                 // columns 4, 5, 6, 7
-    float2 *cc = c + 4 * h;
-    halves_plus(__byte_perm(x0, 0x64646464u, 0x5140u), -1032.0f, cc[0].x, cc[0].y);
-    halves_plus(__byte_perm(x0, 0x64646464u, 0x7362u), -1032.0f, cc[1].x, cc[1].y);
-    halves_plus(__byte_perm(x1, 0x64646464u, 0x5140u), -1032.0f, cc[2].x, cc[2].y);
-    halves_plus(__byte_perm(x1, 0x64646464u, 0x7362u), -1032.0f, cc[3].x, cc[3].y);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) c[4 * h + k] = bytes_minus(ev, od, k, off);
   }
 }
-__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
 // Offset-binary bytes (code + 128) of a lane's 16 columns, 4 columns per word in
 // column order -> exact floats in column pairs (the int8 path after its bias flip).
 __device__ __forceinline__ void unpack_ob_2(const uint32_t (&ob)[4], float2 (&c)[8]) {
+  const float2 off = byte_bias(128);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    halves_plus(__byte_perm(ob[q], 0x64646464u, 0x5140u), -1152.0f, c[2 * q].x, c[2 * q].y);
-    halves_plus(__byte_perm(ob[q], 0x64646464u, 0x7362u), -1152.0f, c[2 * q + 1].x,
-                c[2 * q + 1].y);
+    c[2 * q] = byte_pair_minus(ob[q], 0, off);
+    c[2 * q + 1] = byte_pair_minus(ob[q], 2, off);
   }
 }
 // 16 int4 codes -> offset-binary bytes (code + 128): nibble n -> (n ^ 8) + 120, no carry
@@ -318,8 +337,8 @@ __device__ __forceinline__ DenseLane pack_dense(const uint32_t (&t)[16]) {
   return d;
 }
 
-// 16 dense codes -> exact floats in column pairs: rebuild the offset-binary bytes, drop
-// them into fp16 pairs (1024 + u), add -(1024 + 2^(B-1)) in fp32.
+// 16 dense codes -> exact floats in column pairs: rebuild the offset-binary bytes u
+// (even columns in E, odd in O), then u - 2^(B-1).
 template <int B>
 __device__ __forceinline__ void unpack_dense(const DenseLane &d, float2 (&c)[8]) {
   uint32_t E0 = d.nib0 & 0x0F0F0F0Fu, O0 = (d.nib0 >> 4) & 0x0F0F0F0Fu;
@@ -337,13 +356,11 @@ __device__ __forceinline__ void unpack_dense(const DenseLane &d, float2 (&c)[8])
     E1 |= spread_bit4<B - 1>(d.p1 >> 8);
     O1 |= spread_bit4<B - 1>(d.p1 >> 12);
   }
-  constexpr float bias = -(1024.0f + (float)(1 << (B - 1)));
-  const uint32_t x[4] = {__byte_perm(E0, O0, 0x5140u), __byte_perm(E0, O0, 0x7362u),
-                         __byte_perm(E1, O1, 0x5140u), __byte_perm(E1, O1, 0x7362u)};
+  const float2 off = byte_bias(1 << (B - 1));
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    halves_plus(__byte_perm(x[q], 0x64646464u, 0x5140u), bias, c[2 * q].x, c[2 * q].y);
-    halves_plus(__byte_perm(x[q], 0x64646464u, 0x7362u), bias, c[2 * q + 1].x, c[2 * q + 1].y);
+  for (int k = 0; k < 4; ++k) {
+    c[k] = bytes_minus(E0, O0, k, off);        // columns 2k, 2k + 1
+    c[4 + k] = bytes_minus(E1, O1, k, off);    // columns 8 + 2k, 8 + 2k + 1
   }
 }
 
@@ -417,12 +434,123 @@ __device__ __forceinline__ float recip_nr(float m) {
 // -------------------------------------------------------------------------------------
 // requantize one lane's 16 entries of a value row
 // -------------------------------------------------------------------------------------
-// Dither words of one lane-row: four MurmurHash3 finalizer values of consecutive
-// counters; cbase = tile key + golden * (n0 + 1), n0 the quad index of the lane's first
-// column (see the dither definition).
+// Dither words of one 16-column block: cbase = tile key + golden * (n0 + 1), n0 the
+// quad index of the block's first column (a multiple of 4).
 __device__ __forceinline__ void dither_words(uint32_t cbase, uint32_t (&h)[4]) {
+  const uint32_t bk = dither_block_key(cbase);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) h[q] = fmix32(cbase + 0x9E3779B9u * (uint32_t)q);
+  for (int q = 0; q < 4; ++q) h[q] = dither_word(bk, q);
+}
+
+// -------------------------------------------------------------------------------------
+// exact projection u = S'k for integer codes with one scale per row
+// -------------------------------------------------------------------------------------
+// u_i = fl32(fl64(s_i U_i) 2^-E) with U_i = sum_j c_ij Y_j exact, Y_j = rint(alpha_j k_j
+// 2^E) (ties to even), E = 29 - floor(log2 max_j |alpha_j k_j|) so |Y_j| <= 2^30 (all
+// products zero: E = 0).  Y is kept as four balanced base-256 digits (Y = sum_i 256^i
+// d_i, d_i in [-128, 127]) in digit planes: byte j of plane i is d_i of column j.
+
+// Balanced base-256 digits of |Y| <= 2^30.
+__device__ __forceinline__ void digits4(int Y, int (&d)[4]) {
+  int r = Y;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int di = (int)(int8_t)(r & 0xFF);
+    d[i] = di;
+    r = (r - di) >> 8;
+  }
+  d[3] = r;
+}
+// floor(log2 |x|) of a nonzero finite double (every product of two floats is normal)
+__device__ __forceinline__ int ilog2_d(double x) {
+  return (int)((__double_as_longlong(x) >> 52) & 0x7FF) - 1023;
+}
+__device__ __forceinline__ double pow2_d(int e) {   // 2^e, |e| < 1023
+  return __longlong_as_double((long long)(e + 1023) << 52);
+}
+
+// Digit planes of Y for y (k or q) under decay alpha (alpha_j, or the scalar alpha_s):
+// the whole warp; lane l forms quads l and l + 32 (columns 4 quad .. 4 quad + 3).  plane
+// points to nplanes_stride * 4 bytes per plane, plane i at plane + i * stride.  Returns
+// 2^-E, or NaN if some alpha_j y_j is not finite.
+template <int DK>
+__device__ __forceinline__ double fixed_point_planes(const float *y, const float *alpha, bool diag,
+                                                     float alpha_s, uint8_t *plane, int stride) {
+  const int lane = threadIdx.x & 31;
+  constexpr int NQ = DK / 4, QPL = (NQ + 31) / 32;
+  double pr[QPL][4];
+  int emax = -2000;
+  bool fin = true;
+#pragma unroll
+  for (int qi = 0; qi < QPL; ++qi) {
+    const int quad = lane + 32 * qi;
+    const bool in = quad < NQ;
+    const float4 y4 = in ? reinterpret_cast<const float4 *>(y)[quad] : make_float4(0, 0, 0, 0);
+    const float4 a4 = (in && diag) ? reinterpret_cast<const float4 *>(alpha)[quad]
+                                   : make_float4(alpha_s, alpha_s, alpha_s, alpha_s);
+    pr[qi][0] = (double)a4.x * (double)y4.x;
+    pr[qi][1] = (double)a4.y * (double)y4.y;
+    pr[qi][2] = (double)a4.z * (double)y4.z;
+    pr[qi][3] = (double)a4.w * (double)y4.w;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const double v = pr[qi][c];
+      fin = fin && isfinite(v);
+      if (v != 0.0 && isfinite(v)) emax = max(emax, ilog2_d(v));
+    }
+  }
+#pragma unroll
+  for (int st = 16; st >= 1; st >>= 1) emax = max(emax, __shfl_xor_sync(kFull, emax, st));
+  fin = __all_sync(kFull, fin);
+  const int E = emax == -2000 ? 0 : 29 - emax;
+  const double up = pow2_d(E);
+#pragma unroll
+  for (int qi = 0; qi < QPL; ++qi) {
+    const int quad = lane + 32 * qi;
+    if (quad < NQ) {
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        int dg[4];
+        digits4(fin ? __double2int_rn(pr[qi][c] * up) : 0, dg);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] |= ((uint32_t)dg[i] & 0xFFu) << (8 * c);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(plane + i * stride + 4 * quad) = w[i];
+    }
+  }
+  return fin ? pow2_d(-E) : __longlong_as_double(0x7FF8000000000000ll);
+}
+
+// sum_j c_j Y_j over 16 columns: c as 16 signed bytes (4 words, column order), Y from
+// the four digit planes at the same 16 columns; exact.
+__device__ __forceinline__ long long exact_dot16(const uint32_t (&c)[4], const uint8_t *plane,
+                                                 int stride) {
+  long long U = 0;
+#pragma unroll
+  for (int i = 3; i >= 0; --i) {
+    const uint4 dw = *reinterpret_cast<const uint4 *>(plane + i * stride);
+    int P = __dp4a((int)c[0], (int)dw.x, 0);
+    P = __dp4a((int)c[1], (int)dw.y, P);
+    P = __dp4a((int)c[2], (int)dw.z, P);
+    P = __dp4a((int)c[3], (int)dw.w, P);
+    U = U * 256 + (long long)P;
+  }
+  return U;
+}
+// 16 int4 codes (nibbles, even column low) -> 16 signed bytes in column order
+__device__ __forceinline__ void i4_to_s8(const uint2 &cw, uint32_t (&c)[4]) {
+  const uint32_t w[2] = {cw.x, cw.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t ev = (w[h] & 0x0F0F0F0Fu) ^ 0x08080808u;          // code + 8, even columns
+    const uint32_t od = ((w[h] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // odd columns
+    // (b + 0x78) ^ 0x80 maps b = code + 8 in 0..15 to the code as a signed byte, with no
+    // carry between bytes (b + 0x78 <= 0x87)
+    c[2 * h] = (__byte_perm(ev, od, 0x5140u) + 0x78787878u) ^ 0x80808080u;
+    c[2 * h + 1] = (__byte_perm(ev, od, 0x7362u) + 0x78787878u) ^ 0x80808080u;
+  }
 }
 
 // Largest |x| over one lane's 16 entries (NaN if any entry is NaN).
@@ -565,8 +693,7 @@ __device__ __forceinline__ bool requantize16(const float (&x)[16], int bits, int
   uint32_t t[16];
   if (stochastic) {
     uint32_t h[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) h[q] = fmix32(tkey + 0x9E3779B9u * (n0 + q + 1u));
+    dither_words(tkey + 0x9E3779B9u * (n0 + 1u), h);
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float g = __uint_as_float(__byte_perm(h[e >> 2], kbase, 0x7650u | (e & 3)));

@@ -6,11 +6,15 @@
 //     LORES_EXT = 2: with the per-lane path only
 //   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
 //   -DLORES_DK=<d_k> -DLORES_PAIR=1 -DLORES_MT=<0|1>: the two-rows-per-lane step kernels
-//     (heads of one byte or one nibble per code), single- or multi-token
+//     (heads of one byte or one nibble per code, several scales per row), single- or
+//     multi-token
+//   -DLORES_DK=<d_k> -DLORES_MMA=1: the tensor-core step kernels (heads of one byte or one
+//     nibble per code, one scale per row)
 // The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
 #include "lores_key.cuh"
 #include "lores_pair.cuh"
+#include "lores_mma.cuh"
 
 #define LORES_CAT2(a, b, c, d) a##_##b##_##c##_##d
 #define LORES_CAT(a, b, c, d) LORES_CAT2(a, b, c, d)
@@ -28,13 +32,17 @@ namespace lores {
 #if !defined(LORES_MT)
 #error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_PAIR=1 -DLORES_MT=<0|1>"
 #endif
-StepFn LORES_CAT3(pair_kernels, LORES_DK, LORES_MT)(bool diag, bool delta, bool sr, bool grow) {
+StepFn LORES_CAT3(pair_kernels, LORES_DK, LORES_MT)(bool diag, bool delta, bool sr) {
   constexpr bool kMT = LORES_MT != 0;
-  if (grow)
-    return sr ? pick_pair<LORES_DK, true, true, kMT>(diag, delta)
-              : pick_pair<LORES_DK, false, true, kMT>(diag, delta);
   return sr ? pick_pair<LORES_DK, true, false, kMT>(diag, delta)
             : pick_pair<LORES_DK, false, false, kMT>(diag, delta);
+}
+#elif defined(LORES_MMA)
+#if !defined(LORES_DK)
+#error "compile with -DLORES_DK=<16|32|64|128> -DLORES_MMA=1"
+#endif
+StepFn LORES_CAT1(mma_kernels, LORES_DK)(bool diag, bool delta, bool sr) {
+  return sr ? pick_mma<LORES_DK, true>(diag, delta) : pick_mma<LORES_DK, false>(diag, delta);
 }
 #elif defined(LORES_KEY)
 #if !defined(LORES_DK)

@@ -315,7 +315,7 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
   uint64_t *bars = reinterpret_cast<uint64_t *>(wa);
   float *opart = reinterpret_cast<float *>(wa + 64);
   float *ow = opart + p.opart_floats;
-  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
+  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats) + p.plane_bytes;
   const int per_seq = hi - lo;
   if (per_seq <= 0 || nctas <= 0) return;
   const long long U = (long long)p.B * per_seq;
@@ -496,10 +496,11 @@ StepFn pick_pair(bool diag, bool delta) {
 }
 
 // One function per (key width, single / multi-token), each defined in its own compilation
-// of lores_inst.cu.  grow: one scale per value row (G = d_k).
-#define LORES_DECLARE_PAIR(dk)                                               \
-  StepFn pair_kernels_##dk##_0(bool diag, bool delta, bool sr, bool grow);  \
-  StepFn pair_kernels_##dk##_1(bool diag, bool delta, bool sr, bool grow);
+// of lores_inst.cu: heads with several scales per row (heads with one scale per row take
+// the tensor-core kernel of lores_mma.cuh, or the general kernel).
+#define LORES_DECLARE_PAIR(dk)                                    \
+  StepFn pair_kernels_##dk##_0(bool diag, bool delta, bool sr);  \
+  StepFn pair_kernels_##dk##_1(bool diag, bool delta, bool sr);
 LORES_DECLARE_PAIR(16)
 LORES_DECLARE_PAIR(32)
 LORES_DECLARE_PAIR(64)

@@ -56,11 +56,13 @@ struct StepParams {
   int B, H, d_v, ng, G, units_per_seq;
   uint32_t step_key;
   // shared memory layout: [unit table][warp 0 area][warp 1 area]...; a warp area is
-  // [2 mbarriers | pad to 64][readout partials][row w][stage 0][stage 1]
+  // [2 mbarriers | pad to 64][readout partials][row w][digit planes][stage 0][stage 1]
   int table_bytes;       // bytes of the unit table copy (0: read the table from global)
   int warp_bytes;        // bytes of one warp area
   int opart_floats;      // readout partials per warp (max rows * lanes per row)
   int ow_floats;         // row w per warp (max rows)
+  int plane_bytes;       // exact contractions' scratch per warp: digit planes (8 d_k
+                         // bytes), a tile's k and alpha (8 d_k)
   int st_scales, st_k, st_q, st_v, st_a, stage_bytes;   // stage layout
   // multi-token steps: T tokens, token t reads q, k, v, alpha, beta at t * tok_* and
   // writes o at t * tok_o, with the dither of step step0 + t (keys made on the device)
@@ -240,6 +242,19 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       tkey + 0x9E3779B9u * ((uint32_t)(d.row0 + riw) * (uint32_t)(DK / 4) + (uint32_t)lir * 4u + 1u);
   constexpr uint32_t kCtrPerPass = 0x9E3779B9u * (uint32_t)(RPW * DK / 4);
   uint32_t badmask = 0;                        // bit n: this lane's group was bad in pass n
+  // exact contractions (codes one byte or one nibble each, one scale per row): S'k and
+  // S'q from the digit planes of the fixed-point alpha k and alpha q, built once per unit
+  // (per token)
+  constexpr bool kMayExact = BITS == 8 || BITS == 4;
+  const bool exact = kMayExact && (GROW || p.G == DK);
+  uint8_t *planes = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
+  double sx = 0.0, sxq = 0.0;                  // 2^-E of k and q (NaN: non-finite)
+  if (kMayExact && exact) {
+    __syncwarp();                              // the previous unit's plane reads are done
+    if (DELTA) sx = fixed_point_planes<DK>(sk, sa, DIAG, alpha_s, planes, DK);
+    sxq = fixed_point_planes<DK>(sq, sa, DIAG, alpha_s, planes + 4 * DK, DK);
+    __syncwarp();
+  }
 
 #pragma unroll(FULL ? (BITS == 0 ? 2 : 4) : 1)
   for (int n = 0; n < npass; ++n) {
@@ -253,6 +268,8 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
 
     // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
     float2 sp[8];
+    uint32_t cs[4] = {0u, 0u, 0u, 0u};         // the codes as signed bytes (exact projection)
+    float s_in = 0.0f;
     if (BITS == 32) {
       const float *srow = reinterpret_cast<const float *>(stage + (size_t)lrr * RB) + col0;
       const float2 as = dup2(alpha_s);
@@ -279,13 +296,17 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
           widen_i4_ob(*reinterpret_cast<const uint2 *>(src), ob);
         }
         unpack_ob_2(ob, cf);
-      } else if (w8)
-        unpack_i8_2(BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
-                              : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff),
-                    cf);
-      else
-        unpack_i4_2(*reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + loff), cf);
-      const float s_in = ss[lrr * ng + g];
+      } else if (w8) {
+        const uint4 cw = BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
+                                   : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff);
+        unpack_i8_2(cw, cf);
+        cs[0] = cw.x; cs[1] = cw.y; cs[2] = cw.z; cs[3] = cw.w;
+      } else {
+        const uint2 cw = *reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + loff);
+        unpack_i4_2(cw, cf);
+        if (kMayExact && exact) i4_to_s8(cw, cs);
+      }
+      s_in = ss[lrr * ng + g];
       const float2 s2 = dup2(s_in);
       const float2 a_row = dup2(__fmul_rn(s_in, alpha_s));
 #pragma unroll
@@ -295,7 +316,13 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     // ---- write: w = beta (v - delta (S'k)), x = S' + w k^T ----------------------------
     const float vr = sv[lrr];
     float w;
-    if (DELTA) {
+    if (kMayExact && exact && DELTA) {
+      long long U = exact_dot16(cs, planes + col0, DK);
+#pragma unroll
+      for (int st = 1; st < LPR; st <<= 1) U += __shfl_xor_sync(kFull, U, st);
+      const float u = (float)(((double)s_in * (double)U) * sx);
+      w = __fmul_rn(beta, __fsub_rn(vr, u));
+    } else if (DELTA) {
       float u = dot16_p(sp, kk);
 #pragma unroll
       for (int st = 1; st < LPR; st <<= 1) u = __fadd_rn(u, __shfl_xor_sync(kFull, u, st));
@@ -309,7 +336,17 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     for (int e = 0; e < 8; ++e) x[e] = __ffma2_rn(w2, kk[e], sp[e]);
 
     // ---- readout share: this lane's part of S'q ----------------------------------------
-    const float opv = dot16_p(sp, qq);
+    float opv;
+    if (kMayExact && exact) {
+      // exact: the row's S'q in its first lane's share, zero in the others
+      long long Uq = exact_dot16(cs, planes + 4 * DK + col0, DK);
+#pragma unroll
+      for (int st = 1; st < LPR; st <<= 1) Uq += __shfl_xor_sync(kFull, Uq, st);
+      const float sqr = (float)(((double)s_in * (double)Uq) * sxq);
+      opv = lir == 0 ? sqr : 0.0f;
+    } else {
+      opv = dot16_p(sp, qq);
+    }
     if (active) {
       opart[lr * LPR + lir] = opv;
       if (lir == 0) ow[lr] = w;
@@ -509,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
   uint64_t *bars = reinterpret_cast<uint64_t *>(wa);
   float *opart = reinterpret_cast<float *>(wa + 64);
   float *ow = opart + p.opart_floats;
-  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
+  uint8_t *stages = reinterpret_cast<uint8_t *>(ow + p.ow_floats) + p.plane_bytes;
 
   const UnitDesc *tbl = p.units;
   const int ups = p.units_per_seq;

@@ -117,9 +117,11 @@ typedef struct {
     float *scales_dev;         /* by the handle, valid until lores_destroy): for zero-copy    */
                                /* readers; writes through them must stay inside code_bytes   */
                                /* and scale_count * 4 bytes                                   */
-    int32_t step_kernel;       /* single-token decode kernel: 1 two rows per lane (heads of   */
-                               /* one byte or one nibble per code, full row blocks), 0 the     */
-                               /* general one, 2 the key-axis one                              */
+    int32_t step_kernel;       /* single-token decode kernel: 3 tensor-core contractions     */
+                               /* (heads of one byte or one nibble per code, one scale per     */
+                               /* row, d_k <= 128), 1 two rows per lane (such heads with       */
+                               /* several scales per row, full row blocks), 0 the general      */
+                               /* one, 2 the key-axis one                                      */
 } lores_layout;
 
 /* Create a handle: validate `cfg`, allocate the code pool, the scales and the

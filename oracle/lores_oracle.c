@@ -24,12 +24,18 @@
  *   - The readout o_t = S_t q_t uses S_t = S' + w k^T (S' = S_{t-1} diag(alpha)
  *     in fp32, w in fp32) evaluated exactly, i.e. before requantization and before
  *     the fp32 rounding of the stored entries.
- *   - Products and sums are fp32 with the association written below; the
- *     dot product S'k uses a fixed order (16-column blocks, four interleaved
- *     sequential chains per block by half and column parity, then a pairwise
- *     combine of the block sums, nearest partners first) so that two
- *     implementations that follow it agree bit for bit.  The readout is summed
- *     in double.
+ *   - Products and sums are fp32 with the association written below.  The
+ *     projection u = S'k is exact up to one rounding where the state is integer
+ *     codes with one scale per value row (codes one byte or one nibble each,
+ *     value-axis groups of G = d_k): alpha_j k_j is put on a fixed-point grid
+ *     (Y_j = rint(alpha_j k_j 2^E), |Y_j| <= 2^30), the integer sum
+ *     U_i = sum_j c_ij Y_j is exact, and u_i = fl32(fl64(s_i U_i) 2^-E).
+ *     Elsewhere (fp32 state, several scales per row, bit planes, per-channel
+ *     widths, key-axis scales) S'k uses a fixed fp32 order (16-column blocks,
+ *     four interleaved sequential chains per block by half and column parity,
+ *     then a pairwise combine of the block sums, nearest partners first) so
+ *     that two implementations that follow it agree bit for bit.  The readout
+ *     is summed in double.
  *   - Scale and its inverse: s = m * fl(1/r); inv = r * y, where y ~ 1/m comes
  *     from three Newton-Raphson steps y <- y + y(1 - m y) (fma form) started
  *     from the exponent-reflected seed bits(y0) = 0x7F000000 - bits(m).  The
@@ -42,9 +48,14 @@
  *     1.5 * 2^15, whose float spacing is exactly 1/256, so the fma rounds
  *     x*inv to the nearest 1/256 and adds d/256 exactly.  With d uniform in
  *     0..255 the code is unbiased up to that 1/512-step rounding.
- *   - The dither bytes come from SplitMix64 (Steele, Lea, Flood 2014) and the
- *     MurmurHash3 32-bit finalizer (Appleby), keyed on seed, step, sequence,
- *     head, row and column.
+ *   - The dither bytes come from a counter hash keyed on seed, step, sequence,
+ *     head, row and column: SplitMix64 (Steele, Lea, Flood 2014) and the
+ *     MurmurHash3 32-bit finalizer (Appleby) make the per-tile key; each
+ *     16-column block of a row folds its counter once, and each of its four
+ *     words folds that again with a multiplier of its own.  The
+ *     pages fix no random source; what the method needs (Proposition 3) is a
+ *     dither byte uniform on 0..255 and independent of x and of the other
+ *     entries' bytes, which the tests check statistically.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -frounding-math -fPIC -shared
  * (no fast-math; fmaf is used only where the definition says fma).
@@ -94,13 +105,43 @@ uint32_t lo_tile_key(uint32_t step_key, uint32_t tile_index)
     return lo_fmix32(step_key + 0x85EBCA77u * (tile_index + 1u));
 }
 
-/* Dither byte d in 0..255 for state element (i, j) of a tile.  Four
- * consecutive columns share one 32-bit hash; column j takes byte j mod 4. */
+/* Multiply-fold: the low and high 32-bit halves of the 64-bit product a * b,
+ * XORed. */
+uint32_t lo_mulfold(uint32_t a, uint32_t b)
+{
+    uint64_t p = (uint64_t)a * (uint64_t)b;
+    return (uint32_t)p ^ (uint32_t)(p >> 32);
+}
+
+/* Multipliers of the four words of a 16-column block. */
+static const uint32_t kDitherMul[4] = {0x846CA68Bu, 0xCC9E2D51u, 0x1B873593u, 0xE6546B65u};
+
+/* Dither word q (0..3) of the 16-column block whose counter is c: one multiply-fold of
+ * c, then one with the word's own multiplier. */
+uint32_t lo_dither_word(uint32_t c, int q)
+{
+    return lo_mulfold(lo_mulfold(c, 0x7FEB352Du), kDitherMul[q & 3]);
+}
+
+/* Dither byte d in 0..255 for state element (i, j) of a tile.  Row i is cut into
+ * 16-column blocks; block n4 = i d_k/16 + j/16 has counter c = tile_key + golden *
+ * (4 n4 + 1) (golden = 0x9E3779B9, mod 2^32), and four words, word q for columns
+ * 16 n4 + 4q .. 16 n4 + 4q + 3; column j takes byte j mod 4 of word (j mod 16) / 4. */
 uint32_t lo_dither(uint32_t tile_key, int d_k, int i, int j)
 {
-    uint32_t n = (uint32_t)i * (uint32_t)(d_k / 4) + (uint32_t)(j / 4);
-    uint32_t h = lo_fmix32(tile_key + 0x9E3779B9u * (n + 1u));
+    uint32_t n4 = (uint32_t)i * (uint32_t)(d_k / 16) + (uint32_t)(j / 16);
+    uint32_t h = lo_dither_word(tile_key + 0x9E3779B9u * (4u * n4 + 1u), (j % 16) / 4);
     return (h >> (8 * (j % 4))) & 0xFFu;
+}
+
+/* Dither words of count consecutive 4-column quads of a tile, quads n0, n0 + 1, ...
+ * (quad n = word n mod 4 of block n / 4; for statistical tests of the stream). */
+void lo_dither_words(uint32_t tile_key, uint32_t n0, int count, uint32_t *out)
+{
+    for (int k = 0; k < count; ++k) {
+        uint32_t n = n0 + (uint32_t)k;
+        out[k] = lo_dither_word(tile_key + 0x9E3779B9u * (4u * (n / 4u) + 1u), (int)(n % 4u));
+    }
 }
 
 /* ------------------------------------------------------------------------ */
@@ -306,6 +347,53 @@ float lo_recip_nr(float m)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Exact projection for rows of integer codes with one scale                */
+/* ------------------------------------------------------------------------ */
+
+/* The heads whose projection u = S'k is the exact integer contraction: codes one
+ * byte or one nibble each, one scale per value row. */
+static int exact_projection(const lo_cfg *c)
+{
+    return c->bits != 32 && !is_dense(c) && !c->group_bits && !c->axis && c->group == c->d_k;
+}
+
+/* Fixed-point copy of p_j = alpha_j y_j (exact in double): E = 29 - floor(log2 max|p|)
+ * so that max|p| 2^E lies in [2^29, 2^30), and Y_j = rint(p_j 2^E) (ties to even),
+ * |Y_j| <= 2^30.  All p zero: E = 0, Y = 0.  Returns 0 if some p_j is not finite. */
+int lo_fixed_point(const float *alpha, int diag, const float *y, int n, int32_t *Y, int *E)
+{
+    double m = 0.0;
+    for (int j = 0; j < n; j++) {
+        double p = (double)(diag ? alpha[j] : alpha[0]) * (double)y[j];
+        if (!isfinite(p))
+            return 0;
+        if (fabs(p) > m)
+            m = fabs(p);
+    }
+    int e = 0;
+    *E = 0;
+    if (m > 0.0) {
+        frexp(m, &e);          /* m = f 2^e, f in [1/2, 1): floor(log2 m) = e - 1 */
+        *E = 30 - e;
+    }
+    for (int j = 0; j < n; j++) {
+        double p = (double)(diag ? alpha[j] : alpha[0]) * (double)y[j];
+        Y[j] = (int32_t)nearbyint(ldexp(p, *E));
+    }
+    return 1;
+}
+
+/* u_i = fl32(fl64(s_i U_i) 2^-E) with U_i = sum_j c_ij Y_j, the integer sum exact. */
+float lo_exact_projection(const lo_cfg *c, const uint8_t *codes, float s, int i,
+                          const int32_t *Y, int E)
+{
+    int64_t U = 0;
+    for (int j = 0; j < c->d_k; j++)
+        U += (int64_t)get_code(c, codes, i, j) * (int64_t)Y[j];
+    return (float)ldexp((double)s * (double)U, -E);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Requantization of one value row (Proposition 1 scale, SR or RTN)         */
 /* ------------------------------------------------------------------------ */
 
@@ -413,6 +501,12 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
     float *x = malloc(sizeof(float) * dk);    /* S_t, one row                 */
     float *X = (c->axis && c->bits != 32) ? malloc(sizeof(float) * dk * (size_t)c->d_v) : NULL;
     int flag = 0;
+    /* exact projection: the fixed-point alpha k, once per tile */
+    const int exact = c->delta && exact_projection(c);
+    int32_t *Y = exact ? malloc(sizeof(int32_t) * dk) : NULL;
+    int E = 0, kfinite = 1;
+    if (exact)
+        kfinite = lo_fixed_point(alpha, c->diag, k, dk, Y, &E);
     for (int i = 0; i < c->d_v; i++) {
         /* dequantize and decay: entry (i, j) is c_ij * (s_ig * alpha_j) */
         for (int j = 0; j < dk; j++) {
@@ -426,7 +520,10 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
         }
         /* write: w_i = beta (v_i - delta u_i), u_i = (S' k)_i */
         float w;
-        if (c->delta) {
+        if (exact) {
+            float u = kfinite ? lo_exact_projection(c, (const uint8_t *)state, scales[i], i, Y, E) : NAN;
+            w = beta * (v[i] - u);
+        } else if (c->delta) {
             float u = lo_dot_b16(Sp, k, dk);
             w = beta * (v[i] - u);
         } else {
@@ -461,6 +558,7 @@ int lo_tile_step(const lo_cfg *c, void *state, float *scales,
     }
     free(Sp);
     free(x);
+    free(Y);
     return flag;
 }
 

@@ -35,10 +35,22 @@ def lib():
         L.lo_step_key.argtypes = [C.c_uint64, C.c_uint64]
         L.lo_tile_key.restype = C.c_uint32
         L.lo_tile_key.argtypes = [C.c_uint32, C.c_uint32]
+        L.lo_mulfold.restype = C.c_uint32
+        L.lo_mulfold.argtypes = [C.c_uint32, C.c_uint32]
+        L.lo_dither_word.restype = C.c_uint32
+        L.lo_dither_word.argtypes = [C.c_uint32, C.c_int]
+        L.lo_dither_words.restype = None
+        L.lo_dither_words.argtypes = [C.c_uint32, C.c_uint32, C.c_int, C.c_void_p]
         L.lo_dither.restype = C.c_uint32
         L.lo_dither.argtypes = [C.c_uint32, C.c_int, C.c_int, C.c_int]
         L.lo_dot_b16.restype = C.c_float
         L.lo_dot_b16.argtypes = [C.c_void_p, C.c_void_p, C.c_int]
+        L.lo_fixed_point.restype = C.c_int
+        L.lo_fixed_point.argtypes = [C.c_void_p, C.c_int, C.c_void_p, C.c_int, C.c_void_p,
+                                     C.POINTER(C.c_int)]
+        L.lo_exact_projection.restype = C.c_float
+        L.lo_exact_projection.argtypes = [C.POINTER(LoCfg), C.c_void_p, C.c_float, C.c_int,
+                                          C.c_void_p, C.c_int]
         L.lo_recip_nr.restype = C.c_float
         L.lo_recip_nr.argtypes = [C.c_float]
         L.lo_get_code.restype = C.c_int
@@ -144,6 +156,22 @@ def tile_key(skey, tile_index):
     return int(lib().lo_tile_key(skey, tile_index & 0xFFFFFFFF))
 
 
+def mulfold(a, b):
+    return int(lib().lo_mulfold(a & 0xFFFFFFFF, b & 0xFFFFFFFF))
+
+
+def dither_word(c, q):
+    """Word q of the 16-column block whose counter is c."""
+    return int(lib().lo_dither_word(c & 0xFFFFFFFF, int(q)))
+
+
+def dither_words(tkey, n0, count):
+    """Dither words of quads n0 .. n0 + count - 1 of a tile (uint32 array)."""
+    out = np.empty(count, np.uint32)
+    lib().lo_dither_words(tkey & 0xFFFFFFFF, n0 & 0xFFFFFFFF, count, _p(out))
+    return out
+
+
 def dither(tkey, d_k, i, j):
     return int(lib().lo_dither(tkey, d_k, i, j))
 
@@ -151,6 +179,22 @@ def dither(tkey, d_k, i, j):
 def dot_b16(a, b):
     a, b = _f32(a), _f32(b)
     return float(lib().lo_dot_b16(_p(a), _p(b), a.size))
+
+
+def fixed_point(alpha, y, diag):
+    """(ok, Y, E): the fixed-point copy Y_j = rint(alpha_j y_j 2^E) of the exact projection."""
+    a, yy = _f32(np.atleast_1d(alpha)), _f32(y)
+    Y = np.zeros(yy.size, np.int32)
+    E = C.c_int(0)
+    ok = lib().lo_fixed_point(_p(a), int(diag), _p(yy), yy.size, _p(Y), C.byref(E))
+    return bool(ok), Y, int(E.value)
+
+
+def exact_projection(cfg, codes, s, i, Y, E):
+    """u_i of the exact projection for row i of a head's codes (one scale s per row)."""
+    Y = np.ascontiguousarray(Y, np.int32)
+    return float(np.float32(lib().lo_exact_projection(C.byref(cfg.c), _p(codes), float(np.float32(s)),
+                                                      int(i), _p(Y), int(E))))
 
 
 def recip_nr(m):

@@ -25,13 +25,15 @@ def lib():
     return lores
 
 
-@pytest.mark.parametrize("bits,B,kernel", [([8, 4, 8, 4, 8, 8], 96, 1), ([8, 32, 4, 8, 8, 4], 4, 0)],
-                         ids=["two-rows-per-lane kernel", "general kernel"])
-def test_withheld_copy_times_out_and_the_next_step_is_exact(bits, B, kernel):
+@pytest.mark.parametrize("bits,B,G,kernel", [([8, 4, 8, 4, 8, 8], 96, 128, 3),
+                                             ([8, 4, 8, 4, 8, 8], 96, 32, 1),
+                                             ([8, 32, 4, 8, 8, 4], 4, 128, 0)],
+                         ids=["tensor-core kernel", "two-rows-per-lane kernel", "general kernel"])
+def test_withheld_copy_times_out_and_the_next_step_is_exact(bits, B, G, kernel):
     assert torch.cuda.is_available(), "GPU test needs a CUDA device"
     L = lib()
     wl = synth.Workload("fail", B=B, H=len(bits), d_k=128, d_v=128, steps=5, decay="tau",
-                        outliers=2, seed=21)
+                        group=G, outliers=2, seed=21)
     hp = synth.head_params(wl)
     g = GpuRun(wl, bits, seed=5)
     try:

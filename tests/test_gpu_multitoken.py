@@ -162,13 +162,28 @@ def test_gdn_shape_eight_tokens_per_call():
 
 @pytest.mark.parametrize("diag,delta,sr", [(1, 1, 1), (0, 0, 0)])
 def test_two_rows_per_lane_kernel_tokens_per_call(diag, delta, sr):
-    """Handles that step with the two-rows-per-lane kernel (byte and nibble heads in full
-    row blocks): T tokens per call equal T single-token calls bit for bit."""
+    """Handles that step with the two-rows-per-lane kernel (byte and nibble heads with
+    several scales per row, full row blocks): T tokens per call equal T single-token calls
+    bit for bit."""
     bits = [8, 4, 8, 8, 4, 8, 4, 8]
     wl = synth.Workload("mt-pair", B=72, H=len(bits), d_k=128, d_v=128, steps=8, delta=delta,
-                        diag=diag, group=128, decay="kda" if diag else "tau", outliers=2, seed=9)
+                        diag=diag, group=32, decay="kda" if diag else "tau", outliers=2, seed=9)
     a, b = run_pair(wl, bits, 4, stochastic=sr, chunks=2)
     assert a.layout.step_kernel == 1 and b.layout.step_kernel == 1
+    assert a.check() == lib().LORES_OK
+    a.close()
+    b.close()
+
+
+@pytest.mark.parametrize("diag,delta,sr", [(1, 1, 1), (0, 1, 1), (0, 0, 0)])
+def test_tensor_core_kernel_against_multi_token_calls(diag, delta, sr):
+    """Heads with one scale per row: single-token calls run the tensor-core kernel, T tokens
+    per call the general kernel's exact-projection path.  The two agree bit for bit."""
+    bits = [8, 4, 8, 8, 4, 8, 4, 8]
+    wl = synth.Workload("mt-mma", B=72, H=len(bits), d_k=128, d_v=128, steps=8, delta=delta,
+                        diag=diag, group=128, decay="kda" if diag else "tau", outliers=2, seed=19)
+    a, b = run_pair(wl, bits, 4, stochastic=sr, chunks=2)
+    assert a.layout.step_kernel == 3 and b.layout.step_kernel == 3
     assert a.check() == lib().LORES_OK
     a.close()
     b.close()

@@ -357,11 +357,12 @@ def test_gpu_step_within_bounds_of_the_plain_definition(name, B):
 
 
 PAIR_WIDTHS = [
-    # d_k, d_v, bits, G, delta, diag, sr, B: handles large enough that every row block is
-    # full and the batch fills the GPU, so they step with the two-rows-per-lane kernel
-    (16, 512, [8, 4], 16, 1, 0, 1, 600),
-    (32, 256, [8, 4], 32, 1, 1, 1, 600),
-    (64, 128, [4, 8], 64, 0, 0, 0, 600),
+    # d_k, d_v, bits, G, delta, diag, sr, B: several scales per row, handles large enough
+    # that every row block is full and the batch fills the GPU, so they step with the
+    # two-rows-per-lane kernel
+    (32, 256, [8, 4], 16, 1, 1, 1, 600),
+    (64, 128, [4, 8], 32, 0, 0, 0, 600),
+    (128, 128, [8, 4], 64, 1, 0, 1, 400),
     (256, 64, [8, 4], 64, 1, 1, 1, 300),
 ]
 
@@ -374,5 +375,28 @@ def test_two_rows_per_lane_kernel_every_key_width(d_k, d_v, bits, G, delta, diag
     g = run_free(wl, bits, 21, tiles, 4, stochastic=sr, exact=True)
     try:
         assert g.layout.step_kernel == 1
+    finally:
+        g.close()
+
+
+MMA_WIDTHS = [
+    # d_k, d_v, bits, delta, diag, sr, B: one scale per row (G = d_k), so the tensor-core
+    # kernel; d_v = 24 and 40 leave a last strip of 8 rows in every unit
+    (16, 24, [8, 4], 1, 0, 1, 40),
+    (32, 40, [4, 8], 1, 1, 1, 40),
+    (64, 64, [8, 4, 4], 0, 0, 0, 300),
+    (128, 128, [8, 4, 8], 1, 1, 1, 200),
+    (128, 96, [4, 8], 1, 0, 0, 8),
+]
+
+
+@pytest.mark.parametrize("d_k,d_v,bits,delta,diag,sr,B", MMA_WIDTHS)
+def test_tensor_core_kernel_every_key_width(d_k, d_v, bits, delta, diag, sr, B):
+    wl = synth.Workload("mma-width", B=B, H=len(bits), d_k=d_k, d_v=d_v, steps=4, delta=delta,
+                        diag=diag, group=d_k, decay="kda" if diag else "tau", outliers=2, seed=17)
+    tiles = sample_tiles(wl, bits, 8, seed=2)
+    g = run_free(wl, bits, 23, tiles, 4, stochastic=sr, exact=True)
+    try:
+        assert g.layout.step_kernel == 3
     finally:
         g.close()

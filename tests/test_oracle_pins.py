@@ -109,6 +109,69 @@ def test_dither_adjacent_columns_independent():
         assert abs(c) < 0.03, (off, c)
 
 
+def test_mulfold_is_the_folded_64_bit_product():
+    # the words of the dither stream: (low half XOR high half) of 32 x 32 -> 64-bit
+    # products, checked against Python's exact integer product
+    g = rng(4)
+    for a, b in zip(g.integers(0, 2**32, 200, dtype=np.uint64), g.integers(0, 2**32, 200, dtype=np.uint64)):
+        p = int(a) * int(b)
+        assert O.mulfold(int(a), int(b)) == (p & 0xFFFFFFFF) ^ (p >> 32)
+    mul = (0x846CA68B, 0xCC9E2D51, 0x1B873593, 0xE6546B65)
+    for c in (0, 1, 0xFFFFFFFF, 0x9E3779B9, 123456789):
+        for q in range(4):
+            assert O.dither_word(c, q) == O.mulfold(O.mulfold(c, 0x7FEB352D), mul[q])
+    # lo_dither: block n4 = (row, 16 columns) has counter tile key + golden (4 n4 + 1);
+    # column j takes byte j mod 4 of word (j mod 16) / 4 of its block
+    tk = O.tile_key(O.step_key(3, 1), 7)
+    w = O.dither_words(tk, 0, 64)
+    for i in range(2):
+        for j in range(128):
+            n4 = i * 8 + j // 16
+            c = (tk + 0x9E3779B9 * (4 * n4 + 1)) & 0xFFFFFFFF
+            want = (O.dither_word(c, (j % 16) // 4) >> (8 * (j % 4))) & 0xFF
+            assert O.dither(tk, 128, i, j) == want
+            assert (int(w[i * 32 + j // 4]) >> (8 * (j % 4))) & 0xFF == want
+
+
+def _dither_stream(tk, quads):
+    w = O.dither_words(tk, 0, quads).astype(np.uint64)
+    return np.stack([(w >> np.uint64(8 * j)) & np.uint64(255) for j in range(4)], 1).reshape(-1).astype(np.int64)
+
+
+def test_dither_stream_byte_pairs_uniform():
+    # 2^22 consecutive dither bytes of one tile (a tile's entries in row order): every
+    # pair (d_e, d_e+lag) is uniform over the 65536 cells, for lags inside a word (1-3),
+    # between the words of a 16-column block (4, 8, 12), across blocks (5, 16, 32) and
+    # to the same column of the next row (128 at d_k = 128).  A hash that dropped a
+    # fold, or kept one half of a product, fails this by orders of magnitude.
+    for key in (0x12345678, O.tile_key(O.step_key(9, 2), 5)):
+        d = _dither_stream(key, 2 ** 20)
+        for lag in (1, 2, 3, 4, 5, 8, 12, 16, 32, 128):
+            a = d[:-lag] * 256 + d[lag:]
+            cnt = np.bincount(a, minlength=65536)
+            e = len(a) / 65536
+            chi = ((cnt - e) ** 2 / e).sum() / 65535
+            # chi2 / dof has sd sqrt(2 / 65535) = 0.0055: 6 sd
+            assert abs(chi - 1.0) < 6 * 0.0055, (key, lag, chi)
+
+
+def test_dither_stream_gives_independent_rounding_errors():
+    # Proposition 3's unbiasedness and the variance of a row's rounding error: with
+    # independent uniform dither, floor(x + (d + 1/2)/256) - x has mean ~0 and the sum
+    # over 128 entries has variance sum p(1 - p) (p = frac(x) on the 1/256 grid)
+    d = _dither_stream(O.tile_key(O.step_key(1, 1), 0), 2 ** 20)
+    x = 0.3 + (np.arange(d.size) % 7) * 0.05
+    fr = x - np.floor(x)
+    code = np.floor(x + (d + 0.5) / 256.0)
+    err = code - x
+    rows = err.reshape(-1, 128).sum(1)
+    pv = (fr * (1 - fr)).reshape(-1, 128).sum(1).mean()
+    # the 1/256 grid rounds fr to the nearest 1/256 (here fr is on a 1/20 grid: bias below
+    # 1/512 per entry at most); the row-sum variance of independent Bernoulli errors is pv
+    assert abs(rows.var() / pv - 1.0) < 0.03, rows.var() / pv
+    assert abs(err.mean()) < 2.5e-3, err.mean()
+
+
 # --------------------------------------------------------------------------
 # Fixed-order dot product
 # --------------------------------------------------------------------------
@@ -181,6 +244,85 @@ def test_newton_reciprocal_error_bound():
 # --------------------------------------------------------------------------
 # The recurrence (General recurrence form), quantization off (fp32 state)
 # --------------------------------------------------------------------------
+
+# --------------------------------------------------------------------------
+# Exact projection u = S'k for integer codes with one scale per row
+# --------------------------------------------------------------------------
+
+def test_fixed_point_grid_is_exact_rounding():
+    # Y_j = alpha_j k_j 2^E rounded to the nearest integer (ties to even), with
+    # max |alpha k| 2^E in [2^29, 2^30): checked with exact rationals
+    g = rng(21)
+    for trial in range(12):
+        n = int(g.choice([16, 32, 128, 256]))
+        diag = trial % 2 == 1
+        mag = 10.0 ** g.uniform(-30, 30)
+        k = (g.standard_normal(n) * mag).astype(np.float32)
+        k[g.integers(0, n, 3)] = 0.0
+        alpha = g.uniform(0.1, 1.0, n if diag else 1).astype(np.float32)
+        ok, Y, E = O.fixed_point(alpha, k, diag)
+        assert ok
+        p = [Fraction(float(alpha[j if diag else 0])) * Fraction(float(k[j])) for j in range(n)]
+        m = max(abs(x) for x in p)
+        assert Fraction(2) ** 29 <= m * Fraction(2) ** E < Fraction(2) ** 30, (E, float(m))
+        for j in range(n):
+            assert int(Y[j]) == round(p[j] * Fraction(2) ** E), (j, int(Y[j]))
+    # a tie rounds to even: alpha k 2^E = 2^29 + 1/2 has neighbours 2^29 and 2^29 + 1
+    k = np.array([2.0 ** 29 + 0.5, 1.5, 2.5, -2.5], np.float32)
+    ok, Y, E = O.fixed_point(np.ones(1, np.float32), k, False)
+    assert ok and E == 0 and list(Y) == [2 ** 29, 2, 2, -2]
+    # all zero: E = 0 and Y = 0; a non-finite product is refused
+    ok, Y, E = O.fixed_point(np.ones(1, np.float32), np.zeros(8, np.float32), False)
+    assert ok and E == 0 and not Y.any()
+    assert not O.fixed_point(np.ones(1, np.float32), np.array([1.0, np.inf], np.float32), False)[0]
+    assert not O.fixed_point(np.array([np.nan], np.float32), np.ones(4, np.float32), False)[0]
+
+
+@pytest.mark.parametrize("bits,d_k,diag", [(8, 128, 0), (8, 32, 1), (4, 128, 1), (6, 64, 0)])
+def test_exact_projection_error_bound(bits, d_k, diag):
+    # u_i against the exact rational sum_j c_ij s_i alpha_j k_j: the only errors are the
+    # fixed-point grid (half a step per term), one double rounding and one fp32 rounding
+    g = rng(22 + bits + d_k)
+    cfg, ints, codes, scales = quantized_case(bits, d_k, d_k=d_k, d_v=8, seed=23, diag=diag)
+    k = unit(g.standard_normal(d_k)).astype(np.float32)
+    alpha = g.uniform(0.3, 1.0, d_k if diag else 1).astype(np.float32)
+    ok, Y, E = O.fixed_point(alpha, k, bool(diag))
+    assert ok
+    for i in range(cfg.d_v):
+        s = Fraction(float(scales[i, 0]))
+        u = O.exact_projection(cfg, codes, scales[i, 0], i, Y, E)
+        t = s * sum(int(ints[i, j]) * Fraction(float(alpha[j if diag else 0])) * Fraction(float(k[j]))
+                    for j in range(d_k))
+        grid = s * sum(abs(int(c)) for c in ints[i]) * Fraction(1, 2 ** (E + 1))
+        bound = grid + (abs(t) + grid) * Fraction(1, 2 ** 53) + Fraction(abs(u)) * Fraction(1, 2 ** 24) \
+            + Fraction(1, 2 ** 149)
+        assert abs(Fraction(u) - t) <= bound, (i, u, float(t))
+        # and it is the integer sum itself, rounded: U exact, then fl64, then fl32
+        U = sum(int(ints[i, j]) * int(Y[j]) for j in range(d_k))
+        assert u == float(np.float32(np.ldexp(float(scales[i, 0]) * float(U), -E)))
+
+
+def test_exact_projection_is_what_the_step_uses():
+    # one step of an int8 head with one scale per row: w_i = beta (v_i - u_i) with u the
+    # exact projection (not the fp32 block-order dot); a head with two scales per row keeps
+    # the block order
+    g = rng(24)
+    q, k, v, alpha, beta = draw(1, 128, 8, 25)
+    for group, exact in ((128, True), (64, False)):
+        cfg, ints, codes, scales = quantized_case(8, group, d_k=128, d_v=8, seed=26, diag=0)
+        _, _, x = O.tile_step(cfg, codes.copy(), scales.copy(), q[0], k[0], v[0], alpha[0], beta[0], 7,
+                              want_x=True)
+        ok, Y, E = O.fixed_point(alpha[0], k[0], False)
+        for i in range(cfg.d_v):
+            Sp = (ints[i].astype(np.float32) * np.repeat(scales[i] * alpha[0, 0], group)).astype(np.float32)
+            if exact:
+                u = np.float32(O.exact_projection(cfg, codes, scales[i, 0], i, Y, E))
+            else:
+                u = np.float32(O.dot_b16(Sp, k[0]))
+            w = np.float32(beta[0] * np.float32(v[0, i] - u))
+            xi = (Sp.astype(np.float64) + np.float64(w) * k[0]).astype(np.float32)   # fma: one rounding
+            np.testing.assert_array_equal(x[i], xi)
+
 
 def test_closed_form_no_decay_no_delta():
     # alpha = 1, delta = 0: S_T = sum_t beta_t v_t k_t^T and o_t = S_t q_t
