@@ -110,12 +110,12 @@ def launch_bytes(wl, bits):
 
 
 def kernel_source_hash():
-    """Hash of the decode-step kernels' source (csrc/lores_pair.cuh, csrc/lores_step.cuh,
-    csrc/lores_device.cuh) with comments and blank space removed, so a change of wording
-    leaves it unchanged."""
+    """Hash of the decode-step kernels' source (csrc/lores_mma.cuh, csrc/lores_pair.cuh,
+    csrc/lores_step.cuh, csrc/lores_device.cuh) with comments and blank space removed, so a
+    change of wording leaves it unchanged."""
     import re
     h = hashlib.sha256()
-    for f in ("lores_pair.cuh", "lores_step.cuh", "lores_device.cuh"):
+    for f in ("lores_mma.cuh", "lores_pair.cuh", "lores_step.cuh", "lores_device.cuh"):
         src = open(os.path.join(ROOT, "bit_recurrent_state_lores_b200", "csrc", f)).read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
         src = re.sub(r"//[^\n]*", " ", src)

@@ -38,7 +38,7 @@ def units():
     """(source, extra flags, object name) of every compilation, the slowest first (the
     extended families), so the parallel build does not end on one long unit."""
     out = []
-    for ext in (1, 2, 0):
+    for ext in (1, 4, 3, 2, 0):
         for mt in (1, 0):
             for dk in reversed(KEY_WIDTHS):
                 out.append((INST, [f"-DLORES_DK={dk}", f"-DLORES_MT={mt}", f"-DLORES_EXT={ext}"],

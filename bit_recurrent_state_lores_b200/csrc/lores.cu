@@ -184,12 +184,18 @@ using LoadFn = void (*)(const LoadParams);
 using DequantFn = void (*)(const LoadParams, float *);
 
 // The decode-step kernel of a configuration: mt = multi-token, ext = extended storage.
-// ext: 0 plain kernel, 1 with the dense and per-lane paths, 2 with the per-lane path only
+// ext: 0 plain kernel, 3 plain with the exact contractions (byte and nibble heads with one
+// scale per row), 1 with the dense and per-lane paths, 4 the same with the exact
+// contractions, 2 with the per-lane path only
 static StepFn kernel_for(int dk, bool mt, int ext, bool diag, bool delta, bool sr) {
-#define LORES_PICK_EXT(dk_, m_)                                                \
-  return ext == 2 ? step_kernels_##dk_##_##m_##_2(diag, delta, sr)             \
-                  : (ext == 1 ? step_kernels_##dk_##_##m_##_1(diag, delta, sr) \
-                              : step_kernels_##dk_##_##m_##_0(diag, delta, sr));
+#define LORES_PICK_EXT(dk_, m_)                                                       \
+  switch (ext) {                                                                      \
+    case 1: return step_kernels_##dk_##_##m_##_1(diag, delta, sr);                    \
+    case 2: return step_kernels_##dk_##_##m_##_2(diag, delta, sr);                    \
+    case 3: return step_kernels_##dk_##_##m_##_3(diag, delta, sr);                    \
+    case 4: return step_kernels_##dk_##_##m_##_4(diag, delta, sr);                    \
+    default: return step_kernels_##dk_##_##m_##_0(diag, delta, sr);                   \
+  }
 #define LORES_PICK(dk_)                                                        \
   case dk_:                                                                    \
     if (mt) {                                                                  \
@@ -233,8 +239,8 @@ static StepFn mma_kernel_for(int dk, bool diag, bool delta, bool sr) {
   }
   return nullptr;
 }
-static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr) {
-  return kernel_for(dk, false, 0, diag, delta, sr);
+static StepFn step_kernel_for(int dk, bool diag, bool delta, bool sr, bool exact) {
+  return kernel_for(dk, false, exact ? 3 : 0, diag, delta, sr);
 }
 static KeyFn key_kernel_for(int dk, bool sr, bool load) {
   switch (dk) {
@@ -524,11 +530,15 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
     dense_heads |= h->store[hh] >= 5 && h->store[hh] <= 7;
     lane_heads |= h->store[hh] == 0;
   }
-  const int ext = dense_heads ? 1 : (lane_heads ? 2 : 0);
+  // byte or nibble heads with one scale per row take the exact contractions (u and S'q
+  // as exact integer sums) wherever the general kernel serves them
+  bool exact_heads = false;
+  for (int hh = 0; hh < c.heads; ++hh) exact_heads |= G == dk && (h->store[hh] == 8 || h->store[hh] == 4);
+  const int ext = dense_heads ? (exact_heads ? 4 : 1) : (lane_heads ? 2 : (exact_heads ? 3 : 0));
   // heads that all store one byte or one nibble per code take the tensor-core kernel with
   // one scale per row (d_k up to 128), or else the two-rows-per-lane kernel when cut into
   // full units; any other handle the general one
-  bool pair_heads = ext == 0;
+  bool pair_heads = ext == 0 || ext == 3;   // no dense or per-lane heads
   for (int hh = 0; hh < c.heads; ++hh) pair_heads &= h->store[hh] == 8 || h->store[hh] == 4;
   const bool mma = pair_heads && G == dk && dk <= 128;
   const StepFn general_fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
@@ -1220,7 +1230,8 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   p.st_a = p.st_q + dk * 4;
   p.stage_bytes = stage;
   const int smem = p.table_bytes + kWarps * p.warp_bytes;
-  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic);
+  // one scale per row: the byte and nibble heads take the exact contractions
+  StepFn fn = step_kernel_for(dk, c.decay_diag, c.delta, c.stochastic, G == dk);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
       (fa.maxDynamicSharedSizeBytes < smem &&

@@ -523,6 +523,14 @@ __device__ __forceinline__ double fixed_point_planes(const float *y, const float
   return fin ? pow2_d(-E) : __longlong_as_double(0x7FF8000000000000ll);
 }
 
+// The same as a real call, for the general kernel: it runs once per unit, and its
+// registers must not add to that kernel's inner loop.
+template <int DK>
+__device__ __noinline__ double fixed_point_planes_call(const float *y, const float *alpha, bool diag,
+                                                       float alpha_s, uint8_t *plane, int stride) {
+  return fixed_point_planes<DK>(y, alpha, diag, alpha_s, plane, stride);
+}
+
 // sum_j c_j Y_j over 16 columns: c as 16 signed bytes (4 words, column order), Y from
 // the four digit planes at the same 16 columns; exact.
 __device__ __forceinline__ long long exact_dot16(const uint32_t (&c)[4], const uint8_t *plane,
@@ -538,6 +546,23 @@ __device__ __forceinline__ long long exact_dot16(const uint32_t (&c)[4], const u
     U = U * 256 + (long long)P;
   }
   return U;
+}
+// One row's exact u (if DELTA) and S'q from its lanes' 16 codes each (LPR lanes per row,
+// every lane of the warp taking part): integer sums over the lane's columns, summed over
+// the row's lanes, then fl32(fl64(s U) 2^-E).  planes: digit planes of alpha k at 0 and
+// alpha q at 4 stride, at the lane's first column.
+template <int LPR, bool DELTA>
+__device__ __forceinline__ void exact_row(const uint32_t (&c)[4], const uint8_t *planes, int stride,
+                                          float s, double sxk, double sxq, float &u, float &sq) {
+  long long Uk = DELTA ? exact_dot16(c, planes, stride) : 0ll;
+  long long Uq = exact_dot16(c, planes + 4 * stride, stride);
+#pragma unroll
+  for (int st = 1; st < LPR; st <<= 1) {
+    if (DELTA) Uk += __shfl_xor_sync(kFull, Uk, st);
+    Uq += __shfl_xor_sync(kFull, Uq, st);
+  }
+  u = DELTA ? (float)(((double)s * (double)Uk) * sxk) : 0.0f;
+  sq = (float)(((double)s * (double)Uq) * sxq);
 }
 // 16 int4 codes (nibbles, even column low) -> 16 signed bytes in column order
 __device__ __forceinline__ void i4_to_s8(const uint2 &cw, uint32_t (&c)[4]) {

@@ -4,6 +4,9 @@
 //     LORES_MT  = 1: multi-token steps (lores_decode_steps); 0: single-token steps
 //     LORES_EXT = 1: with the dense 5- to 7-bit and per-lane (per-channel) storage paths
 //     LORES_EXT = 2: with the per-lane path only
+//     LORES_EXT = 3: the plain kernel with the exact contractions (byte and nibble heads
+//                    with one scale per row)
+//     LORES_EXT = 4: the dense and per-lane paths with the exact contractions
 //   -DLORES_DK=<d_k> -DLORES_KEY=1: the key-axis step and loader kernels
 //   -DLORES_DK=<d_k> -DLORES_PAIR=1 -DLORES_MT=<0|1>: the two-rows-per-lane step kernels
 //     (heads of one byte or one nibble per code, several scales per row), single- or
@@ -57,7 +60,7 @@ KeyFn LORES_CAT1(key_kernels, LORES_DK)(bool sr, bool load) {
 }
 #else
 #if !defined(LORES_DK) || !defined(LORES_MT) || !defined(LORES_EXT)
-#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1|2>"
+#error "compile with -DLORES_DK=<16|32|64|128|256> -DLORES_MT=<0|1> -DLORES_EXT=<0|1|2|3|4>"
 #endif
 StepFn LORES_CAT(step_kernels, LORES_DK, LORES_MT, LORES_EXT)(bool diag, bool delta, bool sr) {
   return sr ? pick_step<LORES_DK, true, LORES_MT != 0, LORES_EXT>(diag, delta)

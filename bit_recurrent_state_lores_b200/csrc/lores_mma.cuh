@@ -33,17 +33,19 @@
 
 namespace lores {
 
-// D += A (16 x 32, s8) * B (32 x 8, s8), int32 accumulators
+// D += A (16 x 32, s8) * B (32 x 8, s8), int32 accumulators.  mma.sync is a warp-wide
+// instruction that the whole warp must execute converged: the asm is volatile (not moved
+// or duplicated by the compiler) and the caller issues it right after a __syncwarp.
 __device__ __forceinline__ void mma_k32(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 // D += A (16 x 16, s8) * B (16 x 8, s8)
 __device__ __forceinline__ void mma_k16(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm("mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(b0));
@@ -323,6 +325,7 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, const uint8_t *sta
     mma_load_row<DK, BITS>(stage + (v0 ? r0 : nrows - 1) * RB, tq, c0);
     mma_load_row<DK, BITS>(stage + (v1 ? r1 : nrows - 1) * RB, tq, c1);
     int acc[4] = {0, 0, 0, 0};
+    __syncwarp();                                   // the MMAs need the whole warp converged
     if (DK == 16) {
       mma_k16(acc, c0[0], c1[0], t.bf[0]);
     } else {

@@ -162,7 +162,8 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
 // the last write the requantized rows back into the stage (each lane rewrites the bytes
 // it read; a group's scale is rewritten after the group's lanes have read it), so the
 // next token dequantizes them from shared memory; the last token writes global memory.
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL, bool GROW, bool MT>
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool FULL, bool GROW, bool MT,
+          bool EXACT>
 __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow, int t) {
@@ -245,14 +246,14 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
   // exact contractions (codes one byte or one nibble each, one scale per row): S'k and
   // S'q from the digit planes of the fixed-point alpha k and alpha q, built once per unit
   // (per token)
-  constexpr bool kMayExact = BITS == 8 || BITS == 4;
+  constexpr bool kMayExact = EXACT && (BITS == 8 || BITS == 4);
   const bool exact = kMayExact && (GROW || p.G == DK);
   uint8_t *planes = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
   double sx = 0.0, sxq = 0.0;                  // 2^-E of k and q (NaN: non-finite)
   if (kMayExact && exact) {
     __syncwarp();                              // the previous unit's plane reads are done
-    if (DELTA) sx = fixed_point_planes<DK>(sk, sa, DIAG, alpha_s, planes, DK);
-    sxq = fixed_point_planes<DK>(sq, sa, DIAG, alpha_s, planes + 4 * DK, DK);
+    if (DELTA) sx = fixed_point_planes_call<DK>(sk, sa, DIAG, alpha_s, planes, DK);
+    sxq = fixed_point_planes_call<DK>(sq, sa, DIAG, alpha_s, planes + 4 * DK, DK);
     __syncwarp();
   }
 
@@ -268,7 +269,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
 
     // ---- dequantize and decay: S'_ij = c_ij * (s_ig * alpha_j) ----------------------
     float2 sp[8];
-    uint32_t cs[4] = {0u, 0u, 0u, 0u};         // the codes as signed bytes (exact projection)
+    float u_ex = 0.0f, sq_ex = 0.0f;           // exact contractions: the row's u and S'q
     float s_in = 0.0f;
     if (BITS == 32) {
       const float *srow = reinterpret_cast<const float *>(stage + (size_t)lrr * RB) + col0;
@@ -299,14 +300,25 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       } else if (w8) {
         const uint4 cw = BITS == 0 ? ld16_a8(stage + (size_t)lrr * RB + loff)   // 8-byte aligned
                                    : *reinterpret_cast<const uint4 *>(stage + (size_t)lrr * RB + loff);
+        s_in = ss[lrr * ng + g];
+        if (kMayExact && exact) {
+          // the contractions first, so their digit words and sums are dead before the
+          // floats live
+          const uint32_t cs[4] = {cw.x, cw.y, cw.z, cw.w};
+          exact_row<LPR, DELTA>(cs, planes + col0, DK, s_in, sx, sxq, u_ex, sq_ex);
+        }
         unpack_i8_2(cw, cf);
-        cs[0] = cw.x; cs[1] = cw.y; cs[2] = cw.z; cs[3] = cw.w;
       } else {
         const uint2 cw = *reinterpret_cast<const uint2 *>(stage + (size_t)lrr * RB + loff);
+        s_in = ss[lrr * ng + g];
+        if (kMayExact && exact) {
+          uint32_t cs[4];
+          i4_to_s8(cw, cs);
+          exact_row<LPR, DELTA>(cs, planes + col0, DK, s_in, sx, sxq, u_ex, sq_ex);
+        }
         unpack_i4_2(cw, cf);
-        if (kMayExact && exact) i4_to_s8(cw, cs);
       }
-      s_in = ss[lrr * ng + g];
+      if (DENSE || BITS == 0) s_in = ss[lrr * ng + g];
       const float2 s2 = dup2(s_in);
       const float2 a_row = dup2(__fmul_rn(s_in, alpha_s));
 #pragma unroll
@@ -317,11 +329,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     const float vr = sv[lrr];
     float w;
     if (kMayExact && exact && DELTA) {
-      long long U = exact_dot16(cs, planes + col0, DK);
-#pragma unroll
-      for (int st = 1; st < LPR; st <<= 1) U += __shfl_xor_sync(kFull, U, st);
-      const float u = (float)(((double)s_in * (double)U) * sx);
-      w = __fmul_rn(beta, __fsub_rn(vr, u));
+      w = __fmul_rn(beta, __fsub_rn(vr, u_ex));
     } else if (DELTA) {
       float u = dot16_p(sp, kk);
 #pragma unroll
@@ -339,11 +347,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
     float opv;
     if (kMayExact && exact) {
       // exact: the row's S'q in its first lane's share, zero in the others
-      long long Uq = exact_dot16(cs, planes + 4 * DK + col0, DK);
-#pragma unroll
-      for (int st = 1; st < LPR; st <<= 1) Uq += __shfl_xor_sync(kFull, Uq, st);
-      const float sqr = (float)(((double)s_in * (double)Uq) * sxq);
-      opv = lir == 0 ? sqr : 0.0f;
+      opv = lir == 0 ? sq_ex : 0.0f;
     } else {
       opv = dot16_p(sp, qq);
     }
@@ -472,49 +476,54 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
   __syncwarp();
 }
 
-template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool MT>
+template <int DK, bool DIAG, bool DELTA, bool SR, int BITS, bool MT, bool EXACT>
 __device__ __forceinline__ void compute_any(const StepParams &p, uint8_t *stage, int b,
                                             const UnitDesc &d, float alpha_s, float beta,
                                             float *opart, float *ow, int t) {
   if (BITS == 0) {
     constexpr int RPW = 32 / (DK / 16);
     if (d.nrows % RPW == 0)
-      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false, MT, EXACT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
-      compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT, EXACT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   } else if (d.nrows == full_rows(DK, BITS)) {
     if (p.G == DK)
-      compute_unit<DK, DIAG, DELTA, SR, BITS, true, true, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, true, MT, EXACT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
-      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_unit<DK, DIAG, DELTA, SR, BITS, true, false, MT, EXACT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   } else {
-    compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+    compute_unit<DK, DIAG, DELTA, SR, BITS, false, false, MT, EXACT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   }
 }
 // One unit for one token: the unit's storage class picks the code path.  EXT: 0 the plain
-// kernel (int8 / int4 / fp32 units only, the smallest code); 1 also the dense 5- to 7-bit
-// and per-lane (per-channel) paths; 2 the per-lane path without the dense ones, so a
-// handle with per-channel rows and no dense heads runs with fewer registers live.
+// kernel (int8 / int4 / fp32 units only, the smallest code); 3 the plain kernel with the
+// exact contractions for byte and nibble heads with one scale per row; 1 also the dense 5-
+// to 7-bit and per-lane (per-channel) paths; 4 the same with the exact contractions; 2 the
+// per-lane path without the dense ones, so a handle with per-channel rows and no dense
+// heads runs with fewer registers live.  (The exact contractions live only in the
+// families that need them: their registers would otherwise cost every other path.)
 template <int DK, bool DIAG, bool DELTA, bool SR, bool MT, int EXT>
 __device__ __forceinline__ void compute_bits(const StepParams &p, uint8_t *stage, int b,
                                              const UnitDesc &d, float alpha_s, float beta,
                                              float *opart, float *ow, int t) {
+  constexpr bool EX = EXT == 3 || EXT == 4;
+  constexpr bool DENSE_PATHS = EXT == 1 || EXT == 4;
   if (d.store == 32)
-    compute_any<DK, DIAG, DELTA, SR, 32, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  else if (EXT == 0 || d.store == 4 || d.store == 8) {
+    compute_any<DK, DIAG, DELTA, SR, 32, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  else if (EXT == 0 || EXT == 3 || d.store == 4 || d.store == 8) {
     if (d.store == 4)
-      compute_any<DK, DIAG, DELTA, SR, 4, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_any<DK, DIAG, DELTA, SR, 4, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
-      compute_any<DK, DIAG, DELTA, SR, 8, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_any<DK, DIAG, DELTA, SR, 8, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   } else if (d.store == 0) {
-    compute_any<DK, DIAG, DELTA, SR, 0, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
-  } else if constexpr (EXT == 1) {
+    compute_any<DK, DIAG, DELTA, SR, 0, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+  } else if constexpr (DENSE_PATHS) {
     if (d.store == 6)
-      compute_any<DK, DIAG, DELTA, SR, 6, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_any<DK, DIAG, DELTA, SR, 6, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else if (d.store == 5)
-      compute_any<DK, DIAG, DELTA, SR, 5, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_any<DK, DIAG, DELTA, SR, 5, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
     else
-      compute_any<DK, DIAG, DELTA, SR, 7, MT>(p, stage, b, d, alpha_s, beta, opart, ow, t);
+      compute_any<DK, DIAG, DELTA, SR, 7, MT, EX>(p, stage, b, d, alpha_s, beta, opart, ow, t);
   }
 }
 
@@ -654,7 +663,11 @@ StepFn pick_step(bool diag, bool delta) {
   StepFn step_kernels_##dk##_0_1(bool diag, bool delta, bool sr);  \
   StepFn step_kernels_##dk##_1_1(bool diag, bool delta, bool sr);  \
   StepFn step_kernels_##dk##_0_2(bool diag, bool delta, bool sr);  \
-  StepFn step_kernels_##dk##_1_2(bool diag, bool delta, bool sr);
+  StepFn step_kernels_##dk##_1_2(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_0_3(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_1_3(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_0_4(bool diag, bool delta, bool sr);  \
+  StepFn step_kernels_##dk##_1_4(bool diag, bool delta, bool sr);
 LORES_DECLARE_FAMILY(16)
 LORES_DECLARE_FAMILY(32)
 LORES_DECLARE_FAMILY(64)
