@@ -230,12 +230,12 @@ static StepFn pair_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr) {
   return nullptr;
 }
 // The tensor-core kernel (heads of one byte or one nibble per code, one scale per row).
-static StepFn mma_kernel_for(int dk, bool diag, bool delta, bool sr) {
+static StepFn mma_kernel_for(int dk, bool mt, bool diag, bool delta, bool sr) {
   switch (dk) {
-    case 16: return mma_kernels_16(diag, delta, sr);
-    case 32: return mma_kernels_32(diag, delta, sr);
-    case 64: return mma_kernels_64(diag, delta, sr);
-    case 128: return mma_kernels_128(diag, delta, sr);
+    case 16: return mma_kernels_16(diag, delta, sr, mt);
+    case 32: return mma_kernels_32(diag, delta, sr, mt);
+    case 64: return mma_kernels_64(diag, delta, sr, mt);
+    case 128: return mma_kernels_128(diag, delta, sr, mt);
   }
   return nullptr;
 }
@@ -544,7 +544,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   const StepFn general_fn = kernel_for(dk, false, ext, c.decay_diag, c.delta, c.stochastic);
   const StepFn pair_fn =
       pair_heads && !mma ? pair_kernel_for(dk, false, c.decay_diag, c.delta, c.stochastic) : nullptr;
-  const StepFn mma_fn = mma ? mma_kernel_for(dk, c.decay_diag, c.delta, c.stochastic) : nullptr;
+  const StepFn mma_fn = mma ? mma_kernel_for(dk, false, c.decay_diag, c.delta, c.stochastic) : nullptr;
   StepFn fn = general_fn;
   bool pair = false;
   int split = 1;
@@ -599,7 +599,9 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
                       (c.decay_diag ? dk * 4 : 0);
     const int opart_floats = ((maxrows * LPR + 31) / 32) * 32;     // 128-byte multiples
     const int ow_floats = ((maxrows + 31) / 32) * 32;
-    const int plane_bytes = 16 * dk;     // digit planes (8 d_k), a tile's k and alpha (8 d_k)
+    // digit planes (8 d_k) and a tile's k and alpha (8 d_k): only where exact contractions
+    // run (the tensor-core kernel, or the general kernel's exact families)
+    const int plane_bytes = (mma || exact_heads) ? 16 * dk : 0;
     const int warp_bytes =
         ((64 + 4 * (opart_floats + ow_floats) + plane_bytes + kStages * stage + 127) / 128) * 128;
     const int table = (int)units.size() * (int)sizeof(UnitDesc) <= 16384
@@ -667,9 +669,10 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
   h->step_fn = fn;
   h->pair = pair;
   h->mma = mma;
-  // multi-token calls: the two-rows-per-lane kernel's form, or the general one
-  h->mt_fn = pair ? pair_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic)
-                  : kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic);
+  // multi-token calls: the tensor-core or two-rows-per-lane kernel's form, or the general one
+  h->mt_fn = mma ? mma_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic)
+                 : (pair ? pair_kernel_for(dk, true, c.decay_diag, c.delta, c.stochastic)
+                         : kernel_for(dk, true, ext, c.decay_diag, c.delta, c.stochastic));
   {
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, h->mt_fn) != cudaSuccess ||

@@ -157,6 +157,17 @@ __device__ __forceinline__ void st16_a8(uint8_t *p, uint4 w) {
 // -------------------------------------------------------------------------------------
 // code <-> float
 // -------------------------------------------------------------------------------------
+// Two fp16 halves of a word, each widened to fp32 and added to `bias` in one
+// mixed-precision add (fp16 operand, fp32 operand and result, round to nearest).
+__device__ __forceinline__ void halves_plus(uint32_t w, float bias, float &lo, float &hi) {
+  asm("{\n\t.reg .f16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %3;\n\t"
+      "add.rn.f32.f16 %1, h, %3;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(w), "f"(bias));
+}
+
 // Bytes -> exact floats: a byte b dropped into the low mantissa byte of 2^23 (bits
 // 0x4B0000bb) is the float 2^23 + b, exactly (the float spacing is 1 there); one packed
 // add of -(2^23 + offset) then gives b - offset, exactly, for two bytes at once.
@@ -338,7 +349,10 @@ __device__ __forceinline__ DenseLane pack_dense(const uint32_t (&t)[16]) {
 }
 
 // 16 dense codes -> exact floats in column pairs: rebuild the offset-binary bytes u
-// (even columns in E, odd in O), then u - 2^(B-1).
+// (even columns in E, odd in O), drop them into fp16 pairs (1024 + u: the fp16 spacing is
+// 1 there) and add -(1024 + 2^(B-1)) in fp32.  (The bit-plane path is short of ALU
+// slots, so this route, which puts the conversion on the FMA pipe, suits it better than
+// the byte-into-2^23 route of the other paths.)
 template <int B>
 __device__ __forceinline__ void unpack_dense(const DenseLane &d, float2 (&c)[8]) {
   uint32_t E0 = d.nib0 & 0x0F0F0F0Fu, O0 = (d.nib0 >> 4) & 0x0F0F0F0Fu;
@@ -356,11 +370,13 @@ __device__ __forceinline__ void unpack_dense(const DenseLane &d, float2 (&c)[8])
     E1 |= spread_bit4<B - 1>(d.p1 >> 8);
     O1 |= spread_bit4<B - 1>(d.p1 >> 12);
   }
-  const float2 off = byte_bias(1 << (B - 1));
+  constexpr float bias = -(1024.0f + (float)(1 << (B - 1)));
+  const uint32_t x[4] = {__byte_perm(E0, O0, 0x5140u), __byte_perm(E0, O0, 0x7362u),
+                         __byte_perm(E1, O1, 0x5140u), __byte_perm(E1, O1, 0x7362u)};
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    c[k] = bytes_minus(E0, O0, k, off);        // columns 2k, 2k + 1
-    c[4 + k] = bytes_minus(E1, O1, k, off);    // columns 8 + 2k, 8 + 2k + 1
+  for (int q = 0; q < 4; ++q) {
+    halves_plus(__byte_perm(x[q], 0x64646464u, 0x5140u), bias, c[2 * q].x, c[2 * q].y);
+    halves_plus(__byte_perm(x[q], 0x64646464u, 0x7362u), bias, c[2 * q + 1].x, c[2 * q + 1].y);
   }
 }
 

@@ -12,7 +12,7 @@
 //     (heads of one byte or one nibble per code, several scales per row), single- or
 //     multi-token
 //   -DLORES_DK=<d_k> -DLORES_MMA=1: the tensor-core step kernels (heads of one byte or one
-//     nibble per code, one scale per row)
+//     nibble per code, one scale per row), single- and multi-token
 // The function defined here returns the kernel for the requested modes.
 #include "lores_step.cuh"
 #include "lores_key.cuh"
@@ -44,8 +44,9 @@ StepFn LORES_CAT3(pair_kernels, LORES_DK, LORES_MT)(bool diag, bool delta, bool 
 #if !defined(LORES_DK)
 #error "compile with -DLORES_DK=<16|32|64|128> -DLORES_MMA=1"
 #endif
-StepFn LORES_CAT1(mma_kernels, LORES_DK)(bool diag, bool delta, bool sr) {
-  return sr ? pick_mma<LORES_DK, true>(diag, delta) : pick_mma<LORES_DK, false>(diag, delta);
+StepFn LORES_CAT1(mma_kernels, LORES_DK)(bool diag, bool delta, bool sr, bool mt) {
+  if (mt) return sr ? pick_mma<LORES_DK, true, true>(diag, delta) : pick_mma<LORES_DK, false, true>(diag, delta);
+  return sr ? pick_mma<LORES_DK, true, false>(diag, delta) : pick_mma<LORES_DK, false, false>(diag, delta);
 }
 #elif defined(LORES_KEY)
 #if !defined(LORES_DK)

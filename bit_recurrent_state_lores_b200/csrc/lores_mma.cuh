@@ -155,20 +155,35 @@ __device__ __forceinline__ void s8_floats(uint32_t w, float2 &lo, float2 &hi) {
 }
 
 // Store one chunk's codes (CH columns: words of 4 code bytes) of a row, as bytes or nibbles.
-template <int DK, int BITS>
+// to_stage: the destination is the ring slot (a multi-token call's tokens before the
+// last), written with ordinary stores; otherwise global memory, streaming stores.
+template <int DK, int BITS, bool to_stage>
 __device__ __forceinline__ void mma_store(uint8_t *d, const uint32_t (&wq)[4], bool st) {
   using Gm = MmaGeom<DK>;
   if (!st) return;
   if (BITS == 8) {
-    if (Gm::CH == 16) __stcs(reinterpret_cast<uint4 *>(d), make_uint4(wq[0], wq[1], wq[2], wq[3]));
-    else if (Gm::CH == 8) __stcs(reinterpret_cast<uint2 *>(d), make_uint2(wq[0], wq[1]));
-    else __stcs(reinterpret_cast<unsigned int *>(d), wq[0]);
+    if (Gm::CH == 16) {
+      const uint4 v = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+      if (to_stage) *reinterpret_cast<uint4 *>(d) = v; else __stcs(reinterpret_cast<uint4 *>(d), v);
+    } else if (Gm::CH == 8) {
+      const uint2 v = make_uint2(wq[0], wq[1]);
+      if (to_stage) *reinterpret_cast<uint2 *>(d) = v; else __stcs(reinterpret_cast<uint2 *>(d), v);
+    } else {
+      if (to_stage) *reinterpret_cast<unsigned int *>(d) = wq[0];
+      else __stcs(reinterpret_cast<unsigned int *>(d), wq[0]);
+    }
   } else {
     const uint2 nb = compact_i4(make_uint4(wq[0], Gm::CH >= 8 ? wq[1] : 0u,
                                            Gm::CH == 16 ? wq[2] : 0u, Gm::CH == 16 ? wq[3] : 0u));
-    if (Gm::CH == 16) __stcs(reinterpret_cast<uint2 *>(d), nb);
-    else if (Gm::CH == 8) __stcs(reinterpret_cast<unsigned int *>(d), nb.x);
-    else __stcs(reinterpret_cast<unsigned short *>(d), (unsigned short)nb.x);
+    if (Gm::CH == 16) {
+      if (to_stage) *reinterpret_cast<uint2 *>(d) = nb; else __stcs(reinterpret_cast<uint2 *>(d), nb);
+    } else if (Gm::CH == 8) {
+      if (to_stage) *reinterpret_cast<unsigned int *>(d) = nb.x;
+      else __stcs(reinterpret_cast<unsigned int *>(d), nb.x);
+    } else {
+      if (to_stage) *reinterpret_cast<unsigned short *>(d) = (unsigned short)nb.x;
+      else __stcs(reinterpret_cast<unsigned short *>(d), (unsigned short)nb.x);
+    }
   }
 }
 
@@ -185,12 +200,13 @@ __device__ __forceinline__ uint32_t pack4(const float2 &a, const float2 &b) {
 // (maximum shuffles, Newton steps) overlap.  s2, w2: the rows' old scales and w; snew:
 // their new scales; bad: a row held a non-finite or overflowing entry.  dstA / dstB: the
 // rows in global memory, stored if stA / stB.
-template <int DK, int BITS, bool DIAG, bool SR>
+template <int DK, int BITS, bool DIAG, bool SR, bool TO_STAGE>
 __device__ __forceinline__ void mma_rows2(const uint32_t (&cA)[DK / 16], const uint32_t (&cB)[DK / 16],
                                           float2 s2, const float *sa, float alpha_s, float2 w2,
                                           const float *sk, float r, float inv_r,
                                           uint32_t cbA, uint32_t cbB, uint8_t *dstA, uint8_t *dstB,
-                                          bool stA, bool stB, float2 &snew, bool &badA, bool &badB) {
+                                          bool stA, bool stB, float2 &snew, bool &badA,
+                                          bool &badB) {
   using Gm = MmaGeom<DK>;
   constexpr int NP = DK / 8;                        // column pairs per lane-row
   const int tq = threadIdx.x & 3;
@@ -291,26 +307,30 @@ __device__ __forceinline__ void mma_rows2(const uint32_t (&cA)[DK / 16], const u
       wb[qd] = pack4(tb0, tb1);
     }
     const int boff = BITS == 8 ? Gm::col(tq, c) : Gm::col(tq, c) / 2;
-    mma_store<DK, BITS>(dstA + boff, wa, stA);
-    mma_store<DK, BITS>(dstB + boff, wb, stB);
+    mma_store<DK, BITS, TO_STAGE>(dstA + boff, wa, stA);
+    mma_store<DK, BITS, TO_STAGE>(dstB + boff, wb, stB);
   }
 }
 
 // One unit (rows [row0, row0 + nrows) of one tile) from a ring slot, strip by strip.
 // FULL: the unit is a full row block (full_rows(d_k, BITS) rows, a whole number of
 // strips): the strip count and every row's validity are compile-time facts.
-template <int DK, int BITS, bool DIAG, bool DELTA, bool SR, bool FULL>
-__device__ __forceinline__ void mma_unit(const StepParams &p, const uint8_t *stage, int b,
+// sv: the unit's v rows; go: where its readout rows go; to_stage: write the requantized
+// rows and scales back into the slot (a multi-token call's tokens before the last; every
+// lane rewrites the bytes it read, and a row's scale is rewritten by the row's lane 0 after
+// the row's shuffles, so after all its lanes read it) instead of global memory.
+template <int DK, int BITS, bool DIAG, bool DELTA, bool SR, bool FULL, bool TO_STAGE>
+__device__ __forceinline__ void mma_unit(const StepParams &p, uint8_t *stage, int b,
                                          const UnitDesc &d, const MmaTile<DK, DIAG> &t,
-                                         const float *sk, const float *sa) {
+                                         const float *sk, const float *sa, const float *sv,
+                                         float *go) {
+  constexpr bool to_stage = TO_STAGE;
   constexpr int RB = DK * BITS / 8;                 // bytes of one row
   const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const long long tile = (long long)b * p.H + d.head;
-  const float *ss = reinterpret_cast<const float *>(stage + p.st_scales);
-  const float *sv = reinterpret_cast<const float *>(stage + p.st_v);
-  uint8_t *gcodes = p.codes + (long long)b * p.seq_bytes + d.code_off;
-  float *gs = p.scales + tile * p.d_v + d.row0;
-  float *go = p.o + tile * p.d_v + d.row0;
+  float *ss = reinterpret_cast<float *>(stage + p.st_scales);
+  uint8_t *gcodes = to_stage ? stage : p.codes + (long long)b * p.seq_bytes + d.code_off;
+  float *gs = to_stage ? ss : p.scales + tile * p.d_v + d.row0;
   constexpr int kFull = full_rows(DK, BITS);
   static_assert(kFull % 16 == 0, "a full row block is a whole number of strips");
   const int nrows = FULL ? kFull : d.nrows;
@@ -360,9 +380,9 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, const uint8_t *sta
     const uint32_t cb1 = cb0 + 0x9E3779B9u * (uint32_t)(8 * DK / 4);
     float2 sn;
     bool badA, badB;
-    mma_rows2<DK, BITS, DIAG, SR>(c0, c1, make_float2(sA, sB), sa, t.alpha, make_float2(wA, wB), sk,
-                                  d.r, d.inv_r, cb0, cb1, gcodes + r0 * RB, gcodes + r1 * RB, v0, v1,
-                                  sn, badA, badB);
+    mma_rows2<DK, BITS, DIAG, SR, TO_STAGE>(c0, c1, make_float2(sA, sB), sa, t.alpha, make_float2(wA, wB),
+                                            sk, d.r, d.inv_r, cb0, cb1, gcodes + r0 * RB,
+                                            gcodes + r1 * RB, v0, v1, sn, badA, badB);
     if (tq == 0) {
       if (v0) gs[r0] = sn.x;
       if (v1) gs[r1] = sn.y;
@@ -393,7 +413,7 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, const uint8_t *sta
 // The persistent loop of one warp over the units of one storage class (BITS), as in
 // pair_run: warp gw of W takes units [U gw / W, U (gw + 1) / W) of the class's U units in
 // (sequence, unit) order through a 2-slot ring of bulk copies.
-template <int DK, int BITS, bool DIAG, bool DELTA, bool SR>
+template <int DK, int BITS, bool DIAG, bool DELTA, bool SR, bool MT>
 __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl, uint8_t *wa,
                                         int cta, int nctas, int lo, int hi) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -421,7 +441,7 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
   for (int s = 0; s < kStages && s < count; ++s) {
     const UnitDesc d = tbl[fill.ub];
     const int tl = fill.b * H + d.head;
-    pair_issue<DK, DIAG, false>(p, d, fill.b, fill.ub, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
+    pair_issue<DK, DIAG, MT>(p, d, fill.b, fill.ub, tl != ftile, stages + s * p.stage_bytes, &bars[s]);
     ftile = tl;
     fill.next(lo, hi);
   }
@@ -431,8 +451,8 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
   const float *kkeep = reinterpret_cast<const float *>(planes + 8 * DK);   // the tile's k
   const float *akeep = kkeep + DK;                  // and per-column alpha (DIAG)
   MmaTile<DK, DIAG> t;
-  float beta_c, alpha_c = 0.0f;
-  {
+  float beta_c = 0.0f, alpha_c = 0.0f;
+  if (!MT) {
     const int t0 = cur.b * H + tbl[cur.ub].head;
     beta_c = __ldg(p.beta + t0);
     if (!DIAG) alpha_c = __ldg(p.alpha + t0);
@@ -444,7 +464,7 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
     PairPos nx = cur;
     nx.next(lo, hi);
     float beta_n = 0.0f, alpha_n = 0.0f;
-    if (n + 1 < count) {
+    if (!MT && n + 1 < count) {
       const int tn = nx.b * H + tbl[nx.ub].head;
       beta_n = __ldg(p.beta + tn);
       if (!DIAG) alpha_n = __ldg(p.alpha + tn);
@@ -463,7 +483,40 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
     }
     const UnitDesc d = tbl[cur.ub];
     const int tl = cur.b * H + d.head;
-    if (tl != ctile) {
+    if (MT) {
+      // every token of the unit in turn; the unit's codes and scales stay in the slot
+      for (int tok = 0; tok < p.T; ++tok) {
+        const float *k = p.k + tok * p.tok_qk + (long long)tl * DK;
+        const float *q = p.q + tok * p.tok_qk + (long long)tl * DK;
+        const float *al = p.alpha + tok * p.tok_a + (long long)tl * DK;
+        const float a_s = DIAG ? 0.0f : __ldg(p.alpha + tok * p.tok_a + tl);
+        mma_tile<DK, DIAG>(k, q, al, a_s, planes, t);
+        double kqd = 0.0;
+#pragma unroll
+        for (int j = lane; j < DK; j += 32) kqd = fma((double)__ldg(k + j), (double)__ldg(q + j), kqd);
+#pragma unroll
+        for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
+        t.kq = (float)kqd;
+        t.tkey = tile_key(step_key_dev(p.seed, p.step0 + (uint64_t)tok), (uint32_t)tl);
+        t.beta = __ldg(p.beta + tok * p.tok_b + tl);
+        t.alpha = a_s;
+        const float *sv = p.v + tok * p.tok_v + (long long)tl * p.d_v + d.row0;
+        float *go = p.o + tok * p.tok_o + (long long)tl * p.d_v + d.row0;
+        const bool full = d.nrows == full_rows(DK, BITS);
+        if (tok + 1 < p.T) {                         // not the last token: back to the slot
+          if (full)
+            mma_unit<DK, BITS, DIAG, DELTA, SR, true, true>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+          else
+            mma_unit<DK, BITS, DIAG, DELTA, SR, false, true>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+        } else {
+          if (full)
+            mma_unit<DK, BITS, DIAG, DELTA, SR, true, false>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+          else
+            mma_unit<DK, BITS, DIAG, DELTA, SR, false, false>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+        }
+        __syncwarp();
+      }
+    } else if (tl != ctile) {
       // a new tile: its vectors are in this slot (copied out by mma_tile: a later unit of
       // the tile reuses the slot)
       const float *sk = reinterpret_cast<const float *>(stage + p.st_k);
@@ -479,18 +532,22 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
       t.tkey = tile_key(skey, (uint32_t)tl);
       ctile = tl;
     }
-    t.beta = beta_c;
-    t.alpha = alpha_c;
-    if (d.nrows == full_rows(DK, BITS))
-      mma_unit<DK, BITS, DIAG, DELTA, SR, true>(p, stage, cur.b, d, t, kkeep, akeep);
-    else
-      mma_unit<DK, BITS, DIAG, DELTA, SR, false>(p, stage, cur.b, d, t, kkeep, akeep);
+    if (!MT) {
+      t.beta = beta_c;
+      t.alpha = alpha_c;
+      const float *sv = reinterpret_cast<const float *>(stage + p.st_v);
+      float *go = p.o + ((long long)tl * p.d_v + d.row0);
+      if (d.nrows == full_rows(DK, BITS))
+        mma_unit<DK, BITS, DIAG, DELTA, SR, true, false>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+      else
+        mma_unit<DK, BITS, DIAG, DELTA, SR, false, false>(p, stage, cur.b, d, t, kkeep, akeep, sv, go);
+    }
     __syncwarp();                                   // every lane is done with this slot
     if (n + kStages < count) {
       fence_proxy_async();
       const UnitDesc dn = tbl[fill.ub];
       const int tf = fill.b * H + dn.head;
-      pair_issue<DK, DIAG, false>(p, dn, fill.b, fill.ub, tf != ftile, stage, &bars[s]);
+      pair_issue<DK, DIAG, MT>(p, dn, fill.b, fill.ub, tf != ftile, stage, &bars[s]);
       ftile = tf;
       fill.next(lo, hi);
     }
@@ -504,7 +561,7 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
 // [pair_lo[0], pair_hi[0]) of every sequence) and one nibble per code ([pair_lo[1],
 // pair_hi[1])), all with one scale per value row: CTAs [0, pair_ctas) take the first
 // class, the others the second.
-template <int DK, bool DIAG, bool DELTA, bool SR>
+template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
 __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -518,21 +575,21 @@ __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kerne
   __syncthreads();                                  // the only CTA-wide barrier
   const int cta = (int)blockIdx.x;
   if (cta < p.pair_ctas)
-    mma_run<DK, 8, DIAG, DELTA, SR>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
+    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
   else
-    mma_run<DK, 4, DIAG, DELTA, SR>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
-                                    p.pair_lo[1], p.pair_hi[1]);
+    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
+                                        p.pair_lo[1], p.pair_hi[1]);
 }
 
-template <int DK, bool SR>
+template <int DK, bool SR, bool MT>
 StepFn pick_mma(bool diag, bool delta) {
   if (diag)
-    return delta ? decode_mma_kernel<DK, true, true, SR> : decode_mma_kernel<DK, true, false, SR>;
-  return delta ? decode_mma_kernel<DK, false, true, SR> : decode_mma_kernel<DK, false, false, SR>;
+    return delta ? decode_mma_kernel<DK, true, true, SR, MT> : decode_mma_kernel<DK, true, false, SR, MT>;
+  return delta ? decode_mma_kernel<DK, false, true, SR, MT> : decode_mma_kernel<DK, false, false, SR, MT>;
 }
 
 // One function per key width, each defined in its own compilation of lores_inst.cu.
-#define LORES_DECLARE_MMA(dk) StepFn mma_kernels_##dk(bool diag, bool delta, bool sr);
+#define LORES_DECLARE_MMA(dk) StepFn mma_kernels_##dk(bool diag, bool delta, bool sr, bool mt);
 LORES_DECLARE_MMA(16)
 LORES_DECLARE_MMA(32)
 LORES_DECLARE_MMA(64)

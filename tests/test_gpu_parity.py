@@ -17,7 +17,7 @@ import torch
 from bit_recurrent_state_lores_b200 import synth
 from oracle import oracle as O
 
-from .harness import (GpuRun, OracleTiles, assert_parity, host_tile_inputs, mixed_bits,
+from .harness import (GpuRun, OracleTiles, assert_parity, host_tile_inputs, lib, mixed_bits,
                       rel_l2, sample_tiles, tile_cfg, unpack_fast)
 
 pytestmark = pytest.mark.gpu
@@ -400,3 +400,30 @@ def test_tensor_core_kernel_every_key_width(d_k, d_v, bits, delta, diag, sr, B):
         assert g.layout.step_kernel == 3
     finally:
         g.close()
+
+
+@pytest.mark.parametrize("diag,delta,sr", [(0, 1, 1), (1, 1, 1), (0, 0, 0)])
+def test_general_exact_path_equals_tensor_core_kernel(diag, delta, sr):
+    """The exact contractions of heads with one scale per row have two implementations:
+    the tensor-core kernel, and the general kernel's DP4A path, which a handle takes when it
+    also holds an fp32 head.  Heads 0-3 of handle A (last head int8: tensor-core kernel)
+    and of handle B (last head fp32: general kernel) get the same inputs and the same tile
+    keys, so their readout and state agree bit for bit, step after step."""
+    L = lib()
+    wl = synth.Workload("cross", B=48, H=5, d_k=128, d_v=128, steps=4, delta=delta, diag=diag,
+                        group=128, decay="kda" if diag else "tau", outliers=2, seed=31)
+    hp = synth.head_params(wl)
+    a = GpuRun(wl, [8, 4, 8, 4, 8], 7, stochastic=sr)
+    b = GpuRun(wl, [8, 4, 8, 4, 32], 7, stochastic=sr)
+    try:
+        assert a.layout.step_kernel == 3 and b.layout.step_kernel == 0
+        for t in range(wl.steps):
+            inp = synth.step_inputs(wl, t, hp, device="cuda")
+            oa = a.step(inp, t).clone()
+            ob = b.step(inp, t)
+            assert torch.equal(oa[:, :4], ob[:, :4]), t
+            assert torch.equal(a.dequant()[:, :4], b.dequant()[:, :4]), t
+        assert a.check() == L.LORES_OK and b.check() == L.LORES_OK
+    finally:
+        a.close()
+        b.close()
