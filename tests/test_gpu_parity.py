@@ -390,6 +390,21 @@ MMA_WIDTHS = [
 ]
 
 
+def test_exact_path_at_key_width_256():
+    """d_k = 256 heads with one scale per row: beyond the tensor-core kernel's widths, they
+    take the general kernel's exact contractions (DP4A on the digit planes); parity with
+    the oracle, bit-exact, every step."""
+    bits = [8, 4]
+    wl = synth.Workload("exact-256", B=96, H=len(bits), d_k=256, d_v=64, steps=4, delta=1,
+                        diag=1, group=256, decay="kda", outliers=2, seed=29)
+    tiles = sample_tiles(wl, bits, 8, seed=3)
+    g = run_free(wl, bits, 27, tiles, 4, stochastic=1, exact=True)
+    try:
+        assert g.layout.step_kernel == 0
+    finally:
+        g.close()
+
+
 @pytest.mark.parametrize("d_k,d_v,bits,delta,diag,sr,B", MMA_WIDTHS)
 def test_tensor_core_kernel_every_key_width(d_k, d_v, bits, delta, diag, sr, B):
     wl = synth.Workload("mma-width", B=B, H=len(bits), d_k=d_k, d_v=d_v, steps=4, delta=delta,
