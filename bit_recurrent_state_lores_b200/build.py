@@ -1,12 +1,17 @@
 """Build liblores.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m bit_recurrent_state_lores_b200.build [--verbose]
+    python -m bit_recurrent_state_lores_b200.build [--verbose] [--checked]
 
 csrc/lores.cu (host side, loader, dequantizer) and 45 compilations of csrc/lores_inst.cu
 (one decode-step kernel family per key width x single/multi-token x storage family --
 plain; dense and per-lane; per-lane only --, one two-rows-per-lane family per key width x
 single/multi-token, and one key-axis family per key width) build in parallel, one nvcc
 process per CPU core, then link.
+
+--checked builds liblores_checked.so instead: the same sources compiled with
+LORES_INDEX_CHECKS, so that every global access of the kernels is checked against the
+extent of its buffer first (include/lores.h, lores_index_checked); a debugging build, not
+the product.
 
 No fast-math: the kernels' fp32 rounding is part of the state format, so every
 rounding-sensitive operation is written with explicit round-to-nearest intrinsics
@@ -27,6 +32,7 @@ DEPS = [SRC, INST, os.path.join(CSRC, "lores_step.cuh"), os.path.join(CSRC, "lor
         os.path.join(CSRC, "lores_mma.cuh"),
         os.path.join(ROOT, "include", "lores.h")]
 LIB = os.path.join(PKG, "liblores.so")
+LIB_CHECKED = os.path.join(PKG, "liblores_checked.so")
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-fmad=false", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
@@ -55,11 +61,15 @@ def units():
     return out
 
 
-def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
-    """Compile every unit (up to `jobs` at a time, default: the CPU count), then link."""
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in DEPS)):
-        return LIB
+def build(force: bool = False, verbose: bool = False, jobs: int = 0,
+          checked: bool = False) -> str:
+    """Compile every unit (up to `jobs` at a time, default: the CPU count), then link.
+    checked: the index-checked library instead of the product."""
+    lib = LIB_CHECKED if checked else LIB
+    mode = ["-DLORES_INDEX_CHECKS=1"] if checked else []
+    if (not force and os.path.exists(lib)
+            and os.path.getmtime(lib) >= max(os.path.getmtime(p) for p in DEPS)):
+        return lib
     jobs = jobs or max(1, os.cpu_count() or 1)
     with tempfile.TemporaryDirectory(prefix="lores_build_") as tmp:
         pending = list(units())
@@ -68,7 +78,7 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
             while pending and len(running) < jobs:
                 src, extra, name = pending.pop(0)
                 obj = os.path.join(tmp, name)
-                cmd = [NVCC] + FLAGS + extra + (["-Xptxas=-v"] if verbose else []) + [
+                cmd = [NVCC] + FLAGS + mode + extra + (["-Xptxas=-v"] if verbose else []) + [
                     "-c", "-o", obj, src]
                 running.append((subprocess.Popen(cmd), name))
                 objs.append(obj)
@@ -78,10 +88,10 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
                     p.wait()
                 raise subprocess.CalledProcessError(proc.returncode, f"nvcc ({name})")
         subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o",
-                        LIB + ".tmp"] + objs, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+                        lib + ".tmp"] + objs, check=True)
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    print(build(force=True, verbose="--verbose" in sys.argv, checked="--checked" in sys.argv))

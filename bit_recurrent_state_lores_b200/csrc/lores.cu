@@ -46,6 +46,8 @@ struct LoadParams {
   uint32_t step_key;
   int stochastic;
   int axis;                     // 0: value-axis groups; 1: one scale per key column
+  unsigned *flag;               // the handle's error word
+  LORES_RANGES                  // index-checked build: the extent of every buffer of the launch
 };
 
 template <int DK>
@@ -66,9 +68,10 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   const int bits = f.bits;
   float x[16];
   const float *src = p.S + grr * DK + col0;
+  const bool src_in = LORES_IN(p, kRgS, src, 64);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    const float4 f = __ldg(reinterpret_cast<const float4 *>(src) + c);
+    const float4 f = src_in ? __ldg(reinterpret_cast<const float4 *>(src) + c) : make_float4(0, 0, 0, 0);
     x[4 * c] = f.x; x[4 * c + 1] = f.y; x[4 * c + 2] = f.z; x[4 * c + 3] = f.w;
   }
   uint8_t *tilecodes = p.codes + b * p.seq_bytes + __ldg(p.head_off + head);
@@ -80,28 +83,32 @@ __global__ void __launch_bounds__(kThreads) load_state_kernel(const LoadParams p
   requantize16<LPR>(x, bits == 32 ? 8 : bits, lpg, lane, tkey, n0, p.stochastic, words, s_new,
                     f.store);
   if (!active) return;
+  const bool scale_in = LORES_IN(p, kRgScales, p.scales + grr * p.ng + g, 4);
   if (f.store >= 5 && f.store <= 7) {                 // dense bit planes
     const DenseLane dl{words[0], words[1], words[2], words[3]};
     uint8_t *rowp = tilecodes + (size_t)row * f.rowb;
+    if (!LORES_IN(p, kRgCodes, rowp, f.rowb)) return;
     if (f.store == 5) st_dense<5>(rowp, DK, lir, dl);
     else if (f.store == 6) st_dense<6>(rowp, DK, lir, dl);
     else st_dense<7>(rowp, DK, lir, dl);
-    if (lir % lpg == 0) p.scales[grr * p.ng + g] = s_new;
+    if (lir % lpg == 0 && scale_in) p.scales[grr * p.ng + g] = s_new;
     return;
   }
   uint8_t *dst = tilecodes + (size_t)row * f.rowb + f.off;
   if (bits == 32) {
+    if (LORES_IN(p, kRgCodes, dst, 64))
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
+      for (int c = 0; c < 4; ++c)
+        reinterpret_cast<float4 *>(dst)[c] = make_float4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
     return;
   }
   // lane blocks are 8-byte aligned (16 with one width per head)
-  if (bits != 4)
+  if (!LORES_IN(p, kRgCodes, dst, bits != 4 ? 16 : 8)) {
+  } else if (bits != 4)
     st16_a8(dst, make_uint4(words[0], words[1], words[2], words[3]));
   else
     *reinterpret_cast<uint2 *>(dst) = make_uint2(words[0], words[1]);
-  if (lir % lpg == 0) p.scales[grr * p.ng + g] = s_new;
+  if (lir % lpg == 0 && scale_in) p.scales[grr * p.ng + g] = s_new;
 }
 
 // -------------------------------------------------------------------------------------
@@ -121,6 +128,11 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
   const LaneFmt f = p.fmt[head * (DK / 16) + lir];
   const int bits = f.bits;
   const uint8_t *lanecodes = p.codes + b * p.seq_bytes + p.head_off[head] + (size_t)row * f.rowb + f.off;
+  // (index-checked build: the lane's row must lie in the code pool, its scales in theirs)
+  if (!LORES_IN(p, kRgCodes, lanecodes - f.off, f.rowb)) return;
+  if (bits != 32 && !(p.axis ? LORES_IN(p, kRgScales, p.scales + tile * DK + col0, 64)
+                             : LORES_IN(p, kRgScales, p.scales + grr * p.ng + col0 / p.G, 4)))
+    return;
   float y[16];
   if (bits == 32) {
     const float4 *src = reinterpret_cast<const float4 *>(lanecodes);
@@ -155,8 +167,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const LoadParams p, f
     }
   }
   float4 *dst = reinterpret_cast<float4 *>(out + grr * DK + col0);
+  if (LORES_IN(p, kRgS, dst, 64))
 #pragma unroll
-  for (int c = 0; c < 4; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+    for (int c = 0; c < 4; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
 }
 
 // Adds n to a device step counter (one thread; captured into a CUDA graph together with
@@ -319,6 +332,10 @@ struct lores_handle {
   // staging for lores_decode_step_host
   float *stage_in = nullptr;
   float *stage_o = nullptr;
+  // index-checked build: bytes taken off the end of each buffer's declared extent
+  // (lores_debug_trim_range), and the error word the last lores_check_errors read
+  unsigned long long trim[kRgCount] = {};
+  unsigned last_flags = 0;
 };
 
 namespace {
@@ -378,8 +395,37 @@ LoadParams load_params(const lores_handle *h) {
   p.G = h->G;
   p.stochastic = h->cfg.stochastic;
   p.axis = h->axis;
+  p.flag = h->flag;
   return p;
 }
+
+#ifdef LORES_INDEX_CHECKS
+// Extents of the buffers one launch may touch (T tokens of inputs and outputs; S the fp32
+// state of lores_load_state, or the output of lores_dequant_state), less the handle's trims.
+Ranges ranges_of(const lores_handle *h, const void *q, const void *k, const void *v,
+                 const void *alpha, const void *beta, const void *o, const void *S, int T) {
+  const lores_config &c = h->cfg;
+  const unsigned long long bh = (unsigned long long)c.batch * c.heads, t = (unsigned long long)T;
+  Ranges r{};
+  auto set = [&](int id, const void *ptr, unsigned long long bytes) {
+    r.base[id] = ptr;
+    r.bytes[id] = ptr && bytes > h->trim[id] ? bytes - h->trim[id] : 0;
+  };
+  set(kRgCodes, h->codes, (unsigned long long)c.batch * h->seq_bytes);
+  set(kRgScales, h->scales, (unsigned long long)scale_count_of(h) * 4);
+  set(kRgQ, q, t * bh * c.d_k * 4);
+  set(kRgK, k, t * bh * c.d_k * 4);
+  set(kRgV, v, t * bh * c.d_v * 4);
+  set(kRgAlpha, alpha, t * (c.decay_diag ? bh * c.d_k : bh) * 4);
+  set(kRgBeta, beta, t * bh * 4);
+  set(kRgO, o, t * bh * c.d_v * 4);
+  set(kRgS, S, bh * c.d_v * c.d_k * 4);
+  return r;
+}
+#define LORES_SET_RANGES(params, ...) ((params).rg = ranges_of(h, __VA_ARGS__))
+#else
+#define LORES_SET_RANGES(params, ...) ((void)0)
+#endif
 
 }  // namespace
 
@@ -395,6 +441,7 @@ const char *lores_status_string(lores_status s) {
     case LORES_ERR_UNSUPPORTED: return "unsupported configuration";
     case LORES_ERR_TIMEOUT: return "kernel wait timed out";
     case LORES_ERR_CORRUPT: return "memory around the state was overwritten";
+    case LORES_ERR_INDEX: return "an access fell outside its buffer (index-checked build)";
   }
   return "unknown status";
 }
@@ -862,6 +909,7 @@ static lores_status launch_step(lores_handle *h, const float *q, const float *k,
     kp.S = nullptr;
     kp.step_key = step_key_of(h->cfg.seed, step);
     kp.step_dev = step_dev;
+    LORES_SET_RANGES(kp, q, k, v, alpha, beta, o, nullptr, 1);
     h->key_fn<<<h->key_grid, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
     return cuda_status(cudaGetLastError());
   }
@@ -875,6 +923,7 @@ static lores_status launch_step(lores_handle *h, const float *q, const float *k,
   p.step_key = step_key_of(h->cfg.seed, step);
   p.seed = h->cfg.seed;
   p.step_dev = step_dev;
+  LORES_SET_RANGES(p, q, k, v, alpha, beta, o, nullptr, 1);
   h->step_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
   return cuda_status(cudaGetLastError());
 }
@@ -918,6 +967,7 @@ lores_status lores_decode_steps(lores_handle *h, int32_t T, const float *q, cons
   p.tok_o = tok_v;
   p.seed = c.seed;
   p.step0 = step0;
+  LORES_SET_RANGES(p, q, k, v, alpha, beta, o, nullptr, T);
   h->mt_fn<<<h->grid, kThreads, h->smem, static_cast<cudaStream_t>(stream)>>>(p);
   return cuda_status(cudaGetLastError());
 }
@@ -977,6 +1027,7 @@ lores_status lores_dequant_state(lores_handle *h, float *out, void *stream) {
   DeviceGuard guard(h->cfg.device);
   if (!guard.ok) return LORES_ERR_CUDA;
   LoadParams p = load_params(h);
+  LORES_SET_RANGES(p, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, out, 1);
   const long long threads = p.rows * (h->cfg.d_k / 16);
   const int blocks = (int)((threads + kThreads - 1) / kThreads);
   dequant_kernel_for(h->cfg.d_k)<<<blocks, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p, out);
@@ -991,12 +1042,14 @@ lores_status lores_load_state(lores_handle *h, const float *S, uint64_t step, vo
     KeyParams kp = h->kp;
     kp.S = S;
     kp.step_key = step_key_of(h->cfg.seed, step);
+    LORES_SET_RANGES(kp, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 1);
     h->key_load_fn<<<h->key_load_grid, kThreads, h->key_smem, static_cast<cudaStream_t>(stream)>>>(kp);
     return cuda_status(cudaGetLastError());
   }
   LoadParams p = load_params(h);
   p.S = S;
   p.step_key = step_key_of(h->cfg.seed, step);
+  LORES_SET_RANGES(p, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S, 1);
   const int rpw = 32 / (h->cfg.d_k / 16);
   const long long warps = (p.rows + rpw - 1) / rpw;
   const int blocks = (int)((warps + kWarps - 1) / kWarps);
@@ -1049,6 +1102,31 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
   return LORES_OK;
 }
 
+int32_t lores_index_checked(void) {
+#ifdef LORES_INDEX_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+lores_status lores_debug_trim_range(lores_handle *h, int32_t which, uint64_t bytes) {
+  if (!h || which < 0 || which >= kRgCount) return LORES_ERR_INVALID_ARG;
+#ifdef LORES_INDEX_CHECKS
+  h->trim[which] = bytes;
+  return LORES_OK;
+#else
+  (void)bytes;
+  return LORES_ERR_UNSUPPORTED;
+#endif
+}
+
+lores_status lores_debug_last_flags(lores_handle *h, uint32_t *flags) {
+  if (!h || !flags) return LORES_ERR_INVALID_ARG;
+  *flags = h->last_flags;
+  return LORES_OK;
+}
+
 lores_status lores_set_fault_injection(lores_handle *h, int32_t seq, int32_t unit,
                                        uint32_t wait_us) {
   if (!h || seq < -1 || seq >= h->cfg.batch) return LORES_ERR_INVALID_ARG;
@@ -1072,6 +1150,8 @@ lores_status lores_check_errors(lores_handle *h, void *stream) {
   if (e == cudaSuccess) e = cudaMemcpy(&f, h->flag, sizeof(unsigned), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(h->flag, 0, sizeof(unsigned));
   if (e != cudaSuccess) return cuda_status(e);
+  h->last_flags = f;
+  if (f & kFlagIndex) return LORES_ERR_INDEX;   // (a skipped copy also runs a wait out)
   if (f & kFlagTimeout) return LORES_ERR_TIMEOUT;
   // guard bands around the state
   const long long cb = (long long)h->cfg.batch * h->seq_bytes, sb = scale_count_of(h) * 4;
@@ -1269,6 +1349,19 @@ extern "C" lores_status lores_decode_step_noalloc(const lores_config *cfg, void 
   p.fault_b = -1;
   p.fault_ub = -1;
   p.step_key = step_key_of(c.seed, step);
+#ifdef LORES_INDEX_CHECKS
+  {
+    const unsigned long long bh = (unsigned long long)c.batch * c.heads;
+    const void *base[kRgCount] = {codes, scales, q, k, v, alpha, beta, o, nullptr};
+    const unsigned long long bytes[kRgCount] = {
+        (unsigned long long)c.batch * seq_bytes, bh * dv * ng * 4, bh * dk * 4, bh * dk * 4,
+        bh * dv * 4, (c.decay_diag ? bh * dk : bh) * 4, bh * 4, bh * dv * 4, 0};
+    for (int i = 0; i < kRgCount; ++i) {
+      p.rg.base[i] = base[i];
+      p.rg.bytes[i] = bytes[i];
+    }
+  }
+#endif
   const long long ctas = (p.total_units + kWarps - 1) / kWarps;
   const int grid = (int)std::min<long long>(ctas, (long long)ctas_per_sm * sms);
 

@@ -28,6 +28,9 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 // Flag bits of the handle's sticky device word.
 constexpr unsigned kFlagNonFinite = 1u;
 constexpr unsigned kFlagTimeout = 2u;
+// Index-checked build only: an access fell outside the buffer it belongs to (bit 8 + the
+// buffer's RangeId says which; kRgShared: a bulk copy outside the dynamic shared memory)
+constexpr unsigned kFlagIndex = 4u;
 
 // Bounded waits: a wait on an mbarrier gives up after the launch's limit in nanoseconds of
 // GPU time (%globaltimer; kWaitNs unless a test sets a shorter one), and after kMaxPolls
@@ -141,6 +144,55 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+
+// -------------------------------------------------------------------------------------
+// index-checked build (LORES_INDEX_CHECKS): every global access of the decode, loader and
+// dequantizer kernels names the buffer it belongs to and its byte count; the access runs
+// only if it lies inside that buffer's extent as the host declared it for the launch.
+// Otherwise the kernel raises kFlagIndex and the buffer's bit and skips the access (a
+// skipped bulk copy leaves its barrier short, so the wait runs out and TIMEOUT is raised
+// too).  In the ordinary build LORES_IN is the constant true and costs nothing.
+// -------------------------------------------------------------------------------------
+enum RangeId : int {
+  kRgCodes, kRgScales, kRgQ, kRgK, kRgV, kRgAlpha, kRgBeta, kRgO, kRgS, kRgCount,
+  kRgShared = kRgCount
+};
+struct Ranges {
+  const void *base[kRgCount];
+  unsigned long long bytes[kRgCount];
+};
+
+#ifdef LORES_INDEX_CHECKS
+__device__ __forceinline__ bool range_ok(const Ranges &r, int id, const void *ptr,
+                                         unsigned long long bytes, unsigned *flag) {
+  const unsigned long long lo = reinterpret_cast<unsigned long long>(r.base[id]);
+  const unsigned long long a = reinterpret_cast<unsigned long long>(ptr);
+  if (a >= lo && a - lo <= r.bytes[id] && bytes <= r.bytes[id] - (a - lo)) return true;
+  atomicOr(flag, kFlagIndex | (256u << id));
+  return false;
+}
+
+// A bulk copy's destination [dst, dst + bytes) inside the launch's dynamic shared memory.
+extern __shared__ __align__(16) uint8_t lores_dynamic_smem[];
+__device__ __forceinline__ bool smem_range_ok(const void *dst, unsigned bytes, unsigned *flag) {
+  unsigned size;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(size));
+  const unsigned lo = smem_u32(lores_dynamic_smem), a = smem_u32(dst);
+  if (a >= lo && a - lo <= size && bytes <= size - (a - lo)) return true;
+  atomicOr(flag, kFlagIndex | (256u << kRgShared));
+  return false;
+}
+
+#define LORES_IN(p, id, ptr, bytes) ::lores::range_ok((p).rg, (id), (ptr), (bytes), (p).flag)
+#define LORES_IN_SMEM(p, dst, bytes) ::lores::smem_range_ok((dst), (bytes), (p).flag)
+#define LORES_RANGES ::lores::Ranges rg;
+#define LORES_LDG(p, id, ptr) (LORES_IN(p, id, ptr, 4) ? __ldg(ptr) : 0.0f)
+#else
+#define LORES_LDG(p, id, ptr) __ldg(ptr)
+#define LORES_IN(p, id, ptr, bytes) true
+#define LORES_IN_SMEM(p, dst, bytes) true
+#define LORES_RANGES
+#endif
 
 // 16 code bytes at an address that is only 8-byte aligned (rows of per-channel
 // precision heads: key groups of 8 and 16 bytes back to back), as two 8-byte accesses.

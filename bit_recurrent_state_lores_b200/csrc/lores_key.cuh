@@ -42,6 +42,7 @@ struct KeyParams {
   // scales, k, q, alpha, v at the sm_* offsets inside it; opart, ow, cm are absolute
   int stage0, stage_bytes, nstage;
   int sm_codes, sm_scales, sm_k, sm_q, sm_a, sm_v, sm_opart, sm_ow, sm_cm;
+  LORES_RANGES                  // index-checked build: the extent of every buffer of the launch
 };
 
 using KeyFn = void (*)(const KeyParams);
@@ -54,7 +55,7 @@ using KeyFn = void (*)(const KeyParams);
 // tiny column, or a NaN marker for a bad one.  Every thread of the CTA calls this together.
 template <int DK>
 __device__ __forceinline__ void column_inverses(float (&cm)[16], float *smcm, float r, float inv_r,
-                                                float *gscales, unsigned *flag) {
+                                                float *gscales, unsigned *flag, bool store = true) {
   constexpr int LPR = DK / 16;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int lir = lane % LPR, riw = lane / LPR;
@@ -71,7 +72,7 @@ __device__ __forceinline__ void column_inverses(float (&cm)[16], float *smcm, fl
     for (int w2 = 1; w2 < kWarps; ++w2) m = max_nan(m, smcm[w2 * DK + j]);
     const bool bad = !(m <= 0x1p100f);
     const bool scaled = !bad && m >= 0x1p-100f;
-    gscales[j] = scaled ? __fmul_rn(m, inv_r) : 0.0f;
+    if (store) gscales[j] = scaled ? __fmul_rn(m, inv_r) : 0.0f;
     if (bad) atomicOr(flag, kFlagNonFinite);
     smcm[j] = bad ? __uint_as_float(0x7FC00000u) : (scaled ? __fmul_rn(r, recip_nr(m)) : 0.0f);
   }
@@ -88,12 +89,17 @@ __device__ __forceinline__ void issue_key_tile(const KeyParams &p, long long t, 
   const unsigned cb = (unsigned)(p.d_v * row_bytes(DK, bits)), sb = bits == 32 ? 0u : DK * 4u;
   const unsigned vec = DK * 4, vb = (unsigned)(p.d_v * 4);
   mbar_expect_tx(bar, cb + sb + 2 * vec + vb + (p.diag ? vec : 0u));
-  bulk_g2s(st + p.sm_codes, p.codes + b * p.seq_bytes + __ldg(p.head_off + head), cb, bar);
-  if (sb) bulk_g2s(st + p.sm_scales, p.scales + t * DK, sb, bar);
-  bulk_g2s(st + p.sm_k, p.k + t * DK, vec, bar);
-  bulk_g2s(st + p.sm_q, p.q + t * DK, vec, bar);
-  bulk_g2s(st + p.sm_v, p.v + t * p.d_v, vb, bar);
-  if (p.diag) bulk_g2s(st + p.sm_a, p.alpha + t * DK, vec, bar);
+  // (index-checked build: a copy outside its buffer or the stage is not issued)
+  auto copy = [&](int off, int rid, const void *src, unsigned bytes) {
+    (void)rid;
+    if (LORES_IN(p, rid, src, bytes) && LORES_IN_SMEM(p, st + off, bytes)) bulk_g2s(st + off, src, bytes, bar);
+  };
+  copy(p.sm_codes, kRgCodes, p.codes + b * p.seq_bytes + __ldg(p.head_off + head), cb);
+  if (sb) copy(p.sm_scales, kRgScales, p.scales + t * DK, sb);
+  copy(p.sm_k, kRgK, p.k + t * DK, vec);
+  copy(p.sm_q, kRgQ, p.q + t * DK, vec);
+  copy(p.sm_v, kRgV, p.v + t * p.d_v, vb);
+  if (p.diag) copy(p.sm_a, kRgAlpha, p.alpha + t * DK, vec);
 }
 
 // One tile: STORE is the storage class of the tile's head (4 nibbles, 8 one byte per
@@ -168,8 +174,9 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
     if (LOAD) {
       if (!active) continue;
       const float2 *src = reinterpret_cast<const float2 *>(p.S + (tile * p.d_v + lr) * DK + col0);
+      const bool in = LORES_IN(p, kRgS, src, 64);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = src[e];
+      for (int e = 0; e < 8; ++e) x[e] = in ? src[e] : make_float2(0.0f, 0.0f);
     } else {
       // every lane of the warp takes the shuffles; only real rows keep w and the shares
       const int lrr = active ? lr : 0;
@@ -194,9 +201,10 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
     }
     if (STORE == 32) {
       float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
+      if (LORES_IN(p, kRgCodes, dst, 64))
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        dst[c] = make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y);
+        for (int c = 0; c < 4; ++c)
+          dst[c] = make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y);
 #pragma unroll
       for (int e = 0; e < 8; ++e) bad32 |= !isfinite(x[e].x) || !isfinite(x[e].y);
     } else {
@@ -220,7 +228,7 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
       float acc = 0.0f;
 #pragma unroll
       for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
-      go[r] = __fmaf_rn(ow[r], kq, acc);
+      if (LORES_IN(p, kRgO, go + r, 4)) go[r] = __fmaf_rn(ow[r], kq, acc);
     }
     __syncwarp();
   }
@@ -229,7 +237,8 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
   } else {
     const float r = (float)((1 << (bits - 1)) - 1);
     const float inv_r = __fdiv_rn(1.0f, r);
-    column_inverses<DK>(cm, smcm, r, inv_r, p.scales + tile * DK, p.flag);
+    column_inverses<DK>(cm, smcm, r, inv_r, p.scales + tile * DK, p.flag,
+                        LORES_IN(p, kRgScales, p.scales + tile * DK, DK * 4));
     float2 inv[8];
     unsigned badcols = 0;                        // bit e: column col0 + e is bad
 #pragma unroll
@@ -268,8 +277,9 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
       float2 x[8];
       if (LOAD) {
         const float2 *src = reinterpret_cast<const float2 *>(p.S + (tile * p.d_v + lr) * DK + col0);
+        const bool in = LORES_IN(p, kRgS, src, 64);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = src[e];
+        for (int e = 0; e < 8; ++e) x[e] = in ? src[e] : make_float2(0.0f, 0.0f);
       } else {
         float2 sp[8];
         row_sp(lr, sp);
@@ -296,11 +306,13 @@ __device__ __forceinline__ void key_tile(const KeyParams &p, long long tile, int
         uint2 w = pack_i4(t);
         w.x &= keep[0];
         w.y &= keep[1];
-        *reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8) = w;
+        if (LORES_IN(p, kRgCodes, gcodes + (size_t)lr * RB + lir * 8, 8))
+          *reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + lir * 8) = w;
       } else {
         uint4 w = pack_i8(t);
         w.x &= keep[0]; w.y &= keep[1]; w.z &= keep[2]; w.w &= keep[3];
-        *reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16) = w;
+        if (LORES_IN(p, kRgCodes, gcodes + (size_t)lr * RB + lir * 16, 16))
+          *reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + lir * 16) = w;
       }
     }
   }
@@ -345,8 +357,8 @@ __global__ void __launch_bounds__(kThreads) decode_step_key_kernel(const KeyPara
     const int s = n % p.nstage;
     uint8_t *st = smem + p.stage0 + s * p.stage_bytes;
     const int bits = __ldg(p.head_bits + (int)(tile % p.H));
-    const float alpha_s = (LOAD || p.diag) ? 1.0f : __ldg(p.alpha + tile);
-    const float beta = LOAD ? 0.0f : __ldg(p.beta + tile);
+    const float alpha_s = (LOAD || p.diag) ? 1.0f : LORES_LDG(p, kRgAlpha, p.alpha + tile);
+    const float beta = LOAD ? 0.0f : LORES_LDG(p, kRgBeta, p.beta + tile);
     if (bits == 32)
       key_tile<DK, 32, SR, LOAD>(p, tile, bits, st, alpha_s, beta, skey, opart, ow, smcm);
     else if (bits == 4)

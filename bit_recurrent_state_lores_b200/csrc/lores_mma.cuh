@@ -372,20 +372,23 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, uint8_t *stage, in
     const float wA = DELTA ? __fmul_rn(t.beta, __fsub_rn(vA, uA)) : __fmul_rn(t.beta, vA);
     const float wB = DELTA ? __fmul_rn(t.beta, __fsub_rn(vB, uB)) : __fmul_rn(t.beta, vB);
     if (tq == 0) {
-      if (v0) go[r0] = __fmaf_rn(wA, t.kq, qA);
-      if (v1) go[r1] = __fmaf_rn(wB, t.kq, qB);
+      if (v0 && LORES_IN(p, kRgO, go + r0, 4)) go[r0] = __fmaf_rn(wA, t.kq, qA);
+      if (v1 && LORES_IN(p, kRgO, go + r1, 4)) go[r1] = __fmaf_rn(wB, t.kq, qB);
     }
     // dither counter of the row's quad 0: tile key + golden (row d_k/4 + 1)
     const uint32_t cb0 = t.tkey + 0x9E3779B9u * ((uint32_t)(d.row0 + r0) * (uint32_t)(DK / 4) + 1u);
     const uint32_t cb1 = cb0 + 0x9E3779B9u * (uint32_t)(8 * DK / 4);
     float2 sn;
     bool badA, badB;
+    // (index-checked build: a row outside the code pool is not stored)
+    const bool s0 = v0 && (to_stage || LORES_IN(p, kRgCodes, gcodes + r0 * RB, RB));
+    const bool s1 = v1 && (to_stage || LORES_IN(p, kRgCodes, gcodes + r1 * RB, RB));
     mma_rows2<DK, BITS, DIAG, SR, TO_STAGE>(c0, c1, make_float2(sA, sB), sa, t.alpha, make_float2(wA, wB),
                                             sk, d.r, d.inv_r, cb0, cb1, gcodes + r0 * RB,
-                                            gcodes + r1 * RB, v0, v1, sn, badA, badB);
+                                            gcodes + r1 * RB, s0, s1, sn, badA, badB);
     if (tq == 0) {
-      if (v0) gs[r0] = sn.x;
-      if (v1) gs[r1] = sn.y;
+      if (v0 && (to_stage || LORES_IN(p, kRgScales, gs + r0, 4))) gs[r0] = sn.x;
+      if (v1 && (to_stage || LORES_IN(p, kRgScales, gs + r1, 4))) gs[r1] = sn.y;
     }
     badmask |= (badA && v0 ? 1u : 0u) << (2 * sp);
     badmask |= (badB && v1 ? 1u : 0u) << (2 * sp + 1);
@@ -400,10 +403,11 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, uint8_t *stage, in
         if (!((badmask >> (2 * sp + h)) & 1u)) continue;
         const int r = 16 * sp + g + 8 * h;
         uint8_t *row = gcodes + r * RB;
-        for (int c = 0; c < Gm::NCH; ++c)
-          for (int by = 0; by < Gm::CH * BITS / 8; ++by) row[(BITS == 8 ? Gm::col(tq, c) : Gm::col(tq, c) / 2) + by] = 0;
+        if (to_stage || LORES_IN(p, kRgCodes, row, RB))
+          for (int c = 0; c < Gm::NCH; ++c)
+            for (int by = 0; by < Gm::CH * BITS / 8; ++by) row[(BITS == 8 ? Gm::col(tq, c) : Gm::col(tq, c) / 2) + by] = 0;
         if (tq == 0) {
-          gs[r] = 0.0f;
+          if (to_stage || LORES_IN(p, kRgScales, gs + r, 4)) gs[r] = 0.0f;
           atomicOr(p.flag, kFlagNonFinite);
         }
       }
@@ -454,8 +458,8 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
   float beta_c = 0.0f, alpha_c = 0.0f;
   if (!MT) {
     const int t0 = cur.b * H + tbl[cur.ub].head;
-    beta_c = __ldg(p.beta + t0);
-    if (!DIAG) alpha_c = __ldg(p.alpha + t0);
+    beta_c = LORES_LDG(p, kRgBeta, p.beta + t0);
+    if (!DIAG) alpha_c = LORES_LDG(p, kRgAlpha, p.alpha + t0);
   }
 #pragma unroll 1
   for (int n = 0; n < count; ++n) {
@@ -466,8 +470,8 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
     float beta_n = 0.0f, alpha_n = 0.0f;
     if (!MT && n + 1 < count) {
       const int tn = nx.b * H + tbl[nx.ub].head;
-      beta_n = __ldg(p.beta + tn);
-      if (!DIAG) alpha_n = __ldg(p.alpha + tn);
+      beta_n = LORES_LDG(p, kRgBeta, p.beta + tn);
+      if (!DIAG) alpha_n = LORES_LDG(p, kRgAlpha, p.alpha + tn);
     }
     const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1), p.wait_ns);
     if (!__all_sync(kFull, ok)) {
@@ -489,7 +493,11 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
         const float *k = p.k + tok * p.tok_qk + (long long)tl * DK;
         const float *q = p.q + tok * p.tok_qk + (long long)tl * DK;
         const float *al = p.alpha + tok * p.tok_a + (long long)tl * DK;
-        const float a_s = DIAG ? 0.0f : __ldg(p.alpha + tok * p.tok_a + tl);
+        if (!(LORES_IN(p, kRgK, k, DK * 4) && LORES_IN(p, kRgQ, q, DK * 4) &&
+              LORES_IN(p, kRgV, p.v + tok * p.tok_v + (long long)tl * p.d_v + d.row0, d.nrows * 4) &&
+              (!DIAG || LORES_IN(p, kRgAlpha, al, DK * 4))))
+          continue;                            // index-checked build: vectors out of range
+        const float a_s = DIAG ? 0.0f : LORES_LDG(p, kRgAlpha, p.alpha + tok * p.tok_a + tl);
         mma_tile<DK, DIAG>(k, q, al, a_s, planes, t);
         double kqd = 0.0;
 #pragma unroll
@@ -498,7 +506,7 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
         for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
         t.kq = (float)kqd;
         t.tkey = tile_key(step_key_dev(p.seed, p.step0 + (uint64_t)tok), (uint32_t)tl);
-        t.beta = __ldg(p.beta + tok * p.tok_b + tl);
+        t.beta = LORES_LDG(p, kRgBeta, p.beta + tok * p.tok_b + tl);
         t.alpha = a_s;
         const float *sv = p.v + tok * p.tok_v + (long long)tl * p.d_v + d.row0;
         float *go = p.o + tok * p.tok_o + (long long)tl * p.d_v + d.row0;

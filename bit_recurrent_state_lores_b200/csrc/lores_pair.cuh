@@ -62,15 +62,17 @@ __device__ __forceinline__ void pair_issue(const StepParams &p, const UnitDesc &
     mbar_expect_tx(bar, cbytes + sbytes + vbytes + (vec ? (DIAG ? 3u : 2u) * kVec : 0u));
   __syncwarp();
   const void *src = nullptr;
-  int dst = 0;
+  int dst = 0, rid = kRgCodes;
   unsigned bytes = 0;
   if (lane == 0) { src = p.codes + (long long)b * p.seq_bytes + d.code_off; dst = 0; bytes = cbytes; }
-  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; }
-  if (!MT && lane == 2) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
-  if (vec && lane == 3) { src = p.k + tile * DK; dst = p.st_k; bytes = kVec; }
-  if (vec && lane == 4) { src = p.q + tile * DK; dst = p.st_q; bytes = kVec; }
-  if (vec && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = kVec; }
-  if (bytes && !withhold) bulk_g2s(stage + dst, src, bytes, bar);
+  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; rid = kRgScales; }
+  if (!MT && lane == 2) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; rid = kRgV; }
+  if (vec && lane == 3) { src = p.k + tile * DK; dst = p.st_k; bytes = kVec; rid = kRgK; }
+  if (vec && lane == 4) { src = p.q + tile * DK; dst = p.st_q; bytes = kVec; rid = kRgQ; }
+  if (vec && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = kVec; rid = kRgAlpha; }
+  (void)rid;
+  if (bytes && !withhold && LORES_IN(p, rid, src, bytes) && LORES_IN_SMEM(p, stage + dst, bytes))
+    bulk_g2s(stage + dst, src, bytes, bar);
 }
 
 // 16 codes of one lane's row -> exact floats in column pairs.
@@ -238,14 +240,15 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, uint8_t *stage, i
     uint32_t wA[4], wB[4];
     quantize16<BITS, SR>(spA, dup2(inv2.x), hA, wA);
     quantize16<BITS, SR>(spB, dup2(inv2.y), hB, wB);
-    pair_store<BITS>(gc + oc, wA, MT && to_stage);
-    pair_store<BITS>(gc + oc + RB, wB, MT && to_stage);
+    const bool st = MT && to_stage;
+    if (st || LORES_IN(p, kRgCodes, gc + oc, LB)) pair_store<BITS>(gc + oc, wA, st);
+    if (st || LORES_IN(p, kRgCodes, gc + oc + RB, LB)) pair_store<BITS>(gc + oc + RB, wB, st);
     if (scale_writer) {
       if (GROW) {
-        *reinterpret_cast<float2 *>(gs + orow) = s2;
+        if (st || LORES_IN(p, kRgScales, gs + orow, 8)) *reinterpret_cast<float2 *>(gs + orow) = s2;
       } else {
-        gs[orow * ng] = s2.x;
-        gs[(orow + 1) * ng] = s2.y;
+        if (st || LORES_IN(p, kRgScales, gs + orow * ng, 4)) gs[orow * ng] = s2.x;
+        if (st || LORES_IN(p, kRgScales, gs + (orow + 1) * ng, 4)) gs[(orow + 1) * ng] = s2.y;
       }
     }
     badmask |= (badA ? 1u : 0u) << (2 * n);
@@ -262,8 +265,11 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, uint8_t *stage, i
         const unsigned bal = __ballot_sync(kFull, (badmask >> (2 * n + h)) & 1u);
         if ((bal & rowmask) == 0u) continue;
         const uint32_t z[4] = {0u, 0u, 0u, 0u};
-        pair_store<BITS>(gc + n * 2 * RPW * RB + h * RB, z, MT && to_stage);
-        if (scale_writer) gs[(n * 2 * RPW + h) * ng] = 0.0f;
+        const bool st = MT && to_stage;
+        if (st || LORES_IN(p, kRgCodes, gc + n * 2 * RPW * RB + h * RB, LB))
+          pair_store<BITS>(gc + n * 2 * RPW * RB + h * RB, z, st);
+        if (scale_writer && (st || LORES_IN(p, kRgScales, gs + (n * 2 * RPW + h) * ng, 4)))
+          gs[(n * 2 * RPW + h) * ng] = 0.0f;
         if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
       }
     }
@@ -286,7 +292,7 @@ __device__ __forceinline__ void pair_unit(const StepParams &p, uint8_t *stage, i
 #pragma unroll
       for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
     }
-    go[r] = __fmaf_rn(ow[r], t.kq, acc);
+    if (LORES_IN(p, kRgO, go + r, 4)) go[r] = __fmaf_rn(ow[r], t.kq, acc);
   }
   __syncwarp();
 }
@@ -350,8 +356,8 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
   float beta_c = 0.0f, alpha_c = 0.0f;
   if (!MT) {
     const int t0 = cur.b * H + tbl[cur.ub].head;
-    beta_c = __ldg(p.beta + t0);
-    if (!DIAG) alpha_c = __ldg(p.alpha + t0);
+    beta_c = LORES_LDG(p, kRgBeta, p.beta + t0);
+    if (!DIAG) alpha_c = LORES_LDG(p, kRgAlpha, p.alpha + t0);
   }
 #pragma unroll 1
   for (int n = 0; n < count; ++n) {
@@ -362,8 +368,8 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
     float beta_n = 0.0f, alpha_n = 0.0f;
     if (!MT && n + 1 < count) {
       const int tn = nx.b * H + tbl[nx.ub].head;
-      beta_n = __ldg(p.beta + tn);
-      if (!DIAG) alpha_n = __ldg(p.alpha + tn);
+      beta_n = LORES_LDG(p, kRgBeta, p.beta + tn);
+      if (!DIAG) alpha_n = LORES_LDG(p, kRgAlpha, p.alpha + tn);
     }
     const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1), p.wait_ns);
     if (!__all_sync(kFull, ok)) {
@@ -385,6 +391,10 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
       for (int tok = 0; tok < p.T; ++tok) {
         const float *k = p.k + tok * p.tok_qk + (long long)tl * DK;
         const float *q = p.q + tok * p.tok_qk + (long long)tl * DK;
+        if (!(LORES_IN(p, kRgK, k, DK * 4) && LORES_IN(p, kRgQ, q, DK * 4) &&
+              LORES_IN(p, kRgV, p.v + tok * p.tok_v + (long long)tl * p.d_v + d.row0, d.nrows * 4) &&
+              (!DIAG || LORES_IN(p, kRgAlpha, p.alpha + tok * p.tok_a + (long long)tl * DK, DK * 4))))
+          continue;                            // index-checked build: vectors out of range
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float4 k4 = __ldg(reinterpret_cast<const float4 *>(k + col0) + c);
@@ -407,8 +417,8 @@ __device__ __forceinline__ void pair_run(const StepParams &p, const UnitDesc *tb
         for (int st = 16; st >= 1; st >>= 1) kqd += __shfl_xor_sync(kFull, kqd, st);
         t.kq = (float)kqd;
         t.tkey = tile_key(step_key_dev(p.seed, p.step0 + (uint64_t)tok), (uint32_t)tl);
-        t.beta = __ldg(p.beta + tok * p.tok_b + tl);
-        t.alpha = DIAG ? 0.0f : __ldg(p.alpha + tok * p.tok_a + tl);
+        t.beta = LORES_LDG(p, kRgBeta, p.beta + tok * p.tok_b + tl);
+        t.alpha = DIAG ? 0.0f : LORES_LDG(p, kRgAlpha, p.alpha + tok * p.tok_a + tl);
         pair_unit<DK, DIAG, DELTA, SR, BITS, GROW, MT>(p, stage, cur.b, d, t, opart, ow, tok,
                                                        tok + 1 < p.T);
       }

@@ -80,6 +80,7 @@ struct StepParams {
   // unit fault_ub of sequence fault_b are withheld (fault_b = -1: none)
   unsigned long long wait_ns;
   int fault_b, fault_ub;
+  LORES_RANGES           // index-checked build: the extent of every buffer of the launch
 };
 
 // Step key of the dither: SplitMix64 (Steele, Lea & Flood 2014; Vigna's constants) of the
@@ -139,15 +140,17 @@ __device__ __forceinline__ void issue_unit(const StepParams &p, const UnitDesc *
     mbar_expect_tx(bar, cbytes + sbytes + (MT ? 0u : vbytes + 2 * vec + (DIAG ? vec : 0u)));
   __syncwarp();
   const void *src = nullptr;
-  int dst = 0;
+  int dst = 0, rid = kRgCodes;
   unsigned bytes = 0;
   if (lane == 0) { src = p.codes + (long long)b * p.seq_bytes + d.code_off; dst = 0; bytes = cbytes; }
-  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; }
-  if (!MT && lane == 2) { src = p.k + tile * DK; dst = p.st_k; bytes = vec; }
-  if (!MT && lane == 3) { src = p.q + tile * DK; dst = p.st_q; bytes = vec; }
-  if (!MT && lane == 4) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; }
-  if (!MT && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = vec; }
-  if (bytes && !withhold) bulk_g2s(stage + dst, src, bytes, bar);
+  if (lane == 1) { src = p.scales + (tile * p.d_v + d.row0) * p.ng; dst = p.st_scales; bytes = sbytes; rid = kRgScales; }
+  if (!MT && lane == 2) { src = p.k + tile * DK; dst = p.st_k; bytes = vec; rid = kRgK; }
+  if (!MT && lane == 3) { src = p.q + tile * DK; dst = p.st_q; bytes = vec; rid = kRgQ; }
+  if (!MT && lane == 4) { src = p.v + tile * p.d_v + d.row0; dst = p.st_v; bytes = vbytes; rid = kRgV; }
+  if (!MT && DIAG && lane == 5) { src = p.alpha + tile * DK; dst = p.st_a; bytes = vec; rid = kRgAlpha; }
+  (void)rid;
+  if (bytes && !withhold && LORES_IN(p, rid, src, bytes) && LORES_IN_SMEM(p, stage + dst, bytes))
+    bulk_g2s(stage + dst, src, bytes, bar);
 }
 
 // -------------------------------------------------------------------------------------
@@ -203,6 +206,9 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
                       : reinterpret_cast<const float *>(stage + p.st_a);
   float *ss = reinterpret_cast<float *>(stage + p.st_scales);
   const bool to_stage = MT && t + 1 < p.T;   // not the last token: rows go back to the stage
+  if (MT && !(LORES_IN(p, kRgK, sk, DK * 4) && LORES_IN(p, kRgQ, sq, DK * 4) &&
+              LORES_IN(p, kRgV, sv, d.nrows * 4) && (!DIAG || LORES_IN(p, kRgAlpha, sa, DK * 4))))
+    return;                                  // index-checked build: vectors out of range
   // element pair e holds columns (col0 + 2e, col0 + 2e + 1)
   float2 kk[8], qq[8], aa[8];
 #pragma unroll
@@ -371,9 +377,10 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
             dst[c] = make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y);
         } else {
           float4 *dst = reinterpret_cast<float4 *>(gcodes + (size_t)lr * RB) + lir * 4;
+          if (LORES_IN(p, kRgCodes, dst, 64))
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            __stcs(dst + c, make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y));
+            for (int c = 0; c < 4; ++c)
+              __stcs(dst + c, make_float4(x[2 * c].x, x[2 * c].y, x[2 * c + 1].x, x[2 * c + 1].y));
         }
       }
     } else {
@@ -385,9 +392,10 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
         float2 inv;
         gbad = group_scale(m, rq, rq_inv, inv, s_new);
         const DenseLane dl = quantize16_dense<DB, SR>(x, inv, hw);
-        if (active) {
+        if (active && (to_stage || LORES_IN(p, kRgCodes, gcodes + (size_t)lr * RB, RB))) {
           st_dense<DB>((to_stage ? stage : gcodes) + (size_t)lr * RB, DK, lir, dl);
-          if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = s_new;
+          if (scale_writer && (to_stage || LORES_IN(p, kRgScales, gscales + lr * ng + g, 4)))
+            (to_stage ? ss : gscales)[lr * ng + g] = s_new;
         }
       } else if (BITS == 0) {
         // group scale with every lane, then each lane packs at its own width
@@ -414,17 +422,18 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
             *reinterpret_cast<uint2 *>(stage + (size_t)lr * RB + loff) = make_uint2(words[0], words[1]);
           if (scale_writer) ss[lr * ng + g] = s_new;
         } else {
-          if (w8 && BITS == 0) {
-            uint2 *dst = reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + loff);
+          uint8_t *cdst = gcodes + (size_t)lr * RB + loff;
+          if (!LORES_IN(p, kRgCodes, cdst, w8 ? 16 : 8)) {
+          } else if (w8 && BITS == 0) {
+            uint2 *dst = reinterpret_cast<uint2 *>(cdst);
             __stcs(dst, make_uint2(words[0], words[1]));
             __stcs(dst + 1, make_uint2(words[2], words[3]));
           } else if (w8) {
-            __stcs(reinterpret_cast<uint4 *>(gcodes + (size_t)lr * RB + loff),
-                   make_uint4(words[0], words[1], words[2], words[3]));
+            __stcs(reinterpret_cast<uint4 *>(cdst), make_uint4(words[0], words[1], words[2], words[3]));
           } else
-            __stcs(reinterpret_cast<uint2 *>(gcodes + (size_t)lr * RB + loff),
-                   make_uint2(words[0], words[1]));
-          if (scale_writer) gscales[lr * ng + g] = s_new;
+            __stcs(reinterpret_cast<uint2 *>(cdst), make_uint2(words[0], words[1]));
+          if (scale_writer && LORES_IN(p, kRgScales, gscales + lr * ng + g, 4))
+            gscales[lr * ng + g] = s_new;
         }
       }
     }
@@ -440,17 +449,20 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
       const unsigned bal = __ballot_sync(kFull, (badmask >> n) & 1u);
       const int lr = n * RPW + riw;
       if ((bal & rowmask) == 0u || !(FULL || lr < d.nrows)) continue;
+      const bool sok = to_stage || LORES_IN(p, kRgScales, gscales + lr * ng + g, 4);
       if (DENSE) {
-        st_dense<DENSE ? BITS : 5>((to_stage ? stage : gcodes) + (size_t)lr * RB, DK, lir,
-                                   DenseLane{0u, 0u, 0u, 0u});
-        if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
+        if (to_stage || LORES_IN(p, kRgCodes, gcodes + (size_t)lr * RB, RB))
+          st_dense<DENSE ? BITS : 5>((to_stage ? stage : gcodes) + (size_t)lr * RB, DK, lir,
+                                     DenseLane{0u, 0u, 0u, 0u});
+        if (scale_writer && sok) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
       } else if (BITS != 32) {
         uint8_t *dst = (to_stage ? stage : gcodes) + (size_t)lr * RB + loff;
-        if (w8)
+        if (!to_stage && !LORES_IN(p, kRgCodes, dst, w8 ? 16 : 8)) {
+        } else if (w8)
           st16_a8(dst, make_uint4(0, 0, 0, 0));
         else
           *reinterpret_cast<uint2 *>(dst) = make_uint2(0, 0);
-        if (scale_writer) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
+        if (scale_writer && sok) (to_stage ? ss : gscales)[lr * ng + g] = 0.0f;
       }
       if (lir == 0) atomicOr(p.flag, kFlagNonFinite);
     }
@@ -471,7 +483,7 @@ __device__ __forceinline__ void compute_unit(const StepParams &p, uint8_t *stage
 #pragma unroll
       for (int l = 0; l < LPR; ++l) acc = __fadd_rn(acc, opart[r * LPR + l]);
     }
-    go[r] = __fmaf_rn(ow[r], kq, acc);
+    if (LORES_IN(p, kRgO, go + r, 4)) go[r] = __fmaf_rn(ow[r], kq, acc);
   }
   __syncwarp();
 }
@@ -593,8 +605,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
   float alpha_cur = 0.0f, beta_cur;
   {
     const long long t0 = (long long)cur.b * p.H + tbl[cur.ub].head;
-    beta_cur = __ldg(p.beta + t0);
-    if (!DIAG) alpha_cur = __ldg(p.alpha + t0);
+    beta_cur = LORES_LDG(p, kRgBeta, p.beta + t0);
+    if (!DIAG) alpha_cur = LORES_LDG(p, kRgAlpha, p.alpha + t0);
   }
 
   for (int n = 0; cur.ub < ups; ++n) {
@@ -603,8 +615,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
     float alpha_nx = 0.0f, beta_nx = 0.0f;
     if (nxt.ub < ups) {
       const long long tn = (long long)nxt.b * p.H + tbl[nxt.ub].head;
-      beta_nx = __ldg(p.beta + tn);
-      if (!DIAG) alpha_nx = __ldg(p.alpha + tn);
+      beta_nx = LORES_LDG(p, kRgBeta, p.beta + tn);
+      if (!DIAG) alpha_nx = LORES_LDG(p, kRgAlpha, p.alpha + tn);
     }
     const bool ok = mbar_wait_bounded(&bars[s], (unsigned)((n / kStages) & 1), p.wait_ns);
     if (!__all_sync(kFull, ok)) {
@@ -623,8 +635,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_step_kernel(const StepPara
       // every token of the unit in turn; the unit's rows stay in the stage in between
       const long long tile = (long long)cur.b * p.H + d.head;
       for (int t = 0; t < p.T; ++t) {
-        const float beta_t = __ldg(p.beta + t * p.tok_b + tile);
-        const float alpha_t = DIAG ? 0.0f : __ldg(p.alpha + t * p.tok_a + tile);
+        const float beta_t = LORES_LDG(p, kRgBeta, p.beta + t * p.tok_b + tile);
+        const float alpha_t = DIAG ? 0.0f : LORES_LDG(p, kRgAlpha, p.alpha + t * p.tok_a + tile);
         compute_bits<DK, DIAG, DELTA, SR, MT, EXT>(p, stage, cur.b, d, alpha_t, beta_t, opart, ow, t);
       }
     } else {

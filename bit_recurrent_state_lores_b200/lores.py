@@ -11,6 +11,8 @@ import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblores.so")
+# the index-checked build of the same sources (a debugging aid, not the product)
+CHECKED_LIB_PATH = os.path.join(_PKG, "liblores_checked.so")
 
 LORES_OK = 0
 LORES_ERR_INVALID_ARG = 1
@@ -20,6 +22,7 @@ LORES_ERR_NONFINITE = 4
 LORES_ERR_UNSUPPORTED = 5
 LORES_ERR_TIMEOUT = 6
 LORES_ERR_CORRUPT = 7
+LORES_ERR_INDEX = 8
 
 
 class LoresError(RuntimeError):
@@ -45,11 +48,14 @@ class lores_layout(C.Structure):
                 ("step_kernel", C.c_int32)]
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m "
+def load_library(path=LIB_PATH):
+    """Load a build of the library (the product, or CHECKED_LIB_PATH) and declare its
+    signatures.  The functions below call the module's `_lib`; a caller that wants the
+    index-checked build swaps it in before creating handles."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m "
                           "bit_recurrent_state_lores_b200.build` (needs nvcc)")
-    L = C.CDLL(LIB_PATH)
+    L = C.CDLL(path)
     P, U64, I32, F32 = C.c_void_p, C.c_uint64, C.c_int32, C.c_float
     sig = {
         "lores_create": (I32, [C.POINTER(lores_config), C.POINTER(P)]),
@@ -71,6 +77,9 @@ def _load():
         "lores_set_fault_injection": (I32, [P, I32, I32, C.c_uint32]),
         "lores_assign_bits_by_decay": (I32, [P, I32, F32, I32, I32, P]),
         "lores_status_string": (C.c_char_p, [I32]),
+        "lores_index_checked": (I32, []),
+        "lores_debug_trim_range": (I32, [P, I32, U64]),
+        "lores_debug_last_flags": (I32, [P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -78,7 +87,7 @@ def _load():
     return L
 
 
-_lib = _load()
+_lib = load_library()
 
 
 def _ptr(x):
@@ -222,10 +231,11 @@ def lores_get_layout(h, heads=None):
 
 
 def lores_check_errors(h, stream=None):
-    """Returns the status (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT or
-    LORES_ERR_CORRUPT); raises on other failures."""
+    """Returns the status (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT,
+    LORES_ERR_CORRUPT or LORES_ERR_INDEX); raises on other failures."""
     st = _lib.lores_check_errors(h, _stream(stream))
-    if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT, LORES_ERR_CORRUPT):
+    if st not in (LORES_OK, LORES_ERR_NONFINITE, LORES_ERR_TIMEOUT, LORES_ERR_CORRUPT,
+                  LORES_ERR_INDEX):
         raise LoresError(st, "lores_check_errors")
     return st
 
@@ -235,6 +245,24 @@ def lores_set_fault_injection(h, seq, unit=0, wait_us=0):
     `seq` (-1: none) and bound every wait by `wait_us` microseconds (0: the default)."""
     _check(_lib.lores_set_fault_injection(h, int(seq), int(unit), int(wait_us)),
            "lores_set_fault_injection")
+
+
+def lores_index_checked():
+    """True in the index-checked build."""
+    return bool(_lib.lores_index_checked())
+
+
+def lores_debug_trim_range(h, which, nbytes):
+    """Index-checked build: declare buffer `which` (0 codes, 1 scales, 2 q, 3 k, 4 v,
+    5 alpha, 6 beta, 7 o, 8 the fp32 state) `nbytes` shorter on later launches of h."""
+    _check(_lib.lores_debug_trim_range(h, int(which), int(nbytes)), "lores_debug_trim_range")
+
+
+def lores_debug_last_flags(h):
+    """The raw error word the last lores_check_errors on h read."""
+    f = C.c_uint32()
+    _check(_lib.lores_debug_last_flags(h, C.byref(f)), "lores_debug_last_flags")
+    return f.value
 
 
 def lores_assign_bits_by_decay(mean_decay, frac_high, bits_high=8, bits_low=4):

@@ -51,7 +51,8 @@ typedef enum {
     LORES_ERR_NONFINITE = 4,     /* a state row became non-finite (inf or NaN)            */
     LORES_ERR_UNSUPPORTED = 5,   /* well-formed but not supported (bits, d_k, device)     */
     LORES_ERR_TIMEOUT = 6,       /* a kernel gave up waiting on its own copies            */
-    LORES_ERR_CORRUPT = 7        /* the guard bands around the state were overwritten      */
+    LORES_ERR_CORRUPT = 7,       /* the guard bands around the state were overwritten      */
+    LORES_ERR_INDEX = 8          /* index-checked build: an access fell outside its buffer */
 } lores_status;
 
 typedef struct lores_handle lores_handle;
@@ -266,8 +267,10 @@ lores_status lores_get_layout(const lores_handle *h, lores_layout *out, int64_t 
 
 /* Wait for `stream`, then read and clear the handle's sticky device flag and verify
  * the 256-byte guard bands written around the code pool and the scales at creation.
- * Returns LORES_ERR_TIMEOUT if a kernel gave up waiting on its own copies (its
- * outputs for that call are incomplete), else LORES_ERR_CORRUPT if a guard band was
+ * Returns LORES_ERR_INDEX if (index-checked build only, see lores_index_checked) a
+ * kernel skipped an access outside its buffer, else LORES_ERR_TIMEOUT if a kernel gave
+ * up waiting on its own copies (its outputs for that call are incomplete), else
+ * LORES_ERR_CORRUPT if a guard band was
  * overwritten (a write outside the state: a library defect, or a caller's write
  * through a pointer derived from the state), else LORES_ERR_NONFINITE if any row
  * became non-finite since the last check, else LORES_OK. */
@@ -288,6 +291,32 @@ lores_status lores_check_errors(lores_handle *h, void *stream);
  * UNSUPPORTED (withholding on a key-axis handle). */
 lores_status lores_set_fault_injection(lores_handle *h, int32_t seq, int32_t unit,
                                        uint32_t wait_us);
+
+/* Index-checked build (no counterpart on the pages; a stand-in for a memory sanitizer).
+ * liblores_checked.so is this library compiled with LORES_INDEX_CHECKS: every global
+ * access of the decode, loader and dequantizer kernels (bulk copies, their shared-memory
+ * destinations, loads, stores) is first checked against the extent of the buffer it
+ * belongs to, as the host declares it for the launch:
+ *   0 code pool (B * seq_code_bytes)   1 scales (scale_count floats)
+ *   2 q, 3 k (T*B*H*d_k floats)        4 v (T*B*H*d_v)     5 alpha (T*B*H, d_k if diagonal)
+ *   6 beta (T*B*H)                     7 o (T*B*H*d_v)     8 the fp32 state of
+ *   lores_load_state / lores_dequant_state (B*H*d_v*d_k floats)
+ * An access outside its buffer is skipped and raises the handle's INDEX flag together
+ * with bit 8 + the buffer's number (bit 17: a copy outside the launch's shared memory);
+ * a skipped copy leaves its barrier short, so that warp's wait runs out as well.  Outputs
+ * are bit-identical to the ordinary build's when nothing is out of range.
+ *
+ * lores_index_checked: 1 in the index-checked build, 0 in the ordinary one.
+ * lores_debug_trim_range: declare buffer `which` (0..8 above) `bytes` shorter than it is
+ * on every later launch of h, so that the checks see accesses at its end as out of range
+ * (the memory itself is untouched, so nothing can fault); bytes = 0 restores it.  Errors:
+ * INVALID_ARG (NULL, which outside 0..8); UNSUPPORTED in the ordinary build.
+ * lores_debug_last_flags: the raw error word the last lores_check_errors on h read
+ * (bit 0 NONFINITE, bit 1 TIMEOUT, bit 2 INDEX, bits 8.. the buffers).  Errors:
+ * INVALID_ARG (NULL). */
+int32_t lores_index_checked(void);
+lores_status lores_debug_trim_range(lores_handle *h, int32_t which, uint64_t bytes);
+lores_status lores_debug_last_flags(lores_handle *h, uint32_t *flags);
 
 /* Decay-based mixed precision (Table 5 text): the round(frac_high * H) heads with
  * the largest mean decay (slowest to forget) get bits_high, the others bits_low;

@@ -27,11 +27,25 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), f"liblores.so does not export {n}"
     assert "lores_decode_step" in names and "lores_create" in names
+    assert lib.lores_index_checked() == 0
+
+
+def test_checked_library_exports_the_same_symbols():
+    """The index-checked debugging build (when built) exports the same ABI and says so."""
+    from bit_recurrent_state_lores_b200 import lores as L
+    if not os.path.exists(L.CHECKED_LIB_PATH):
+        pytest.skip("liblores_checked.so is not built")
+    lib = L.load_library(L.CHECKED_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"liblores_checked.so does not export {n}"
+    assert lib.lores_index_checked() == 1
+    assert lib.lores_debug_trim_range(None, 0, 0) == L.LORES_ERR_INVALID_ARG
+    assert lib.lores_debug_last_flags(None, None) == L.LORES_ERR_INVALID_ARG
 
 
 def test_status_strings():
     from bit_recurrent_state_lores_b200 import lores as L
-    for s in range(7):
+    for s in range(9):
         assert L.lores_status_string(s) and "unknown" not in L.lores_status_string(s)
     assert "unknown" in L.lores_status_string(99)
 
