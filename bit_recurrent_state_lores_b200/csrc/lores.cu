@@ -706,7 +706,7 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
         h->sp.pair_hi[0] = n8;
         h->sp.pair_lo[1] = n8;
         h->sp.pair_hi[1] = (int)units.size();
-        h->sp.pair_ctas = (int)c8;
+        h->sp.pair_ctas = (int)c8;          // (the tensor-core kernel runs both in every CTA)
       }
       break;
     }

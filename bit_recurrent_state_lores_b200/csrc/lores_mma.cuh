@@ -416,12 +416,13 @@ __device__ __forceinline__ void mma_unit(const StepParams &p, uint8_t *stage, in
 
 // The persistent loop of one warp over the units of one storage class (BITS), as in
 // pair_run: warp gw of W takes units [U gw / W, U (gw + 1) / W) of the class's U units in
-// (sequence, unit) order through a 2-slot ring of bulk copies.
+// (sequence, unit) order through a 2-slot ring of bulk copies; bar0: the first of the
+// warp's barrier slots the ring uses.
 template <int DK, int BITS, bool DIAG, bool DELTA, bool SR, bool MT>
 __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl, uint8_t *wa,
-                                        int cta, int nctas, int lo, int hi) {
+                                        int cta, int nctas, int lo, int hi, int bar0 = 0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(wa);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wa) + bar0;
   float *ow = reinterpret_cast<float *>(wa + 64) + p.opart_floats;
   uint8_t *planes = reinterpret_cast<uint8_t *>(ow + p.ow_floats);
   uint8_t *stages = planes + p.plane_bytes;
@@ -567,8 +568,7 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
 
 // Persistent kernel over the units of heads stored one byte per code (table entries
 // [pair_lo[0], pair_hi[0]) of every sequence) and one nibble per code ([pair_lo[1],
-// pair_hi[1])), all with one scale per value row: CTAs [0, pair_ctas) take the first
-// class, the others the second.
+// pair_hi[1])), all with one scale per value row (pair_ctas is not used).
 template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
 __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -581,12 +581,13 @@ __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kerne
     tbl = stbl;
   }
   __syncthreads();                                  // the only CTA-wide barrier
+  // Every CTA takes its share of the byte class, then its share of the nibble class, so
+  // that an SM runs one class's body at a time (CTAs of both classes side by side on one
+  // SM thrash its instruction cache).  The second class's ring takes fresh barriers.
   const int cta = (int)blockIdx.x;
-  if (cta < p.pair_ctas)
-    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
-  else
-    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
-                                        p.pair_lo[1], p.pair_hi[1]);
+  mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[0], p.pair_hi[0]);
+  mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[1], p.pair_hi[1],
+                                      kStages);
 }
 
 template <int DK, bool SR, bool MT>
