@@ -706,7 +706,12 @@ lores_status lores_create(const lores_config *cfg, lores_handle **out) {
         h->sp.pair_hi[0] = n8;
         h->sp.pair_lo[1] = n8;
         h->sp.pair_hi[1] = (int)units.size();
-        h->sp.pair_ctas = (int)c8;          // (the tensor-core kernel runs both in every CTA)
+        h->sp.pair_ctas = (int)c8;
+        // The tensor-core kernel with two or more units per warp: every CTA takes both
+        // classes in turn, so an SM runs one body at a time (side by side they thrash its
+        // instruction cache).  With fewer, the classes stay in their own CTAs: in turn
+        // they would add a unit's latency to a warp's.
+        if (mma && e8 > 0 && e4 > 0 && total >= 2 * warp_slots) h->sp.pair_ctas = -1;
       }
       break;
     }

@@ -568,7 +568,8 @@ __device__ __forceinline__ void mma_run(const StepParams &p, const UnitDesc *tbl
 
 // Persistent kernel over the units of heads stored one byte per code (table entries
 // [pair_lo[0], pair_hi[0]) of every sequence) and one nibble per code ([pair_lo[1],
-// pair_hi[1])), all with one scale per value row (pair_ctas is not used).
+// pair_hi[1])), all with one scale per value row.  pair_ctas < 0: every CTA takes both
+// classes in turn; else CTAs [0, pair_ctas) take the first class, the others the second.
 template <int DK, bool DIAG, bool DELTA, bool SR, bool MT>
 __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kernel(const StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -581,13 +582,21 @@ __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kerne
     tbl = stbl;
   }
   __syncthreads();                                  // the only CTA-wide barrier
-  // Every CTA takes its share of the byte class, then its share of the nibble class, so
-  // that an SM runs one class's body at a time (CTAs of both classes side by side on one
-  // SM thrash its instruction cache).  The second class's ring takes fresh barriers.
   const int cta = (int)blockIdx.x;
-  mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[0], p.pair_hi[0]);
-  mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[1], p.pair_hi[1],
-                                      kStages);
+  if (p.pair_ctas < 0) {
+    // Every CTA takes its share of the byte class, then its share of the nibble class, so
+    // that an SM runs one class's body at a time (CTAs of both classes side by side on one
+    // SM thrash its instruction cache).  The second class's ring takes fresh barriers.
+    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[0], p.pair_hi[0]);
+    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[1], p.pair_hi[1],
+                                        kStages);
+  } else if (cta < p.pair_ctas) {
+    // about one unit per warp: the classes run side by side, CTAs [0, pair_ctas) the first
+    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
+  } else {
+    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
+                                        p.pair_lo[1], p.pair_hi[1]);
+  }
 }
 
 template <int DK, bool SR, bool MT>
