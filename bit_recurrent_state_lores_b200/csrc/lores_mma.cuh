@@ -582,21 +582,19 @@ __global__ void __launch_bounds__(kThreads, LORES_MMA_MIN_CTAS) decode_mma_kerne
     tbl = stbl;
   }
   __syncthreads();                                  // the only CTA-wide barrier
-  const int cta = (int)blockIdx.x;
-  if (p.pair_ctas < 0) {
-    // Every CTA takes its share of the byte class, then its share of the nibble class, so
-    // that an SM runs one class's body at a time (CTAs of both classes side by side on one
-    // SM thrash its instruction cache).  The second class's ring takes fresh barriers.
-    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[0], p.pair_hi[0]);
-    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, (int)gridDim.x, p.pair_lo[1], p.pair_hi[1],
-                                        kStages);
-  } else if (cta < p.pair_ctas) {
-    // about one unit per warp: the classes run side by side, CTAs [0, pair_ctas) the first
-    mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, cta, p.pair_ctas, p.pair_lo[0], p.pair_hi[0]);
-  } else {
-    mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, cta - p.pair_ctas, (int)gridDim.x - p.pair_ctas,
-                                        p.pair_lo[1], p.pair_hi[1]);
-  }
+  // pair_ctas < 0: every CTA takes its share of the byte class, then its share of the
+  // nibble class, so that an SM runs one class's body at a time (CTAs of both classes side
+  // by side on one SM thrash its instruction cache).  Else CTAs [0, pair_ctas) take the
+  // byte class and the others the nibble class (about one unit per warp: in turn, the
+  // classes would add a unit's latency to a warp's).  The nibble ring takes fresh barriers.
+  const int cta = (int)blockIdx.x, grid = (int)gridDim.x;
+  const bool both = p.pair_ctas < 0;
+  const int c8 = both || cta < p.pair_ctas ? cta : 0;
+  const int n8 = both ? grid : (cta < p.pair_ctas ? p.pair_ctas : 0);
+  const int c4 = both ? cta : cta - p.pair_ctas;
+  const int n4 = both ? grid : (cta < p.pair_ctas ? 0 : grid - p.pair_ctas);
+  mma_run<DK, 8, DIAG, DELTA, SR, MT>(p, tbl, wa, c8, n8, p.pair_lo[0], p.pair_hi[0]);
+  mma_run<DK, 4, DIAG, DELTA, SR, MT>(p, tbl, wa, c4, n4, p.pair_lo[1], p.pair_hi[1], kStages);
 }
 
 template <int DK, bool SR, bool MT>
